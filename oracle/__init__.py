@@ -1,0 +1,254 @@
+"""Plain CPU oracle for the Hadamard-rotated, tensor-wise quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  It shares no code with the CUDA
+library and never imports it.
+
+The arithmetic lives in ``hq_oracle.c`` (plain C, fp32 FWHT without FMA contraction, RNE
+quantizers, int32 / fp64 GEMMs); this module only marshals numpy arrays into it and composes
+the three GEMMs of one linear layer the way the pages describe them:
+
+* "HALO: Hadamard-Assisted Lower-Precision Optimization for LLMs", "Approach": right-hand
+  Hadamard on X and W in the forward pass, left-hand Hadamard on the output gradient in the
+  backward pass (HALO-2), tensor-wise quantization.
+* "Training Transformers with 4-bit Integers", section 3.3: a block-diagonal transform of
+  H_k blocks applied to both operands of a product cancels in the product; section 3.1:
+  the integer product is dequantized by the two scales.
+
+Every rotation runs along the contraction dimension of its GEMM:
+
+    forward   Y  = X  W^T   contraction over K (d_in):  X along K, W along K
+    backward  dX = dY W     contraction over N (d_out): dY along N, W along N
+    backward  dW = dY^T X   contraction over M (tokens): dY along M, X along M  (left-hand)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libhq_oracle.so")
+
+INT8, FP8_E4M3 = 0, 1
+F32, BF16 = 0, 1
+
+OK, ERR_ARG, ERR_SHAPE, ERR_NONFINITE = 0, 1, 2, 5
+
+GCC_FLAGS = ["-O3", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile hq_oracle.c into libhq_oracle.so next to it (plain gcc, no CUDA)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.hq_oracle_rotate.argtypes = [p, i32, i64, i64, i32, i32, p]
+        L.hq_oracle_rotate.restype = i32
+        L.hq_oracle_quantize.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p]
+        L.hq_oracle_quantize.restype = i32
+        L.hq_oracle_quantize_rotated.argtypes = [p, i64, i32, p, p]
+        L.hq_oracle_quantize_rotated.restype = i32
+        L.hq_oracle_fwht_block.argtypes = [p, i32]
+        L.hq_oracle_fwht_block.restype = None
+        L.hq_oracle_norm_const.argtypes = [i32]
+        L.hq_oracle_norm_const.restype = ctypes.c_float
+        L.hq_oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.hq_oracle_e4m3_decode.restype = ctypes.c_double
+        L.hq_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.hq_oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.hq_oracle_bf16_from_f64.argtypes = [ctypes.c_double]
+        L.hq_oracle_bf16_from_f64.restype = ctypes.c_uint16
+        L.hq_oracle_bf16_from_f32.argtypes = [ctypes.c_float]
+        L.hq_oracle_bf16_from_f32.restype = ctypes.c_uint16
+        L.hq_oracle_gemm_i8.argtypes = [p, p, i64, i64, i64, p, i64, p]
+        L.hq_oracle_gemm_i8.restype = None
+        L.hq_oracle_gemm_f8.argtypes = [p, p, i64, i64, i64, p, i64, p]
+        L.hq_oracle_gemm_f8.restype = None
+        L.hq_oracle_epilogue.argtypes = [p, i32, i64, ctypes.c_float, ctypes.c_float, p, p]
+        L.hq_oracle_epilogue.restype = None
+        _lib = L
+    return _lib
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: oracle status {status}")
+        self.status = status
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _src(x: np.ndarray):
+    """Accept fp32 arrays or bf16 bit patterns stored as uint16."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.uint16:
+        return x, BF16
+    raise TypeError(f"oracle source must be float32 or bf16 bits (uint16), got {x.dtype}")
+
+
+# ------------------------------------------------------------------------------- primitives
+
+def fwht_block(x: np.ndarray) -> np.ndarray:
+    """Unnormalised fp32 Sylvester FWHT of one block (length k), stage h = 1, 2, ..., k/2."""
+    buf = np.array(x, dtype=np.float32, copy=True)
+    lib().hq_oracle_fwht_block(_ptr(buf), buf.size)
+    return buf
+
+
+def norm_const(k: int) -> np.float32:
+    return np.float32(lib().hq_oracle_norm_const(k))
+
+
+def rotate(x: np.ndarray, dim: int, k: int) -> np.ndarray:
+    """y = blockdiag(H_k / sqrt(k)) applied along `dim` of x[rows][cols], in fp32.
+
+    dim=1: along columns, result [rows][cols].  dim=0: along rows, result [cols][rows]
+    (rotated dimension innermost, i.e. K-major for the GEMM that contracts it)."""
+    x, dt = _src(x)
+    rows, cols = x.shape
+    y = np.empty((rows, cols) if dim == 1 else (cols, rows), dtype=np.float32)
+    st = lib().hq_oracle_rotate(_ptr(x), dt, rows, cols, dim, k, _ptr(y))
+    if st != OK:
+        raise OracleError(st, "rotate")
+    return y
+
+
+def quantize_rotated(y: np.ndarray, fmt: int):
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    codes = np.empty(y.shape, dtype=np.uint8)
+    scale = np.zeros(1, dtype=np.float32)
+    st = lib().hq_oracle_quantize_rotated(_ptr(y), y.size, fmt, _ptr(codes), _ptr(scale))
+    if st != OK:
+        raise OracleError(st, "quantize")
+    return codes, np.float32(scale[0])
+
+
+def quantize(x: np.ndarray, dim: int, k: int, fmt: int):
+    """hq_quantize's definition: rotate along `dim`, tensor-wise absmax, RNE codes.
+
+    Returns (codes uint8 with the rotated dim innermost, fp32 scale)."""
+    x, dt = _src(x)
+    rows, cols = x.shape
+    codes = np.empty((rows, cols) if dim == 1 else (cols, rows), dtype=np.uint8)
+    scale = np.zeros(1, dtype=np.float32)
+    st = lib().hq_oracle_quantize(_ptr(x), dt, rows, cols, dim, k, fmt, _ptr(codes), _ptr(scale))
+    if st != OK:
+        raise OracleError(st, "quantize")
+    return codes, np.float32(scale[0])
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().hq_oracle_e4m3_decode(code)
+
+
+def e4m3_encode(x: float) -> int:
+    return lib().hq_oracle_e4m3_encode(x)
+
+
+E4M3_TABLE = None
+
+
+def e4m3_table() -> np.ndarray:
+    """Decoded value of each of the 256 e4m3 codes (NaN for 0x7F / 0xFF)."""
+    global E4M3_TABLE
+    if E4M3_TABLE is None:
+        E4M3_TABLE = np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    return E4M3_TABLE
+
+
+def bf16_from_f64(v: float) -> int:
+    return lib().hq_oracle_bf16_from_f64(v)
+
+
+def bf16_from_f32(v: float) -> int:
+    return lib().hq_oracle_bf16_from_f32(v)
+
+
+def gemm(A: np.ndarray, B: np.ndarray, fmt: int, rows=None) -> np.ndarray:
+    """C[i][j] = sum_l A[i][l] B[j][l] over codes (both operands contraction-innermost).
+
+    INT8: int32 accumulators.  FP8: exact fp64 accumulators.  `rows` selects rows of A."""
+    A = np.ascontiguousarray(A)
+    B = np.ascontiguousarray(B)
+    M, K = A.shape
+    N, K2 = B.shape
+    if K != K2:
+        raise ValueError("contraction lengths differ")
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        R, rp = rows.size, _ptr(rows)
+    else:
+        R, rp = M, None
+    if fmt == INT8:
+        C = np.empty((R, N), dtype=np.int32)
+        lib().hq_oracle_gemm_i8(_ptr(A.view(np.int8)), _ptr(B.view(np.int8)), M, N, K, rp,
+                                R, _ptr(C))
+    else:
+        C = np.empty((R, N), dtype=np.float64)
+        lib().hq_oracle_gemm_f8(_ptr(A.view(np.uint8)), _ptr(B.view(np.uint8)), M, N, K, rp,
+                                R, _ptr(C))
+    return C
+
+
+def epilogue(acc: np.ndarray, sa: float, sb: float):
+    """Dequantize accumulators to bf16 bit patterns.
+
+    Returns (ref, fast): ref = bf16(fp64(acc)*sa*sb); fast = bf16(fp32(acc)*fp32(sa*sb))."""
+    acc = np.ascontiguousarray(acc)
+    kind = 0 if acc.dtype == np.int32 else 1
+    if kind == 1:
+        acc = acc.astype(np.float64, copy=False)
+    ref = np.empty(acc.shape, dtype=np.uint16)
+    fast = np.empty(acc.shape, dtype=np.uint16)
+    lib().hq_oracle_epilogue(_ptr(acc), kind, acc.size, float(sa), float(sb), _ptr(ref),
+                             _ptr(fast))
+    return ref, fast
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------------------------------- the layer
+
+def _gemm_layer(a_src, a_dim, b_src, b_dim, k, fmt, rows=None):
+    qa, sa = quantize(a_src, a_dim, k, fmt)
+    qb, sb = quantize(b_src, b_dim, k, fmt)
+    acc = gemm(qa, qb, fmt, rows)
+    ref, fast = epilogue(acc, sa, sb)
+    return dict(qa=qa, sa=sa, qb=qb, sb=sb, acc=acc, ref=ref, fast=fast)
+
+
+def linear_fwd(X, W, k, fmt, rows=None):
+    """Y[M][N] = (X H)(W H)^T, both operands rotated along K (HALO right-hand rotation)."""
+    return _gemm_layer(X, 1, W, 1, k, fmt, rows)
+
+
+def linear_bwd_dx(dY, W, k, fmt, rows=None):
+    """dX[M][K] = dY W: dY rotated along N (its columns), W rotated along N (its rows)."""
+    return _gemm_layer(dY, 1, W, 0, k, fmt, rows)
+
+
+def linear_bwd_dw(dY, X, k, fmt, rows=None):
+    """dW[N][K] = dY^T X: both rotated along the token dimension M (HALO-2 left-hand)."""
+    return _gemm_layer(dY, 0, X, 0, k, fmt, rows)
