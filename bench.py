@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark: one HALO-2 linear layer, forward + both backward GEMMs, on B200.
+
+A step is the whole hot path over one batch: the six Hadamard-rotate + quantize passes
+(X along K and M, W along K and N, dY along N and M) and the three tcgen05 GEMMs with the
+dequantizing epilogue (Y = X W^T, dX = dY W, dW = dY^T X).  Workload: Llama-style MLP
+up-projection, 4096 tokens (batch 4 x seq 1024), d_in 4096 -> d_out 11008, bf16 inputs,
+INT8 codes, k = 256, synthetic seeded inputs (N(0,1) activations with 1% outlier channels
+x U[30,100], N(0,0.02) weights, Student-t(3) x 1e-3 output gradients).
+
+Prints one JSON line (rank 0).  `value` = 6*M*N*K / device time per step (TOPS), inputs
+resident in HBM; `e2e` = the same metric through the public API with the inputs copied
+from pinned host memory and the three outputs copied back inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun every rank runs its own replica (weak scaling, no collective on the data
+path); times are the max over ranks.  `--impl reference` times the CPU oracle (the plain
+reference implementation of the method) on a token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hadamard_rotated_precision_b200 import synthetic  # noqa: E402
+
+WORKLOAD_ID = 2
+METRIC = "HALO-2 linear fwd+bwd TOPS, % of INT8/FP8 tensor peak; FWHT+quant HBM GB/s"
+UNIT = "TOPS"
+INT8_OVER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25)
+GEMM_SRC = os.path.join(ROOT, "hadamard_rotated_precision_b200", "csrc", "gemm_tcgen05.cuh")
+QUANT_SRC = os.path.join(ROOT, "hadamard_rotated_precision_b200", "csrc", "fwht_quant.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CPU_SAMPLE_TOKENS = 512
+REF_STEP_TOKENS = 256
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def file_digest(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def recorded_traffic(kind: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if that summary was
+    taken on the current source of the kernel (else None)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(kind)
+    if not e:
+        return None
+    src = GEMM_SRC if kind.startswith("gemm") else QUANT_SRC
+    if e.get("source_sha") != file_digest(src):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="hq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU (oracle)
+
+def oracle_layer_seconds(d, k: int, fmt: int) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.linear_fwd(d["X"], d["W"], k, fmt)
+    oracle.linear_bwd_dx(d["dY"], d["W"], k, fmt)
+    oracle.linear_bwd_dw(d["dY"], d["X"], k, fmt)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, tokens: int):
+    """The oracle, untuned, on a token-prefix sample of the workload (full K, N, k, format)."""
+    import oracle
+    L = w.layers[0]
+    d = synthetic.draw(w, 0, M=tokens)
+    fmt = 0 if w.fmt == "int8" else 1
+    secs = oracle_layer_seconds(d, w.k, fmt)
+    ops = 6.0 * tokens * L.K * L.N
+    return {"value": ops / secs / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{L.name} layer fwd+dX+dW at {tokens} of {L.M} tokens (K={L.K}, N={L.N}, "
+                      f"k={w.k}, {w.fmt}), {secs:.2f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = synthetic.WORKLOADS[WORKLOAD_ID]
+    L = w.layers[0]
+    d = synthetic.draw(w, 0, M=REF_STEP_TOKENS)
+    fmt = 0 if w.fmt == "int8" else 1
+    for _ in range(args.warmup):
+        oracle_layer_seconds(d, w.k, fmt)
+    total = 0.0
+    for _ in range(args.steps):
+        total += oracle_layer_seconds(d, w.k, fmt)
+    ops = 6.0 * REF_STEP_TOKENS * L.K * L.N
+    value = ops * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: M={L.M} K={L.K} N={L.N} k={w.k} {w.fmt} bf16 inputs",
+                   "step_sample_tokens": REF_STEP_TOKENS, "parallelism": "rank 0 only (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": f"each step: fwd+dX+dW at {REF_STEP_TOKENS} of {L.M} tokens"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU
+
+def run_gpu(args):
+    import torch
+    import hadamard_rotated_precision_b200 as hq
+    from hadamard_rotated_precision_b200 import build
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    build.build()
+    hq.lib()
+
+    w = synthetic.WORKLOADS[WORKLOAD_ID]
+    L = w.layers[0]
+    M, K, N, k = L.M, L.K, L.N, w.k
+    fmt = hq.HQ_INT8 if w.fmt == "int8" else hq.HQ_FP8_E4M3
+    d = synthetic.draw(w, 0)
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+    X, W, dY = dev(d["X"]), dev(d["W"]), dev(d["dY"])
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+    dW = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+    qX_K = torch.empty(M, K, dtype=torch.uint8, device=device)
+    qW_K = torch.empty(N, K, dtype=torch.uint8, device=device)
+    qdY_N = torch.empty(M, N, dtype=torch.uint8, device=device)
+    qW_N = torch.empty(K, N, dtype=torch.uint8, device=device)
+    qdY_M = torch.empty(N, M, dtype=torch.uint8, device=device)
+    qX_M = torch.empty(K, M, dtype=torch.uint8, device=device)
+    scales = torch.empty(8, dtype=torch.float32, device=device)
+    qws = torch.empty(hq.hq_quantize_workspace_bytes(), dtype=torch.uint8, device=device)
+    lws = torch.empty(hq.hq_linear_workspace_bytes(M, K, N), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    # (GEMM operands, output) of the three GEMMs; each operand = (src, dim, codes, scale index)
+    gemms = (
+        ((X, 1, qX_K, 0), (W, 1, qW_K, 1), Y),
+        ((dY, 1, qdY_N, 2), (W, 0, qW_N, 3), dX),
+        ((dY, 0, qdY_M, 4), (X, 0, qX_M, 5), dW),
+    )
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    # Pre-marshalled C-ABI calls (the same entry points the Python wrappers use), so the host
+    # enqueues the 15 launches of a step far ahead of the device.
+    L_ = hq.lib()
+    sh = stream.cuda_stream
+    ws_n = qws.numel()
+    calls = []
+    for a, b, out in gemms:
+        qcalls = [(src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt,
+                   codes.data_ptr(), scales[si:si + 1].data_ptr(), qws.data_ptr(), ws_n, sh)
+                  for src, dim, codes, si in (a, b)]
+        gm, gk = a[2].shape
+        gn = b[2].shape[0]
+        gcall = (a[2].data_ptr(), scales[a[3]:a[3] + 1].data_ptr(), b[2].data_ptr(),
+                 scales[b[3]:b[3] + 1].data_ptr(), gm, gn, gk, fmt, hq.HQ_OUT_BF16, out.data_ptr(), sh)
+        calls.append((qcalls, gcall))
+
+    def step(events=None):
+        for gi, (qcalls, gcall) in enumerate(calls):
+            if events is not None:
+                events[gi][0].record(stream)
+            for qc in qcalls:
+                st = L_.hq_quantize(*qc)
+                if st:
+                    raise hq.HQError(st, "hq_quantize")
+            if events is not None:
+                events[gi][1].record(stream)
+            st = L_.hq_gemm(*gcall)
+            if st:
+                raise hq.HQError(st, "hq_gemm")
+            if events is not None:
+                events[gi][2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if hq.hq_get_error(stream) != 0:
+        raise SystemExit("device status error during warm-up")
+
+    # ---------------------------------------------------------------- timed region (device)
+    per_step = [[[ev(), ev(), ev()] for _ in range(3)] for _ in range(args.steps)]
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            flush.zero_()  # L2 flush (256 MiB > 126 MB L2), outside the step's events
+            step(per_step[s])
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    status = hq.hq_get_error(stream)
+    quant_ms = sum(e[g][0].elapsed_time(e[g][1]) for e in per_step for g in range(3))
+    gemm_ms = sum(e[g][1].elapsed_time(e[g][2]) for e in per_step for g in range(3))
+    step_ms_local = (quant_ms + gemm_ms) / args.steps
+    step_ms = reduce_max(step_ms_local, world, device)
+    gemm_ms_launch = reduce_max(gemm_ms / (3 * args.steps), world, device)
+    quant_ms_launch = reduce_max(quant_ms / (6 * args.steps), world, device)
+    launches = 15 * args.steps  # per step: 6 quantizations x 2 kernels + 3 GEMMs
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    hX = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True).copy_(X)
+    hW = torch.empty(N, K, dtype=torch.bfloat16, pin_memory=True).copy_(W)
+    hdY = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True).copy_(dY)
+    hY = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+    hdX = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
+    hdW = torch.empty(N, K, dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        X.copy_(hX, non_blocking=True)
+        W.copy_(hW, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        hq.hq_linear_fwd(X, W, k, fmt, out=Y, workspace=lws, stream=stream)
+        hq.hq_linear_bwd_dx(dY, W, k, fmt, out=dX, workspace=lws, stream=stream)
+        hq.hq_linear_bwd_dw(dY, X, k, fmt, out=dW, workspace=lws, stream=stream)
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(dX, non_blocking=True)
+        hdW.copy_(dW, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world, device)
+    status |= hq.hq_get_error(stream)
+
+    # ---------------------------------------------------------------- report
+    ops = 6.0 * M * N * K
+    value = world * ops / (step_ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_sus"] * INT8_OVER_BF16
+    gemm_ops = 2.0 * M * N * K
+    gemm_tops = gemm_ops / (gemm_ms_launch * 1e-3) / 1e12
+    elem = 2  # bf16 source bytes
+    quant_bytes = (elem + 1) * (2 * M * K + 2 * N * K + 2 * M * N)  # six rotations
+    quant_gbs = quant_bytes / (quant_ms_launch * 6 * 1e-3) / 1e9
+    traffic = recorded_traffic("gemm_int8_llama_up_proj")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": f"{w.name}: M={M} K={K} N={N} k={k} {w.fmt} codes, bf16 inputs",
+                   "l2": "flushed between steps (256 MiB write, outside the step timing)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel<int8,bf16 out> (tcgen05 kind::i8)",
+                     "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tops / int8_peak, "traffic": traffic,
+                     "peak_note": f"{peaks['src']} sustained bf16 {peaks['bf16_sus']} x {INT8_OVER_BF16} (nominal INT8/bf16 ratio); ops = 2*M*N*K per launch"},
+        "fwht_quant": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm"],
+                       "frac": quant_gbs / peaks["hbm"], "bytes_per_step": quant_bytes,
+                       "ms_per_step": quant_ms_launch * 6, "note": "algorithmic bytes: bf16 source read once + 1-byte codes, six rotations"},
+        "gemm_ms_per_step": gemm_ms_launch * 3,
+        "frac_of_int8_peak_end_to_end": value / world / int8_peak,
+        "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": elem * (M * K + N * K + M * N),
+                "d2h_bytes_per_step": elem * (M * N + M * K + N * K),
+                "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "device_status": int(status),
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, CPU_SAMPLE_TOKENS)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0 if status == 0 else 1
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

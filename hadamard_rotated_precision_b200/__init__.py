@@ -1,0 +1,241 @@
+"""Python binding of libhq.so: Hadamard-rotated, tensor-wise quantized INT8/FP8 linear layer
+for B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels; PyTorch provides device memory and streams.  The functions carry the names of the
+C entry points declared in include/hq.h.  There is no CPU fallback: CPU tensors, a missing
+library or a non-sm_100 device raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+HQ_OK = 0
+HQ_INT8, HQ_FP8_E4M3 = 0, 1
+HQ_F32, HQ_BF16 = 0, 1
+HQ_OUT_BF16, HQ_OUT_ACC = 0, 1
+HQ_MAX_K_INT8 = 133143
+
+STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_ARG", 2: "HQ_ERR_SHAPE", 3: "HQ_ERR_DTYPE",
+                4: "HQ_ERR_ALIGN", 5: "HQ_ERR_NONFINITE", 6: "HQ_ERR_TIMEOUT", 7: "HQ_ERR_CUDA",
+                8: "HQ_ERR_WORKSPACE", 9: "HQ_ERR_UNSUPPORTED"}
+
+EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_gemm", "hq_linear_workspace_bytes",
+           "hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw", "hq_get_error",
+           "hq_last_cuda_error", "hq_status_string", "hq_version")
+
+
+class HQError(RuntimeError):
+    def __init__(self, status: int, where: str, cuda_error: int = 0):
+        name = STATUS_NAMES.get(status, str(status))
+        msg = f"{where}: {name}"
+        if status == 7:
+            msg += f" (cudaError {cuda_error})"
+        super().__init__(msg)
+        self.status = status
+        self.cuda_error = cuda_error
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhq.so (built in-tree by ``build.build()``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libhq.so is not built ({LIB_PATH}); run "
+                              "`python -m hadamard_rotated_precision_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.hq_quantize_workspace_bytes.argtypes = []
+        L.hq_quantize_workspace_bytes.restype = sz
+        L.hq_quantize.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p, sz, p]
+        L.hq_quantize.restype = i32
+        L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
+        L.hq_gemm.restype = i32
+        L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]
+        L.hq_linear_workspace_bytes.restype = sz
+        for name in ("hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw"):
+            f = getattr(L, name)
+            f.argtypes = [p, p, i32, i64, i64, i64, i32, i32, p, p, sz, p]
+            f.restype = i32
+        L.hq_get_error.argtypes = [p]
+        L.hq_get_error.restype = i32
+        L.hq_last_cuda_error.argtypes = []
+        L.hq_last_cuda_error.restype = i32
+        L.hq_status_string.argtypes = [i32]
+        L.hq_status_string.restype = ctypes.c_char_p
+        L.hq_version.argtypes = []
+        L.hq_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != HQ_OK:
+        raise HQError(status, where, lib().hq_last_cuda_error() if status == 7 else 0)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _dev_tensor(t, name: str):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _src_dtype(t, name: str) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return HQ_F32
+    if t.dtype == torch.bfloat16:
+        return HQ_BF16
+    raise TypeError(f"{name} must be float32 or bfloat16, got {t.dtype}")
+
+
+def _fmt(fmt) -> int:
+    if fmt in (HQ_INT8, "int8"):
+        return HQ_INT8
+    if fmt in (HQ_FP8_E4M3, "fp8", "fp8_e4m3"):
+        return HQ_FP8_E4M3
+    raise ValueError(f"unknown format {fmt!r}")
+
+
+def hq_quantize_workspace_bytes() -> int:
+    return int(lib().hq_quantize_workspace_bytes())
+
+
+def hq_linear_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_workspace_bytes(M, K, N))
+
+
+def _workspace(nbytes: int, device, workspace=None):
+    torch = _torch()
+    if workspace is None:
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    _dev_tensor(workspace, "workspace")
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError("workspace too small")
+    return workspace
+
+
+def hq_quantize(src, dim: int, k: int, fmt, codes=None, scale=None, workspace=None,
+                stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """Rotate `src` [rows][cols] along `dim` with blockdiag(H_k)/sqrt(k), quantize it
+    tensor-wise.  Returns (codes uint8 with the rotated dim innermost, scale fp32[1])."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    shape = (rows, cols) if dim == 1 else (cols, rows)
+    if codes is None:
+        codes = torch.empty(shape, dtype=torch.uint8, device=src.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=src.device)
+    _dev_tensor(codes, "codes")
+    _dev_tensor(scale, "scale")
+    ws = _workspace(hq_quantize_workspace_bytes(), src.device, workspace)
+    st = lib().hq_quantize(src.data_ptr(), dt, rows, cols, dim, k, _fmt(fmt), codes.data_ptr(),
+                           scale.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                           _stream_handle(stream))
+    _check(st, "hq_quantize")
+    return codes, scale
+
+
+def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None):
+    """out[M][N] = sum_l A[i][l] B[j][l] on codes (both contraction-innermost), dequantized
+    to bf16 by scale_a*scale_b (HQ_OUT_BF16) or raw int32/fp32 accumulators (HQ_OUT_ACC)."""
+    torch = _torch()
+    _dev_tensor(A, "A")
+    _dev_tensor(B, "B")
+    M, K = A.shape
+    N, K2 = B.shape
+    if K != K2:
+        raise ValueError("contraction lengths differ")
+    f = _fmt(fmt)
+    if out is None:
+        if out_kind == HQ_OUT_BF16:
+            dtype = torch.bfloat16
+        else:
+            dtype = torch.int32 if f == HQ_INT8 else torch.float32
+        out = torch.empty((M, N), dtype=dtype, device=A.device)
+    _dev_tensor(out, "out")
+    sa = scale_a.data_ptr() if scale_a is not None else None
+    sb = scale_b.data_ptr() if scale_b is not None else None
+    st = lib().hq_gemm(A.data_ptr(), sa, B.data_ptr(), sb, M, N, K, f, out_kind, out.data_ptr(),
+                       _stream_handle(stream))
+    _check(st, "hq_gemm")
+    return out
+
+
+def _linear(name, a, b, M, K, N, out_shape, k, fmt, out, workspace, stream):
+    torch = _torch()
+    _dev_tensor(a, "a")
+    _dev_tensor(b, "b")
+    dt = _src_dtype(a, "a")
+    if _src_dtype(b, "b") != dt:
+        raise TypeError("both operands must have the same dtype")
+    if out is None:
+        out = torch.empty(out_shape, dtype=torch.bfloat16, device=a.device)
+    _dev_tensor(out, "out")
+    ws = _workspace(hq_linear_workspace_bytes(M, K, N), a.device, workspace)
+    st = getattr(lib(), name)(a.data_ptr(), b.data_ptr(), dt, M, K, N, k, _fmt(fmt),
+                              out.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                              _stream_handle(stream))
+    _check(st, name)
+    return out
+
+
+def hq_linear_fwd(X, W, k: int, fmt, out=None, workspace=None, stream=None):
+    """Y[M][N] = (X H)(W H)^T, X [M][K], W [N][K]: HALO right-hand rotation along K."""
+    M, K = X.shape
+    N = W.shape[0]
+    return _linear("hq_linear_fwd", X, W, M, K, N, (M, N), k, fmt, out, workspace, stream)
+
+
+def hq_linear_bwd_dx(dY, W, k: int, fmt, out=None, workspace=None, stream=None):
+    """dX[M][K] = dY W with dY and W rotated along N (d_out)."""
+    M, N = dY.shape
+    K = W.shape[1]
+    return _linear("hq_linear_bwd_dx", dY, W, M, K, N, (M, K), k, fmt, out, workspace, stream)
+
+
+def hq_linear_bwd_dw(dY, X, k: int, fmt, out=None, workspace=None, stream=None):
+    """dW[N][K] = dY^T X with dY and X rotated along the tokens M (HALO-2 left-hand)."""
+    M, N = dY.shape
+    K = X.shape[1]
+    return _linear("hq_linear_bwd_dw", dY, X, M, K, N, (N, K), k, fmt, out, workspace, stream)
+
+
+def hq_get_error(stream=None) -> int:
+    """Synchronise the stream and return/clear the device status word (0 = HQ_OK)."""
+    return int(lib().hq_get_error(_stream_handle(stream)))
+
+
+def hq_status_string(status: int) -> str:
+    return lib().hq_status_string(status).decode()
+
+
+def hq_version() -> int:
+    return int(lib().hq_version())

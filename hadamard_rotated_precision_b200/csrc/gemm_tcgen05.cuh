@@ -1,0 +1,300 @@
+// Low-precision GEMM on the 5th-generation tensor cores with a fused dequantization epilogue.
+//
+//   C[i][j] = sum_l A[i][l] * B[j][l]          A: [M][K] codes, B: [N][K] codes (both K-major)
+//   out[i][j] = bf16( fp32(C[i][j]) * fp32(s_a * s_b) )       (or the raw accumulator)
+//
+// Method: "Training Transformers with 4-bit Integers", section 3.1 (the integer product is
+// computed on integer tensor cores and dequantized back to floating point by the scales)
+// and section 3.3 (the Hadamard rotation of both operands cancels in the product, so the
+// GEMM runs directly on the rotated codes); "HALO: Hadamard-Assisted Lower-Precision
+// Optimization for LLMs" (INT8 / FP8 operands with one tensor-wise scale each).
+//
+// Kernel shape (one CTA per SM, persistent over output tiles):
+//   tile 128 x 256, K step 128 bytes (one 128-byte swizzle atom per operand row), 4-stage
+//   shared-memory ring fed by TMA (no multicast), tcgen05.mma (kind::i8 / kind::f8f6f4,
+//   M=128 N=256 K=32) issued by one thread into a TMEM accumulator, two accumulators
+//   (2 x 256 TMEM columns) so the epilogue of tile t overlaps the main loop of tile t+1.
+//   warp 0: TMA producer; warp 1: TMEM allocator + MMA issuer; warps 2-5: epilogue
+//   (warp w reads TMEM lanes 32*(w%4) .. +31 = output rows of that quarter tile).
+// Every wait on an mbarrier is bounded (about a second); on expiry the kernel records
+// HQ_ERR_TIMEOUT in the status word, the other roles stop, in-flight copies and MMAs are
+// drained with bounded waits, TMEM is freed and the CTA exits.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "sm100_ptx.cuh"
+
+namespace hq {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;  // bytes == elements for 8-bit operands
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;  // K of one tcgen05.mma for 8-bit operands
+constexpr int A_STAGE_BYTES = BM * BK;
+constexpr int B_STAGE_BYTES = BN * BK;
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int ACC_BUFS = 2;
+constexpr int TMEM_COLS = ACC_BUFS * BN;  // 512: the whole tensor memory of the SM
+constexpr int NUM_THREADS = 192;
+constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8 + 16;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s per wait
+
+enum Fmt : int { kInt8 = 0, kFp8 = 1 };
+enum Out : int { kOutBf16 = 0, kOutAcc = 1 };
+
+// Instruction descriptor: dense, D = s32 (int8) / f32 (fp8), A = B = s8 / e4m3, both K-major,
+// N = 256, M = 128.
+template <int FMT>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  return (uint32_t(FMT == kInt8 ? 2 : 1) << 4)     // D format
+         | (uint32_t(FMT == kInt8 ? 1 : 0) << 7)   // A format
+         | (uint32_t(FMT == kInt8 ? 1 : 0) << 10)  // B format
+         | (uint32_t(BN >> 3) << 17)               // N / 8
+         | (uint32_t(BM >> 4) << 24);              // M / 16
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row core groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4)      // start address
+         | (uint64_t(1) << 16)                   // leading-dimension offset (unused, 1)
+         | (uint64_t(1024 >> 4) << 32)           // stride offset between 8-row groups
+         | (uint64_t(1) << 46)                   // descriptor version (sm_100)
+         | (uint64_t(2) << 61);                  // 128-byte swizzle
+}
+
+struct Shared {
+  uint8_t* a;
+  uint8_t* b;
+  uint64_t* bars;
+  uint32_t* tmem_holder;
+  volatile int* abort_flag;
+};
+
+__device__ __forceinline__ Shared carve(uint8_t* raw) {
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  Shared s;
+  s.a = base;
+  s.b = base + STAGES * A_STAGE_BYTES;
+  s.bars = reinterpret_cast<uint64_t*>(s.b + STAGES * B_STAGE_BYTES);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + NUM_BARS);
+  s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_holder + 1);
+  return s;
+}
+
+// Bounded wait; gives up when the flag is raised by another role or after WAIT_LIMIT_NS.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned int* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      *abort_flag = 1;
+      atomicCAS(status, 0u, 6u /* HQ_ERR_TIMEOUT */);
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used to drain work already in flight).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, unsigned int* status) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      atomicCAS(status, 0u, 6u);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int& m_blk, int& n_blk) {
+  m_blk = tile % num_m;  // M fastest: concurrent CTAs share B tiles and sweep A
+  n_blk = tile / num_m;
+}
+
+template <int FMT, int OUT>
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void* out, int64_t row,
+                                            int col0, int N, float sab) {
+  if (OUT == kOutBf16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + row * N + col0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (col0 + 8 * q + 8 > N) break;
+      uint32_t pk[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 8 * q + 2 * e;
+        float x0, x1;
+        if (FMT == kInt8) {
+          x0 = __int2float_rn(static_cast<int>(r[i]));
+          x1 = __int2float_rn(static_cast<int>(r[i + 1]));
+        } else {
+          x0 = __uint_as_float(r[i]);
+          x1 = __uint_as_float(r[i + 1]);
+        }
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(x0, sab), __fmul_rn(x1, sab));
+        pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(o + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  } else {
+    uint32_t* o = reinterpret_cast<uint32_t*>(out) + row * N + col0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (col0 + 4 * q + 4 > N) break;
+      *reinterpret_cast<uint4*>(o + 4 * q) = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+    }
+  }
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+            const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
+            int M, int N, int K, unsigned int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  const Shared sh = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + BK - 1) / BK;
+
+  auto bar = [&](int i) { return ptx::smem_u32(sh.bars + i); };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto empty_bar = [&](int s) { return bar(STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar(2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * STAGES + ACC_BUFS + b); };
+  const uint32_t drain_bar = bar(2 * STAGES + 2 * ACC_BUFS);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < ACC_BUFS; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 4);  // one arrive per epilogue warp
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *sh.abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmap_a);
+    ptx::prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(sh.tmem_holder), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before_sync();
+  __syncthreads();
+  ptx::tc_fence_after_sync();
+  const uint32_t tmem_base = *sh.tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(tile, num_m, m_blk, n_blk);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+          ptx::tma_load_2d(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, kb * BK, m_blk * BM, full_bar(stage));
+          ptx::tma_load_2d(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, kb * BK, n_blk * BN, full_bar(stage));
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // every copy this thread started has landed before the CTA may exit
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) drain_wait(full_bar(s), (issued_parity >> s) & 1u, status);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<FMT>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, sh.abort_flag, status)) break;
+        ptx::tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, sh.abort_flag, status)) { ok = false; break; }
+          ptx::tc_fence_after_sync();
+          const uint32_t a_addr = ptx::smem_u32(sh.a + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = ptx::smem_u32(sh.b + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_addr + kk * UMMA_K);
+            const uint64_t bd = smem_desc_sw128(b_addr + kk * UMMA_K);
+            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            if (FMT == kInt8) ptx::mma_i8(d_tmem, ad, bd, idesc, accumulate);
+            else ptx::mma_f8(d_tmem, ad, bd, idesc, accumulate);
+          }
+          ptx::tc_commit(empty_bar(stage));  // frees the smem stage once these MMAs retire
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::tc_commit(tfull_bar(acc));  // accumulator complete
+        if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all MMAs issued by this thread have retired before TMEM is released
+      ptx::tc_commit(drain_bar);
+      drain_wait(drain_bar, 0, status);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const float sab = (OUT == kOutBf16) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int m_blk, n_blk;
+      tile_coords(tile, num_m, m_blk, n_blk);
+      int ok = 0;
+      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, sh.abort_flag, status) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      ptx::tc_fence_after_sync();
+      const int64_t row = int64_t(m_blk) * BM + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
+        ptx::tmem_ld_wait();
+        const int col0 = n_blk * BN + c * 32;
+        if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+      }
+      ptx::tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+      if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  ptx::tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after_sync();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+}  // namespace hq

@@ -1,0 +1,395 @@
+// Host side of libhq.so: argument validation, workspace carving, TMA descriptor encoding
+// and kernel launches behind the C ABI declared in include/hq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "hq.h"
+#include "fwht_quant.cuh"
+#include "gemm_tcgen05.cuh"
+
+namespace {
+
+// Per-device status word: written by kernels on a device-side error, read and cleared by
+// hq_get_error().
+__device__ unsigned int g_hq_status;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxPartials = 4096;  // upper bound on the absmax pass's grid
+constexpr size_t kPartialBytes = kMaxPartials * sizeof(float);
+constexpr size_t kAlign = 256;
+
+thread_local int t_last_cuda_error = 0;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sms = 0;
+  unsigned int* status = nullptr;
+  unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+hq_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return HQ_ERR_CUDA;
+}
+
+// Current device's cached properties; fills them on first use.
+hq_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return cuda_fail(e);
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_hq_status)) != cudaSuccess) return cuda_fail(e);
+    d.supported = (major == 10);
+    d.sms = sms;
+    d.status = static_cast<unsigned int*>(p);
+    d.ready = true;
+  }
+  if (!d.supported) return HQ_ERR_UNSUPPORTED;
+  *out = &d;
+  return HQ_OK;
+}
+
+hq_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                                     cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (q != cudaDriverEntryPointSuccess || !p) return cuda_fail(cudaErrorNotSupported);
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return HQ_OK;
+}
+
+bool valid_k(int k) { return k == 16 || k == 32 || k == 64 || k == 128 || k == 256; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// ------------------------------------------------------------------ quantization launches
+
+template <typename SrcT, int K>
+cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim, hq_fmt fmt,
+                         uint8_t* codes, float* scale, float* partials, const DeviceInfo& d,
+                         cudaStream_t st) {
+  const SrcT* src = static_cast<const SrcT*>(src_v);
+  using namespace hq;
+  if (dim == 1) {
+    const int64_t n_chunks8 = rows * cols / 8;
+    const int64_t n_groups = ((n_chunks8 + 31) / 32 + kRowsUnroll - 1) / kRowsUnroll;
+    const int64_t warps = kQuantThreads / 32;
+    int64_t grid = (n_groups + warps - 1) / warps;
+    grid = std::max<int64_t>(1, std::min<int64_t>(grid, std::min<int64_t>(int64_t(d.sms) * 4, kMaxPartials)));
+    const int g = static_cast<int>(grid);
+    fwhtq_rows_kernel<SrcT, K, kModeAbsmax><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
+    if (fmt == HQ_INT8)
+      fwhtq_rows_kernel<SrcT, K, kModeInt8><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
+    else
+      fwhtq_rows_kernel<SrcT, K, kModeFp8><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
+  } else {
+    constexpr int tcols = 8 * (16 / static_cast<int>(sizeof(SrcT)));
+    const int64_t n_tiles = ((rows + kColsTileRows - 1) / kColsTileRows) * ((cols + tcols - 1) / tcols);
+    int64_t grid = std::max<int64_t>(1, std::min<int64_t>(n_tiles, std::min<int64_t>(int64_t(d.sms) * 2, kMaxPartials)));
+    const int g = static_cast<int>(grid);
+    fwhtq_cols_kernel<SrcT, K, kModeAbsmax><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+    if (fmt == HQ_INT8)
+      fwhtq_cols_kernel<SrcT, K, kModeInt8><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+    else
+      fwhtq_cols_kernel<SrcT, K, kModeFp8><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+  }
+  return cudaGetLastError();
+}
+
+template <typename SrcT>
+cudaError_t launch_quant_k(const void* src, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
+                           uint8_t* codes, float* scale, float* partials, const DeviceInfo& d,
+                           cudaStream_t st) {
+  switch (k) {
+    case 16: return launch_quant<SrcT, 16>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+    case 32: return launch_quant<SrcT, 32>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+    case 64: return launch_quant<SrcT, 64>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+    case 128: return launch_quant<SrcT, 128>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+    default: return launch_quant<SrcT, 256>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+  }
+}
+
+__global__ void set_scale_one_kernel(float* scale) { *scale = 1.0f; }
+
+hq_status check_quant_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                           hq_fmt fmt, const void* codes, const float* scale) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if ((dim != 0 && dim != 1) || !valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (rows < 0 || cols < 0 || !scale) return HQ_ERR_ARG;
+  if (rows == 0 || cols == 0) return HQ_OK;
+  if (!src || !codes) return HQ_ERR_ARG;
+  if (dim == 1 && cols % k != 0) return HQ_ERR_SHAPE;
+  if (dim == 0 && (rows % k != 0 || cols % 16 != 0)) return HQ_ERR_SHAPE;
+  if (rows > (int64_t(1) << 40) / cols) return HQ_ERR_SHAPE;
+  if (!aligned16(src) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scale) & 3u)) return HQ_ERR_ALIGN;
+  return HQ_OK;
+}
+
+hq_status quantize_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                        hq_fmt fmt, void* codes, float* scale, float* partials, const DeviceInfo& d,
+                        cudaStream_t st) {
+  if (rows == 0 || cols == 0) {
+    set_scale_one_kernel<<<1, 1, 0, st>>>(scale);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  cudaError_t e = (dt == HQ_BF16)
+                      ? launch_quant_k<__nv_bfloat16>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, d, st)
+                      : launch_quant_k<float>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------ GEMM launches
+
+hq_status encode_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  hq_status s = tensor_map_encoder(&enc);
+  if (s != HQ_OK) return s;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(hq::gemm::BK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return HQ_OK;
+}
+
+template <int FMT, int OUT>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
+                        void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st) {
+  auto kernel = hq::gemm::gemm_kernel<FMT, OUT>;
+  const unsigned bit = 1u << (FMT * 2 + OUT);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!(d.gemm_attr_set & bit)) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(hq::gemm::SMEM_BYTES));
+      if (e != cudaSuccess) return e;
+      d.gemm_attr_set |= bit;
+    }
+  }
+  const int tiles = ((M + hq::gemm::BM - 1) / hq::gemm::BM) * ((N + hq::gemm::BN - 1) / hq::gemm::BN);
+  const int grid = std::max(1, std::min(tiles, d.sms));
+  kernel<<<grid, hq::gemm::NUM_THREADS, hq::gemm::SMEM_BYTES, st>>>(ta, tb, sa, sb, out, M, N, K, d.status);
+  return cudaGetLastError();
+}
+
+hq_status check_gemm_args(const void* A, const float* sa, const void* B, const float* sb, int64_t M,
+                          int64_t N, int64_t K, hq_fmt fmt, hq_out ok, const void* out) {
+  if ((fmt != HQ_INT8 && fmt != HQ_FP8_E4M3) || (ok != HQ_OUT_BF16 && ok != HQ_OUT_ACC)) return HQ_ERR_ARG;
+  if (M < 0 || N < 0 || K < 0) return HQ_ERR_ARG;
+  if (M == 0 || N == 0) return HQ_OK;
+  if (!out) return HQ_ERR_ARG;
+  if (K > 0 && (!A || !B)) return HQ_ERR_ARG;
+  if (ok == HQ_OUT_BF16 && (!sa || !sb)) return HQ_ERR_ARG;
+  if (K % 16 != 0 || N % 16 != 0) return HQ_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
+  if (fmt == HQ_INT8 && K > HQ_MAX_K_INT8) return HQ_ERR_SHAPE;
+  if (!aligned16(out) || (K > 0 && (!aligned16(A) || !aligned16(B)))) return HQ_ERR_ALIGN;
+  if ((sa && (reinterpret_cast<uintptr_t>(sa) & 3u)) || (sb && (reinterpret_cast<uintptr_t>(sb) & 3u))) return HQ_ERR_ALIGN;
+  return HQ_OK;
+}
+
+hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
+                    int64_t K, hq_fmt fmt, hq_out ok, void* out, DeviceInfo& d, cudaStream_t st) {
+  if (M == 0 || N == 0) return HQ_OK;
+  if (K == 0) {
+    const size_t elem = ok == HQ_OUT_BF16 ? 2 : 4;
+    cudaError_t e = cudaMemsetAsync(out, 0, size_t(M) * size_t(N) * elem, st);
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  CUtensorMap ta, tb;
+  hq_status s = encode_codes_map(&ta, A, M, K, hq::gemm::BM);
+  if (s != HQ_OK) return s;
+  if ((s = encode_codes_map(&tb, B, N, K, hq::gemm::BN)) != HQ_OK) return s;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
+  cudaError_t e;
+  using namespace hq::gemm;
+  if (fmt == HQ_INT8)
+    e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                          : launch_gemm<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+  else
+    e = ok == HQ_OUT_BF16 ? launch_gemm<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                          : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------ the linear layer
+
+struct LinearWs {
+  uint8_t* codes_a;
+  uint8_t* codes_b;
+  float* scale_a;
+  float* scale_b;
+  float* partials;
+};
+
+size_t linear_ws_bytes(int64_t a_bytes, int64_t b_bytes) {
+  return align_up(size_t(a_bytes)) + align_up(size_t(b_bytes)) + kAlign + kPartialBytes;
+}
+
+hq_status carve_linear_ws(void* ws, size_t ws_bytes, int64_t a_bytes, int64_t b_bytes, LinearWs* out) {
+  if (!ws || ws_bytes < linear_ws_bytes(a_bytes, b_bytes)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HQ_ERR_ALIGN;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  out->codes_a = p;
+  p += align_up(size_t(a_bytes));
+  out->codes_b = p;
+  p += align_up(size_t(b_bytes));
+  out->scale_a = reinterpret_cast<float*>(p);
+  out->scale_b = reinterpret_cast<float*>(p) + 4;
+  p += kAlign;
+  out->partials = reinterpret_cast<float*>(p);
+  return HQ_OK;
+}
+
+struct Operand {
+  const void* src;
+  int64_t rows, cols;
+  int dim;
+};
+
+// Quantize both operands along the shared contraction dimension, then run the GEMM.
+hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, hq_dtype dt, int k,
+                      hq_fmt fmt, void* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (gm < 0 || gn < 0 || gk < 0) return HQ_ERR_ARG;
+  if (gm % k || gn % k || gk % k) return HQ_ERR_SHAPE;
+  if (gm == 0 || gn == 0) return HQ_OK;
+  if (!out) return HQ_ERR_ARG;
+  if (gk > 0 && (!a.src || !b.src)) return HQ_ERR_ARG;
+  if (fmt == HQ_INT8 && gk > HQ_MAX_K_INT8) return HQ_ERR_SHAPE;
+  if (gm >= (int64_t(1) << 31) || gn >= (int64_t(1) << 31) || gk >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
+  if (!aligned16(out) || (gk > 0 && (!aligned16(a.src) || !aligned16(b.src)))) return HQ_ERR_ALIGN;
+  LinearWs w;
+  hq_status s = carve_linear_ws(ws, ws_bytes, gm * gk, gn * gk, &w);
+  if (s != HQ_OK) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  if (gk > 0) {
+    if ((s = quantize_impl(a.src, dt, a.rows, a.cols, a.dim, k, fmt, w.codes_a, w.scale_a, w.partials, *d, st)) != HQ_OK) return s;
+    if ((s = quantize_impl(b.src, dt, b.rows, b.cols, b.dim, k, fmt, w.codes_b, w.scale_b, w.partials, *d, st)) != HQ_OK) return s;
+  }
+  return gemm_impl(w.codes_a, w.scale_a, w.codes_b, w.scale_b, gm, gn, gk, fmt, HQ_OUT_BF16, out, *d, st);
+}
+
+}  // namespace
+
+// ====================================================================== exported C ABI
+
+extern "C" {
+
+size_t hq_quantize_workspace_bytes(void) { return kPartialBytes; }
+
+hq_status hq_quantize(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                      hq_fmt fmt, void* codes, float* scale, void* workspace, size_t ws_bytes,
+                      hq_stream_t stream) {
+  hq_status s = check_quant_args(src, dt, rows, cols, dim, k, fmt, codes, scale);
+  if (s != HQ_OK) return s;
+  if (rows > 0 && cols > 0) {
+    if (!workspace || ws_bytes < kPartialBytes) return HQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  }
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  return quantize_impl(src, dt, rows, cols, dim, k, fmt, codes, scale, static_cast<float*>(workspace), *d,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_gemm(const void* A, const float* scale_a, const void* B, const float* scale_b, int64_t M,
+                  int64_t N, int64_t K, hq_fmt fmt, hq_out out_kind, void* out, hq_stream_t stream) {
+  hq_status s = check_gemm_args(A, scale_a, B, scale_b, M, N, K, fmt, out_kind, out);
+  if (s != HQ_OK || M == 0 || N == 0) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  return gemm_impl(A, scale_a, B, scale_b, M, N, K, fmt, out_kind, out, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  size_t best = 0;
+  best = std::max(best, linear_ws_bytes(M * K, N * K));  // forward
+  best = std::max(best, linear_ws_bytes(M * N, K * N));  // dX
+  best = std::max(best, linear_ws_bytes(N * M, K * M));  // dW
+  return best;
+}
+
+hq_status hq_linear_fwd(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                        hq_fmt fmt, void* Y, void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  return linear_gemm(Operand{X, M, K, 1}, Operand{W, N, K, 1}, M, N, K, dt, k, fmt, Y, workspace, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_linear_bwd_dx(const void* dY, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                           hq_fmt fmt, void* dX, void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  return linear_gemm(Operand{dY, M, N, 1}, Operand{W, N, K, 0}, M, K, N, dt, k, fmt, dX, workspace, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                           hq_fmt fmt, void* dW, void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  return linear_gemm(Operand{dY, M, N, 0}, Operand{X, M, K, 0}, N, K, M, dt, k, fmt, dW, workspace, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_get_error(hq_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  DeviceInfo* d = nullptr;
+  hq_status s = device_info(&d);
+  if (s != HQ_OK) return s;
+  unsigned int v = 0;
+  if ((e = cudaMemcpyAsync(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemsetAsync(d->status, 0, sizeof(v), st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e);
+  return static_cast<hq_status>(v);
+}
+
+int hq_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char* hq_status_string(hq_status status) {
+  switch (status) {
+    case HQ_OK: return "ok";
+    case HQ_ERR_ARG: return "invalid argument";
+    case HQ_ERR_SHAPE: return "unsupported shape";
+    case HQ_ERR_DTYPE: return "unsupported dtype";
+    case HQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case HQ_ERR_NONFINITE: return "non-finite value in a rotated operand";
+    case HQ_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
+    case HQ_ERR_CUDA: return "CUDA runtime error";
+    case HQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case HQ_ERR_UNSUPPORTED: return "device is not sm_100";
+  }
+  return "unknown status";
+}
+
+int hq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+/*
+ * hq.h -- C ABI of libhq.so: Hadamard-rotated, tensor-wise quantized INT8 / FP8 linear layer
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on the subject):
+ *  - "Training Transformers with 4-bit Integers", section 3.3 "Hadamard Quantization": both
+ *    operands of a matmul are multiplied by a block-diagonal matrix of k x k Hadamard blocks
+ *    H_k before quantization; the transform cancels in the product.  Section 3.1: symmetric
+ *    integer range, integer product dequantized back to floating point by the scales.
+ *  - "HALO: Hadamard-Assisted Lower-Precision Optimization for LLMs", "Approach": in the
+ *    forward pass X and W are rotated on the right (along d_in); in the backward pass the
+ *    output gradient is rotated on the left (along tokens) for the weight gradient (HALO-2);
+ *    tensor-wise scales; INT8 or FP8 operands ("Key results", "Limitations").
+ *
+ * Readings taken where the pages are silent (all implemented identically by the test oracle):
+ *  - H_k is Sylvester's natural-order Hadamard matrix, normalised by fp32(1/sqrt(k)); the
+ *    transform is an fp32 FWHT with stages h = 1, 2, ..., k/2, no fused multiply-add.
+ *  - Every rotation runs along the contraction dimension of its GEMM (forward: K; dX: N;
+ *    dW: the tokens M), with the same k everywhere.
+ *  - Tensor-wise absmax a of the rotated tensor.  INT8: codes clamp(rne(y*fp32(127/a)),
+ *    -127, 127), scale fp32(a/127).  FP8 (E4M3FN): codes e4m3_rne_satfinite(y*fp32(448/a)),
+ *    scale fp32(a/448).  a == 0: scale 1, codes 0.
+ *  - Epilogue: out = bf16_rne(fp32(acc) * fp32(scale_a * scale_b)).
+ *
+ * Conventions for every call:
+ *  - All tensors are dense row-major device buffers owned by the caller; the library never
+ *    allocates or frees memory and keeps no state except a per-device status word.
+ *  - Every device pointer must be 16-byte aligned (else HQ_ERR_ALIGN).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *    Argument errors are returned synchronously before anything is launched.  Errors found
+ *    on the device (non-finite operand, an internal wait that expired) are recorded in the
+ *    status word and returned by hq_get_error(); outputs are unspecified after an error.
+ *  - Codes are 1 byte each (int8 two's complement, or e4m3 bits) stored with the rotated
+ *    (contraction) dimension innermost.  Scales are one fp32 each, in device memory.
+ *  - k is one of 16, 32, 64, 128, 256.
+ */
+#ifndef HQ_H_
+#define HQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HQ_API __attribute__((visibility("default")))
+#else
+#define HQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* hq_stream_t;
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_ARG = 1,         /* null pointer, unknown enum value, negative size, bad k or dim */
+  HQ_ERR_SHAPE = 2,       /* rotated dim not a multiple of k, other dim not a multiple of 16,
+                             or a size limit exceeded */
+  HQ_ERR_DTYPE = 3,       /* unknown source dtype */
+  HQ_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+  HQ_ERR_NONFINITE = 5,   /* device: a rotated operand contained NaN or Inf */
+  HQ_ERR_TIMEOUT = 6,     /* device: a bounded wait inside a kernel expired */
+  HQ_ERR_CUDA = 7,        /* a CUDA runtime call failed (hq_last_cuda_error() tells which) */
+  HQ_ERR_WORKSPACE = 8,   /* workspace pointer missing or smaller than required */
+  HQ_ERR_UNSUPPORTED = 9  /* the current device is not sm_100 */
+} hq_status;
+
+typedef enum { HQ_INT8 = 0, HQ_FP8_E4M3 = 1 } hq_fmt;
+typedef enum { HQ_F32 = 0, HQ_BF16 = 1 } hq_dtype;
+typedef enum {
+  HQ_OUT_BF16 = 0, /* dequantized bf16 */
+  HQ_OUT_ACC = 1   /* raw accumulators: int32 for HQ_INT8, fp32 for HQ_FP8_E4M3 */
+} hq_out;
+
+/* Largest contraction length the INT8 path accepts: 127*127*K must stay below 2^31 so the
+ * int32 accumulator cannot overflow. */
+#define HQ_MAX_K_INT8 133143
+
+/* ------------------------------------------------------------------------------------------
+ * hq_quantize -- rotate a matrix along one dimension with blockdiag(H_k)/sqrt(k) and quantize
+ * it tensor-wise ("Training Transformers with 4-bit Integers", section 3.3; HALO "Approach").
+ *
+ *   src     [rows][cols], dtype `dt` (fp32 or bf16).
+ *   dim     1: rotate along cols (cols % k == 0);  codes are [rows][cols].
+ *           0: rotate along rows (rows % k == 0);  codes are [cols][rows] (transposed so the
+ *              rotated dimension is innermost); cols must be a multiple of 16.
+ *   codes   rows*cols bytes, device.      scale   1 fp32, device (dequantization step).
+ *   workspace / ws_bytes: >= hq_quantize_workspace_bytes() bytes of device scratch (partial
+ *           maxima); contents need no initialisation and are not preserved.
+ * Runs two kernels on `stream`: rotation + absmax partials, then rotation + codes.
+ * rows == 0 or cols == 0 writes scale = 1 and no codes.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_quantize_workspace_bytes(void);
+HQ_API hq_status hq_quantize(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                      hq_fmt fmt, void* codes, float* scale, void* workspace, size_t ws_bytes,
+                      hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * hq_gemm -- low-precision GEMM on the tcgen05 tensor cores with the dequantization epilogue
+ * ("Training Transformers with 4-bit Integers", section 3.1: INT32 product dequantized).
+ *
+ *   A [M][K] codes, B [N][K] codes (both contraction-innermost, as hq_quantize writes them),
+ *   scale_a / scale_b: device fp32 scalars (may be NULL when out_kind == HQ_OUT_ACC).
+ *   out [M][N]: bf16  = bf16(fp32(acc) * fp32(scale_a*scale_b))   (HQ_OUT_BF16)
+ *               int32 / fp32 raw accumulators                     (HQ_OUT_ACC)
+ *   K and N must be multiples of 16 (K <= HQ_MAX_K_INT8 for INT8); M is free.
+ *   K == 0 writes zeros; M == 0 or N == 0 does nothing.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_gemm(const void* A, const float* scale_a, const void* B, const float* scale_b,
+                  int64_t M, int64_t N, int64_t K, hq_fmt fmt, hq_out out_kind, void* out,
+                  hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * The three GEMMs of one linear layer Y = X W^T with M tokens, K = d_in, N = d_out, each
+ * with both operands rotated along its contraction dimension and quantized tensor-wise
+ * (HALO-2: right-hand rotation of X and W forward, left-hand rotation of dY for dW).
+ *   X [M][K], W [N][K], dY [M][N] in dtype `dt`; outputs bf16.
+ *   M, K, N: multiples of k (and of 16).
+ *   workspace: >= hq_linear_workspace_bytes(M, K, N) bytes of device scratch (codes, scales,
+ *   partial maxima); no initialisation needed, not preserved between calls.
+ * Each call launches 5 kernels on `stream` (2 per quantization + the GEMM).
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/* Y[M][N] = (X H)(W H)^T: X and W rotated along K. */
+HQ_API hq_status hq_linear_fwd(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K,
+                        int64_t N, int k, hq_fmt fmt, void* Y, void* workspace, size_t ws_bytes,
+                        hq_stream_t stream);
+
+/* dX[M][K] = (dY H)(W^T H)^T: dY rotated along N (its columns), W along N (its rows). */
+HQ_API hq_status hq_linear_bwd_dx(const void* dY, const void* W, hq_dtype dt, int64_t M, int64_t K,
+                           int64_t N, int k, hq_fmt fmt, void* dX, void* workspace,
+                           size_t ws_bytes, hq_stream_t stream);
+
+/* dW[N][K] = (dY^T H)(X^T H)^T: dY and X rotated along the tokens M (left-hand rotation). */
+HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, int64_t M, int64_t K,
+                           int64_t N, int k, hq_fmt fmt, void* dW, void* workspace,
+                           size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Status.
+ * ---------------------------------------------------------------------------------------- */
+/* Synchronises `stream`, then returns and clears the current device's status word (HQ_OK,
+ * HQ_ERR_NONFINITE or HQ_ERR_TIMEOUT), or HQ_ERR_CUDA if the stream reported an error. */
+HQ_API hq_status hq_get_error(hq_stream_t stream);
+/* The cudaError_t of the most recent HQ_ERR_CUDA on this thread (0 if none). */
+HQ_API int hq_last_cuda_error(void);
+HQ_API const char* hq_status_string(hq_status status);
+/* 10000 * major + 100 * minor + patch. */
+HQ_API int hq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H_ */

@@ -82,6 +82,8 @@ def lib():
         L.hq_oracle_gemm_f8.restype = None
         L.hq_oracle_epilogue.argtypes = [p, i32, i64, ctypes.c_float, ctypes.c_float, p, p]
         L.hq_oracle_epilogue.restype = None
+        L.hq_oracle_threads.argtypes = []
+        L.hq_oracle_threads.restype = i32
         _lib = L
     return _lib
 
@@ -223,6 +225,11 @@ def epilogue(acc: np.ndarray, sa: float, sb: float):
     lib().hq_oracle_epilogue(_ptr(acc), kind, acc.size, float(sa), float(sb), _ptr(ref),
                              _ptr(fast))
     return ref, fast
+
+
+def threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(lib().hq_oracle_threads())
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

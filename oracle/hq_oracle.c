@@ -33,6 +33,7 @@
  * INT8 GEMM accumulates in int32 (exact while 127*127*K < 2^31).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -41,6 +42,9 @@
 #define ORC_ERR_ARG 1
 #define ORC_ERR_SHAPE 2
 #define ORC_ERR_NONFINITE 5
+
+/* Threads the OpenMP loops below will use (reported with CPU timings). */
+int hq_oracle_threads(void) { return omp_get_max_threads(); }
 
 /* ---------------------------------------------------------------- bf16 <-> fp32 */
 
@@ -68,7 +72,7 @@ static double round_to_format(double v, int p, int emin) {
     return v < 0 ? -r : r;
 }
 
-/* fp32 -> bf16 bits, round to nearest even (bf16: 8 significand bits, emin -126). */
+/* double -> bf16 bits, one rounding to nearest even (bf16: 8 significand bits, emin -126). */
 uint16_t hq_oracle_bf16_from_f64(double v) {
     double r = round_to_format(v, 8, -126);
     float f = (float)r; /* exact: r has 8 significant bits */

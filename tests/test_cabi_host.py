@@ -1,0 +1,136 @@
+"""CPU-only checks of the C ABI library: it builds, loads, exports every symbol the header
+declares, and rejects bad arguments synchronously (these paths return before any CUDA call,
+so no GPU is needed; fake but 16-byte-aligned addresses are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hadamard_rotated_precision_b200 as hq
+from hadamard_rotated_precision_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hq.h")
+
+FAKE = 0x10000      # aligned, never dereferenced: every call below fails validation first
+FAKE_MIS = 0x10002  # misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return hq.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"HQ_API\s+[\w\s\*]+?\b(hq_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(hq.EXPORTS)
+
+
+def test_status_strings_and_version(L):
+    for s in range(10):
+        assert hq.hq_status_string(s)
+    assert hq.hq_version() >= 100
+
+
+def test_workspace_sizes(L):
+    q = hq.hq_quantize_workspace_bytes()
+    assert q >= 4096 * 4
+    M, K, N = 4096, 4096, 11008
+    need = hq.hq_linear_workspace_bytes(M, K, N)
+    assert need >= max(M * K + N * K, M * N + K * N, N * M + K * M) + q
+    assert hq.hq_linear_workspace_bytes(-1, 2, 3) == 0
+
+
+def _q(L, src=FAKE, dt=hq.HQ_BF16, rows=64, cols=256, dim=1, k=16, fmt=0, codes=FAKE, scale=FAKE,
+       ws=FAKE, wsb=1 << 20):
+    return L.hq_quantize(src, dt, rows, cols, dim, k, fmt, codes, scale, ws, wsb, None)
+
+
+def test_quantize_argument_errors(L):
+    assert _q(L, dt=7) == 3
+    assert _q(L, k=24) == 1
+    assert _q(L, k=512) == 1
+    assert _q(L, dim=2) == 1
+    assert _q(L, fmt=3) == 1
+    assert _q(L, rows=-1) == 1
+    assert _q(L, scale=None) == 1
+    assert _q(L, src=None) == 1
+    assert _q(L, cols=250) == 2                      # not a multiple of k along dim 1
+    assert _q(L, dim=0, rows=60) == 2                # not a multiple of k along dim 0
+    assert _q(L, dim=0, rows=64, cols=24) == 2       # other dim not a multiple of 16
+    assert _q(L, src=FAKE_MIS) == 4
+    assert _q(L, codes=FAKE_MIS) == 4
+    assert _q(L, ws=None) == 8
+    assert _q(L, wsb=16) == 8
+    assert _q(L, ws=FAKE_MIS) == 4
+
+
+def _g(L, A=FAKE, sa=FAKE, B=FAKE, sb=FAKE, M=128, N=256, K=128, fmt=0, out_kind=0, out=FAKE):
+    return L.hq_gemm(A, sa, B, sb, M, N, K, fmt, out_kind, out, None)
+
+
+def test_gemm_argument_errors(L):
+    assert _g(L, fmt=2) == 1
+    assert _g(L, out_kind=2) == 1
+    assert _g(L, M=-1) == 1
+    assert _g(L, out=None) == 1
+    assert _g(L, A=None) == 1
+    assert _g(L, sa=None) == 1                # bf16 output needs the scales
+    assert _g(L, K=40) == 2
+    assert _g(L, N=100) == 2
+    assert _g(L, K=133152) == 2               # INT8 accumulator bound (127^2 K < 2^31)
+    assert _g(L, M=1 << 31) == 2
+    assert _g(L, A=FAKE_MIS) == 4
+    assert _g(L, out=FAKE_MIS) == 4
+    assert _g(L, M=0) == 0                    # empty: nothing to do, no launch
+    assert _g(L, N=0) == 0
+
+
+def _lin(L, name, M=256, K=512, N=256, k=64, dt=hq.HQ_BF16, fmt=0, out=FAKE, ws=FAKE, wsb=1 << 30):
+    return getattr(L, name)(FAKE, FAKE, dt, M, K, N, k, fmt, out, ws, wsb, None)
+
+
+@pytest.mark.parametrize("name", ("hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw"))
+def test_linear_argument_errors(L, name):
+    assert _lin(L, name, dt=9) == 3
+    assert _lin(L, name, k=8) == 1
+    assert _lin(L, name, fmt=5) == 1
+    assert _lin(L, name, M=100) == 2
+    assert _lin(L, name, K=100) == 2
+    assert _lin(L, name, N=100) == 2
+    assert _lin(L, name, out=None) == 1
+    assert _lin(L, name, out=FAKE_MIS) == 4
+    assert _lin(L, name, ws=None) == 8
+    assert _lin(L, name, wsb=1024) == 8
+    big = 133248  # multiple of 64 above the INT8 contraction bound
+    if name == "hq_linear_fwd":
+        assert _lin(L, name, K=big) == 2
+    elif name == "hq_linear_bwd_dx":
+        assert _lin(L, name, N=big) == 2
+    else:
+        assert _lin(L, name, M=big) == 2
+
+
+def test_python_binding_rejects_cpu_tensors(L):
+    import torch
+    with pytest.raises(TypeError):
+        hq.hq_quantize(torch.zeros(16, 16), 1, 16, "int8")
+    with pytest.raises(TypeError):
+        hq.hq_linear_fwd(torch.zeros(16, 16), torch.zeros(16, 16), 16, "int8")
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(hq, "_lib", None)
+    monkeypatch.setattr(hq, "LIB_PATH", str(tmp_path / "libhq.so"))
+    with pytest.raises(ImportError):
+        hq.lib()

@@ -1,0 +1,280 @@
+"""GPU parity of the CUDA path (called through the C ABI) against the CPU oracle.
+
+Bar (stated for the method, see include/hq.h for the readings):
+  * quantized codes and scales: bit-exact;
+  * INT8 GEMM int32 accumulators: bit-exact;
+  * bf16 outputs: within 1 bf16 ulp of the oracle's fp64-dequantized value (and, for INT8,
+    bit-exact with the oracle's evaluation of the device epilogue formula);
+  * FP8 path: relative Frobenius error of the output <= 2e-3 against the oracle's exact
+    fp64 product of the same codes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import hadamard_rotated_precision_b200 as hq
+from hadamard_rotated_precision_b200 import synthetic
+from _helpers import to_device, bf16_bits, bits_to_f32, sample_rows, bf16_ulp_diff, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+KS = (16, 32, 64, 128, 256)
+FMTS = (oracle.INT8, oracle.FP8_E4M3)
+FP8_TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup(oracle_lib):
+    from hadamard_rotated_precision_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    hq.lib()
+    yield
+    assert hq.hq_get_error() == 0
+
+
+def _quant_check(x_np, dim, k, fmt):
+    codes, scale = hq.hq_quantize(to_device(x_np), dim, k, fmt)
+    want_codes, want_scale = oracle.quantize(x_np, dim, k, fmt)
+    got = codes.cpu().numpy()
+    assert got.shape == want_codes.shape
+    mism = np.count_nonzero(got != want_codes)
+    assert mism == 0, f"{mism} code mismatches of {got.size}"
+    got_scale = scale.cpu().numpy()[0]
+    assert got_scale.view(np.uint32) == np.float32(want_scale).view(np.uint32)
+    return codes, scale
+
+
+def _outlier_input(rows, cols, seed, dtype):
+    x = synthetic.tiny_random((rows, cols), seed)
+    x[:, 3 % cols] *= 60.0
+    x[:, (cols // 2) % cols] *= -35.0
+    return synthetic.to_bf16_bits(x) if dtype == "bf16" else x
+
+
+# ------------------------------------------------------------------------------ quantize
+
+@pytest.mark.parametrize("dtype", ("f32", "bf16"))
+@pytest.mark.parametrize("k", KS)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_along_cols_ragged(dtype, k, fmt):
+    # 37 rows x 5k cols: the element count is not a multiple of the 256-element warp chunk
+    # nor of the per-step 1024 elements, so the tail paths run
+    x = _outlier_input(37, 5 * k, 10 + k, dtype)
+    _quant_check(x, 1, k, fmt)
+
+
+@pytest.mark.parametrize("dtype", ("f32", "bf16"))
+@pytest.mark.parametrize("k", KS)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_along_rows_ragged(dtype, k, fmt):
+    # rows = 3 tiles of 256 + 2k (ragged last row tile); cols = 208: ragged column tile
+    x = _outlier_input(768 + 2 * k, 208, 20 + k, dtype)
+    _quant_check(x, 0, k, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_large_grid(fmt):
+    # big enough that every CTA runs several grid-stride steps in both passes
+    x = _outlier_input(2048, 4096, 3, "bf16")
+    _quant_check(x, 1, 256, fmt)
+    _quant_check(x, 0, 64, fmt)
+
+
+def test_quantize_zero_tensor():
+    for dim in (0, 1):
+        for fmt in FMTS:
+            codes, scale = hq.hq_quantize(torch.zeros(64, 64, device="cuda"), dim, 16, fmt)
+            assert scale.item() == 1.0 and int(codes.count_nonzero()) == 0
+
+
+def test_quantize_single_outlier():
+    x = np.zeros((32, 256), np.float32)
+    x[5, 100] = 1000.0
+    for dim in (0, 1):
+        _quant_check(x, dim, 32, oracle.INT8)
+        _quant_check(x, dim, 32, oracle.FP8_E4M3)
+
+
+@pytest.mark.parametrize("bad", (float("nan"), float("inf")))
+def test_quantize_nonfinite_sets_status(bad):
+    x = torch.randn(64, 128, device="cuda")
+    x[7, 9] = bad
+    assert hq.hq_get_error() == 0
+    hq.hq_quantize(x, 1, 64, "int8")
+    assert hq.hq_get_error() == 5
+    assert hq.hq_get_error() == 0  # cleared
+    hq.hq_quantize(x, 0, 64, "fp8")
+    assert hq.hq_get_error() == 5
+
+
+def test_quantize_empty():
+    codes, scale = hq.hq_quantize(torch.zeros(0, 64, device="cuda"), 1, 16, "int8")
+    assert codes.numel() == 0 and scale.item() == 1.0
+
+
+def test_argument_errors():
+    x = torch.randn(64, 96, device="cuda")
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_quantize(x, 1, 64, "int8")  # 96 % 64 != 0
+    assert e.value.status == 2
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_quantize(x, 1, 24, "int8")
+    assert e.value.status == 1
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_quantize(torch.randn(64, 24, device="cuda"), 0, 16, "int8")  # cols % 16
+    assert e.value.status == 2
+    buf = torch.randn(64 * 64 + 4, device="cuda")
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_quantize(buf[1:1 + 64 * 64].view(64, 64), 1, 16, "int8")
+    assert e.value.status == 4
+    with pytest.raises(hq.HQError) as e:  # K = 40 is not a multiple of 16
+        hq.hq_gemm(torch.zeros(128, 40, dtype=torch.uint8, device="cuda"), None,
+                   torch.zeros(128, 40, dtype=torch.uint8, device="cuda"), None, "int8", hq.HQ_OUT_ACC)
+    assert e.value.status == 2
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_linear_fwd(torch.randn(64, 256, device="cuda"), torch.randn(100, 256, device="cuda"), 16, "int8")
+    assert e.value.status == 2
+    with pytest.raises(TypeError):
+        hq.hq_quantize(torch.randn(16, 16), 1, 16, "int8")  # CPU tensor: no fallback
+
+
+# ------------------------------------------------------------------------------ GEMM
+
+def _rand_codes(shape, fmt, seed):
+    r = np.random.default_rng(seed)
+    if fmt == oracle.INT8:
+        return r.integers(-127, 128, size=shape).astype(np.int8).view(np.uint8)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    return r.choice(finite, size=shape)
+
+
+GEMM_SHAPES = [(128, 256, 128), (200, 272, 400), (384, 768, 1024), (64, 16, 16), (1, 32, 48),
+               (300, 512, 12608 // 64 * 16)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_int8_accumulators_exact(M, N, K):
+    A = _rand_codes((M, K), oracle.INT8, M + K)
+    B = _rand_codes((N, K), oracle.INT8, N + 7 * K)
+    acc = hq.hq_gemm(torch.from_numpy(A).cuda(), None, torch.from_numpy(B).cuda(), None, "int8",
+                     hq.HQ_OUT_ACC)
+    want = oracle.gemm(A, B, oracle.INT8)
+    np.testing.assert_array_equal(acc.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES[:4])
+def test_gemm_int8_bf16_epilogue(M, N, K):
+    A = _rand_codes((M, K), oracle.INT8, 3 * M + K)
+    B = _rand_codes((N, K), oracle.INT8, 5 * N + K)
+    sa = np.float32(0.0173)
+    sb = np.float32(2.9e-4)
+    out = hq.hq_gemm(torch.from_numpy(A).cuda(), torch.tensor([sa], device="cuda"),
+                     torch.from_numpy(B).cuda(), torch.tensor([sb], device="cuda"), "int8")
+    ref, fast = oracle.epilogue(oracle.gemm(A, B, oracle.INT8), sa, sb)
+    got = bf16_bits(out)
+    np.testing.assert_array_equal(got, fast)
+    assert bf16_ulp_diff(got, ref).max() <= 1
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES[:5])
+def test_gemm_fp8(M, N, K):
+    A = _rand_codes((M, K), oracle.FP8_E4M3, 11 * M + K)
+    B = _rand_codes((N, K), oracle.FP8_E4M3, 13 * N + K)
+    At, Bt = torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda()
+    acc = hq.hq_gemm(At, None, Bt, None, "fp8", hq.HQ_OUT_ACC)
+    want = oracle.gemm(A, B, oracle.FP8_E4M3)
+    assert rel_fro(acc.cpu().numpy(), want) <= FP8_TOL
+    sa, sb = np.float32(0.011), np.float32(0.0037)
+    out = hq.hq_gemm(At, torch.tensor([sa], device="cuda"), Bt, torch.tensor([sb], device="cuda"), "fp8")
+    ref, _ = oracle.epilogue(want, sa, sb)
+    assert rel_fro(bits_to_f32(bf16_bits(out)), bits_to_f32(ref)) <= FP8_TOL
+
+
+def test_gemm_k_zero_writes_zeros():
+    a = torch.zeros(32, 0, dtype=torch.uint8, device="cuda")
+    out = torch.full((32, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    b = torch.zeros(64, 0, dtype=torch.uint8, device="cuda")
+    s = torch.ones(1, device="cuda")
+    hq.hq_gemm(a, s, b, s, "int8", out=out)
+    assert int(out.count_nonzero()) == 0
+
+
+# ------------------------------------------------------------------------------ the layer
+
+def _layer_check(d, k, fmt, rows_sample=None, tag=""):
+    """All three GEMMs of one layer: codes, scales, accumulators (via the split entry points)
+    and the fused linear entry points' bf16 outputs."""
+    X, W, dY = d["X"], d["W"], d["dY"]
+    Xd, Wd, dYd = to_device(X), to_device(W), to_device(dY)
+    cases = (
+        ("fwd", hq.hq_linear_fwd, (Xd, Wd), oracle.linear_fwd, (X, W), (X, 1), (W, 1)),
+        ("dx", hq.hq_linear_bwd_dx, (dYd, Wd), oracle.linear_bwd_dx, (dY, W), (dY, 1), (W, 0)),
+        ("dw", hq.hq_linear_bwd_dw, (dYd, Xd), oracle.linear_bwd_dw, (dY, X), (dY, 0), (X, 0)),
+    )
+    for name, gfun, gargs, ofun, oargs, (a_src, a_dim), (b_src, b_dim) in cases:
+        out = gfun(*gargs, k, fmt)
+        n_out_rows = out.shape[0]
+        rows = None if rows_sample is None else sample_rows(n_out_rows, seed=n_out_rows)
+        want = ofun(*oargs, k, fmt, rows=rows)
+        # codes and scales of both operands, bit-exact
+        qa, sa = hq.hq_quantize(to_device(a_src), a_dim, k, fmt)
+        qb, sb = hq.hq_quantize(to_device(b_src), b_dim, k, fmt)
+        assert np.array_equal(qa.cpu().numpy(), want["qa"]), f"{tag}{name}: A codes"
+        assert np.array_equal(qb.cpu().numpy(), want["qb"]), f"{tag}{name}: B codes"
+        assert sa.cpu().numpy()[0] == want["sa"] and sb.cpu().numpy()[0] == want["sb"], f"{tag}{name}: scales"
+        got = bf16_bits(out)
+        if rows is not None:
+            got = got[rows]
+        if fmt == oracle.INT8:
+            acc = hq.hq_gemm(qa, None, qb, None, fmt, hq.HQ_OUT_ACC).cpu().numpy()
+            if rows is not None:
+                acc = acc[rows]
+            np.testing.assert_array_equal(acc, want["acc"], err_msg=f"{tag}{name}: int32")
+            np.testing.assert_array_equal(got, want["fast"], err_msg=f"{tag}{name}: bf16 formula")
+            assert bf16_ulp_diff(got, want["ref"]).max() <= 1, f"{tag}{name}: ulp"
+        else:
+            e = rel_fro(bits_to_f32(got), bits_to_f32(want["ref"]))
+            assert e <= FP8_TOL, f"{tag}{name}: fp8 rel fro {e}"
+    assert hq.hq_get_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_layer_tiny_workload(fmt):
+    w = synthetic.WORKLOADS[1]
+    _layer_check(synthetic.draw(w), w.k, fmt)
+
+
+@pytest.mark.parametrize("wid", (2, 3, 4))
+def test_layer_token_prefix(wid):
+    """Each workload at its full K and N but a 512-token prefix (exact, full comparison)."""
+    w = synthetic.WORKLOADS[wid]
+    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
+    for li in range(len(w.layers)):
+        _layer_check(synthetic.draw(w, li, M=512), w.k, fmt, tag=f"{w.name}/{li}/")
+
+
+@pytest.mark.parametrize("wid", (1, 2, 3, 4))
+def test_layer_full_size(wid):
+    """Each workload at its full size (the bench's launch configuration), outputs compared on
+    sampled rows; codes and scales compared in full."""
+    w = synthetic.WORKLOADS[wid]
+    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
+    for li in range(len(w.layers)):
+        _layer_check(synthetic.draw(w, li), w.k, fmt, rows_sample=True, tag=f"{w.name}/{li}/")
+
+
+@pytest.mark.parametrize("fmt_name,k", synthetic.WORKLOADS[5].sweep)
+def test_llama_block_sweep_o_proj(fmt_name, k):
+    """Llama-2-7B block sweep over formats and k on the 4096 -> 4096 projection (8192 tokens)."""
+    w = synthetic.WORKLOADS[5]
+    fmt = oracle.INT8 if fmt_name == "int8" else oracle.FP8_E4M3
+    _layer_check(synthetic.draw(w, 1), k, fmt, rows_sample=True, tag=f"o/{fmt_name}/{k}/")
+
+
+@pytest.mark.parametrize("li", (0, 2, 4))
+def test_llama_block_other_shapes(li):
+    """qkv (4096 -> 12288), gate (4096 -> 11008) and down (11008 -> 4096) at INT8 k=256."""
+    w = synthetic.WORKLOADS[5]
+    _layer_check(synthetic.draw(w, li), 256, oracle.INT8, rows_sample=True, tag=f"{li}/")
