@@ -420,13 +420,50 @@ def run_gpu(args):
     return 0 if status == 0 else 1
 
 
+def run_kernel_case(args):
+    """One small standalone invocation of a hot kernel, for profiler captures: a warm-up
+    call, then the captured call(s).  Inputs exceed L2 (126 MB) but stay near 200 MB."""
+    import torch
+    import hadamard_rotated_precision_b200 as hq
+    from hadamard_rotated_precision_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(0)
+    case = args.kernel_case
+    if case.startswith("gemm"):
+        fmt = "fp8" if case == "gemm_fp8" else "int8"
+        M, N, K = 4096, 11008, 4096
+        A = torch.randint(-127, 128, (M, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        B = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        if fmt == "fp8":
+            A = A & 0x77  # finite e4m3 codes, magnitude <= 240
+            B = B & 0x77
+        s = torch.full((1,), 0.01, device="cuda")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        for _ in range(2):
+            hq.hq_gemm(A, s, B, s, fmt, out=out)
+    else:
+        rows, cols, dim = (11008, 4096, 1) if case == "quant_rows" else (11008, 4096, 0)
+        x = torch.randn(rows, cols, generator=g, device="cuda").to(torch.bfloat16)
+        for _ in range(2):
+            hq.hq_quantize(x, dim, 256, "int8")
+    torch.cuda.synchronize()
+    st = hq.hq_get_error()
+    print(json.dumps({"kernel_case": case, "status": st}))
+    return 0 if st == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
+    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "quant_rows", "quant_cols"),
+                    help="run one small standalone kernel case (for profiler captures) and exit")
     args = ap.parse_args(argv)
+    if args.kernel_case:
+        return run_kernel_case(args)
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
