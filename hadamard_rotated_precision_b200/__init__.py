@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_ARG", 2: "HQ_ERR_SHAPE", 3: "HQ_ERR_DTYPE
                 4: "HQ_ERR_ALIGN", 5: "HQ_ERR_NONFINITE", 6: "HQ_ERR_TIMEOUT", 7: "HQ_ERR_CUDA",
                 8: "HQ_ERR_WORKSPACE", 9: "HQ_ERR_UNSUPPORTED"}
 
-EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_gemm", "hq_linear_workspace_bytes",
+EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc", "hq_gemm", "hq_linear_workspace_bytes",
            "hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw", "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.hq_quantize_workspace_bytes.restype = sz
         L.hq_quantize.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p, sz, p]
         L.hq_quantize.restype = i32
+        L.hq_quantize_noalloc.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p]
+        L.hq_quantize_noalloc.restype = i32
         L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm.restype = i32
         L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]

@@ -299,6 +299,50 @@ hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, 
   return gemm_impl(w.codes_a, w.scale_a, w.codes_b, w.scale_b, gm, gn, gk, fmt, HQ_OUT_BF16, out, *d, st);
 }
 
+// ------------------------------------------------------------------ allocation-free quantize
+
+// Scratch for hq_quantize_noalloc: the absmax pass's per-CTA partial maxima, in a fixed
+// array every device that loads the library keeps until exit.  Host code never uses the name
+// as an address: the device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) float g_noalloc_partials[HQ_NOALLOC_MAX_PARTIALS];
+
+struct NoAllocSlot {
+  bool ready = false;
+  float* partials = nullptr;
+};
+NoAllocSlot g_noalloc[kMaxDevices];
+
+hq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocSlot& s = g_noalloc[dev];
+  if (!s.ready) {
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_partials)) != cudaSuccess) return cuda_fail(e);
+    s.partials = static_cast<float*>(p);
+    s.ready = true;
+  }
+  *out = s.partials;
+  return HQ_OK;
+}
+
+// CTAs the absmax pass will launch for this shape (the same rule as launch_quant).
+int64_t quant_grid(hq_dtype dt, int64_t rows, int64_t cols, int dim, int sms) {
+  if (dim == 1) {
+    const int64_t n_chunks8 = rows * cols / 8;
+    const int64_t n_groups = ((n_chunks8 + 31) / 32 + hq::kRowsUnroll - 1) / hq::kRowsUnroll;
+    const int64_t warps = hq::kQuantThreads / 32;
+    const int64_t grid = (n_groups + warps - 1) / warps;
+    return std::max<int64_t>(1, std::min<int64_t>(grid, std::min<int64_t>(int64_t(sms) * 4, kMaxPartials)));
+  }
+  const int64_t tcols = 8 * (16 / (dt == HQ_BF16 ? 2 : 4));
+  const int64_t n_tiles = ((rows + hq::kColsTileRows - 1) / hq::kColsTileRows) * ((cols + tcols - 1) / tcols);
+  return std::max<int64_t>(1, std::min<int64_t>(n_tiles, std::min<int64_t>(int64_t(sms) * 2, kMaxPartials)));
+}
+
 }  // namespace
 
 // ====================================================================== exported C ABI
@@ -356,6 +400,20 @@ hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, int64_t M
                            hq_fmt fmt, void* dW, void* workspace, size_t ws_bytes, hq_stream_t stream) {
   return linear_gemm(Operand{dY, M, N, 0}, Operand{X, M, K, 0}, N, K, M, dt, k, fmt, dW, workspace, ws_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                              hq_fmt fmt, void* codes, float* scale, hq_stream_t stream) {
+  hq_status s = check_quant_args(src, dt, rows, cols, dim, k, fmt, codes, scale);
+  if (s != HQ_OK) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  float* partials = nullptr;
+  if ((s = noalloc_scratch(&partials)) != HQ_OK) return s;
+  if (rows > 0 && cols > 0 && quant_grid(dt, rows, cols, dim, d->sms) > HQ_NOALLOC_MAX_PARTIALS)
+    return HQ_ERR_WORKSPACE;
+  return quantize_impl(src, dt, rows, cols, dim, k, fmt, codes, scale, partials, *d,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 hq_status hq_get_error(hq_stream_t stream) {

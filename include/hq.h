@@ -140,6 +140,35 @@ HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, in
                            size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * hq_quantize_noalloc -- hq_quantize for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call: it exists for integration only.  Some callers
+ * receive nothing but their input and output buffers and may not allocate: plugin code run
+ * inside another engine's execution step, code under a fixed device-memory budget, or code
+ * on a latency-critical path where cudaMalloc (which can synchronise the device and can fail
+ * when memory is fragmented) is not allowed.  Such a caller cannot provide the scratch that
+ * hq_quantize takes as `workspace`.
+ *
+ * Same arguments, results and errors as hq_quantize, without the workspace.  Its scratch (the
+ * per-CTA partial maxima of the absmax pass) lives in a fixed array inside the library:
+ * HQ_NOALLOC_MAX_PARTIALS fp32 values (16 KiB), held on every GPU that loads the library until
+ * the process exits.  The quantizer never launches more CTAs than that on current parts; a
+ * launch that would need more partials than the array holds is refused with
+ * HQ_ERR_WORKSPACE, and sizes beyond hq_quantize's own limits get the same errors as there.
+ * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ *
+ * The first call on a device looks up the array's device address (once per device, with
+ * that device current); make that first call before any stream capture.  All calls share
+ * the one array and it keeps the last call's contents (nothing in it needs clearing between
+ * calls: each call writes every entry it later reads).  Calls whose kernels overlap on the
+ * GPU race on the array: run them on one stream, or otherwise order them.
+ * ---------------------------------------------------------------------------------------- */
+#define HQ_NOALLOC_MAX_PARTIALS 4096
+HQ_API hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols,
+                                     int dim, int k, hq_fmt fmt, void* codes, float* scale,
+                                     hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Status.
  * ---------------------------------------------------------------------------------------- */
 /* Synchronises `stream`, then returns and clears the current device's status word (HQ_OK,
