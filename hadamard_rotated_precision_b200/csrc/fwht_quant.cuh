@@ -29,6 +29,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+#include "sm100_ptx.cuh"
 #include <cfloat>
 #include <cstdint>
 
@@ -187,22 +188,188 @@ __device__ __forceinline__ QuantParams finish_absmax(const float* partials, int 
   return p;
 }
 
+// ------------------------------------------------------------------ packed-fp32 helpers
+
+// Every helper is one fp32 round-to-nearest-even op per lane (f32x2 on sm_100), so results
+// are bit-identical to the scalar __fadd_rn / __fsub_rn / __fmul_rn sequence.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);  // a - b, one rounding
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// Butterfly stages h = 1, 2, ..., H/2 over NV float2 registers holding 2*NV consecutive
+// in-block positions (register index = position).  h = 1 pairs the halves of one float2.
+template <int H, int NV>
+__device__ __forceinline__ void stages_low(float2 (&v)[NV]) {
+  if constexpr (H >= 2) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = v[i].x, b = v[i].y;
+      v[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+  }
+#pragma unroll
+  for (int h2 = 1; h2 < H / 2; h2 <<= 1) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if (i & h2) continue;
+      const float2 a = v[i], b = v[i + h2];
+      v[i] = add2(a, b);
+      v[i + h2] = sub2(a, b);
+    }
+  }
+}
+
+// Stages whose partner lives in another lane (xor mask m): the lower holder keeps a + b, the
+// upper one b' - a' = fma(-1, own, partner), a single rounding either way.
+template <int NV>
+__device__ __forceinline__ void stage_lanes(float2 (&v)[NV], int m, int lane) {
+  const float sg = (lane & m) ? -1.0f : 1.0f;
+  const float2 s2 = make_float2(sg, sg);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float2 p;
+    p.x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, m);
+    p.y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, m);
+    v[i] = __ffma2_rn(s2, v[i], p);
+  }
+}
+
+// max over |x| that turns any NaN into NaN (three-input max on sm_100).
+__device__ __forceinline__ float absmax3(float m, float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+  return r;
+}
+
+// Partial of pass 1 from a per-thread max of the *unnormalised* |t|: the normalisation is
+// a positive scaling, and fp32 rounding is monotone, so max|fp32(t*c)| = fp32(max|t| * c).
+__device__ __forceinline__ void write_partial_unnormalised(float amax_t, float c, float* partials,
+                                                           float* scratch) {
+  const float m = block_max(amax_t != amax_t ? INFINITY : amax_t, scratch);
+  if (threadIdx.x == 0) partials[blockIdx.x] = __fmul_rn(m, c);
+}
+
+// Codes of 4 consecutive elements packed little-endian into one word.
+template <int MODE>
+__device__ __forceinline__ uint32_t codes4(float2 z0, float2 z1) {
+  if constexpr (MODE == kModeInt8) {
+    // z + 1.5*2^23 rounds to an integer with ties to even (|z| <= 127.00001 < 2^22); the low
+    // byte of the sum's bit pattern is that integer in two's complement.  |z| <= 127 after
+    // rounding because |y| <= a and inv = fp32(127/a), so no clamp is needed.  The add is the
+    // scalar __fadd_rn, which is never contracted with the multiply that produced z: a fused
+    // multiply-add would round y*inv only once and flip codes whose product lies within an
+    // ulp of a half-integer.
+    constexpr float mg = 12582912.0f;
+    const uint32_t b0 = __float_as_uint(__fadd_rn(z0.x, mg)), b1 = __float_as_uint(__fadd_rn(z0.y, mg));
+    const uint32_t b2 = __float_as_uint(__fadd_rn(z1.x, mg)), b3 = __float_as_uint(__fadd_rn(z1.y, mg));
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+  } else {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(z0, __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(z1, __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+  }
+}
+
 // ------------------------------------------------------------------ dim = 1 (contiguous)
 
-// A warp-chunk is 32 lanes x 8 elements = 256 consecutive elements: a whole number of
-// k-blocks for every k <= 256.  Each warp processes U consecutive warp-chunks per step.
-constexpr int kRowsUnroll = 4;
+// Each thread owns 32 consecutive elements (one warp step = 1024 elements), so in-block index
+// bits 0..4 are register bits.  For k >= 64 the warp exchanges its 1024 values through a
+// 4 KB shared-memory slice so that each thread then holds index bits {0, 1, 5, 6, 7}
+// (bits 2, 3, 4 and the 256-element group become lane bits) and the stages for bits 5.. run
+// in registers too: no shuffles.  The slice is XOR-swizzled at 16-byte granularity,
+// chunk c -> c ^ ((c >> 3) & 7), which makes both the write and the read conflict-free.
+constexpr int kRowsPerThread = 32;
+constexpr int kRowsWarpElems = 32 * kRowsPerThread;
 
-template <typename SrcT, int K, int MODE>
+template <typename SrcT>
+struct RowsRaw {
+  static constexpr int W = 16 * static_cast<int>(sizeof(SrcT)) / 2;  // 32-bit words per thread
+};
+
+template <bool LAST_USE>
+__device__ __forceinline__ void ld_32B(const void* p, uint32_t* r) {
+  if (LAST_USE)
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+  else
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+
+// (the L2 eviction hint exists only for the 32-byte form)
+template <bool LAST_USE>
+__device__ __forceinline__ void ld_16B(const void* p, uint32_t* r) {
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "l"(p));
+}
+
+// Load a thread's 32 elements starting at element `e` (two halves of 16; a half past the end
+// of the tensor reads as zeros).  WIDE: 32-byte loads (source 32-byte aligned).
+template <typename SrcT, bool WIDE, bool LAST_USE>
+__device__ __forceinline__ void load_rows32(const SrcT* src, int64_t n, int64_t e,
+                                            uint32_t (&raw)[RowsRaw<SrcT>::W]) {
+  constexpr int HW = RowsRaw<SrcT>::W / 2;  // words per half (8 for bf16, 16 for fp32)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t eh = e + 16 * h;
+    if (eh < n) {
+      const char* p = reinterpret_cast<const char*>(src + eh);
+#pragma unroll
+      for (int q = 0; q < HW; q += (WIDE ? 8 : 4)) {
+        if (WIDE) ld_32B<LAST_USE>(p + 4 * q, raw + h * HW + q);
+        else ld_16B<LAST_USE>(p + 4 * q, raw + h * HW + q);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < HW; ++q) raw[h * HW + q] = 0u;
+    }
+  }
+}
+
+template <typename SrcT>
+__device__ __forceinline__ void unpack_rows32(const uint32_t (&raw)[RowsRaw<SrcT>::W], float2 (&v)[16]) {
+  if constexpr (sizeof(SrcT) == 2) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      v[i] = make_float2(__uint_as_float(raw[i] << 16), __uint_as_float(raw[i] & 0xFFFF0000u));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = make_float2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1]));
+  }
+}
+
+// Warp-level exchange: before, thread t holds elements 32t + r (r = register index 0..31);
+// after, thread t holds elements 4*(t&7) + (r&3) + 32*(r>>2) + 256*(t>>3).
+__device__ __forceinline__ void exchange_rows(float2 (&v)[16], float4* slice, int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    slice[8 * lane + (j ^ (lane & 7))] = make_float4(v[2 * j].x, v[2 * j].y, v[2 * j + 1].x, v[2 * j + 1].y);
+  __syncwarp();
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const float4 f = slice[(((lane & 7) ^ b) + 8 * b) + 64 * (lane >> 3)];
+    v[2 * b] = make_float2(f.x, f.y);
+    v[2 * b + 1] = make_float2(f.z, f.w);
+  }
+  __syncwarp();
+}
+
+template <typename SrcT, int K, int MODE, bool WIDE>
 __global__ void __launch_bounds__(kQuantThreads)
-fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n_chunks8, uint8_t* __restrict__ codes,
+fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__ codes,
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
                   unsigned int* __restrict__ status) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
-  constexpr int U = kRowsUnroll;
   constexpr bool QUANT = MODE != kModeAbsmax;
+  constexpr bool EXCH = K >= 64;
+  constexpr int RW = RowsRaw<SrcT>::W;
+  __shared__ __align__(16) float4 xch[EXCH ? kQuantThreads * 8 : 1];
   __shared__ float scratch[32];
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float c = __frsqrt_rn(static_cast<float>(K));
 
   QuantParams qp{0.0f, false, false};
@@ -210,67 +377,206 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n_chunks8, uint8_t* __re
     qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status);
     if (qp.abort) return;
   }
+  const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
 
-  const int64_t warps_per_cta = kQuantThreads / 32;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps_per_cta + (threadIdx.x >> 5);
-  const int64_t tw = static_cast<int64_t>(gridDim.x) * warps_per_cta;
-  const int64_t n_wchunks = (n_chunks8 + 31) / 32;
-  const int64_t n_groups = (n_wchunks + U - 1) / U;
-
+  const int64_t wpc = kQuantThreads / 32;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * wpc + warp;
+  const int64_t tw = static_cast<int64_t>(gridDim.x) * wpc;
+  const int64_t n_units = (n + kRowsWarpElems - 1) / kRowsWarpElems;
   float amax = 0.0f;
-  bool bad = false;
-  if (gw < n_groups) {
-    const int64_t last = gw + tw * ((n_groups - 1 - gw) / tw);
-    // pass 1 walks forward, pass 2 backward (L2 reuse of the tail pass 1 read last)
-    for (int64_t g = QUANT ? last : gw; QUANT ? g >= 0 : g < n_groups; g += QUANT ? -tw : tw) {
-      float v[U][8];
+  if (gw < n_units) {
+    // pass 1 walks forward, pass 2 backward (its first reads hit what pass 1 left in L2)
+    const int64_t last = gw + tw * ((n_units - 1 - gw) / tw);
+    const int64_t first = QUANT ? last : gw;
+    const int64_t step = QUANT ? -tw : tw;
+    uint32_t raw[RW];
+    load_rows32<SrcT, WIDE, QUANT>(src, n, first * kRowsWarpElems + 32 * lane, raw);
+    for (int64_t u = first; QUANT ? u >= 0 : u < n_units; u += step) {
+      float2 v[16];
+      unpack_rows32<SrcT>(raw, v);
+      const int64_t nu = u + step;
+      if (QUANT ? nu >= 0 : nu < n_units)
+        load_rows32<SrcT, WIDE, QUANT>(src, n, nu * kRowsWarpElems + 32 * lane, raw);
+      stages_low<(K < 32 ? K : 32), 16>(v);
+      if constexpr (EXCH) {
+        exchange_rows(v, xch + warp * 256, lane);
+        // index bits 5.. are register-index bits 2.. = float2-index bits 1..
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t ch = (g * U + u) * 32 + lane;
-        if (ch < n_chunks8) {
-          load8<SrcT, QUANT>(src + ch * 8, v[u]);
-        } else {
+        for (int h2 = 2; h2 < K / 16; h2 <<= 1) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+          for (int i = 0; i < 16; ++i) {
+            if (i & h2) continue;
+            const float2 a = v[i], b = v[i + h2];
+            v[i] = add2(a, b);
+            v[i + h2] = sub2(a, b);
+          }
         }
       }
+      if constexpr (!QUANT) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        butterfly_regs8(v[u]);
-        butterfly_lanes<K, 8>(v[u], lane);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[u][i] = __fmul_rn(v[u][i], c);
-      }
-      if (!QUANT) {
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float ay = fabsf(v[u][i]);
-            bad |= !(ay <= FLT_MAX);
-            amax = fmaxf(amax, ay);
-          }
+        for (int i = 0; i < 16; ++i) amax = absmax3(amax, v[i].x, v[i].y);
       } else {
+        const int64_t ub = u * kRowsWarpElems;
+        uint32_t w[8];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int64_t ch = (g * U + u) * 32 + lane;
-          if (ch < n_chunks8)
-            __stcs(reinterpret_cast<uint2*>(codes + ch * 8), codes8<MODE>(v[u], qp.inv, qp.zero));
+        for (int j = 0; j < 8; ++j)
+          w[j] = qp.zero ? 0u : codes4<MODE>(mul2(mul2(v[2 * j], c2), inv2), mul2(mul2(v[2 * j + 1], c2), inv2));
+        if constexpr (!EXCH) {
+          const int64_t e = ub + 32 * lane;
+          if (e < n) *reinterpret_cast<uint4*>(codes + e) = make_uint4(w[0], w[1], w[2], w[3]);
+          if (e + 16 < n) *reinterpret_cast<uint4*>(codes + e + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+          const int64_t e0 = ub + 256 * (lane >> 3) + 4 * (lane & 7);
+#pragma unroll
+          for (int b = 0; b < 8; ++b)
+            if (e0 + 32 * b < n) *reinterpret_cast<uint32_t*>(codes + e0 + 32 * b) = w[b];
         }
       }
     }
   }
-  if (!QUANT) write_partial(amax, bad, partials, scratch);
+  if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
 }
 
-// ------------------------------------------------------------------ dim = 0 (strided)
+// ------------------------------------------------------------------ dim = 0, bf16 source
+
+// A CTA tile is 256 rows x 64 bf16 columns (32 KB), double-buffered in shared memory with
+// cp.async (zero-filled past the tensor's edge).  Warp w owns the tile's 8 columns of 16-byte
+// chunk w; ldmatrix.trans turns four 8x8 blocks at a time into column-major fragments so that
+// thread t holds 64 consecutive rows (64*(t&3) + 0..63) of column 8w + t/4: in-block row bits
+// 0..5 are register bits, bits 6 and 7 lane bits (shuffles only for k = 128, 256).  The
+// codes of a thread are 64 contiguous bytes of the transposed output.
+constexpr int kColsTileRows2 = 256;
+constexpr int kColsTileCols2 = 64;
+constexpr size_t kColsSmemBytes2 = 2ull * kColsTileRows2 * 128;  // two 32 KB tiles
+
+// 16-byte chunk swizzle of tile row rho: row bit 0 -> bit 0, row bits 6, 7 -> bits 1, 2, so
+// the 8 rows one ldmatrix matrix reads (rows differing in bits 0, 6, 7) hit distinct banks.
+__device__ __forceinline__ int cols_swz(int rho) { return (rho & 1) | ((rho >> 5) & 6); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+template <int K, int MODE>
+__global__ void __launch_bounds__(kQuantThreads)
+fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols,
+                       uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
+                       float* __restrict__ scale_out, unsigned int* __restrict__ status) {
+  static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  constexpr bool QUANT = MODE != kModeAbsmax;
+  extern __shared__ __align__(128) uint4 tiles[];  // [2][256 rows][8 chunks]
+  __shared__ float scratch[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float c = __frsqrt_rn(static_cast<float>(K));
+
+  QuantParams qp{0.0f, false, false};
+  if (QUANT) {
+    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status);
+    if (qp.abort) return;
+  }
+  const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
+
+  const int64_t n_rt = (rows + kColsTileRows2 - 1) / kColsTileRows2;
+  const int64_t n_ct = (cols + kColsTileCols2 - 1) / kColsTileCols2;
+  const int64_t n_tiles = n_rt * n_ct;
+  float amax = 0.0f;
+
+  // load a tile: thread T copies 16-byte chunk (T & 7) of rows (T >> 3) + 32 j
+  auto issue = [&](int buf, int64_t t) {
+    const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+    const int ch = threadIdx.x & 7;
+    const int64_t gc = c0 + 8 * ch;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int rho = (threadIdx.x >> 3) + 32 * j;
+      const int64_t gr = r0 + rho;
+      const bool ok = gr < rows && gc < cols;
+      const __nv_bfloat16* g = ok ? src + gr * cols + gc : src;
+      cp_async16(ptx::smem_u32(&tiles[(buf * kColsTileRows2 + rho) * 8 + (ch ^ cols_swz(rho))]), g, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+
+  const int64_t G = gridDim.x, b0 = blockIdx.x;
+  if (b0 < n_tiles) {
+    const int64_t last = b0 + G * ((n_tiles - 1 - b0) / G);
+    const int64_t first = QUANT ? last : b0;
+    const int64_t step = QUANT ? -G : G;
+    int buf = 0;
+    issue(0, first);
+    for (int64_t t = first; QUANT ? t >= 0 : t < n_tiles; t += step) {
+      const int64_t nt = t + step;
+      const bool has_next = QUANT ? nt >= 0 : nt < n_tiles;
+      if (has_next) {
+        issue(buf ^ 1, nt);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      // gather: 8 x (ldmatrix.x4.trans) -> 64 consecutive rows of one column per thread
+      float2 v[32];
+      {
+        const int m = lane >> 3, q = lane & 7;
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const int rho = (q & 1) + 2 * m + 8 * kc + 64 * (q >> 1);
+          uint32_t r[4];
+          ldmatrix_x4_trans(ptx::smem_u32(&tiles[(buf * kColsTileRows2 + rho) * 8 + (warp ^ cols_swz(rho))]), r);
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm)
+            v[4 * kc + mm] = make_float2(__uint_as_float(r[mm] << 16), __uint_as_float(r[mm] & 0xFFFF0000u));
+        }
+      }
+      __syncthreads();  // buffer free for the next-but-one tile's copies
+      stages_low<(K < 64 ? K : 64), 32>(v);
+      if constexpr (K >= 128) stage_lanes<32>(v, 1, lane);
+      if constexpr (K >= 256) stage_lanes<32>(v, 2, lane);
+      if constexpr (!QUANT) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = absmax3(amax, v[i].x, v[i].y);
+      } else {
+        const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+        const int64_t col = c0 + 8 * warp + (lane >> 2);
+        const int64_t row = r0 + 64 * (lane & 3);
+        if (col < cols) {
+          uint8_t* o = codes + col * rows + row;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (row + 16 * j < rows) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = 8 * j + 2 * e;
+                w[e] = qp.zero ? 0u : codes4<MODE>(mul2(mul2(v[i], c2), inv2), mul2(mul2(v[i + 1], c2), inv2));
+              }
+              *reinterpret_cast<uint4*>(o + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      }
+      buf ^= 1;
+    }
+  }
+  if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
+}
+
+// ------------------------------------------------------------------ dim = 0, fp32 source
 
 constexpr int kColsTileRows = 256;   // rows per tile: 32 lanes x 8 registers
 constexpr int kColsTileBytes = 128;  // bytes of each source row per tile (8 x 16-byte chunks)
 
 template <typename SrcT, int K, int MODE>
 __global__ void __launch_bounds__(kQuantThreads)
-fwhtq_cols_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
+fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
                   float* __restrict__ scale_out, unsigned int* __restrict__ status) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");

@@ -31,6 +31,9 @@ struct DeviceInfo {
   int sms = 0;
   unsigned int* status = nullptr;
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
+  unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation
+  unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
+  int pair_clusters = 0;       // co-resident 2-CTA clusters of the pair GEMM
 };
 
 std::mutex g_mu;
@@ -87,41 +90,74 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ quantization launches
 
-template <typename SrcT, int K>
-cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim, hq_fmt fmt,
-                         uint8_t* codes, float* scale, float* partials, const DeviceInfo& d,
-                         cudaStream_t st) {
-  const SrcT* src = static_cast<const SrcT*>(src_v);
+// CTAs of both quantization passes for a shape (the absmax pass writes one partial per CTA).
+int64_t quant_grid(hq_dtype dt, int64_t rows, int64_t cols, int dim, int sms) {
+  int64_t want, cap;
+  if (dim == 1) {
+    const int64_t units = (rows * cols + hq::kRowsWarpElems - 1) / hq::kRowsWarpElems;
+    want = (units + hq::kQuantThreads / 32 - 1) / (hq::kQuantThreads / 32);
+    cap = int64_t(sms) * 4;
+  } else if (dt == HQ_BF16) {
+    want = ((rows + hq::kColsTileRows2 - 1) / hq::kColsTileRows2) *
+           ((cols + hq::kColsTileCols2 - 1) / hq::kColsTileCols2);
+    cap = int64_t(sms) * 2;
+  } else {
+    const int64_t tcols = 8 * (16 / 4);
+    want = ((rows + hq::kColsTileRows - 1) / hq::kColsTileRows) * ((cols + tcols - 1) / tcols);
+    cap = int64_t(sms) * 2;
+  }
+  return std::max<int64_t>(1, std::min<int64_t>(want, std::min<int64_t>(cap, kMaxPartials)));
+}
+
+template <int K, int MODE>
+cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
+  constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
+  const unsigned bit = 1u << (kIdx * 3 + MODE);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (d.cols_attr_set & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(hq::fwhtq_cols_bf16_kernel<K, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(hq::kColsSmemBytes2));
+  if (e == cudaSuccess) d.cols_attr_set |= bit;
+  return e;
+}
+
+template <typename SrcT, int K, int MODE>
+cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes,
+                        float* scale, float* partials, int g, DeviceInfo& d, cudaStream_t st) {
   using namespace hq;
   if (dim == 1) {
-    const int64_t n_chunks8 = rows * cols / 8;
-    const int64_t n_groups = ((n_chunks8 + 31) / 32 + kRowsUnroll - 1) / kRowsUnroll;
-    const int64_t warps = kQuantThreads / 32;
-    int64_t grid = (n_groups + warps - 1) / warps;
-    grid = std::max<int64_t>(1, std::min<int64_t>(grid, std::min<int64_t>(int64_t(d.sms) * 4, kMaxPartials)));
-    const int g = static_cast<int>(grid);
-    fwhtq_rows_kernel<SrcT, K, kModeAbsmax><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
-    if (fmt == HQ_INT8)
-      fwhtq_rows_kernel<SrcT, K, kModeInt8><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
+    const int64_t n = rows * cols;
+    if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0)
+      fwhtq_rows_kernel<SrcT, K, MODE, true><<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, g, scale, d.status);
     else
-      fwhtq_rows_kernel<SrcT, K, kModeFp8><<<g, kQuantThreads, 0, st>>>(src, n_chunks8, codes, partials, g, scale, d.status);
+      fwhtq_rows_kernel<SrcT, K, MODE, false><<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, g, scale, d.status);
+  } else if constexpr (sizeof(SrcT) == 2) {
+    cudaError_t e = cols_bf16_smem_attr<K, MODE>(d);
+    if (e != cudaSuccess) return e;
+    fwhtq_cols_bf16_kernel<K, MODE><<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
   } else {
-    constexpr int tcols = 8 * (16 / static_cast<int>(sizeof(SrcT)));
-    const int64_t n_tiles = ((rows + kColsTileRows - 1) / kColsTileRows) * ((cols + tcols - 1) / tcols);
-    int64_t grid = std::max<int64_t>(1, std::min<int64_t>(n_tiles, std::min<int64_t>(int64_t(d.sms) * 2, kMaxPartials)));
-    const int g = static_cast<int>(grid);
-    fwhtq_cols_kernel<SrcT, K, kModeAbsmax><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
-    if (fmt == HQ_INT8)
-      fwhtq_cols_kernel<SrcT, K, kModeInt8><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
-    else
-      fwhtq_cols_kernel<SrcT, K, kModeFp8><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+    fwhtq_cols_f32_kernel<SrcT, K, MODE><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
   }
   return cudaGetLastError();
 }
 
+template <typename SrcT, int K>
+cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim, hq_fmt fmt,
+                         uint8_t* codes, float* scale, float* partials, DeviceInfo& d,
+                         cudaStream_t st) {
+  const SrcT* src = static_cast<const SrcT*>(src_v);
+  using namespace hq;
+  const int g = static_cast<int>(quant_grid(sizeof(SrcT) == 2 ? HQ_BF16 : HQ_F32, rows, cols, dim, d.sms));
+  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, g, d, st);
+  if (e != cudaSuccess) return e;
+  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g, d, st);
+  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g, d, st);
+}
+
 template <typename SrcT>
 cudaError_t launch_quant_k(const void* src, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
-                           uint8_t* codes, float* scale, float* partials, const DeviceInfo& d,
+                           uint8_t* codes, float* scale, float* partials, DeviceInfo& d,
                            cudaStream_t st) {
   switch (k) {
     case 16: return launch_quant<SrcT, 16>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
@@ -149,7 +185,7 @@ hq_status check_quant_args(const void* src, hq_dtype dt, int64_t rows, int64_t c
 }
 
 hq_status quantize_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
-                        hq_fmt fmt, void* codes, float* scale, float* partials, const DeviceInfo& d,
+                        hq_fmt fmt, void* codes, float* scale, float* partials, DeviceInfo& d,
                         cudaStream_t st) {
   if (rows == 0 || cols == 0) {
     set_scale_one_kernel<<<1, 1, 0, st>>>(scale);
@@ -215,6 +251,60 @@ hq_status check_gemm_args(const void* A, const float* sa, const void* B, const f
   return HQ_OK;
 }
 
+template <int FMT, int OUT>
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
+                             void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st) {
+  namespace gp = hq::gemm::pair;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT>;
+  const unsigned bit = 1u << (FMT * 2 + OUT);
+  int max_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!(d.pair_attr_set & bit)) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(gp::SMEM_BYTES));
+      if (e != cudaSuccess) return e;
+      d.pair_attr_set |= bit;
+    }
+    if (d.pair_clusters <= 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (d.sms / 2));
+      q.blockDim = dim3(hq::gemm::NUM_THREADS);
+      q.dynamicSmemBytes = gp::SMEM_BYTES;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int n = 0;
+      cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &q);
+      if (e != cudaSuccess) return e;
+      d.pair_clusters = n > 0 ? n : 1;
+    }
+    max_pairs = d.pair_clusters;
+  }
+  const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + gp::BN - 1) / gp::BN);
+  const int pairs = std::max(1, std::min(tiles, max_pairs));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(hq::gemm::NUM_THREADS);
+  cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, sa, sb, out, M, N, K, d.status);
+}
+
+// GEMMs with at least one full 256-row pair tile run on CTA pairs; smaller M on single CTAs.
+constexpr int64_t kPairMinRows = 256;
+
 hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
                     int64_t K, hq_fmt fmt, hq_out ok, void* out, DeviceInfo& d, cudaStream_t st) {
   if (M == 0 || N == 0) return HQ_OK;
@@ -223,19 +313,29 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     cudaError_t e = cudaMemsetAsync(out, 0, size_t(M) * size_t(N) * elem, st);
     return e == cudaSuccess ? HQ_OK : cuda_fail(e);
   }
+  const bool pair = M >= kPairMinRows;
   CUtensorMap ta, tb;
-  hq_status s = encode_codes_map(&ta, A, M, K, hq::gemm::BM);
+  hq_status s = encode_codes_map(&ta, A, M, K, pair ? hq::gemm::pair::HALF : hq::gemm::BM);
   if (s != HQ_OK) return s;
-  if ((s = encode_codes_map(&tb, B, N, K, hq::gemm::BN)) != HQ_OK) return s;
+  if ((s = encode_codes_map(&tb, B, N, K, pair ? hq::gemm::pair::HALF : hq::gemm::BN)) != HQ_OK) return s;
   const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
   cudaError_t e;
   using namespace hq::gemm;
-  if (fmt == HQ_INT8)
-    e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                          : launch_gemm<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
-  else
-    e = ok == HQ_OUT_BF16 ? launch_gemm<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                          : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+  if (pair) {
+    if (fmt == HQ_INT8)
+      e = ok == HQ_OUT_BF16 ? launch_gemm_pair<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                            : launch_gemm_pair<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+    else
+      e = ok == HQ_OUT_BF16 ? launch_gemm_pair<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                            : launch_gemm_pair<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+  } else {
+    if (fmt == HQ_INT8)
+      e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                            : launch_gemm<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+    else
+      e = ok == HQ_OUT_BF16 ? launch_gemm<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
+                            : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+  }
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -327,20 +427,6 @@ hq_status noalloc_scratch(float** out) {
   }
   *out = s.partials;
   return HQ_OK;
-}
-
-// CTAs the absmax pass will launch for this shape (the same rule as launch_quant).
-int64_t quant_grid(hq_dtype dt, int64_t rows, int64_t cols, int dim, int sms) {
-  if (dim == 1) {
-    const int64_t n_chunks8 = rows * cols / 8;
-    const int64_t n_groups = ((n_chunks8 + 31) / 32 + hq::kRowsUnroll - 1) / hq::kRowsUnroll;
-    const int64_t warps = hq::kQuantThreads / 32;
-    const int64_t grid = (n_groups + warps - 1) / warps;
-    return std::max<int64_t>(1, std::min<int64_t>(grid, std::min<int64_t>(int64_t(sms) * 4, kMaxPartials)));
-  }
-  const int64_t tcols = 8 * (16 / (dt == HQ_BF16 ? 2 : 4));
-  const int64_t n_tiles = ((rows + hq::kColsTileRows - 1) / hq::kColsTileRows) * ((cols + tcols - 1) / tcols);
-  return std::max<int64_t>(1, std::min<int64_t>(n_tiles, std::min<int64_t>(int64_t(sms) * 2, kMaxPartials)));
 }
 
 }  // namespace
