@@ -296,5 +296,196 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
   }
 }
 
+
+// ====================================================================== CTA-pair variant
+//
+// A cluster of two CTAs on the two SMs of a TPC computes a 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32 per instruction): CTA r of the pair holds
+// rows 128 r .. 128 r + 127 of the A tile and rows 128 r .. of the B tile (its half of N) in
+// its own shared memory, and the 128 x 256 accumulator of its rows in its own TMEM.  Per CTA a
+// stage is 16 KB of A + 16 KB of B (half of the single-CTA kernel's B traffic per output), so
+// six stages fit.  Only CTA 0 issues MMAs; both CTAs load their own tiles (no multicast), the
+// loads of both count on CTA 0's "full" barrier, and CTA 0's commits arrive on the barriers of
+// both CTAs.  Epilogue warps of both CTAs report a drained accumulator to CTA 0.
+namespace pair {
+
+constexpr int BM = 256;  // rows per pair tile (128 per CTA)
+constexpr int BN = 256;
+constexpr int HALF = 128;
+constexpr int STAGES = 6;
+constexpr int A_STAGE_BYTES = HALF * BK;
+constexpr int B_STAGE_BYTES = HALF * BK;
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // per CTA
+constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8 + 16;
+
+template <int FMT>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  return (uint32_t(FMT == kInt8 ? 2 : 1) << 4) | (uint32_t(FMT == kInt8 ? 1 : 0) << 7) |
+         (uint32_t(FMT == kInt8 ? 1 : 0) << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ Shared carve(uint8_t* raw) {
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  Shared s;
+  s.a = base;
+  s.b = base + STAGES * A_STAGE_BYTES;
+  s.bars = reinterpret_cast<uint64_t*>(s.b + STAGES * B_STAGE_BYTES);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + NUM_BARS);
+  s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_holder + 1);
+  return s;
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
+                 int M, int N, int K, unsigned int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  const Shared sh = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + BK - 1) / BK;
+
+  auto bar = [&](int i) { return ptx::smem_u32(sh.bars + i); };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto empty_bar = [&](int s) { return bar(STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar(2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar(2 * STAGES + ACC_BUFS + b); };
+  const uint32_t drain_bar = bar(2 * STAGES + 2 * ACC_BUFS);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full_bar(s), 1);   // used in CTA 0: its producer's arrive + both CTAs' bytes
+      ptx::mbar_init(empty_bar(s), 1);  // CTA 0's commit, multicast to both CTAs
+    }
+    for (int b = 0; b < ACC_BUFS; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 8);  // used in CTA 0: 4 epilogue warps x 2 CTAs
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *sh.abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmap_a);
+    ptx::prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(ptx::smem_u32(sh.tmem_holder), TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before_sync();
+  ptx::cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
+  ptx::tc_fence_after_sync();
+  const uint32_t tmem_base = *sh.tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
+          const uint32_t fb = ptx::mapa_shared(full_bar(stage), 0);
+          if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          ptx::tma_load_2d_pair(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, kb * BK,
+                                m_blk * BM + int(rank) * HALF, fb);
+          ptx::tma_load_2d_pair(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, kb * BK,
+                                n_blk * BN + int(rank) * HALF, fb);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // CTA 0 sees both CTAs' copies complete on its barriers; CTA 1 is held by the final
+      // cluster barrier until CTA 0 got here
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) drain_wait(full_bar(s), (issued_parity >> s) & 1u, status);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (CTA 0)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = instr_desc<FMT>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+        if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, sh.abort_flag, status)) break;
+        ptx::tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, sh.abort_flag, status)) { ok = false; break; }
+          ptx::tc_fence_after_sync();
+          const uint32_t a_addr = ptx::smem_u32(sh.a + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = ptx::smem_u32(sh.b + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_addr + kk * UMMA_K);
+            const uint64_t bd = smem_desc_sw128(b_addr + kk * UMMA_K);
+            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            if (FMT == kInt8) ptx::mma_i8_pair(d_tmem, ad, bd, idesc, accumulate);
+            else ptx::mma_f8_pair(d_tmem, ad, bd, idesc, accumulate);
+          }
+          ptx::tc_commit_pair_mc(empty_bar(stage), 0x3);  // both CTAs' stage is free
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::tc_commit_pair_mc(tfull_bar(acc), 0x3);  // both halves of the accumulator ready
+        if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+      }
+      ptx::tc_commit_pair(drain_bar);
+      drain_wait(drain_bar, 0, status);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const float sab = (OUT == kOutBf16) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair_id; tile < num_tiles; tile += num_pairs) {
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      int ok = 0;
+      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, sh.abort_flag, status) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      ptx::tc_fence_after_sync();
+      const int64_t row = int64_t(m_blk) * BM + int(rank) * HALF + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
+        ptx::tmem_ld_wait();
+        const int col0 = n_blk * BN + c * 32;
+        if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+      }
+      ptx::tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
+      if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  ptx::tc_fence_before_sync();
+  ptx::cluster_sync();  // no CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    ptx::tc_fence_after_sync();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace pair
+
 }  // namespace gemm
 }  // namespace hq
