@@ -25,8 +25,11 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_ARG", 2: "HQ_ERR_SHAPE", 3: "HQ_ERR_DTYPE
                 4: "HQ_ERR_ALIGN", 5: "HQ_ERR_NONFINITE", 6: "HQ_ERR_TIMEOUT", 7: "HQ_ERR_CUDA",
                 8: "HQ_ERR_WORKSPACE", 9: "HQ_ERR_UNSUPPORTED"}
 
-EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc", "hq_gemm", "hq_linear_workspace_bytes",
-           "hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw", "hq_get_error",
+EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
+           "hq_quantize_dual_workspace_bytes", "hq_quantize_dual", "hq_gemm",
+           "hq_linear_workspace_bytes", "hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw",
+           "hq_linear_fwd_bwd_workspace_bytes", "hq_linear_fwd_bwd", "hq_selftest_gemm_timeout",
+           "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
 
@@ -59,6 +62,14 @@ def lib() -> ctypes.CDLL:
         L.hq_quantize.restype = i32
         L.hq_quantize_noalloc.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p]
         L.hq_quantize_noalloc.restype = i32
+        L.hq_quantize_dual_workspace_bytes.argtypes = []
+        L.hq_quantize_dual_workspace_bytes.restype = sz
+        L.hq_quantize_dual.argtypes = [p, i32, i64, i64, i32, i32, p, p, p, p, p, sz, p]
+        L.hq_quantize_dual.restype = i32
+        L.hq_linear_fwd_bwd_workspace_bytes.argtypes = [i64, i64, i64]
+        L.hq_linear_fwd_bwd_workspace_bytes.restype = sz
+        L.hq_linear_fwd_bwd.argtypes = [p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, sz, p]
+        L.hq_linear_fwd_bwd.restype = i32
         L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm.restype = i32
         L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]
@@ -67,6 +78,8 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.argtypes = [p, p, i32, i64, i64, i64, i32, i32, p, p, sz, p]
             f.restype = i32
+        L.hq_selftest_gemm_timeout.argtypes = [p, p, p, i64, i64, i64, p]
+        L.hq_selftest_gemm_timeout.restype = i32
         L.hq_get_error.argtypes = [p]
         L.hq_get_error.restype = i32
         L.hq_last_cuda_error.argtypes = []
@@ -163,6 +176,64 @@ def hq_quantize(src, dim: int, k: int, fmt, codes=None, scale=None, workspace=No
                            _stream_handle(stream))
     _check(st, "hq_quantize")
     return codes, scale
+
+
+def hq_quantize_dual_workspace_bytes() -> int:
+    return int(lib().hq_quantize_dual_workspace_bytes())
+
+
+def hq_quantize_dual(src, k: int, fmt, codes_c=None, scale_c=None, codes_r=None, scale_r=None,
+                     workspace=None, stream=None):
+    """Both rotations of `src` [rows][cols] at once.  Returns (codes_c [rows][cols], scale_c,
+    codes_r [cols][rows], scale_r): rotated along cols and along rows respectively."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    dev = src.device
+    codes_c = torch.empty((rows, cols), dtype=torch.uint8, device=dev) if codes_c is None else codes_c
+    codes_r = torch.empty((cols, rows), dtype=torch.uint8, device=dev) if codes_r is None else codes_r
+    scale_c = torch.empty(1, dtype=torch.float32, device=dev) if scale_c is None else scale_c
+    scale_r = torch.empty(1, dtype=torch.float32, device=dev) if scale_r is None else scale_r
+    for t, n in ((codes_c, "codes_c"), (codes_r, "codes_r"), (scale_c, "scale_c"), (scale_r, "scale_r")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_quantize_dual_workspace_bytes(), dev, workspace)
+    st = lib().hq_quantize_dual(src.data_ptr(), dt, rows, cols, k, _fmt(fmt), codes_c.data_ptr(),
+                                scale_c.data_ptr(), codes_r.data_ptr(), scale_r.data_ptr(),
+                                ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_quantize_dual")
+    return codes_c, scale_c, codes_r, scale_r
+
+
+def hq_linear_fwd_bwd_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_fwd_bwd_workspace_bytes(M, K, N))
+
+
+def hq_linear_fwd_bwd(X, W, dY, k: int, fmt, Y=None, dX=None, dW=None, workspace=None, stream=None):
+    """The layer step: (Y, dX, dW) = (X W^T, dY W, dY^T X), every operand quantized once in both
+    rotations."""
+    torch = _torch()
+    for t, n in ((X, "X"), (W, "W"), (dY, "dY")):
+        _dev_tensor(t, n)
+    dt = _src_dtype(X, "X")
+    if _src_dtype(W, "W") != dt or _src_dtype(dY, "dY") != dt:
+        raise TypeError("X, W and dY must have the same dtype")
+    M, K = X.shape
+    N = W.shape[0]
+    dev = X.device
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if Y is None else Y
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if dW is None else dW
+    for t, n in ((Y, "Y"), (dX, "dX"), (dW, "dW")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_fwd_bwd_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_fwd_bwd(X.data_ptr(), W.data_ptr(), dY.data_ptr(), dt, M, K, N, k, _fmt(fmt),
+                                 Y.data_ptr(), dX.data_ptr(), dW.data_ptr(), ws.data_ptr(),
+                                 ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_linear_fwd_bwd")
+    return Y, dX, dW
 
 
 def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None):

@@ -15,8 +15,8 @@
 //
 // Data movement (HBM-bound; log2(k) <= 8 adds per element against 3-5 bytes moved):
 //   pass 1 rotates and reduces the absmax into one partial per CTA, pass 2 reduces the
-//   partials, rotates again and writes the 1-byte codes.  Pass 2 walks the tensor in the
-//   reverse order of pass 1 so its first reads hit what pass 1 left in L2.
+//   partials, rotates again and writes the 1-byte codes.  Consecutive passes over the same
+//   tensor walk it in opposite directions so each starts on what the previous left in L2.
 //   * along the contiguous dimension (dim = 1): each thread owns 8 consecutive elements
 //     (one 16-byte bf16 load or two fp32 loads), bits 0-2 of the in-block index live in
 //     registers, bits 3.. across lanes (warp shuffles); 8 code bytes per thread, 256
@@ -362,7 +362,7 @@ template <typename SrcT, int K, int MODE, bool WIDE>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__ codes,
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
-                  unsigned int* __restrict__ status) {
+                  unsigned int* __restrict__ status, int reverse) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr bool EXCH = K >= 64;
@@ -385,18 +385,18 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
   const int64_t n_units = (n + kRowsWarpElems - 1) / kRowsWarpElems;
   float amax = 0.0f;
   if (gw < n_units) {
-    // pass 1 walks forward, pass 2 backward (its first reads hit what pass 1 left in L2)
+    // alternate passes over a tensor walk it in opposite directions, so each pass starts on
+    // what the previous one left in L2
     const int64_t last = gw + tw * ((n_units - 1 - gw) / tw);
-    const int64_t first = QUANT ? last : gw;
-    const int64_t step = QUANT ? -tw : tw;
-    uint32_t raw[RW];
-    load_rows32<SrcT, WIDE, QUANT>(src, n, first * kRowsWarpElems + 32 * lane, raw);
-    for (int64_t u = first; QUANT ? u >= 0 : u < n_units; u += step) {
+    const int64_t first = reverse ? last : gw;
+    const int64_t step = reverse ? -tw : tw;
+    // two units in flight per thread: the loads of unit u + 2 step go out while u is computed
+    auto valid = [&](int64_t u) { return reverse ? u >= 0 : u < n_units; };
+    auto body = [&](uint32_t (&raw)[RW], int64_t u) {
       float2 v[16];
       unpack_rows32<SrcT>(raw, v);
-      const int64_t nu = u + step;
-      if (QUANT ? nu >= 0 : nu < n_units)
-        load_rows32<SrcT, WIDE, QUANT>(src, n, nu * kRowsWarpElems + 32 * lane, raw);
+      const int64_t nu = u + 2 * step;
+      if (valid(nu)) load_rows32<SrcT, WIDE, QUANT>(src, n, nu * kRowsWarpElems + 32 * lane, raw);
       stages_low<(K < 32 ? K : 32), 16>(v);
       if constexpr (EXCH) {
         exchange_rows(v, xch + warp * 256, lane);
@@ -432,6 +432,14 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
             if (e0 + 32 * b < n) *reinterpret_cast<uint32_t*>(codes + e0 + 32 * b) = w[b];
         }
       }
+    };
+    uint32_t raw0[RW], raw1[RW];
+    load_rows32<SrcT, WIDE, QUANT>(src, n, first * kRowsWarpElems + 32 * lane, raw0);
+    if (valid(first + step)) load_rows32<SrcT, WIDE, QUANT>(src, n, (first + step) * kRowsWarpElems + 32 * lane, raw1);
+    for (int64_t u = first; valid(u); u += 2 * step) {
+      body(raw0, u);
+      if (!valid(u + step)) break;
+      body(raw1, u + step);
     }
   }
   if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
@@ -439,15 +447,16 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
 
 // ------------------------------------------------------------------ dim = 0, bf16 source
 
-// A CTA tile is 256 rows x 64 bf16 columns (32 KB), double-buffered in shared memory with
-// cp.async (zero-filled past the tensor's edge).  Warp w owns the tile's 8 columns of 16-byte
+// A CTA tile is 256 rows x 64 bf16 columns (32 KB); a 3-tile ring in shared memory is filled
+// by cp.async (zero-filled past the tensor's edge), two tiles ahead of the one computed.  Warp w owns the tile's 8 columns of 16-byte
 // chunk w; ldmatrix.trans turns four 8x8 blocks at a time into column-major fragments so that
 // thread t holds 64 consecutive rows (64*(t&3) + 0..63) of column 8w + t/4: in-block row bits
 // 0..5 are register bits, bits 6 and 7 lane bits (shuffles only for k = 128, 256).  The
 // codes of a thread are 64 contiguous bytes of the transposed output.
 constexpr int kColsTileRows2 = 256;
 constexpr int kColsTileCols2 = 64;
-constexpr size_t kColsSmemBytes2 = 2ull * kColsTileRows2 * 128;  // two 32 KB tiles
+constexpr int kColsStages2 = 3;
+constexpr size_t kColsSmemBytes2 = size_t(kColsStages2) * kColsTileRows2 * 128;  // 3 x 32 KB tiles
 
 // 16-byte chunk swizzle of tile row rho: row bit 0 -> bit 0, row bits 6, 7 -> bits 1, 2, so
 // the 8 rows one ldmatrix matrix reads (rows differing in bits 0, 6, 7) hit distinct banks.
@@ -469,10 +478,10 @@ template <int K, int MODE>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols,
                        uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
-                       float* __restrict__ scale_out, unsigned int* __restrict__ status) {
+                       float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
-  extern __shared__ __align__(128) uint4 tiles[];  // [2][256 rows][8 chunks]
+  extern __shared__ __align__(128) uint4 tiles[];  // [3][256 rows][8 chunks]
   __shared__ float scratch[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float c = __frsqrt_rn(static_cast<float>(K));
@@ -508,15 +517,18 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
   const int64_t G = gridDim.x, b0 = blockIdx.x;
   if (b0 < n_tiles) {
     const int64_t last = b0 + G * ((n_tiles - 1 - b0) / G);
-    const int64_t first = QUANT ? last : b0;
-    const int64_t step = QUANT ? -G : G;
+    const int64_t first = reverse ? last : b0;
+    const int64_t step = reverse ? -G : G;
+    auto valid = [&](int64_t t) { return reverse ? t >= 0 : t < n_tiles; };
     int buf = 0;
     issue(0, first);
-    for (int64_t t = first; QUANT ? t >= 0 : t < n_tiles; t += step) {
-      const int64_t nt = t + step;
-      const bool has_next = QUANT ? nt >= 0 : nt < n_tiles;
-      if (has_next) {
-        issue(buf ^ 1, nt);
+    if (valid(first + step)) issue(1, first + step);
+    for (int64_t t = first; valid(t); t += step) {
+      // keep two tiles in flight; wait only for this tile's copies
+      if (valid(t + 2 * step)) {
+        issue(buf == 0 ? 2 : buf - 1, t + 2 * step);
+        cp_async_wait<2>();
+      } else if (valid(t + step)) {
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
@@ -536,7 +548,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
             v[4 * kc + mm] = make_float2(__uint_as_float(r[mm] << 16), __uint_as_float(r[mm] & 0xFFFF0000u));
         }
       }
-      __syncthreads();  // buffer free for the next-but-one tile's copies
+      __syncthreads();  // buffer free before the copies issued next iteration reuse it
       stages_low<(K < 64 ? K : 64), 32>(v);
       if constexpr (K >= 128) stage_lanes<32>(v, 1, lane);
       if constexpr (K >= 256) stage_lanes<32>(v, 2, lane);
@@ -563,7 +575,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
           }
         }
       }
-      buf ^= 1;
+      buf = buf == 2 ? 0 : buf + 1;
     }
   }
   if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
@@ -578,7 +590,7 @@ template <typename SrcT, int K, int MODE>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
-                  float* __restrict__ scale_out, unsigned int* __restrict__ status) {
+                  float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr int CPC = 16 / static_cast<int>(sizeof(SrcT));  // columns per 16-byte chunk
@@ -604,7 +616,7 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
     const int64_t G = gridDim.x;
     const int64_t b = blockIdx.x;
     const int64_t last = b + G * ((n_tiles - 1 - b) / G);
-    for (int64_t t = QUANT ? last : b; QUANT ? t >= 0 : t < n_tiles; t += QUANT ? -G : G) {
+    for (int64_t t = reverse ? last : b; reverse ? t >= 0 : t < n_tiles; t += reverse ? -G : G) {
       const int64_t r0 = (t / n_ct) * kColsTileRows;
       const int64_t c0 = (t % n_ct) * TCOLS;
       __syncthreads();  // previous tile's gather is done before the tile is overwritten

@@ -156,7 +156,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
             const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
-            int M, int N, int K, unsigned int* __restrict__ status) {
+            int M, int N, int K, unsigned int* __restrict__ status, int skip_first_load) {
   extern __shared__ uint8_t smem_raw[];
   const Shared sh = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -208,6 +208,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         tile_coords(tile, num_m, m_blk, n_blk);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
+          if (skip_first_load && tile == static_cast<int>(blockIdx.x) && kb == 0) {
+            // test hook: leave the first stage un-armed so the MMA warp's bounded wait on it
+            // expires (HQ_ERR_TIMEOUT) and every role takes the abort path
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            continue;
+          }
           ptx::mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
           ptx::tma_load_2d(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, kb * BK, m_blk * BM, full_bar(stage));
           ptx::tma_load_2d(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, kb * BK, n_blk * BN, full_bar(stage));

@@ -90,23 +90,44 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ quantization launches
 
-// CTAs of both quantization passes for a shape (the absmax pass writes one partial per CTA).
-int64_t quant_grid(hq_dtype dt, int64_t rows, int64_t cols, int dim, int sms) {
-  int64_t want, cap;
+// Work units of a quantization pass (warp steps along the contiguous dimension, or tiles).
+int64_t quant_units(hq_dtype dt, int64_t rows, int64_t cols, int dim) {
   if (dim == 1) {
     const int64_t units = (rows * cols + hq::kRowsWarpElems - 1) / hq::kRowsWarpElems;
-    want = (units + hq::kQuantThreads / 32 - 1) / (hq::kQuantThreads / 32);
-    cap = int64_t(sms) * 4;
-  } else if (dt == HQ_BF16) {
-    want = ((rows + hq::kColsTileRows2 - 1) / hq::kColsTileRows2) *
-           ((cols + hq::kColsTileCols2 - 1) / hq::kColsTileCols2);
-    cap = int64_t(sms) * 2;
-  } else {
-    const int64_t tcols = 8 * (16 / 4);
-    want = ((rows + hq::kColsTileRows - 1) / hq::kColsTileRows) * ((cols + tcols - 1) / tcols);
-    cap = int64_t(sms) * 2;
+    return (units + hq::kQuantThreads / 32 - 1) / (hq::kQuantThreads / 32);
   }
-  return std::max<int64_t>(1, std::min<int64_t>(want, std::min<int64_t>(cap, kMaxPartials)));
+  if (dt == HQ_BF16)
+    return ((rows + hq::kColsTileRows2 - 1) / hq::kColsTileRows2) *
+           ((cols + hq::kColsTileCols2 - 1) / hq::kColsTileCols2);
+  const int64_t tcols = 8 * (16 / 4);
+  return ((rows + hq::kColsTileRows - 1) / hq::kColsTileRows) * ((cols + tcols - 1) / tcols);
+}
+
+// Upper bound on the CTAs of any quantization pass (the partial-maxima capacity it needs).
+int64_t quant_grid(hq_dtype dt, int64_t rows, int64_t cols, int dim, int sms) {
+  return std::max<int64_t>(1, std::min<int64_t>(quant_units(dt, rows, cols, dim),
+                                                std::min<int64_t>(int64_t(sms) * 4, kMaxPartials)));
+}
+
+// Co-resident CTAs per SM of a kernel (cached): grids never exceed one full wave, so no
+// pass ends with a partial second wave.
+int blocks_per_sm(const void* fn, size_t smem) {
+  static std::mutex mu;
+  static const void* keys[512];
+  static int vals[512];
+  static int n = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (keys[i] == fn) return vals[i];
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fn, hq::kQuantThreads, smem) != cudaSuccess || b < 1) b = 1;
+  b = std::min(b, 4);
+  if (n < 512) {
+    keys[n] = fn;
+    vals[n] = b;
+    ++n;
+  }
+  return b;
 }
 
 template <int K, int MODE>
@@ -122,37 +143,92 @@ cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
   return e;
 }
 
+// Launch one pass; returns its grid through *grid (the absmax pass's grid is the number of
+// partials the code pass reduces).
 template <typename SrcT, int K, int MODE>
 cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes,
-                        float* scale, float* partials, int g, DeviceInfo& d, cudaStream_t st) {
+                        float* scale, float* partials, int n_partials, int reverse, DeviceInfo& d,
+                        cudaStream_t st, int* grid) {
   using namespace hq;
+  const int64_t units = quant_units(sizeof(SrcT) == 2 ? HQ_BF16 : HQ_F32, rows, cols, dim);
+  auto grid_for = [&](const void* fn, size_t smem) {
+    const int64_t cap = std::min<int64_t>(int64_t(d.sms) * blocks_per_sm(fn, smem), kMaxPartials);
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, cap)));
+  };
+  int g = 1;
   if (dim == 1) {
     const int64_t n = rows * cols;
-    if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0)
-      fwhtq_rows_kernel<SrcT, K, MODE, true><<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, g, scale, d.status);
-    else
-      fwhtq_rows_kernel<SrcT, K, MODE, false><<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, g, scale, d.status);
+    if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0) {
+      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, true>;
+      g = grid_for(reinterpret_cast<const void*>(fn), 0);
+      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+    } else {
+      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, false>;
+      g = grid_for(reinterpret_cast<const void*>(fn), 0);
+      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+    }
   } else if constexpr (sizeof(SrcT) == 2) {
     cudaError_t e = cols_bf16_smem_attr<K, MODE>(d);
     if (e != cudaSuccess) return e;
-    fwhtq_cols_bf16_kernel<K, MODE><<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+    auto fn = fwhtq_cols_bf16_kernel<K, MODE>;
+    g = grid_for(reinterpret_cast<const void*>(fn), kColsSmemBytes2);
+    fn<<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
   } else {
-    fwhtq_cols_f32_kernel<SrcT, K, MODE><<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, g, scale, d.status);
+    auto fn = fwhtq_cols_f32_kernel<SrcT, K, MODE>;
+    g = grid_for(reinterpret_cast<const void*>(fn), 0);
+    fn<<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
   }
+  *grid = g;
   return cudaGetLastError();
 }
 
+// One operand, one rotation: absmax pass forward, code pass backward.
 template <typename SrcT, int K>
 cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim, hq_fmt fmt,
                          uint8_t* codes, float* scale, float* partials, DeviceInfo& d,
                          cudaStream_t st) {
   const SrcT* src = static_cast<const SrcT*>(src_v);
   using namespace hq;
-  const int g = static_cast<int>(quant_grid(sizeof(SrcT) == 2 ? HQ_BF16 : HQ_F32, rows, cols, dim, d.sms));
-  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, g, d, st);
+  int g1 = 0, g2 = 0;
+  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, 0, 0, d, st, &g1);
   if (e != cudaSuccess) return e;
-  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g, d, st);
-  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g, d, st);
+  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g1, 1, d, st, &g2);
+  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g1, 1, d, st, &g2);
+}
+
+// One operand, both rotations: the four passes run back to back, alternating direction, so
+// after the first only what L2 cannot hold is read from HBM again.
+template <typename SrcT, int K>
+cudaError_t launch_dual(const void* src_v, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
+                        float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
+                        DeviceInfo& d, cudaStream_t st) {
+  const SrcT* src = static_cast<const SrcT*>(src_v);
+  using namespace hq;
+  int gc = 0, gr = 0, g = 0;
+  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 1, codes_c, scale_c, part_c, 0, 0, d, st, &gc);
+  if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 0, codes_r, scale_r, part_r, 0, 1, d, st, &gr);
+  if (e != cudaSuccess) return e;
+  if (fmt == HQ_INT8) {
+    e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, d, st, &g);
+    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, d, st, &g);
+  } else {
+    e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, d, st, &g);
+    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, d, st, &g);
+  }
+  return e;
+}
+
+template <typename SrcT>
+cudaError_t launch_dual_k(const void* src, int64_t rows, int64_t cols, int k, hq_fmt fmt, uint8_t* codes_c,
+                          float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
+                          DeviceInfo& d, cudaStream_t st) {
+  switch (k) {
+    case 16: return launch_dual<SrcT, 16>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 32: return launch_dual<SrcT, 32>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 64: return launch_dual<SrcT, 64>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 128: return launch_dual<SrcT, 128>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    default: return launch_dual<SrcT, 256>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+  }
 }
 
 template <typename SrcT>
@@ -217,7 +293,8 @@ hq_status encode_codes_map(CUtensorMap* map, const void* base, int64_t rows, int
 
 template <int FMT, int OUT>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
-                        void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st) {
+                        void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st,
+                        int skip_first_load = 0) {
   auto kernel = hq::gemm::gemm_kernel<FMT, OUT>;
   const unsigned bit = 1u << (FMT * 2 + OUT);
   {
@@ -231,7 +308,8 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const floa
   }
   const int tiles = ((M + hq::gemm::BM - 1) / hq::gemm::BM) * ((N + hq::gemm::BN - 1) / hq::gemm::BN);
   const int grid = std::max(1, std::min(tiles, d.sms));
-  kernel<<<grid, hq::gemm::NUM_THREADS, hq::gemm::SMEM_BYTES, st>>>(ta, tb, sa, sb, out, M, N, K, d.status);
+  kernel<<<grid, hq::gemm::NUM_THREADS, hq::gemm::SMEM_BYTES, st>>>(ta, tb, sa, sb, out, M, N, K, d.status,
+                                                                     skip_first_load);
   return cudaGetLastError();
 }
 
@@ -399,6 +477,68 @@ hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, 
   return gemm_impl(w.codes_a, w.scale_a, w.codes_b, w.scale_b, gm, gn, gk, fmt, HQ_OUT_BF16, out, *d, st);
 }
 
+// ------------------------------------------------------------------ quantize once, both rotations
+
+hq_status check_dual_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
+                          const void* codes_c, const float* scale_c, const void* codes_r, const float* scale_r) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (rows < 0 || cols < 0 || !scale_c || !scale_r) return HQ_ERR_ARG;
+  if (rows == 0 || cols == 0) return HQ_OK;
+  if (!src || !codes_c || !codes_r) return HQ_ERR_ARG;
+  if (rows % k != 0 || cols % k != 0) return HQ_ERR_SHAPE;
+  if (rows > (int64_t(1) << 40) / cols) return HQ_ERR_SHAPE;
+  if (!aligned16(src) || !aligned16(codes_c) || !aligned16(codes_r)) return HQ_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(scale_c) & 3u) || (reinterpret_cast<uintptr_t>(scale_r) & 3u)) return HQ_ERR_ALIGN;
+  return HQ_OK;
+}
+
+hq_status dual_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt, void* codes_c,
+                    float* scale_c, void* codes_r, float* scale_r, float* part_c, float* part_r, DeviceInfo& d,
+                    cudaStream_t st) {
+  if (rows == 0 || cols == 0) {
+    set_scale_one_kernel<<<1, 1, 0, st>>>(scale_c);
+    set_scale_one_kernel<<<1, 1, 0, st>>>(scale_r);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  uint8_t* cc = static_cast<uint8_t*>(codes_c);
+  uint8_t* cr = static_cast<uint8_t*>(codes_r);
+  cudaError_t e = dt == HQ_BF16
+                      ? launch_dual_k<__nv_bfloat16>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st)
+                      : launch_dual_k<float>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// Workspace of hq_linear_fwd_bwd: six code tensors, six scales, two partial buffers.
+struct StepWs {
+  uint8_t *xq, *xqt, *wq, *wqt, *dyq, *dyqt;
+  float* scales;  // x_c, x_r, w_c, w_r, dy_c, dy_r
+  float *part_c, *part_r;
+};
+
+size_t step_ws_bytes(int64_t M, int64_t K, int64_t N) {
+  return 2 * (align_up(size_t(M * K)) + align_up(size_t(N * K)) + align_up(size_t(M * N))) + kAlign +
+         2 * kPartialBytes;
+}
+
+hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t N, StepWs* w) {
+  if (!ws || ws_bytes < step_ws_bytes(M, K, N)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HQ_ERR_ALIGN;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  auto take = [&](size_t n) { uint8_t* r = p; p += align_up(n); return r; };
+  w->xq = take(size_t(M * K));
+  w->xqt = take(size_t(M * K));
+  w->wq = take(size_t(N * K));
+  w->wqt = take(size_t(N * K));
+  w->dyq = take(size_t(M * N));
+  w->dyqt = take(size_t(M * N));
+  w->scales = reinterpret_cast<float*>(take(kAlign));
+  w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
+  w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  return HQ_OK;
+}
+
 // ------------------------------------------------------------------ allocation-free quantize
 
 // Scratch for hq_quantize_noalloc: the absmax pass's per-CTA partial maxima, in a fixed
@@ -488,6 +628,59 @@ hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, int64_t M
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t hq_quantize_dual_workspace_bytes(void) { return 2 * kPartialBytes; }
+
+hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
+                           void* codes_c, float* scale_c, void* codes_r, float* scale_r, void* workspace,
+                           size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_dual_args(src, dt, rows, cols, k, fmt, codes_c, scale_c, codes_r, scale_r);
+  if (s != HQ_OK) return s;
+  if (rows > 0 && cols > 0) {
+    if (!workspace || ws_bytes < 2 * kPartialBytes) return HQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  }
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  float* part = static_cast<float*>(workspace);
+  return dual_impl(src, dt, rows, cols, k, fmt, codes_c, scale_c, codes_r, scale_r, part, part + kMaxPartials,
+                   *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  return step_ws_bytes(M, K, N);
+}
+
+hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt, int64_t M, int64_t K,
+                            int64_t N, int k, hq_fmt fmt, void* Y, void* dX, void* dW, void* workspace,
+                            size_t ws_bytes, hq_stream_t stream) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0) return HQ_ERR_ARG;
+  if (M % k || K % k || N % k) return HQ_ERR_SHAPE;
+  if (M == 0 || K == 0 || N == 0) return HQ_ERR_SHAPE;
+  if (!X || !W || !dY || !Y || !dX || !dW) return HQ_ERR_ARG;
+  if (fmt == HQ_INT8 && (M > HQ_MAX_K_INT8 || K > HQ_MAX_K_INT8 || N > HQ_MAX_K_INT8)) return HQ_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || !aligned16(Y) || !aligned16(dX) || !aligned16(dW))
+    return HQ_ERR_ALIGN;
+  StepWs w;
+  hq_status s = carve_step_ws(workspace, ws_bytes, M, K, N, &w);
+  if (s != HQ_OK) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* sc = w.scales;
+  // X [M][K]: along K (forward) and along M (dW);  W [N][K]: along K (forward) and along N (dX)
+  if ((s = dual_impl(X, dt, M, K, k, fmt, w.xq, sc + 0, w.xqt, sc + 1, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
+  if ((s = dual_impl(W, dt, N, K, k, fmt, w.wq, sc + 2, w.wqt, sc + 3, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st)) != HQ_OK) return s;
+  // dY [M][N]: along N (dX) and along M (dW)
+  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.dyq, sc + 4, w.dyqt, sc + 5, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
+  return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
+}
+
 hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
                               hq_fmt fmt, void* codes, float* scale, hq_stream_t stream) {
   hq_status s = check_quant_args(src, dt, rows, cols, dim, k, fmt, codes, scale);
@@ -500,6 +693,21 @@ hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_
     return HQ_ERR_WORKSPACE;
   return quantize_impl(src, dt, rows, cols, dim, k, fmt, codes, scale, partials, *d,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int64_t M, int64_t N, int64_t K,
+                                   hq_stream_t stream) {
+  hq_status s = check_gemm_args(A, nullptr, B, nullptr, M, N, K, HQ_INT8, HQ_OUT_ACC, out);
+  if (s != HQ_OK) return s;
+  if (M <= 0 || N <= 0 || K <= 0 || M > 4096 || N > 4096 || K > 4096) return HQ_ERR_SHAPE;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  CUtensorMap ta, tb;
+  if ((s = encode_codes_map(&ta, A, M, K, hq::gemm::BM)) != HQ_OK) return s;
+  if ((s = encode_codes_map(&tb, B, N, K, hq::gemm::BN)) != HQ_OK) return s;
+  cudaError_t e = launch_gemm<hq::gemm::kInt8, hq::gemm::kOutAcc>(ta, tb, nullptr, nullptr, out, int(M), int(N),
+                                                                  int(K), *d, reinterpret_cast<cudaStream_t>(stream), 1);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
 hq_status hq_get_error(hq_stream_t stream) {

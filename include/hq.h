@@ -140,6 +140,36 @@ HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, in
                            size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * hq_quantize_dual -- both rotations of one matrix in one call ("HALO" Approach: quantized
+ * rotated tensors are kept and reused; each operand of the layer is needed rotated along each
+ * of its two dimensions).  Results are bit-identical to two hq_quantize calls:
+ *   codes_c [rows][cols] + scale_c: rotated along cols  (hq_quantize dim = 1)
+ *   codes_r [cols][rows] + scale_r: rotated along rows  (hq_quantize dim = 0)
+ * rows and cols must both be multiples of k.  The four passes (two absmax, two code passes)
+ * run back to back in alternating directions so that after the first one most source reads
+ * are served by L2.  workspace: >= hq_quantize_dual_workspace_bytes() bytes.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_quantize_dual_workspace_bytes(void);
+HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k,
+                                  hq_fmt fmt, void* codes_c, float* scale_c, void* codes_r,
+                                  float* scale_r, void* workspace, size_t ws_bytes,
+                                  hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * hq_linear_fwd_bwd -- the whole layer step: Y = X W^T, dX = dY W and dW = dY^T X, each GEMM
+ * on operands rotated along its contraction dimension, with X, W and dY each quantized once in
+ * both rotations (3 x hq_quantize_dual + 3 GEMMs, 15 kernels).  Outputs equal those of
+ * hq_linear_fwd, hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
+ *   X [M][K], W [N][K], dY [M][N] (dtype dt); Y [M][N], dX [M][K], dW [N][K] bf16.
+ *   M, K, N: positive multiples of k.  workspace: >= hq_linear_fwd_bwd_workspace_bytes().
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt,
+                                   int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt, void* Y,
+                                   void* dX, void* dW, void* workspace, size_t ws_bytes,
+                                   hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * hq_quantize_noalloc -- hq_quantize for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this call: it exists for integration only.  Some callers
@@ -167,6 +197,19 @@ HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, in
 HQ_API hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols,
                                      int dim, int k, hq_fmt fmt, void* codes, float* scale,
                                      hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * hq_selftest_gemm_timeout -- test hook for the device-side failure path (no counterpart on
+ * the pages).  Runs the single-CTA INT8 GEMM (raw accumulators) on caller buffers
+ * A [M][K], B [N][K], out [M][N] int32 with its first pipeline stage deliberately left
+ * un-armed: the MMA warp's bounded wait on it expires after about one second, the kernel
+ * records HQ_ERR_TIMEOUT in the status word, every role stops, copies and MMAs in flight
+ * are drained, tensor memory is freed and the kernel returns.  hq_get_error() then reports
+ * HQ_ERR_TIMEOUT and the CUDA context stays usable.  out is unspecified.
+ * Shapes as hq_gemm, each of M, N, K at most 4096.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int64_t M,
+                                          int64_t N, int64_t K, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Status.

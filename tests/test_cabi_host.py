@@ -121,6 +121,36 @@ def test_linear_argument_errors(L, name):
         assert _lin(L, name, M=big) == 2
 
 
+def test_dual_and_step_argument_errors(L):
+    q = lambda **kw: L.hq_quantize_dual(kw.get("src", FAKE), kw.get("dt", hq.HQ_BF16), kw.get("rows", 256),
+                                        kw.get("cols", 256), kw.get("k", 64), kw.get("fmt", 0),
+                                        kw.get("cc", FAKE), kw.get("sc", FAKE), kw.get("cr", FAKE),
+                                        kw.get("sr", FAKE), kw.get("ws", FAKE), kw.get("wsb", 1 << 20), None)
+    assert q(dt=4) == 3
+    assert q(k=48) == 1
+    assert q(sr=None) == 1
+    assert q(rows=100) == 2
+    assert q(cols=96) == 2
+    assert q(cr=FAKE_MIS) == 4
+    assert q(ws=None) == 8
+    assert q(wsb=100) == 8
+    assert hq.hq_quantize_dual_workspace_bytes() >= 2 * hq.hq_quantize_workspace_bytes()
+    f = lambda **kw: L.hq_linear_fwd_bwd(FAKE, FAKE, FAKE, kw.get("dt", hq.HQ_BF16), kw.get("M", 256),
+                                         kw.get("K", 512), kw.get("N", 256), kw.get("k", 64), 0,
+                                         kw.get("Y", FAKE), FAKE, FAKE, kw.get("ws", FAKE),
+                                         kw.get("wsb", 1 << 34), None)
+    assert f(dt=5) == 3
+    assert f(k=20) == 1
+    assert f(M=100) == 2
+    assert f(M=0) == 2
+    assert f(Y=None) == 1
+    assert f(Y=FAKE_MIS) == 4
+    assert f(ws=None) == 8
+    assert f(wsb=1000) == 8
+    M, K, N = 4096, 4096, 11008
+    assert hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N) >= 2 * (M * K + N * K + M * N)
+
+
 def test_python_binding_rejects_cpu_tensors(L):
     import torch
     with pytest.raises(TypeError):

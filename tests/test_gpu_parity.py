@@ -140,6 +140,19 @@ def test_argument_errors():
         hq.hq_quantize(torch.randn(16, 16), 1, 16, "int8")  # CPU tensor: no fallback
 
 
+@pytest.mark.parametrize("dtype", ("f32", "bf16"))
+@pytest.mark.parametrize("k", KS)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_dual(dtype, k, fmt):
+    """Both rotations from one call equal the oracle's two quantizations bit for bit."""
+    x = _outlier_input(512 + 2 * k, 3 * k, 40 + k, dtype)
+    cc, sc, cr, sr = hq.hq_quantize_dual(to_device(x), k, fmt)
+    for codes, scale, dim in ((cc, sc, 1), (cr, sr, 0)):
+        want_codes, want_scale = oracle.quantize(x, dim, k, fmt)
+        assert np.array_equal(codes.cpu().numpy(), want_codes), f"dim {dim}"
+        assert scale.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32)
+
+
 # ------------------------------------------------------------------------------ GEMM
 
 def _rand_codes(shape, fmt, seed):
@@ -238,6 +251,34 @@ def _layer_check(d, k, fmt, rows_sample=None, tag=""):
             e = rel_fro(bits_to_f32(got), bits_to_f32(want["ref"]))
             assert e <= FP8_TOL, f"{tag}{name}: fp8 rel fro {e}"
     assert hq.hq_get_error() == 0
+
+
+def _fwd_bwd_check(d, k, fmt, rows_sample=None, tag=""):
+    """hq_linear_fwd_bwd (quantize once, both rotations) equals the three separate layer
+    entry points bit for bit, and those are checked against the oracle by _layer_check."""
+    Xd, Wd, dYd = to_device(d["X"]), to_device(d["W"]), to_device(d["dY"])
+    Y, dX, dW = hq.hq_linear_fwd_bwd(Xd, Wd, dYd, k, fmt)
+    sep = (hq.hq_linear_fwd(Xd, Wd, k, fmt), hq.hq_linear_bwd_dx(dYd, Wd, k, fmt),
+           hq.hq_linear_bwd_dw(dYd, Xd, k, fmt))
+    for name, a, b in zip(("Y", "dX", "dW"), (Y, dX, dW), sep):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{tag}{name}"
+    assert hq.hq_get_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_fwd_bwd_tiny_workload(fmt):
+    w = synthetic.WORKLOADS[1]
+    d = synthetic.draw(w)
+    _layer_check(d, w.k, fmt)
+    _fwd_bwd_check(d, w.k, fmt)
+
+
+@pytest.mark.parametrize("wid", (2, 3, 4))
+def test_fwd_bwd_full_size(wid):
+    w = synthetic.WORKLOADS[wid]
+    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
+    for li in range(len(w.layers)):
+        _fwd_bwd_check(synthetic.draw(w, li), w.k, fmt, tag=f"{w.name}/{li}/")
 
 
 @pytest.mark.parametrize("fmt", FMTS)
