@@ -510,6 +510,34 @@ hq_status dual_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, in
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
+// Per-device side stream of hq_linear_fwd_bwd (created on first use, kept until exit) and the
+// events that fork it from / join it to the caller's stream.  Enqueueing is serialised by a
+// mutex, so concurrent callers on one device interleave correctly (their side work shares
+// the one side stream).
+struct SideStream {
+  bool ready = false;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join_dx = nullptr, join_dw = nullptr;
+};
+SideStream g_side[kMaxDevices];
+std::mutex g_side_mu;
+
+hq_status side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  SideStream& ss = g_side[dev];
+  if (!ss.ready) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    for (cudaEvent_t* ev : {&ss.fork, &ss.join_dx, &ss.join_dw})
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+    ss.ready = true;
+  }
+  *out = &ss;
+  return HQ_OK;
+}
+
 // Workspace of hq_linear_fwd_bwd: six code tensors, six scales, two partial buffers.
 struct StepWs {
   uint8_t *xq, *xqt, *wq, *wqt, *dyq, *dyqt;
@@ -670,14 +698,28 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* sc = w.scales;
-  // X [M][K]: along K (forward) and along M (dW);  W [N][K]: along K (forward) and along N (dX)
-  if ((s = dual_impl(X, dt, M, K, k, fmt, w.xq, sc + 0, w.xqt, sc + 1, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
-  if ((s = dual_impl(W, dt, N, K, k, fmt, w.wq, sc + 2, w.wqt, sc + 3, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
+  float* sc = w.scales;  // x_K, x_M, w_K, w_N, dy_N, dy_M
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  if ((s = side_stream(&ss)) != HQ_OK) return s;
+  cudaError_t e;
+  if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+  // side stream: the four rotations the forward GEMM does not need, in the order the
+  // backward GEMMs need them; they run alongside the forward quantizations and GEMM
+  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((s = quantize_impl(dY, dt, M, N, 1, k, fmt, w.dyq, sc + 4, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dx, ss->s)) != cudaSuccess) return cuda_fail(e);
+  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, w.dyqt, sc + 5, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
+  // caller's stream: forward operands, forward GEMM, then the backward GEMMs as their codes land
+  if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.wq, sc + 2, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st)) != HQ_OK) return s;
-  // dY [M][N]: along N (dX) and along M (dW)
-  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.dyq, sc + 4, w.dyqt, sc + 5, w.part_c, w.part_r, *d, st)) != HQ_OK) return s;
+  if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
   if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
+  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
 }
 

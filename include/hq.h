@@ -157,11 +157,15 @@ HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, in
 
 /* ------------------------------------------------------------------------------------------
  * hq_linear_fwd_bwd -- the whole layer step: Y = X W^T, dX = dY W and dW = dY^T X, each GEMM
- * on operands rotated along its contraction dimension, with X, W and dY each quantized once in
- * both rotations (3 x hq_quantize_dual + 3 GEMMs, 15 kernels).  Outputs equal those of
- * hq_linear_fwd, hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
+ * on operands rotated along its contraction dimension, every operand rotation computed once
+ * (six quantizations + three GEMMs, 15 kernels).  Outputs equal those of hq_linear_fwd,
+ * hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
  *   X [M][K], W [N][K], dY [M][N] (dtype dt); Y [M][N], dX [M][K], dW [N][K] bf16.
  *   M, K, N: positive multiples of k.  workspace: >= hq_linear_fwd_bwd_workspace_bytes().
+ * The four rotations the forward GEMM does not use (W along N, dY along N, X along M, dY
+ * along M) run on a per-device side stream that the library creates on first use (with two
+ * events) and forks from / joins back to `stream` with events, so they overlap the forward
+ * quantizations and GEMM; everything is complete when `stream` reaches the end of the call.
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
 HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt,
