@@ -314,6 +314,7 @@ def run_gpu(args):
         side.wait_event(fork)
         rec(ev_side, 0, side)
         run(q_side_dx, L_.hq_quantize, "hq_quantize")
+        rec(ev_side, 2, side)
         j_dx = torch.cuda.Event()
         j_dx.record(side)
         run(q_side_dw, L_.hq_quantize, "hq_quantize")
@@ -343,7 +344,7 @@ def run_gpu(args):
 
     # ---------------------------------------------------------------- timed region (device)
     ev_main = [[ev() for _ in range(7)] for _ in range(args.steps)]
-    ev_side = [[ev() for _ in range(2)] for _ in range(args.steps)]
+    ev_side = [[ev() for _ in range(3)] for _ in range(args.steps)]
     barrier(world, device)
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clocks:
@@ -357,10 +358,41 @@ def run_gpu(args):
     step_ms_local = sum(e[0].elapsed_time(e[6]) for e in ev_main) / args.steps
     gemm_ms = sum(e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) + e[5].elapsed_time(e[6]) for e in ev_main)
     quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev_main) + sum(e[0].elapsed_time(e[1]) for e in ev_side)
+    def mean_ms(pairs):
+        return sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    phases = {
+        "main_quant_fwd_operands": mean_ms((e[0], e[1]) for e in ev_main),
+        "gemm_fwd": mean_ms((e[1], e[2]) for e in ev_main),
+        "wait_side_dx": mean_ms((e[2], e[3]) for e in ev_main),
+        "gemm_dx": mean_ms((e[3], e[4]) for e in ev_main),
+        "wait_side_dw": mean_ms((e[4], e[5]) for e in ev_main),
+        "gemm_dw": mean_ms((e[5], e[6]) for e in ev_main),
+        "side_quant_dx_operands": mean_ms((e[0], e[2]) for e in ev_side),
+        "side_quant_dw_operands": mean_ms((e[2], e[1]) for e in ev_side),
+    }
     step_ms = reduce_max(step_ms_local, world, device)
     gemm_ms_launch = reduce_max(gemm_ms / (3 * args.steps), world, device)
     quant_ms_step = reduce_max(quant_ms / args.steps, world, device)
     launches = 15 * args.steps  # per step: 6 quantizations x 2 kernels + 3 GEMMs
+
+    # ---------------------------------------------------------------- quantizer alone
+    # The six rotations one after another on one stream (nothing overlapping), L2 flushed
+    # before each, to report the quantization kernels' own throughput.
+    alone_ms = 0.0
+    reps = max(3, min(args.steps, 10))
+    for _ in range(reps):
+        for c in q_main + [quant(*(src_args[:4]), ws_main, sh) for src_args in
+                           ((W, 0, qW_N, 3), (dY, 1, qdY_N, 4), (X, 0, qX_M, 1), (dY, 0, qdY_M, 5))]:
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record(stream)
+            st = L_.hq_quantize(*c)
+            if st:
+                raise hq.HQError(st, "hq_quantize")
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            alone_ms += a.elapsed_time(b)
+    alone_ms_step = reduce_max(alone_ms / reps, world, device)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     # Every step copies X, W, dY from pinned host memory, runs hq_linear_fwd_bwd and copies Y,
@@ -439,9 +471,12 @@ def run_gpu(args):
                      "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
                      "frac": gemm_tops / int8_peak, "traffic": traffic,
                      "peak_note": f"{peaks['src']} burst bf16 {peaks['bf16']} x {INT8_OVER_BF16} (nominal INT8/bf16 ratio; the timed region lasts tens of ms, clocks stay at max); ops = 2*M*N*K per launch"},
-        "fwht_quant": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm"],
-                       "frac": quant_gbs / peaks["hbm"], "bytes_per_step": quant_bytes,
-                       "ms_per_step": quant_ms_step, "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each) / summed event time of the quantization launches on both streams (the side stream's overlap the forward GEMM)"},
+        "fwht_quant": {"achieved_gbs": quant_bytes / (alone_ms_step * 1e-3) / 1e9, "peak_gbs": peaks["hbm"],
+                       "frac": quant_bytes / (alone_ms_step * 1e-3) / 1e9 / peaks["hbm"],
+                       "bytes_per_step": quant_bytes, "ms_per_step": alone_ms_step,
+                       "in_step_gbs": quant_gbs, "in_step_ms": quant_ms_step,
+                       "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each); achieved: the six rotations timed alone with CUDA events, L2 flushed before each; in_step: summed event time of the same launches inside the overlapped step (sharing the GPU with the GEMMs)"},
+        "phases_ms": phases,
         "gemm_ms_per_step": gemm_ms_launch * 3,
         "schedule": "forward operands + GEMM on the main stream; the other four rotations on a side stream overlapping them",
         "frac_of_int8_peak_end_to_end": value / world / int8_peak,
