@@ -421,15 +421,21 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           w[j] = qp.zero ? 0u : codes4<MODE>(mul2(mul2(v[2 * j], c2), inv2), mul2(mul2(v[2 * j + 1], c2), inv2));
+        const bool full = ub + kRowsWarpElems <= n;  // all but a ragged last unit
         if constexpr (!EXCH) {
           const int64_t e = ub + 32 * lane;
-          if (e < n) *reinterpret_cast<uint4*>(codes + e) = make_uint4(w[0], w[1], w[2], w[3]);
-          if (e + 16 < n) *reinterpret_cast<uint4*>(codes + e + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+          if (full || e < n) *reinterpret_cast<uint4*>(codes + e) = make_uint4(w[0], w[1], w[2], w[3]);
+          if (full || e + 16 < n) *reinterpret_cast<uint4*>(codes + e + 16) = make_uint4(w[4], w[5], w[6], w[7]);
         } else {
           const int64_t e0 = ub + 256 * (lane >> 3) + 4 * (lane & 7);
+          if (full) {
 #pragma unroll
-          for (int b = 0; b < 8; ++b)
-            if (e0 + 32 * b < n) *reinterpret_cast<uint32_t*>(codes + e0 + 32 * b) = w[b];
+            for (int b = 0; b < 8; ++b) *reinterpret_cast<uint32_t*>(codes + e0 + 32 * b) = w[b];
+          } else {
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+              if (e0 + 32 * b < n) *reinterpret_cast<uint32_t*>(codes + e0 + 32 * b) = w[b];
+          }
         }
       }
     };
