@@ -315,40 +315,51 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
 // both CTAs.  Epilogue warps of both CTAs report a drained accumulator to CTA 0.
 namespace pair {
 
-constexpr int BM = 256;  // rows per pair tile (128 per CTA)
-constexpr int BN = 256;
-constexpr int HALF = 128;
-constexpr int STAGES = 6;
-constexpr int A_STAGE_BYTES = HALF * BK;
-constexpr int B_STAGE_BYTES = HALF * BK;
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // per CTA
-constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
-constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8 + 16;
+constexpr int BM = 256;    // rows per pair tile (128 per CTA)
+constexpr int HALF = 128;  // A rows per CTA
 
-template <int FMT>
+// Tile geometry for an N tile of BN_ (256 or 128) columns: each CTA holds BN_/2 rows of B.
+template <int BN_>
+struct Geo {
+  static constexpr int BN = BN_;
+  static constexpr int B_ROWS = BN_ / 2;
+  static constexpr int A_STAGE_BYTES = HALF * BK;
+  static constexpr int B_STAGE_BYTES = B_ROWS * BK;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // per CTA
+  static constexpr int STAGES = (6 * (16384 + 16384)) / STAGE_BYTES;  // 192 KB of stages
+  static constexpr int TMEM_COLS = ACC_BUFS * BN_;                      // 512 or 256
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+  static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8 + 16;
+};
+
+template <int FMT, int BN_>
 __host__ __device__ constexpr uint32_t instr_desc() {
   return (uint32_t(FMT == kInt8 ? 2 : 1) << 4) | (uint32_t(FMT == kInt8 ? 1 : 0) << 7) |
-         (uint32_t(FMT == kInt8 ? 1 : 0) << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+         (uint32_t(FMT == kInt8 ? 1 : 0) << 10) | (uint32_t(BN_ >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 }
 
+template <class G>
 __device__ __forceinline__ Shared carve(uint8_t* raw) {
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   Shared s;
   s.a = base;
-  s.b = base + STAGES * A_STAGE_BYTES;
-  s.bars = reinterpret_cast<uint64_t*>(s.b + STAGES * B_STAGE_BYTES);
-  s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + NUM_BARS);
+  s.b = base + G::STAGES * G::A_STAGE_BYTES;
+  s.bars = reinterpret_cast<uint64_t*>(s.b + G::STAGES * G::B_STAGE_BYTES);
+  s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + G::NUM_BARS);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_holder + 1);
   return s;
 }
 
-template <int FMT, int OUT>
+template <int FMT, int OUT, int BN_>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
                  int M, int N, int K, unsigned int* __restrict__ status) {
+  using G = Geo<BN_>;
+  constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
+  constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
-  const Shared sh = carve(smem_raw);
+  const Shared sh = carve<G>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
@@ -405,7 +416,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           ptx::tma_load_2d_pair(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, kb * BK,
                                 m_blk * BM + int(rank) * HALF, fb);
           ptx::tma_load_2d_pair(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, kb * BK,
-                                n_blk * BN + int(rank) * HALF, fb);
+                                n_blk * BN + int(rank) * G::B_ROWS, fb);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -420,7 +431,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (CTA 0)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = instr_desc<FMT>();
+      constexpr uint32_t idesc = instr_desc<FMT, BN_>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;

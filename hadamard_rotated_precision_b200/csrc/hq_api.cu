@@ -33,7 +33,6 @@ struct DeviceInfo {
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
   unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
-  int pair_clusters = 0;       // co-resident 2-CTA clusters of the pair GEMM
 };
 
 std::mutex g_mu;
@@ -329,46 +328,51 @@ hq_status check_gemm_args(const void* A, const float* sa, const void* B, const f
   return HQ_OK;
 }
 
-template <int FMT, int OUT>
-cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
-                             void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st) {
-  namespace gp = hq::gemm::pair;
-  auto kernel = gp::gemm_pair_kernel<FMT, OUT>;
-  const unsigned bit = 1u << (FMT * 2 + OUT);
-  int max_pairs = 0;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!(d.pair_attr_set & bit)) {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(gp::SMEM_BYTES));
-      if (e != cudaSuccess) return e;
-      d.pair_attr_set |= bit;
-    }
-    if (d.pair_clusters <= 0) {
-      cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * (d.sms / 2));
-      q.blockDim = dim3(hq::gemm::NUM_THREADS);
-      q.dynamicSmemBytes = gp::SMEM_BYTES;
-      cudaLaunchAttribute qa[1];
-      qa[0].id = cudaLaunchAttributeClusterDimension;
-      qa[0].val.clusterDim.x = 2;
-      qa[0].val.clusterDim.y = 1;
-      qa[0].val.clusterDim.z = 1;
-      q.attrs = qa;
-      q.numAttrs = 1;
-      int n = 0;
-      cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &q);
-      if (e != cudaSuccess) return e;
-      d.pair_clusters = n > 0 ? n : 1;
-    }
-    max_pairs = d.pair_clusters;
+// Co-resident 2-CTA clusters of a pair-GEMM instantiation (cached per device).
+int pair_clusters(const void* kernel, size_t smem, int sms) {
+  static std::mutex mu;
+  static const void* keys[64];
+  static int devs[64], vals[64];
+  static int n = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (keys[i] == kernel && devs[i] == dev) return vals[i];
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3(2 * (sms / 2));
+  q.blockDim = dim3(hq::gemm::NUM_THREADS);
+  q.dynamicSmemBytes = smem;
+  cudaLaunchAttribute qa[1];
+  qa[0].id = cudaLaunchAttributeClusterDimension;
+  qa[0].val.clusterDim.x = 2;
+  qa[0].val.clusterDim.y = 1;
+  qa[0].val.clusterDim.z = 1;
+  q.attrs = qa;
+  q.numAttrs = 1;
+  int c = 0;
+  if (cudaOccupancyMaxActiveClusters(&c, kernel, &q) != cudaSuccess || c < 1) c = sms / 2;
+  if (n < 64) {
+    keys[n] = kernel;
+    devs[n] = dev;
+    vals[n] = c;
+    ++n;
   }
-  const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + gp::BN - 1) / gp::BN);
-  const int pairs = std::max(1, std::min(tiles, max_pairs));
+  return c;
+}
+
+template <int FMT, int OUT, int BN>
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
+                             void* out, int M, int N, int K, int clusters, DeviceInfo& d, cudaStream_t st) {
+  namespace gp = hq::gemm::pair;
+  using G = gp::Geo<BN>;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN>;
+  const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN);
+  const int pairs = std::max(1, std::min(tiles, clusters));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(hq::gemm::NUM_THREADS);
-  cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+  cfg.dynamicSmemBytes = G::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -377,7 +381,39 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  (void)d;
   return cudaLaunchKernelEx(&cfg, kernel, ta, tb, sa, sb, out, M, N, K, d.status);
+}
+
+// Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
+template <int FMT, int OUT, int BN>
+cudaError_t pair_prepare(DeviceInfo& d, int* clusters) {
+  namespace gp = hq::gemm::pair;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN>;
+  const unsigned bit = 1u << ((FMT * 2 + OUT) * 2 + (BN == 256 ? 0 : 1));
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!(d.pair_attr_set & bit)) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(gp::Geo<BN>::SMEM_BYTES));
+      if (e != cudaSuccess) return e;
+      d.pair_attr_set |= bit;
+    }
+  }
+  *clusters = pair_clusters(reinterpret_cast<const void*>(kernel), gp::Geo<BN>::SMEM_BYTES, d.sms);
+  return cudaSuccess;
+}
+
+// N tile of the pair GEMM: whichever of 256 and 128 finishes in fewer tile-times, counting
+// whole waves of `clusters`.  A 128-wide tile takes 0.78 of a 256-wide one's time on B200
+// (it needs 1.5x the operand bytes per MAC; measured on the 4096^2 x 11008 dX GEMM: 196 us
+// with 128-wide tiles in 7 waves against 126 us with 256-wide tiles in 4), so 128 wins only
+// when there are fewer 256-wide tiles than clusters.  Ties keep 256.
+int pick_pair_bn(int M, int N, int clusters) {
+  const int m_tiles = (M + hq::gemm::pair::BM - 1) / hq::gemm::pair::BM;
+  const int64_t w256 = (int64_t(m_tiles) * ((N + 255) / 256) + clusters - 1) / clusters;
+  const int64_t w128 = (int64_t(m_tiles) * ((N + 127) / 128) + clusters - 1) / clusters;
+  return (double(w128) * 0.78 < double(w256)) ? 128 : 256;
 }
 
 // GEMMs with at least one full 256-row pair tile run on CTA pairs; smaller M on single CTAs.
@@ -392,20 +428,36 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     return e == cudaSuccess ? HQ_OK : cuda_fail(e);
   }
   const bool pair = M >= kPairMinRows;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
+  using namespace hq::gemm;
+  cudaError_t e;
+  int bn = 256, clusters = 0;
+  if (pair) {
+    // both N tiles of this instantiation pair are prepared; the cluster counts are equal in
+    // practice (one CTA per SM either way)
+    if (fmt == HQ_INT8) {
+      e = ok == HQ_OUT_BF16 ? pair_prepare<kInt8, kOutBf16, 256>(d, &clusters) : pair_prepare<kInt8, kOutAcc, 256>(d, &clusters);
+      if (e == cudaSuccess) { int c2; e = ok == HQ_OUT_BF16 ? pair_prepare<kInt8, kOutBf16, 128>(d, &c2) : pair_prepare<kInt8, kOutAcc, 128>(d, &c2); }
+    } else {
+      e = ok == HQ_OUT_BF16 ? pair_prepare<kFp8, kOutBf16, 256>(d, &clusters) : pair_prepare<kFp8, kOutAcc, 256>(d, &clusters);
+      if (e == cudaSuccess) { int c2; e = ok == HQ_OUT_BF16 ? pair_prepare<kFp8, kOutBf16, 128>(d, &c2) : pair_prepare<kFp8, kOutAcc, 128>(d, &c2); }
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    bn = pick_pair_bn(m, n, clusters);
+  }
   CUtensorMap ta, tb;
   hq_status s = encode_codes_map(&ta, A, M, K, pair ? hq::gemm::pair::HALF : hq::gemm::BM);
   if (s != HQ_OK) return s;
-  if ((s = encode_codes_map(&tb, B, N, K, pair ? hq::gemm::pair::HALF : hq::gemm::BN)) != HQ_OK) return s;
-  const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
-  cudaError_t e;
-  using namespace hq::gemm;
+  if ((s = encode_codes_map(&tb, B, N, K, pair ? uint32_t(bn / 2) : uint32_t(hq::gemm::BN))) != HQ_OK) return s;
   if (pair) {
+#define HQ_PAIR_LAUNCH(F, O)                                                                   \
+  (bn == 256 ? launch_gemm_pair<F, O, 256>(ta, tb, sa, sb, out, m, n, kk, clusters, d, st) \
+             : launch_gemm_pair<F, O, 128>(ta, tb, sa, sb, out, m, n, kk, clusters, d, st))
     if (fmt == HQ_INT8)
-      e = ok == HQ_OUT_BF16 ? launch_gemm_pair<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                            : launch_gemm_pair<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+      e = ok == HQ_OUT_BF16 ? HQ_PAIR_LAUNCH(kInt8, kOutBf16) : HQ_PAIR_LAUNCH(kInt8, kOutAcc);
     else
-      e = ok == HQ_OUT_BF16 ? launch_gemm_pair<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                            : launch_gemm_pair<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+      e = ok == HQ_OUT_BF16 ? HQ_PAIR_LAUNCH(kFp8, kOutBf16) : HQ_PAIR_LAUNCH(kFp8, kOutAcc);
+#undef HQ_PAIR_LAUNCH
   } else {
     if (fmt == HQ_INT8)
       e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
