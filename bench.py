@@ -499,6 +499,86 @@ def run_gpu(args):
     return 0 if status == 0 else 1
 
 
+def run_sweep(args):
+    """Every workload's layer (and the Llama-2-7B block over INT8/FP8 x k): the whole step
+    through hq_linear_fwd_bwd, each GEMM alone and each rotation alone, CUDA events, L2
+    flushed before every timed launch group.  One JSON line per point."""
+    import torch
+    import hadamard_rotated_precision_b200 as hq
+    from hadamard_rotated_precision_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    int8_peak = peaks["bf16"] * INT8_OVER_BF16
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    L_ = hq.lib()
+    reps = max(3, args.steps)
+
+    def timed(fn):
+        for _ in range(2):
+            flush.zero_()
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / reps
+
+    out_lines = []
+    for wid in sorted(synthetic.WORKLOADS):
+        w = synthetic.WORKLOADS[wid]
+        points = list(w.sweep) if w.sweep else [(w.fmt, w.k)]
+        for li, Lr in enumerate(w.layers):
+            d = synthetic.draw(w, li)
+            def dev_t(a):
+                if a.dtype == np.uint16:
+                    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                return torch.from_numpy(a).to(dev)
+            X, W, dY = dev_t(d["X"]), dev_t(d["W"]), dev_t(d["dY"])
+            M, K, N = Lr.M, Lr.K, Lr.N
+            ws = torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N), dtype=torch.uint8, device=dev)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+            dW = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+            for fmt_name, k in points:
+                fmt = hq.HQ_INT8 if fmt_name == "int8" else hq.HQ_FP8_E4M3
+                step_ms = timed(lambda: hq.hq_linear_fwd_bwd(X, W, dY, k, fmt, Y=Y, dX=dX, dW=dW, workspace=ws))
+                codes = {}
+                quant_ms = 0.0
+                for name, src, dim in (("XK", X, 1), ("XM", X, 0), ("WK", W, 1), ("WN", W, 0), ("DN", dY, 1), ("DM", dY, 0)):
+                    c_out = torch.empty((src.shape[0], src.shape[1]) if dim == 1 else (src.shape[1], src.shape[0]),
+                                        dtype=torch.uint8, device=dev)
+                    sc = torch.empty(1, dtype=torch.float32, device=dev)
+                    quant_ms += timed(lambda: hq.hq_quantize(src, dim, k, fmt, codes=c_out, scale=sc))
+                    codes[name] = (c_out, sc)
+                gemm_ms = 0.0
+                for a, b, o in (("XK", "WK", Y), ("DN", "WN", dX), ("DM", "XM", dW)):
+                    (ca, sa), (cb, sb) = codes[a], codes[b]
+                    gemm_ms += timed(lambda: hq.hq_gemm(ca, sa, cb, sb, fmt, out=o))
+                elem = X.element_size()
+                qbytes = (elem + 1) * 2 * (M * K + N * K + M * N)
+                ops = 6.0 * M * N * K
+                line = {"workload": w.name, "layer": Lr.name, "M": M, "K": K, "N": N, "fmt": fmt_name, "k": k,
+                        "dtype": "bf16" if elem == 2 else "f32",
+                        "step_ms": step_ms, "step_tops": ops / (step_ms * 1e-3) / 1e12,
+                        "gemm_ms": gemm_ms, "gemm_tops": ops / (gemm_ms * 1e-3) / 1e12,
+                        "gemm_frac_of_peak": ops / (gemm_ms * 1e-3) / 1e12 / int8_peak,
+                        "quant_ms": quant_ms, "quant_gbs": qbytes / (quant_ms * 1e-3) / 1e9,
+                        "quant_frac_of_hbm": qbytes / (quant_ms * 1e-3) / 1e9 / peaks["hbm"],
+                        "status": hq.hq_get_error()}
+                out_lines.append(line)
+                print(json.dumps(line), flush=True)
+            del X, W, dY, ws, Y, dX, dW
+            torch.cuda.empty_cache()
+    return 0 if all(l["status"] == 0 for l in out_lines) else 1
+
+
 def run_kernel_case(args):
     """One small standalone invocation of a hot kernel, for profiler captures: a warm-up
     call, then the captured call(s).  Inputs exceed L2 (126 MB) but stay near 200 MB."""
@@ -540,9 +620,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
     ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "quant_rows", "quant_cols"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every workload (one JSON line per workload/layer/format/k) and exit")
     args = ap.parse_args(argv)
     if args.kernel_case:
         return run_kernel_case(args)
+    if args.sweep:
+        return run_sweep(args)
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
