@@ -28,7 +28,9 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_ARG", 2: "HQ_ERR_SHAPE", 3: "HQ_ERR_DTYPE
 EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_quantize_dual_workspace_bytes", "hq_quantize_dual", "hq_gemm",
            "hq_linear_workspace_bytes", "hq_linear_fwd", "hq_linear_bwd_dx", "hq_linear_bwd_dw",
-           "hq_linear_fwd_bwd_workspace_bytes", "hq_linear_fwd_bwd", "hq_selftest_gemm_timeout",
+           "hq_linear_fwd_bwd_workspace_bytes", "hq_linear_fwd_bwd",
+           "hq_linear_fwd_save_workspace_bytes", "hq_linear_fwd_save",
+           "hq_linear_bwd_workspace_bytes", "hq_linear_bwd", "hq_selftest_gemm_timeout",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -70,6 +72,13 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_fwd_bwd_workspace_bytes.restype = sz
         L.hq_linear_fwd_bwd.argtypes = [p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, sz, p]
         L.hq_linear_fwd_bwd.restype = i32
+        for name in ("hq_linear_fwd_save_workspace_bytes", "hq_linear_bwd_workspace_bytes"):
+            getattr(L, name).argtypes = [i64, i64, i64]
+            getattr(L, name).restype = sz
+        L.hq_linear_fwd_save.argtypes = [p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, sz, p]
+        L.hq_linear_fwd_save.restype = i32
+        L.hq_linear_bwd.argtypes = [p, p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, sz, p]
+        L.hq_linear_bwd.restype = i32
         L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm.restype = i32
         L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]
@@ -234,6 +243,64 @@ def hq_linear_fwd_bwd(X, W, dY, k: int, fmt, Y=None, dX=None, dW=None, workspace
                                  ws.numel() * ws.element_size(), _stream_handle(stream))
     _check(st, "hq_linear_fwd_bwd")
     return Y, dX, dW
+
+
+def hq_linear_fwd_save_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_fwd_save_workspace_bytes(M, K, N))
+
+
+def hq_linear_fwd_save(X, W, k: int, fmt, Y=None, xqt=None, xqt_scale=None, workspace=None, stream=None):
+    """Y = X W^T, and X's codes rotated along the tokens (xqt [K][M] uint8 + device scale) kept
+    for hq_linear_bwd.  Returns (Y, xqt, xqt_scale)."""
+    torch = _torch()
+    _dev_tensor(X, "X")
+    _dev_tensor(W, "W")
+    dt = _src_dtype(X, "X")
+    if _src_dtype(W, "W") != dt:
+        raise TypeError("X and W must have the same dtype")
+    M, K = X.shape
+    N = W.shape[0]
+    dev = X.device
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if Y is None else Y
+    xqt = torch.empty((K, M), dtype=torch.uint8, device=dev) if xqt is None else xqt
+    xqt_scale = torch.empty((1,), dtype=torch.float32, device=dev) if xqt_scale is None else xqt_scale
+    for t, n in ((Y, "Y"), (xqt, "xqt"), (xqt_scale, "xqt_scale")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_fwd_save_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_fwd_save(X.data_ptr(), W.data_ptr(), dt, M, K, N, k, _fmt(fmt), Y.data_ptr(),
+                                  xqt.data_ptr(), xqt_scale.data_ptr(), ws.data_ptr(),
+                                  ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_linear_fwd_save")
+    return Y, xqt, xqt_scale
+
+
+def hq_linear_bwd_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_bwd_workspace_bytes(M, K, N))
+
+
+def hq_linear_bwd(dY, W, xqt, xqt_scale, k: int, fmt, dX=None, dW=None, workspace=None, stream=None):
+    """(dX, dW) = (dY W, dY^T X) with X given by the codes hq_linear_fwd_save kept."""
+    torch = _torch()
+    for t, n in ((dY, "dY"), (W, "W"), (xqt, "xqt"), (xqt_scale, "xqt_scale")):
+        _dev_tensor(t, n)
+    dt = _src_dtype(dY, "dY")
+    if _src_dtype(W, "W") != dt:
+        raise TypeError("dY and W must have the same dtype")
+    M, N = dY.shape
+    K = W.shape[1]
+    if tuple(xqt.shape) != (K, M):
+        raise ValueError(f"xqt must be [K][M] = [{K}][{M}]")
+    dev = dY.device
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if dW is None else dW
+    for t, n in ((dX, "dX"), (dW, "dW")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_bwd_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_bwd(dY.data_ptr(), W.data_ptr(), xqt.data_ptr(), xqt_scale.data_ptr(), dt, M, K, N, k,
+                             _fmt(fmt), dX.data_ptr(), dW.data_ptr(), ws.data_ptr(),
+                             ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_linear_bwd")
+    return dX, dW
 
 
 def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None):

@@ -619,6 +619,45 @@ hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t
   return HQ_OK;
 }
 
+// Shape and format checks shared by the multi-GEMM layer calls (every one of M, K, N is a
+// contraction length of one of the layer's GEMMs and a rotated dimension).
+hq_status check_step_shape(hq_dtype dt, int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0) return HQ_ERR_ARG;
+  if (M % k || K % k || N % k) return HQ_ERR_SHAPE;
+  if (M == 0 || K == 0 || N == 0) return HQ_ERR_SHAPE;
+  if (fmt == HQ_INT8 && (M > HQ_MAX_K_INT8 || K > HQ_MAX_K_INT8 || N > HQ_MAX_K_INT8)) return HQ_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
+  return HQ_OK;
+}
+
+// Workspace of hq_linear_fwd_save (X along K, W along K) and hq_linear_bwd (dY along N,
+// W along N, dY along M): up to three code tensors, scales, two partial buffers.
+size_t codes_ws_bytes(int64_t b0, int64_t b1, int64_t b2) {
+  return align_up(size_t(b0)) + align_up(size_t(b1)) + align_up(size_t(b2)) + kAlign + 2 * kPartialBytes;
+}
+
+struct CodesWs {
+  uint8_t* c[3];
+  float* scales;
+  float *part_c, *part_r;
+};
+
+hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int64_t b2, CodesWs* w) {
+  if (!ws || ws_bytes < codes_ws_bytes(b0, b1, b2)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HQ_ERR_ALIGN;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  auto take = [&](size_t n) { uint8_t* r = p; p += align_up(n); return r; };
+  w->c[0] = take(size_t(b0));
+  w->c[1] = take(size_t(b1));
+  w->c[2] = take(size_t(b2));
+  w->scales = reinterpret_cast<float*>(take(kAlign));
+  w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
+  w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  return HQ_OK;
+}
+
 // ------------------------------------------------------------------ allocation-free quantize
 
 // Scratch for hq_quantize_noalloc: the absmax pass's per-CTA partial maxima, in a fixed
@@ -734,18 +773,13 @@ size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
 hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt, int64_t M, int64_t K,
                             int64_t N, int k, hq_fmt fmt, void* Y, void* dX, void* dW, void* workspace,
                             size_t ws_bytes, hq_stream_t stream) {
-  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
-  if (M < 0 || K < 0 || N < 0) return HQ_ERR_ARG;
-  if (M % k || K % k || N % k) return HQ_ERR_SHAPE;
-  if (M == 0 || K == 0 || N == 0) return HQ_ERR_SHAPE;
+  hq_status s = check_step_shape(dt, M, K, N, k, fmt);
+  if (s != HQ_OK) return s;
   if (!X || !W || !dY || !Y || !dX || !dW) return HQ_ERR_ARG;
-  if (fmt == HQ_INT8 && (M > HQ_MAX_K_INT8 || K > HQ_MAX_K_INT8 || N > HQ_MAX_K_INT8)) return HQ_ERR_SHAPE;
-  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || !aligned16(Y) || !aligned16(dX) || !aligned16(dW))
     return HQ_ERR_ALIGN;
   StepWs w;
-  hq_status s = carve_step_ws(workspace, ws_bytes, M, K, N, &w);
+  s = carve_step_ws(workspace, ws_bytes, M, K, N, &w);
   if (s != HQ_OK) return s;
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
@@ -773,6 +807,80 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
   if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
+}
+
+size_t hq_linear_fwd_save_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  return codes_ws_bytes(M * K, N * K, 0);
+}
+
+hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                             hq_fmt fmt, void* Y, void* xqt_codes, float* xqt_scale, void* workspace,
+                             size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_step_shape(dt, M, K, N, k, fmt);
+  if (s != HQ_OK) return s;
+  if (!X || !W || !Y || !xqt_codes || !xqt_scale) return HQ_ERR_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || !aligned16(xqt_codes) ||
+      (reinterpret_cast<uintptr_t>(xqt_scale) & 3u))
+    return HQ_ERR_ALIGN;
+  CodesWs w;
+  if ((s = carve_codes_ws(workspace, ws_bytes, M * K, N * K, 0, &w)) != HQ_OK) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  if ((s = side_stream(&ss)) != HQ_OK) return s;
+  cudaError_t e;
+  if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+  // side stream: the codes kept for the weight gradient
+  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, xqt_codes, xqt_scale, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
+  // caller's stream: the forward operands and GEMM
+  if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.c[0], w.scales + 0, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.c[1], w.scales + 1, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st)) != HQ_OK)
+    return s;
+  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
+  return HQ_OK;
+}
+
+size_t hq_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  return codes_ws_bytes(M * N, K * N, N * M);
+}
+
+hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, const float* xqt_scale, hq_dtype dt,
+                        int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt, void* dX, void* dW, void* workspace,
+                        size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_step_shape(dt, M, K, N, k, fmt);
+  if (s != HQ_OK) return s;
+  if (!dY || !W || !xqt_codes || !xqt_scale || !dX || !dW) return HQ_ERR_ARG;
+  if (!aligned16(dY) || !aligned16(W) || !aligned16(xqt_codes) || !aligned16(dX) || !aligned16(dW) ||
+      (reinterpret_cast<uintptr_t>(xqt_scale) & 3u))
+    return HQ_ERR_ALIGN;
+  CodesWs w;
+  if ((s = carve_codes_ws(workspace, ws_bytes, M * N, K * N, N * M, &w)) != HQ_OK) return s;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* sc = w.scales;  // dy_N, w_N, dy_M
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  if ((s = side_stream(&ss)) != HQ_OK) return s;
+  cudaError_t e;
+  if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+  // side stream: dY along the tokens, for the weight gradient
+  if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, w.c[2], sc + 2, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
+  // caller's stream: dX operands and GEMM, then dW once dY's second rotation has landed
+  if ((s = quantize_impl(dY, dt, M, N, 1, k, fmt, w.c[0], sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.c[1], sc + 1, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.c[0], sc + 0, w.c[1], sc + 1, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
+  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
+  return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
 }
 
 hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,

@@ -174,6 +174,40 @@ HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY,
                                    hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Training flow with saved codes ("HALO" Approach: the quantized rotated tensors are kept for
+ * the backward pass instead of the bf16 activation, which halves the activation memory).
+ *
+ * hq_linear_fwd_save -- Y = X W^T like hq_linear_fwd, and in the same call X rotated along the
+ * tokens M and quantized: xqt_codes [K][M] (1 byte per element, M innermost) and the device
+ * scalar *xqt_scale, exactly the codes and scale hq_quantize(X, dim = 0) gives.  Keep them
+ * for hq_linear_bwd; X itself is then not needed after the forward.
+ *   X [M][K], W [N][K] (dtype dt); Y [M][N] bf16; M, K, N positive multiples of k.
+ *   workspace: >= hq_linear_fwd_save_workspace_bytes(M, K, N) bytes (not preserved).
+ * X along M runs on the library's per-device side stream (see hq_linear_fwd_bwd), alongside
+ * the forward quantizations and GEMM; all outputs are complete when `stream` reaches the end
+ * of the call.
+ *
+ * hq_linear_bwd -- dX = dY W and dW = dY^T X from the saved codes: dY is quantized once in
+ * both rotations (along N for dX, along M for dW; the latter on the side stream), W along N,
+ * then the two GEMMs.  Outputs equal those of hq_linear_bwd_dx and hq_linear_bwd_dw (the
+ * latter given the X the codes came from) bit for bit.
+ *   dY [M][N], W [N][K] (dtype dt); xqt_codes [K][M] and xqt_scale from hq_linear_fwd_save
+ *   with the same M, K, k and fmt (not checked: the library cannot tell codes apart);
+ *   dX [M][K], dW [N][K] bf16.  workspace: >= hq_linear_bwd_workspace_bytes(M, K, N).
+ * Errors: as hq_linear_fwd_bwd; a null xqt_codes or xqt_scale is HQ_ERR_ARG.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_linear_fwd_save_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t M,
+                                    int64_t K, int64_t N, int k, hq_fmt fmt, void* Y,
+                                    void* xqt_codes, float* xqt_scale, void* workspace,
+                                    size_t ws_bytes, hq_stream_t stream);
+HQ_API size_t hq_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes,
+                               const float* xqt_scale, hq_dtype dt, int64_t M, int64_t K,
+                               int64_t N, int k, hq_fmt fmt, void* dX, void* dW, void* workspace,
+                               size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * hq_quantize_noalloc -- hq_quantize for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this call: it exists for integration only.  Some callers

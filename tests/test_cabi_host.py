@@ -151,12 +151,49 @@ def test_dual_and_step_argument_errors(L):
     assert hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N) >= 2 * (M * K + N * K + M * N)
 
 
+def test_saved_codes_flow_argument_errors(L):
+    fs = lambda **kw: L.hq_linear_fwd_save(FAKE, FAKE, kw.get("dt", hq.HQ_BF16), kw.get("M", 256),
+                                           kw.get("K", 512), kw.get("N", 256), kw.get("k", 64), 0,
+                                           kw.get("Y", FAKE), kw.get("xqt", FAKE), kw.get("sx", FAKE),
+                                           kw.get("ws", FAKE), kw.get("wsb", 1 << 34), None)
+    assert fs(dt=2) == 3
+    assert fs(k=12) == 1
+    assert fs(M=96) == 2                     # tokens not a multiple of k: no rotation along M
+    assert fs(N=0) == 2
+    assert fs(xqt=None) == 1
+    assert fs(sx=None) == 1
+    assert fs(xqt=FAKE_MIS) == 4
+    assert fs(sx=FAKE + 2) == 4
+    assert fs(ws=None) == 8
+    assert fs(wsb=4096) == 8
+    b = lambda **kw: L.hq_linear_bwd(FAKE, FAKE, kw.get("xqt", FAKE), kw.get("sx", FAKE),
+                                     kw.get("dt", hq.HQ_BF16), kw.get("M", 256), kw.get("K", 512),
+                                     kw.get("N", 256), kw.get("k", 64), kw.get("fmt", 1),
+                                     kw.get("dX", FAKE), kw.get("dW", FAKE), kw.get("ws", FAKE),
+                                     kw.get("wsb", 1 << 34), None)
+    assert b(dt=3) == 3
+    assert b(fmt=4) == 1
+    assert b(K=80) == 2
+    assert b(M=133248, K=128, N=128, fmt=0) == 2   # INT8 contraction bound on the dW GEMM
+    assert b(xqt=None) == 1
+    assert b(dW=None) == 1
+    assert b(dX=FAKE_MIS) == 4
+    assert b(ws=None) == 8
+    assert b(wsb=4096) == 8
+    M, K, N = 4096, 4096, 11008
+    assert hq.hq_linear_fwd_save_workspace_bytes(M, K, N) >= M * K + N * K
+    assert hq.hq_linear_bwd_workspace_bytes(M, K, N) >= 2 * M * N + K * N
+    assert hq.hq_linear_bwd_workspace_bytes(-1, 1, 1) == 0
+
+
 def test_python_binding_rejects_cpu_tensors(L):
     import torch
     with pytest.raises(TypeError):
         hq.hq_quantize(torch.zeros(16, 16), 1, 16, "int8")
     with pytest.raises(TypeError):
         hq.hq_linear_fwd(torch.zeros(16, 16), torch.zeros(16, 16), 16, "int8")
+    with pytest.raises(TypeError):
+        hq.hq_linear_fwd_save(torch.zeros(16, 16), torch.zeros(16, 16), 16, "int8")
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

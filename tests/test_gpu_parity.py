@@ -265,12 +265,31 @@ def _fwd_bwd_check(d, k, fmt, rows_sample=None, tag=""):
     assert hq.hq_get_error() == 0
 
 
+def _saved_codes_check(d, k, fmt, tag=""):
+    """Training flow: hq_linear_fwd_save keeps X's token-rotated codes (equal to the oracle's
+    quantization of X along M bit for bit), and hq_linear_bwd from those codes gives the same
+    dX and dW as the separate entry points given X itself."""
+    X = d["X"]
+    Xd, Wd, dYd = to_device(X), to_device(d["W"]), to_device(d["dY"])
+    Y, xqt, sx = hq.hq_linear_fwd_save(Xd, Wd, k, fmt)
+    want_codes, want_scale = oracle.quantize(X, 0, k, fmt)
+    assert np.array_equal(xqt.cpu().numpy(), want_codes), f"{tag}saved codes"
+    assert sx.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32), f"{tag}saved scale"
+    dX, dW = hq.hq_linear_bwd(dYd, Wd, xqt, sx, k, fmt)
+    sep = (hq.hq_linear_fwd(Xd, Wd, k, fmt), hq.hq_linear_bwd_dx(dYd, Wd, k, fmt),
+           hq.hq_linear_bwd_dw(dYd, Xd, k, fmt))
+    for name, a, b in zip(("Y", "dX", "dW"), (Y, dX, dW), sep):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{tag}{name}"
+    assert hq.hq_get_error() == 0
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_fwd_bwd_tiny_workload(fmt):
     w = synthetic.WORKLOADS[1]
     d = synthetic.draw(w)
     _layer_check(d, w.k, fmt)
     _fwd_bwd_check(d, w.k, fmt)
+    _saved_codes_check(d, w.k, fmt)
 
 
 @pytest.mark.parametrize("wid", (2, 3, 4))
@@ -278,44 +297,21 @@ def test_fwd_bwd_full_size(wid):
     w = synthetic.WORKLOADS[wid]
     fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
     for li in range(len(w.layers)):
-        _fwd_bwd_check(synthetic.draw(w, li), w.k, fmt, tag=f"{w.name}/{li}/")
+        d = synthetic.draw(w, li)
+        _fwd_bwd_check(d, w.k, fmt, tag=f"{w.name}/{li}/")
+        _saved_codes_check(d, w.k, fmt, tag=f"{w.name}/{li}/")
 
 
+@pytest.mark.parametrize("dtype", ("f32", "bf16"))
+@pytest.mark.parametrize("k", KS)
 @pytest.mark.parametrize("fmt", FMTS)
-def test_layer_tiny_workload(fmt):
-    w = synthetic.WORKLOADS[1]
-    _layer_check(synthetic.draw(w), w.k, fmt)
-
-
-@pytest.mark.parametrize("wid", (2, 3, 4))
-def test_layer_token_prefix(wid):
-    """Each workload at its full K and N but a 512-token prefix (exact, full comparison)."""
-    w = synthetic.WORKLOADS[wid]
-    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
-    for li in range(len(w.layers)):
-        _layer_check(synthetic.draw(w, li, M=512), w.k, fmt, tag=f"{w.name}/{li}/")
-
-
-@pytest.mark.parametrize("wid", (1, 2, 3, 4))
-def test_layer_full_size(wid):
-    """Each workload at its full size (the bench's launch configuration), outputs compared on
-    sampled rows; codes and scales compared in full."""
-    w = synthetic.WORKLOADS[wid]
-    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
-    for li in range(len(w.layers)):
-        _layer_check(synthetic.draw(w, li), w.k, fmt, rows_sample=True, tag=f"{w.name}/{li}/")
-
-
-@pytest.mark.parametrize("fmt_name,k", synthetic.WORKLOADS[5].sweep)
-def test_llama_block_sweep_o_proj(fmt_name, k):
-    """Llama-2-7B block sweep over formats and k on the 4096 -> 4096 projection (8192 tokens)."""
-    w = synthetic.WORKLOADS[5]
-    fmt = oracle.INT8 if fmt_name == "int8" else oracle.FP8_E4M3
-    _layer_check(synthetic.draw(w, 1), k, fmt, rows_sample=True, tag=f"o/{fmt_name}/{k}/")
-
-
-@pytest.mark.parametrize("li", (0, 2, 4))
-def test_llama_block_other_shapes(li):
-    """qkv (4096 -> 12288), gate (4096 -> 11008) and down (11008 -> 4096) at INT8 k=256."""
-    w = synthetic.WORKLOADS[5]
-    _layer_check(synthetic.draw(w, li), 256, oracle.INT8, rows_sample=True, tag=f"{li}/")
+def test_saved_codes_every_k(dtype, k, fmt):
+    """The saved-codes flow at every k, both formats and both source dtypes, on a layer of
+    3k tokens, 2k inputs and 5k outputs (several GEMM tiles only at the larger k)."""
+    M, K, N = 3 * k, 2 * k, 5 * k
+    X = _outlier_input(M, K, 70 + k, dtype)
+    W = synthetic.tiny_random((N, K), 80 + k, scale=0.02)
+    dY = synthetic.tiny_random((M, N), 90 + k, scale=1e-3)
+    if dtype == "bf16":
+        W, dY = synthetic.to_bf16_bits(W), synthetic.to_bf16_bits(dY)
+    _saved_codes_check({"X": X, "W": W, "dY": dY}, k, fmt, tag=f"{dtype}/{k}/{fmt}/")
