@@ -69,6 +69,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 struct Shared {
   uint8_t* a;
   uint8_t* b;
+  uint8_t* epi;  // pair kernel: bf16 output boxes staged for TMA stores
   uint64_t* bars;
   uint32_t* tmem_holder;
   volatile int* abort_flag;
@@ -79,6 +80,7 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   Shared s;
   s.a = base;
   s.b = base + STAGES * A_STAGE_BYTES;
+  s.epi = nullptr;
   s.bars = reinterpret_cast<uint64_t*>(s.b + STAGES * B_STAGE_BYTES);
   s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + NUM_BARS);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_holder + 1);
@@ -329,7 +331,11 @@ struct Geo {
   static constexpr int STAGES = (6 * (16384 + 16384)) / STAGE_BYTES;  // 192 KB of stages
   static constexpr int TMEM_COLS = ACC_BUFS * BN_;                      // 512 or 256
   static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
-  static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8 + 16;
+  // bf16 epilogue: each of the 4 epilogue warps owns two 32 x 32 bf16 boxes (2 KB each)
+  static constexpr int EPI_BOX_BYTES = 32 * 32 * 2;
+  static constexpr int EPI_BYTES = 4 * 2 * EPI_BOX_BYTES;
+  static constexpr size_t SMEM_BYTES =
+      1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
 };
 
 template <int FMT, int BN_>
@@ -344,7 +350,8 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   Shared s;
   s.a = base;
   s.b = base + G::STAGES * G::A_STAGE_BYTES;
-  s.bars = reinterpret_cast<uint64_t*>(s.b + G::STAGES * G::B_STAGE_BYTES);
+  s.epi = s.b + G::STAGES * G::B_STAGE_BYTES;  // 1024-byte aligned
+  s.bars = reinterpret_cast<uint64_t*>(s.epi + G::EPI_BYTES);
   s.tmem_holder = reinterpret_cast<uint32_t*>(s.bars + G::NUM_BARS);
   s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_holder + 1);
   return s;
@@ -353,8 +360,9 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
 template <int FMT, int OUT, int BN_>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
-                 int M, int N, int K, unsigned int* __restrict__ status) {
+                 const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
+                 const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
+                 unsigned int* __restrict__ status) {
   using G = Geo<BN_>;
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
@@ -390,6 +398,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     ptx::fence_proxy_async_smem();
     ptx::prefetch_tmap(&tmap_a);
     ptx::prefetch_tmap(&tmap_b);
+    if (OUT == kOutBf16) ptx::prefetch_tmap(&tmap_out);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(ptx::smem_u32(sh.tmem_holder), TMEM_COLS);
@@ -468,6 +477,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int quarter = warp & 3;
     const float sab = (OUT == kOutBf16) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
+    const uint32_t epi_base = ptx::smem_u32(sh.epi) + uint32_t(quarter) * 2u * G::EPI_BOX_BYTES;
+    int last_box = -1;  // box of this warp's most recent TMA store
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair_id; tile < num_tiles; tile += num_pairs) {
@@ -477,21 +488,75 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       ptx::tc_fence_after_sync();
-      const int64_t row = int64_t(m_blk) * BM + int(rank) * HALF + quarter * 32 + lane;
+      const int row0 = m_blk * BM + int(rank) * HALF + quarter * 32;  // first row of this warp
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
+      if constexpr (OUT == kOutBf16) {
+        // Chunk c (32 columns) goes TMEM -> registers -> bf16 box in shared memory -> TMA
+        // store.  The TMEM read of chunk c + 1 is in flight while chunk c is converted, and
+        // the stores run asynchronously; a buffer is rewritten only once the store that last
+        // used it has read it.
+        uint32_t r[2][32];
+        ptx::tmem_ld_32x32b_x32(t_row, r[0]);
+        ptx::tmem_ld_wait(r[0]);
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          if (c + 1 < BN / 32) ptx::tmem_ld_32x32b_x32(t_row + uint32_t((c + 1) * 32), r[(c + 1) & 1]);
+          const int b = c & 1;
+          const uint32_t box = epi_base + uint32_t(b) * G::EPI_BOX_BYTES;
+          if (lane == 0) {
+            if (b == last_box) ptx::bulk_wait_read<0>();
+            else ptx::bulk_wait_read<1>();
+          }
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 8 * q + 2 * e;
+              float x0, x1;
+              if (FMT == kInt8) {
+                x0 = __int2float_rn(static_cast<int>(r[b][i]));
+                x1 = __int2float_rn(static_cast<int>(r[b][i + 1]));
+              } else {
+                x0 = __uint_as_float(r[b][i]);
+                x1 = __uint_as_float(r[b][i + 1]);
+              }
+              const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(x0, sab), __fmul_rn(x1, sab));
+              pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            ptx::st_shared_v4(box + uint32_t(lane * 64 + q * 16), pk[0], pk[1], pk[2], pk[3]);
+          }
+          ptx::fence_proxy_async_smem();  // the box is visible to the TMA engine
+          __syncwarp();
+          const int col0 = n_blk * BN + c * 32;
+          if (col0 < N && row0 < M) {  // boxes reaching past the edge are clipped by TMA
+            if (lane == 0) {
+              ptx::tma_store_2d(&tmap_out, box, col0, row0);
+              ptx::bulk_commit();
+            }
+            last_box = b;
+          }
+          if (c + 1 < BN / 32) ptx::tmem_ld_wait(r[(c + 1) & 1]);
+        }
+      } else {
+        const int64_t row = int64_t(row0) + lane;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
-        ptx::tmem_ld_wait();
-        const int col0 = n_blk * BN + c * 32;
-        if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
+          ptx::tmem_ld_wait();
+          const int col0 = n_blk * BN + c * 32;
+          if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+        }
       }
       ptx::tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
+    // every store of this warp has completed (and its shared memory been read) before exit
+    if (OUT == kOutBf16 && lane == 0) ptx::bulk_wait<0>();
   }
 
   ptx::tc_fence_before_sync();

@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "hq.h"
@@ -290,6 +291,22 @@ hq_status encode_codes_map(CUtensorMap* map, const void* base, int64_t rows, int
   return HQ_OK;
 }
 
+// bf16 output [rows][cols] as 32 x 32 boxes for the pair GEMM's TMA-store epilogue.
+hq_status encode_out_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  hq_status s = tensor_map_encoder(&enc);
+  if (s != HQ_OK) return s;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return HQ_OK;
+}
+
 template <int FMT, int OUT>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
                         void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st,
@@ -362,8 +379,9 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
 }
 
 template <int FMT, int OUT, int BN>
-cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
-                             void* out, int M, int N, int K, int clusters, DeviceInfo& d, cudaStream_t st) {
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
+                             const float* sb, void* out, int M, int N, int K, int clusters, DeviceInfo& d,
+                             cudaStream_t st) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN>;
   auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN>;
@@ -382,7 +400,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   (void)d;
-  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, sa, sb, out, M, N, K, d.status);
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status);
 }
 
 // Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
@@ -450,9 +468,12 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
   if (s != HQ_OK) return s;
   if ((s = encode_codes_map(&tb, B, N, K, pair ? uint32_t(bn / 2) : uint32_t(hq::gemm::BN))) != HQ_OK) return s;
   if (pair) {
-#define HQ_PAIR_LAUNCH(F, O)                                                                   \
-  (bn == 256 ? launch_gemm_pair<F, O, 256>(ta, tb, sa, sb, out, m, n, kk, clusters, d, st) \
-             : launch_gemm_pair<F, O, 128>(ta, tb, sa, sb, out, m, n, kk, clusters, d, st))
+    CUtensorMap to;  // read by the bf16 epilogue only
+    std::memset(&to, 0, sizeof(to));
+    if (ok == HQ_OUT_BF16 && (s = encode_out_map(&to, out, M, N)) != HQ_OK) return s;
+#define HQ_PAIR_LAUNCH(F, O)                                                                       \
+  (bn == 256 ? launch_gemm_pair<F, O, 256>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st) \
+             : launch_gemm_pair<F, O, 128>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st))
     if (fmt == HQ_INT8)
       e = ok == HQ_OUT_BF16 ? HQ_PAIR_LAUNCH(kInt8, kOutBf16) : HQ_PAIR_LAUNCH(kInt8, kOutAcc);
     else

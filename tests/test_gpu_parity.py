@@ -191,6 +191,31 @@ def test_gemm_int8_bf16_epilogue(M, N, K):
     assert bf16_ulp_diff(got, ref).max() <= 1
 
 
+# CTA-pair kernel (M >= 256) with ragged row and column edges: its bf16 epilogue stores 32 x 32
+# boxes with TMA, clipped at the tensor's edge, and skips boxes wholly past it.
+PAIR_EDGE_SHAPES = [(520, 400, 256), (300, 48, 512), (256, 16, 128), (777, 1040, 384)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_EDGE_SHAPES)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_gemm_pair_bf16_edges(M, N, K, fmt):
+    A = _rand_codes((M, K), fmt, 17 * M + K)
+    B = _rand_codes((N, K), fmt, 19 * N + K)
+    sa, sb = np.float32(0.0123), np.float32(7.1e-4)
+    out = torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    hq.hq_gemm(torch.from_numpy(A).cuda(), torch.tensor([sa], device="cuda"), torch.from_numpy(B).cuda(),
+               torch.tensor([sb], device="cuda"), fmt, out=out)
+    got = bf16_bits(out)
+    ref, fast = oracle.epilogue(oracle.gemm(A, B, fmt), sa, sb)
+    if fmt == oracle.INT8:
+        np.testing.assert_array_equal(got, fast)
+        assert bf16_ulp_diff(got, ref).max() <= 1
+    else:
+        assert rel_fro(bits_to_f32(got), bits_to_f32(ref)) <= FP8_TOL
+    # nothing outside [M][N] exists to be written; every element inside was written
+    assert not np.any(got == np.uint16(0x4040)) or np.count_nonzero(bits_to_f32(ref) == 3.0) > 0
+
+
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES[:5])
 def test_gemm_fp8(M, N, K):
     A = _rand_codes((M, K), oracle.FP8_E4M3, 11 * M + K)
