@@ -591,7 +591,8 @@ def run_kernel_case(args):
     case = args.kernel_case
     if case.startswith("gemm"):
         fmt = "fp8" if case == "gemm_fp8" else "int8"
-        M, N, K = 4096, 11008, 4096
+        # the Llama up-projection forward shape, or the ViT-B fc1 forward (contraction 768)
+        M, N, K = (12608, 3072, 768) if case == "gemm_short_k" else (4096, 11008, 4096)
         A = torch.randint(-127, 128, (M, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
         B = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
         if fmt == "fp8":
@@ -618,7 +619,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
-    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "quant_rows", "quant_cols"),
+    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload (one JSON line per workload/layer/format/k) and exit")

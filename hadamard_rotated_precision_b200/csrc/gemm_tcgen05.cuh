@@ -321,22 +321,32 @@ constexpr int BM = 256;    // rows per pair tile (128 per CTA)
 constexpr int HALF = 128;  // A rows per CTA
 
 // Tile geometry for an N tile of BN_ (256 or 128) columns: each CTA holds BN_/2 rows of B.
-template <int BN_>
+// The bf16 epilogue stages output boxes of 32 rows x 64 columns (4 KB, 128-byte swizzle) in
+// shared memory for TMA stores.  Default shape: a 192 KB operand ring and two boxes per
+// epilogue warp.  SHORT_K (contractions of at most kShortKBlocks k-blocks, where a tile's main
+// loop is shorter than writing its output): a 128 KB ring and room for the warp's whole
+// tile share, so the accumulator is released as soon as it has been read and the stores
+// stream out while the next tiles are computed.
+template <int BN_, bool SHORT_K = false>
 struct Geo {
   static constexpr int BN = BN_;
   static constexpr int B_ROWS = BN_ / 2;
   static constexpr int A_STAGE_BYTES = HALF * BK;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // per CTA
-  static constexpr int STAGES = (6 * (16384 + 16384)) / STAGE_BYTES;  // 192 KB of stages
+  static constexpr int STAGES = ((SHORT_K ? 4 : 6) * (16384 + 16384)) / STAGE_BYTES;
   static constexpr int TMEM_COLS = ACC_BUFS * BN_;                      // 512 or 256
   static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
-  // bf16 epilogue: each of the 4 epilogue warps owns two 32 x 32 bf16 boxes (2 KB each)
-  static constexpr int EPI_BOX_BYTES = 32 * 32 * 2;
-  static constexpr int EPI_BYTES = 4 * 2 * EPI_BOX_BYTES;
+  static constexpr int BOX_COLS = 64;
+  static constexpr int BOX_BYTES = 32 * BOX_COLS * 2;
+  static constexpr int CHUNKS = BN_ / BOX_COLS;         // 64-column chunks per tile and warp
+  static constexpr int NB = SHORT_K ? CHUNKS : 2;       // boxes per epilogue warp
+  static constexpr int EPI_BYTES = 4 * NB * BOX_BYTES;  // four epilogue warps
   static constexpr size_t SMEM_BYTES =
       1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
 };
+
+constexpr int kShortKBlocks = 8;  // K <= 1024 bytes: the SHORT_K shape
 
 template <int FMT, int BN_>
 __host__ __device__ constexpr uint32_t instr_desc() {
@@ -357,13 +367,13 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   return s;
 }
 
-template <int FMT, int OUT, int BN_>
+template <int FMT, int OUT, int BN_, bool SHORT_K>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
                  unsigned int* __restrict__ status) {
-  using G = Geo<BN_>;
+  using G = Geo<BN_, SHORT_K>;
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -477,8 +487,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int quarter = warp & 3;
     const float sab = (OUT == kOutBf16) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
-    const uint32_t epi_base = ptx::smem_u32(sh.epi) + uint32_t(quarter) * 2u * G::EPI_BOX_BYTES;
-    int last_box = -1;  // box of this warp's most recent TMA store
+    // bf16 output: chunk j (64 columns) of this warp's 32 rows goes TMEM -> registers -> a
+    // swizzled 32 x 64 box in shared memory -> TMA store (asynchronous).  Box b of the warp's
+    // NB boxes is rewritten only once the store that last used it has read it.
+    const uint32_t epi_base = ptx::smem_u32(sh.epi) + uint32_t(quarter) * uint32_t(G::NB * G::BOX_BYTES);
+    int box_group[G::NB];  // commit index of the store that last used each box (-1: none)
+#pragma unroll
+    for (int b = 0; b < G::NB; ++b) box_group[b] = -1;
+    int ncommit = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair_id; tile < num_tiles; tile += num_pairs) {
@@ -491,53 +507,56 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       const int row0 = m_blk * BM + int(rank) * HALF + quarter * 32;  // first row of this warp
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
       if constexpr (OUT == kOutBf16) {
-        // Chunk c (32 columns) goes TMEM -> registers -> bf16 box in shared memory -> TMA
-        // store.  The TMEM read of chunk c + 1 is in flight while chunk c is converted, and
-        // the stores run asynchronously; a buffer is rewritten only once the store that last
-        // used it has read it.
-        uint32_t r[2][32];
-        ptx::tmem_ld_32x32b_x32(t_row, r[0]);
-        ptx::tmem_ld_wait(r[0]);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          if (c + 1 < BN / 32) ptx::tmem_ld_32x32b_x32(t_row + uint32_t((c + 1) * 32), r[(c + 1) & 1]);
-          const int b = c & 1;
-          const uint32_t box = epi_base + uint32_t(b) * G::EPI_BOX_BYTES;
-          if (lane == 0) {
-            if (b == last_box) ptx::bulk_wait_read<0>();
-            else ptx::bulk_wait_read<1>();
+        for (int j = 0; j < G::CHUNKS; ++j) {
+          uint32_t r0[32], r1[32];
+          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64), r0);
+          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64 + 32), r1);
+          ptx::tmem_ld_wait(r0);
+          ptx::reg_fence(r1);
+          if (j == G::CHUNKS - 1) {  // the accumulator has been read: the MMA may reuse it
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
+          }
+          const int b = j % G::NB;
+          const uint32_t box = epi_base + uint32_t(b * G::BOX_BYTES);
+          if (lane == 0 && box_group[b] >= 0) {
+            if (ncommit - 1 - box_group[b] >= G::NB - 1) ptx::bulk_wait_read<G::NB - 1>();
+            else ptx::bulk_wait_read<0>();
           }
           __syncwarp();
+          // row `lane` of the box: 16-byte chunk q (columns 8q .. 8q+7) at q ^ (lane & 7)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 8; ++q) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int i = 8 * q + 2 * e;
+              const int i = 8 * (q & 3) + 2 * e;
+              const uint32_t u0 = q < 4 ? r0[i] : r1[i], u1 = q < 4 ? r0[i + 1] : r1[i + 1];
               float x0, x1;
               if (FMT == kInt8) {
-                x0 = __int2float_rn(static_cast<int>(r[b][i]));
-                x1 = __int2float_rn(static_cast<int>(r[b][i + 1]));
+                x0 = __int2float_rn(static_cast<int>(u0));
+                x1 = __int2float_rn(static_cast<int>(u1));
               } else {
-                x0 = __uint_as_float(r[b][i]);
-                x1 = __uint_as_float(r[b][i + 1]);
+                x0 = __uint_as_float(u0);
+                x1 = __uint_as_float(u1);
               }
               const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(x0, sab), __fmul_rn(x1, sab));
               pk[e] = *reinterpret_cast<const uint32_t*>(&h);
             }
-            ptx::st_shared_v4(box + uint32_t(lane * 64 + q * 16), pk[0], pk[1], pk[2], pk[3]);
+            ptx::st_shared_v4(box + uint32_t(lane * 128 + ((q ^ (lane & 7)) << 4)), pk[0], pk[1], pk[2], pk[3]);
           }
           ptx::fence_proxy_async_smem();  // the box is visible to the TMA engine
           __syncwarp();
-          const int col0 = n_blk * BN + c * 32;
+          const int col0 = n_blk * BN + j * G::BOX_COLS;
           if (col0 < N && row0 < M) {  // boxes reaching past the edge are clipped by TMA
             if (lane == 0) {
               ptx::tma_store_2d(&tmap_out, box, col0, row0);
               ptx::bulk_commit();
             }
-            last_box = b;
+            box_group[b] = ncommit++;
           }
-          if (c + 1 < BN / 32) ptx::tmem_ld_wait(r[(c + 1) & 1]);
         }
       } else {
         const int64_t row = int64_t(row0) + lane;
@@ -549,10 +568,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           const int col0 = n_blk * BN + c * 32;
           if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
         }
+        ptx::tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
       }
-      ptx::tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
     // every store of this warp has completed (and its shared memory been read) before exit

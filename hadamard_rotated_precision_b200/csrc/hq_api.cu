@@ -291,17 +291,18 @@ hq_status encode_codes_map(CUtensorMap* map, const void* base, int64_t rows, int
   return HQ_OK;
 }
 
-// bf16 output [rows][cols] as 32 x 32 boxes for the pair GEMM's TMA-store epilogue.
+// bf16 output [rows][cols] as 32-row x 64-column boxes (128-byte rows, 128-byte swizzle) for
+// the pair GEMM's TMA-store epilogue.
 hq_status encode_out_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   hq_status s = tensor_map_encoder(&enc);
   if (s != HQ_OK) return s;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t box[2] = {64, 32};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
   return HQ_OK;
@@ -378,13 +379,13 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
   return c;
 }
 
-template <int FMT, int OUT, int BN>
+template <int FMT, int OUT, int BN, bool SK>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
                              const float* sb, void* out, int M, int N, int K, int clusters, DeviceInfo& d,
                              cudaStream_t st) {
   namespace gp = hq::gemm::pair;
-  using G = gp::Geo<BN>;
-  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN>;
+  using G = gp::Geo<BN, SK>;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK>;
   const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN);
   const int pairs = std::max(1, std::min(tiles, clusters));
   cudaLaunchConfig_t cfg = {};
@@ -404,21 +405,22 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
 }
 
 // Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
-template <int FMT, int OUT, int BN>
+template <int FMT, int OUT, int BN, bool SK>
 cudaError_t pair_prepare(DeviceInfo& d, int* clusters) {
   namespace gp = hq::gemm::pair;
-  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN>;
-  const unsigned bit = 1u << ((FMT * 2 + OUT) * 2 + (BN == 256 ? 0 : 1));
+  using G = gp::Geo<BN, SK>;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK>;
+  const unsigned bit = 1u << (((FMT * 2 + OUT) * 2 + (BN == 256 ? 0 : 1)) * 2 + (SK ? 1 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!(d.pair_attr_set & bit)) {
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(gp::Geo<BN>::SMEM_BYTES));
+                                           static_cast<int>(G::SMEM_BYTES));
       if (e != cudaSuccess) return e;
       d.pair_attr_set |= bit;
     }
   }
-  *clusters = pair_clusters(reinterpret_cast<const void*>(kernel), gp::Geo<BN>::SMEM_BYTES, d.sms);
+  *clusters = pair_clusters(reinterpret_cast<const void*>(kernel), G::SMEM_BYTES, d.sms);
   return cudaSuccess;
 }
 
@@ -450,16 +452,25 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
   using namespace hq::gemm;
   cudaError_t e;
   int bn = 256, clusters = 0;
+  // short contractions whose output is bf16 use the SHORT_K shape (fewer operand stages, the
+  // whole output tile staged for TMA stores)
+  const bool sk = pair && ok == HQ_OUT_BF16 && (K + hq::gemm::BK - 1) / hq::gemm::BK <= hq::gemm::pair::kShortKBlocks;
   if (pair) {
-    // both N tiles of this instantiation pair are prepared; the cluster counts are equal in
+    // both N tiles of the chosen instantiation are prepared; the cluster counts are equal in
     // practice (one CTA per SM either way)
+#define HQ_PAIR_PREP(F, O, SKV)                                        \
+  e = pair_prepare<F, O, 256, SKV>(d, &clusters);                      \
+  if (e == cudaSuccess) { int c2; e = pair_prepare<F, O, 128, SKV>(d, &c2); }
     if (fmt == HQ_INT8) {
-      e = ok == HQ_OUT_BF16 ? pair_prepare<kInt8, kOutBf16, 256>(d, &clusters) : pair_prepare<kInt8, kOutAcc, 256>(d, &clusters);
-      if (e == cudaSuccess) { int c2; e = ok == HQ_OUT_BF16 ? pair_prepare<kInt8, kOutBf16, 128>(d, &c2) : pair_prepare<kInt8, kOutAcc, 128>(d, &c2); }
+      if (ok == HQ_OUT_ACC) { HQ_PAIR_PREP(kInt8, kOutAcc, false) }
+      else if (sk) { HQ_PAIR_PREP(kInt8, kOutBf16, true) }
+      else { HQ_PAIR_PREP(kInt8, kOutBf16, false) }
     } else {
-      e = ok == HQ_OUT_BF16 ? pair_prepare<kFp8, kOutBf16, 256>(d, &clusters) : pair_prepare<kFp8, kOutAcc, 256>(d, &clusters);
-      if (e == cudaSuccess) { int c2; e = ok == HQ_OUT_BF16 ? pair_prepare<kFp8, kOutBf16, 128>(d, &c2) : pair_prepare<kFp8, kOutAcc, 128>(d, &c2); }
+      if (ok == HQ_OUT_ACC) { HQ_PAIR_PREP(kFp8, kOutAcc, false) }
+      else if (sk) { HQ_PAIR_PREP(kFp8, kOutBf16, true) }
+      else { HQ_PAIR_PREP(kFp8, kOutBf16, false) }
     }
+#undef HQ_PAIR_PREP
     if (e != cudaSuccess) return cuda_fail(e);
     bn = pick_pair_bn(m, n, clusters);
   }
@@ -471,13 +482,17 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     CUtensorMap to;  // read by the bf16 epilogue only
     std::memset(&to, 0, sizeof(to));
     if (ok == HQ_OUT_BF16 && (s = encode_out_map(&to, out, M, N)) != HQ_OK) return s;
-#define HQ_PAIR_LAUNCH(F, O)                                                                       \
-  (bn == 256 ? launch_gemm_pair<F, O, 256>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st) \
-             : launch_gemm_pair<F, O, 128>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st))
+#define HQ_PAIR_LAUNCH(F, O, SKV)                                                                    \
+  (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st) \
+             : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st))
     if (fmt == HQ_INT8)
-      e = ok == HQ_OUT_BF16 ? HQ_PAIR_LAUNCH(kInt8, kOutBf16) : HQ_PAIR_LAUNCH(kInt8, kOutAcc);
+      e = ok == HQ_OUT_ACC ? HQ_PAIR_LAUNCH(kInt8, kOutAcc, false)
+          : sk             ? HQ_PAIR_LAUNCH(kInt8, kOutBf16, true)
+                           : HQ_PAIR_LAUNCH(kInt8, kOutBf16, false);
     else
-      e = ok == HQ_OUT_BF16 ? HQ_PAIR_LAUNCH(kFp8, kOutBf16) : HQ_PAIR_LAUNCH(kFp8, kOutAcc);
+      e = ok == HQ_OUT_ACC ? HQ_PAIR_LAUNCH(kFp8, kOutAcc, false)
+          : sk             ? HQ_PAIR_LAUNCH(kFp8, kOutBf16, true)
+                           : HQ_PAIR_LAUNCH(kFp8, kOutBf16, false);
 #undef HQ_PAIR_LAUNCH
   } else {
     if (fmt == HQ_INT8)
