@@ -372,7 +372,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
-                 unsigned int* __restrict__ status) {
+                 unsigned int* __restrict__ status, int splits, uint32_t* __restrict__ part_ws,
+                 int* __restrict__ counters) {
   using G = Geo<BN_, SHORT_K>;
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
@@ -385,6 +386,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
+  // Work item i: tile i % num_tiles, k-block range of split i / num_tiles (splits = 1: the
+  // whole contraction).  With splits = 2 each half writes its partial accumulator to part_ws;
+  // the warp slab that finishes second adds the other half and writes the output.
+  const int num_items = num_tiles * splits;
+  const int kb_per = (num_kb + splits - 1) / splits;
 
   auto bar = [&](int i) { return ptx::smem_u32(sh.bars + i); };
   auto full_bar = [&](int s) { return bar(s); };
@@ -426,9 +432,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+      for (int item = pair_id; item < num_items && ok; item += num_pairs) {
+        const int tile = item % num_tiles, split = item / num_tiles;
         const int m_blk = tile % num_m, n_blk = tile / num_m;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int kb_end = min(num_kb, (split + 1) * kb_per);
+        for (int kb = split * kb_per; kb < kb_end; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
           const uint32_t fb = ptx::mapa_shared(full_bar(stage), 0);
           if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
@@ -456,11 +464,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
+      for (int item = pair_id; item < num_items && ok; item += num_pairs) {
+        const int split = item / num_tiles;
+        const int kb_begin = split * kb_per, kb_end = min(num_kb, kb_begin + kb_per);
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, sh.abort_flag, status)) break;
         ptx::tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!wait_bounded(full_bar(stage), phase, sh.abort_flag, status)) { ok = false; break; }
           ptx::tc_fence_after_sync();
           const uint32_t a_addr = ptx::smem_u32(sh.a + stage * A_STAGE_BYTES);
@@ -469,7 +479,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             const uint64_t ad = smem_desc_sw128(a_addr + kk * UMMA_K);
             const uint64_t bd = smem_desc_sw128(b_addr + kk * UMMA_K);
-            const uint32_t accumulate = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accumulate = (kb > kb_begin || kk > 0) ? 1u : 0u;
             if (FMT == kInt8) ptx::mma_i8_pair(d_tmem, ad, bd, idesc, accumulate);
             else ptx::mma_f8_pair(d_tmem, ad, bd, idesc, accumulate);
           }
@@ -497,7 +507,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     int ncommit = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair_id; tile < num_tiles; tile += num_pairs) {
+    for (int item = pair_id; item < num_items; item += num_pairs) {
+      const int tile = item % num_tiles, split = item / num_tiles;
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       int ok = 0;
       if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, sh.abort_flag, status) ? 1 : 0;
@@ -507,13 +518,61 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       const int row0 = m_blk * BM + int(rank) * HALF + quarter * 32;  // first row of this warp
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
       if constexpr (OUT == kOutBf16) {
+        // split contraction: publish this half's partial slab (32 rows x BN, stored so that a
+        // warp's 16-byte stores are contiguous), then count it; the half that counts second
+        // adds the other's partial to its own and writes the output, the first is done.
+        const uint32_t* peer = nullptr;
+        int* slab_counter = nullptr;
+        bool emit = true;
+        if (splits > 1) {
+          const size_t slab_words = size_t(32) * BN;
+          const size_t slab = size_t(tile) * 8 + size_t(rank) * 4 + quarter;  // [tile][rank][quarter]
+          uint32_t* mine = part_ws + (size_t(split) * num_tiles * 8 + slab) * slab_words;
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
+            ptx::tmem_ld_wait(r);
 #pragma unroll
-        for (int j = 0; j < G::CHUNKS; ++j) {
+            for (int v = 0; v < 8; ++v)
+              ptx::st_global_cg_v4(mine + size_t((c * 8 + v) * 32 + lane) * 4, r[4 * v], r[4 * v + 1], r[4 * v + 2],
+                                   r[4 * v + 3]);
+          }
+          __threadfence();
+          __syncwarp();
+          slab_counter = counters + slab;
+          int prev = 0;
+          if (lane == 0) prev = atomicAdd(slab_counter, 1);
+          prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+          emit = prev == splits - 1;
+          if (emit) {
+            __threadfence();  // the other half's partial is visible
+            peer = part_ws + (size_t(1 - split) * num_tiles * 8 + slab) * slab_words;
+          } else {  // the accumulator has been read: the MMA may reuse it
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < G::CHUNKS && emit; ++j) {
           uint32_t r0[32], r1[32];
           ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64), r0);
           ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64 + 32), r1);
           ptx::tmem_ld_wait(r0);
           ptx::reg_fence(r1);
+          if (peer) {  // own + other half: one rounding per element (fp32) or exact (int32)
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              const int c = 2 * j + (v >> 3);
+              const uint4 q = ptx::ld_global_cg_v4(peer + size_t((c * 8 + (v & 7)) * 32 + lane) * 4);
+              uint32_t* rr = (v < 8 ? r0 : r1) + 4 * (v & 7);
+              const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                rr[e] = FMT == kInt8 ? rr[e] + qq[e] : __float_as_uint(__fadd_rn(__uint_as_float(rr[e]), __uint_as_float(qq[e])));
+            }
+          }
           if (j == G::CHUNKS - 1) {  // the accumulator has been read: the MMA may reuse it
             ptx::tc_fence_before_sync();
             __syncwarp();
@@ -558,6 +617,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             box_group[b] = ncommit++;
           }
         }
+        if (peer && lane == 0) *slab_counter = 0;  // both halves counted: ready for the next launch
       } else {
         const int64_t row = int64_t(row0) + lane;
 #pragma unroll 1

@@ -381,13 +381,13 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
 
 template <int FMT, int OUT, int BN, bool SK>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
-                             const float* sb, void* out, int M, int N, int K, int clusters, DeviceInfo& d,
-                             cudaStream_t st) {
+                             const float* sb, void* out, int M, int N, int K, int clusters, int splits,
+                             uint32_t* part_ws, int* counters, DeviceInfo& d, cudaStream_t st) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN, SK>;
   auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK>;
-  const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN);
-  const int pairs = std::max(1, std::min(tiles, clusters));
+  const int items = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN) * splits;
+  const int pairs = std::max(1, std::min(items, clusters));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(hq::gemm::NUM_THREADS);
@@ -401,7 +401,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   (void)d;
-  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status);
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, splits, part_ws, counters);
 }
 
 // Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
@@ -439,8 +439,38 @@ int pick_pair_bn(int M, int N, int clusters) {
 // GEMMs with at least one full 256-row pair tile run on CTA pairs; smaller M on single CTAs.
 constexpr int64_t kPairMinRows = 256;
 
+// Split contraction for GEMMs with too few 256 x 256 tiles to fill the clusters (the weight
+// gradient of a layer with few outputs and many tokens): two halves of the k-blocks per tile,
+// when that at least cuts the waves by 30% (so the exchange of fp32/int32 partials pays off)
+// and each half keeps 8 or more k-blocks.  Workspace: both halves' partial tiles (fp32/int32)
+// and one arrival counter per 32-row slab.
+constexpr int kRefClusters = 74;  // workspace sizing: the clusters of a 148-SM B200
+
+int pick_splits(int64_t M, int64_t N, int64_t K, int clusters) {
+  if (M < kPairMinRows || clusters <= 0) return 1;
+  const int64_t num_kb = (K + hq::gemm::BK - 1) / hq::gemm::BK;
+  if (num_kb < 16) return 1;
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t w1 = (tiles + clusters - 1) / clusters, w2 = (2 * tiles + clusters - 1) / clusters;
+  return double(w2) * 0.5 <= 0.7 * double(w1) ? 2 : 1;
+}
+
+size_t split_part_bytes(int64_t M, int64_t N) {
+  return size_t(2) * size_t((M + 255) / 256) * size_t((N + 255) / 256) * 256 * 256 * 4;
+}
+size_t split_counter_bytes(int64_t M, int64_t N) {
+  return align_up(size_t((M + 255) / 256) * size_t((N + 255) / 256) * 8 * sizeof(int));
+}
+
+// Workspace a GEMM of the layer may use for a split contraction (0 when it never splits).
+size_t split_ws_bytes(int64_t M, int64_t N, int64_t K) {
+  if (pick_splits(M, N, K, kRefClusters) < 2) return 0;
+  return split_part_bytes(M, N) + split_counter_bytes(M, N);
+}
+
 hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
-                    int64_t K, hq_fmt fmt, hq_out ok, void* out, DeviceInfo& d, cudaStream_t st) {
+                    int64_t K, hq_fmt fmt, hq_out ok, void* out, DeviceInfo& d, cudaStream_t st,
+                    void* split_ws = nullptr, size_t split_ws_len = 0) {
   if (M == 0 || N == 0) return HQ_OK;
   if (K == 0) {
     const size_t elem = ok == HQ_OUT_BF16 ? 2 : 4;
@@ -474,6 +504,18 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     if (e != cudaSuccess) return cuda_fail(e);
     bn = pick_pair_bn(m, n, clusters);
   }
+  int splits = 1;
+  uint32_t* part_ws = nullptr;
+  int* counters = nullptr;
+  if (pair && !sk && ok == HQ_OUT_BF16 && split_ws && pick_splits(M, N, K, clusters) == 2 &&
+      split_ws_len >= split_part_bytes(M, N) + split_counter_bytes(M, N)) {
+    splits = 2;
+    bn = 256;
+    counters = static_cast<int*>(split_ws);
+    part_ws = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(split_ws) + split_counter_bytes(M, N));
+    e = cudaMemsetAsync(counters, 0, split_counter_bytes(M, N), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   CUtensorMap ta, tb;
   hq_status s = encode_codes_map(&ta, A, M, K, pair ? hq::gemm::pair::HALF : hq::gemm::BM);
   if (s != HQ_OK) return s;
@@ -482,9 +524,11 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     CUtensorMap to;  // read by the bf16 epilogue only
     std::memset(&to, 0, sizeof(to));
     if (ok == HQ_OUT_BF16 && (s = encode_out_map(&to, out, M, N)) != HQ_OK) return s;
-#define HQ_PAIR_LAUNCH(F, O, SKV)                                                                    \
-  (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st) \
-             : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, d, st))
+#define HQ_PAIR_LAUNCH(F, O, SKV)                                                                       \
+  (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
+                                                counters, d, st)                                             \
+             : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
+                                                counters, d, st))
     if (fmt == HQ_INT8)
       e = ok == HQ_OUT_ACC ? HQ_PAIR_LAUNCH(kInt8, kOutAcc, false)
           : sk             ? HQ_PAIR_LAUNCH(kInt8, kOutBf16, true)
@@ -513,14 +557,17 @@ struct LinearWs {
   float* scale_a;
   float* scale_b;
   float* partials;
+  void* split;  // split-contraction scratch of the GEMM (split_len bytes, may be 0)
+  size_t split_len;
 };
 
-size_t linear_ws_bytes(int64_t a_bytes, int64_t b_bytes) {
-  return align_up(size_t(a_bytes)) + align_up(size_t(b_bytes)) + kAlign + kPartialBytes;
+size_t linear_ws_bytes(int64_t a_bytes, int64_t b_bytes, size_t split_bytes) {
+  return align_up(size_t(a_bytes)) + align_up(size_t(b_bytes)) + kAlign + kPartialBytes + align_up(split_bytes);
 }
 
-hq_status carve_linear_ws(void* ws, size_t ws_bytes, int64_t a_bytes, int64_t b_bytes, LinearWs* out) {
-  if (!ws || ws_bytes < linear_ws_bytes(a_bytes, b_bytes)) return HQ_ERR_WORKSPACE;
+hq_status carve_linear_ws(void* ws, size_t ws_bytes, int64_t a_bytes, int64_t b_bytes, size_t split_bytes,
+                          LinearWs* out) {
+  if (!ws || ws_bytes < linear_ws_bytes(a_bytes, b_bytes, split_bytes)) return HQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return HQ_ERR_ALIGN;
   uint8_t* p = static_cast<uint8_t*>(ws);
   out->codes_a = p;
@@ -531,6 +578,9 @@ hq_status carve_linear_ws(void* ws, size_t ws_bytes, int64_t a_bytes, int64_t b_
   out->scale_b = reinterpret_cast<float*>(p) + 4;
   p += kAlign;
   out->partials = reinterpret_cast<float*>(p);
+  p += kPartialBytes;
+  out->split = split_bytes ? p : nullptr;
+  out->split_len = split_bytes;
   return HQ_OK;
 }
 
@@ -554,7 +604,7 @@ hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, 
   if (gm >= (int64_t(1) << 31) || gn >= (int64_t(1) << 31) || gk >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
   if (!aligned16(out) || (gk > 0 && (!aligned16(a.src) || !aligned16(b.src)))) return HQ_ERR_ALIGN;
   LinearWs w;
-  hq_status s = carve_linear_ws(ws, ws_bytes, gm * gk, gn * gk, &w);
+  hq_status s = carve_linear_ws(ws, ws_bytes, gm * gk, gn * gk, split_ws_bytes(gm, gn, gk), &w);
   if (s != HQ_OK) return s;
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
@@ -562,7 +612,8 @@ hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, 
     if ((s = quantize_impl(a.src, dt, a.rows, a.cols, a.dim, k, fmt, w.codes_a, w.scale_a, w.partials, *d, st)) != HQ_OK) return s;
     if ((s = quantize_impl(b.src, dt, b.rows, b.cols, b.dim, k, fmt, w.codes_b, w.scale_b, w.partials, *d, st)) != HQ_OK) return s;
   }
-  return gemm_impl(w.codes_a, w.scale_a, w.codes_b, w.scale_b, gm, gn, gk, fmt, HQ_OUT_BF16, out, *d, st);
+  return gemm_impl(w.codes_a, w.scale_a, w.codes_b, w.scale_b, gm, gn, gk, fmt, HQ_OUT_BF16, out, *d, st,
+                   w.split, w.split_len);
 }
 
 // ------------------------------------------------------------------ quantize once, both rotations
@@ -631,11 +682,17 @@ struct StepWs {
   uint8_t *xq, *xqt, *wq, *wqt, *dyq, *dyqt;
   float* scales;  // x_c, x_r, w_c, w_r, dy_c, dy_r
   float *part_c, *part_r;
+  void* split;  // split-contraction scratch shared by the GEMMs (they run in stream order)
+  size_t split_len;
 };
+
+size_t step_split_bytes(int64_t M, int64_t K, int64_t N) {
+  return std::max({split_ws_bytes(M, N, K), split_ws_bytes(M, K, N), split_ws_bytes(N, K, M)});
+}
 
 size_t step_ws_bytes(int64_t M, int64_t K, int64_t N) {
   return 2 * (align_up(size_t(M * K)) + align_up(size_t(N * K)) + align_up(size_t(M * N))) + kAlign +
-         2 * kPartialBytes;
+         2 * kPartialBytes + align_up(step_split_bytes(M, K, N));
 }
 
 hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t N, StepWs* w) {
@@ -652,6 +709,8 @@ hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t
   w->scales = reinterpret_cast<float*>(take(kAlign));
   w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
   w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  w->split_len = step_split_bytes(M, K, N);
+  w->split = w->split_len ? take(w->split_len) : nullptr;
   return HQ_OK;
 }
 
@@ -670,18 +729,22 @@ hq_status check_step_shape(hq_dtype dt, int64_t M, int64_t K, int64_t N, int k, 
 
 // Workspace of hq_linear_fwd_save (X along K, W along K) and hq_linear_bwd (dY along N,
 // W along N, dY along M): up to three code tensors, scales, two partial buffers.
-size_t codes_ws_bytes(int64_t b0, int64_t b1, int64_t b2) {
-  return align_up(size_t(b0)) + align_up(size_t(b1)) + align_up(size_t(b2)) + kAlign + 2 * kPartialBytes;
+size_t codes_ws_bytes(int64_t b0, int64_t b1, int64_t b2, size_t split_bytes) {
+  return align_up(size_t(b0)) + align_up(size_t(b1)) + align_up(size_t(b2)) + kAlign + 2 * kPartialBytes +
+         align_up(split_bytes);
 }
 
 struct CodesWs {
   uint8_t* c[3];
   float* scales;
   float *part_c, *part_r;
+  void* split;  // split-contraction scratch of the GEMMs (they run in stream order)
+  size_t split_len;
 };
 
-hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int64_t b2, CodesWs* w) {
-  if (!ws || ws_bytes < codes_ws_bytes(b0, b1, b2)) return HQ_ERR_WORKSPACE;
+hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int64_t b2, size_t split_bytes,
+                         CodesWs* w) {
+  if (!ws || ws_bytes < codes_ws_bytes(b0, b1, b2, split_bytes)) return HQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return HQ_ERR_ALIGN;
   uint8_t* p = static_cast<uint8_t*>(ws);
   auto take = [&](size_t n) { uint8_t* r = p; p += align_up(n); return r; };
@@ -691,6 +754,8 @@ hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int6
   w->scales = reinterpret_cast<float*>(take(kAlign));
   w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
   w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  w->split_len = split_bytes;
+  w->split = split_bytes ? take(split_bytes) : nullptr;
   return HQ_OK;
 }
 
@@ -759,9 +824,9 @@ hq_status hq_gemm(const void* A, const float* scale_a, const void* B, const floa
 size_t hq_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M < 0 || K < 0 || N < 0) return 0;
   size_t best = 0;
-  best = std::max(best, linear_ws_bytes(M * K, N * K));  // forward
-  best = std::max(best, linear_ws_bytes(M * N, K * N));  // dX
-  best = std::max(best, linear_ws_bytes(N * M, K * M));  // dW
+  best = std::max(best, linear_ws_bytes(M * K, N * K, split_ws_bytes(M, N, K)));  // forward
+  best = std::max(best, linear_ws_bytes(M * N, K * N, split_ws_bytes(M, K, N)));  // dX
+  best = std::max(best, linear_ws_bytes(N * M, K * M, split_ws_bytes(N, K, M)));  // dW
   return best;
 }
 
@@ -838,16 +903,20 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
   // caller's stream: forward operands, forward GEMM, then the backward GEMMs as their codes land
   if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.wq, sc + 2, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split, w.split_len)) !=
+      HQ_OK)
+    return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
-  if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st, w.split,
+                     w.split_len)) != HQ_OK)
+    return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
-  return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
+  return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split, w.split_len);
 }
 
 size_t hq_linear_fwd_save_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M < 0 || K < 0 || N < 0) return 0;
-  return codes_ws_bytes(M * K, N * K, 0);
+  return codes_ws_bytes(M * K, N * K, 0, split_ws_bytes(M, N, K));
 }
 
 hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
@@ -860,7 +929,7 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
       (reinterpret_cast<uintptr_t>(xqt_scale) & 3u))
     return HQ_ERR_ALIGN;
   CodesWs w;
-  if ((s = carve_codes_ws(workspace, ws_bytes, M * K, N * K, 0, &w)) != HQ_OK) return s;
+  if ((s = carve_codes_ws(workspace, ws_bytes, M * K, N * K, 0, split_ws_bytes(M, N, K), &w)) != HQ_OK) return s;
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -876,7 +945,8 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
   // caller's stream: the forward operands and GEMM
   if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.c[0], w.scales + 0, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.c[1], w.scales + 1, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st)) != HQ_OK)
+  if ((s = gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split,
+                     w.split_len)) != HQ_OK)
     return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return HQ_OK;
@@ -884,7 +954,7 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
 
 size_t hq_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   if (M < 0 || K < 0 || N < 0) return 0;
-  return codes_ws_bytes(M * N, K * N, N * M);
+  return codes_ws_bytes(M * N, K * N, N * M, std::max(split_ws_bytes(M, K, N), split_ws_bytes(N, K, M)));
 }
 
 hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, const float* xqt_scale, hq_dtype dt,
@@ -897,7 +967,9 @@ hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, co
       (reinterpret_cast<uintptr_t>(xqt_scale) & 3u))
     return HQ_ERR_ALIGN;
   CodesWs w;
-  if ((s = carve_codes_ws(workspace, ws_bytes, M * N, K * N, N * M, &w)) != HQ_OK) return s;
+  if ((s = carve_codes_ws(workspace, ws_bytes, M * N, K * N, N * M,
+                          std::max(split_ws_bytes(M, K, N), split_ws_bytes(N, K, M)), &w)) != HQ_OK)
+    return s;
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -914,9 +986,12 @@ hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, co
   // caller's stream: dX operands and GEMM, then dW once dY's second rotation has landed
   if ((s = quantize_impl(dY, dt, M, N, 1, k, fmt, w.c[0], sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.c[1], sc + 1, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = gemm_impl(w.c[0], sc + 0, w.c[1], sc + 1, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(w.c[0], sc + 0, w.c[1], sc + 1, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st, w.split,
+                     w.split_len)) != HQ_OK)
+    return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
-  return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st);
+  return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split,
+                   w.split_len);
 }
 
 hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,

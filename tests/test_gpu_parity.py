@@ -340,3 +340,69 @@ def test_saved_codes_every_k(dtype, k, fmt):
     if dtype == "bf16":
         W, dY = synthetic.to_bf16_bits(W), synthetic.to_bf16_bits(dY)
     _saved_codes_check({"X": X, "W": W, "dY": dY}, k, fmt, tag=f"{dtype}/{k}/{fmt}/")
+
+
+# Weight gradients with few output tiles and a long token contraction run as two halves of
+# the contraction whose partial sums are combined in the GEMM (split contraction): ragged
+# output edges, both formats, through the layer entry points and the layer step.
+SPLIT_SHAPES = [(4096, 272, 400), (8192, 256, 256), (3072, 768, 512)]
+
+
+@pytest.mark.parametrize("M,K,N", SPLIT_SHAPES)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_split_contraction_dw(M, K, N, fmt):
+    k = 16
+    X = _outlier_input(M, K, 3 + K, "bf16")
+    dY = synthetic.to_bf16_bits(synthetic.tiny_random((M, N), 5 + N, scale=1e-3))
+    W = synthetic.to_bf16_bits(synthetic.tiny_random((N, K), 7 + K, scale=0.02))
+    d = {"X": X, "W": W, "dY": dY}
+    out = hq.hq_linear_bwd_dw(to_device(dY), to_device(X), k, fmt)
+    want = oracle.linear_bwd_dw(dY, X, k, fmt)
+    got = bf16_bits(out)
+    if fmt == oracle.INT8:
+        np.testing.assert_array_equal(got, want["fast"])
+        assert bf16_ulp_diff(got, want["ref"]).max() <= 1
+    else:
+        assert rel_fro(bits_to_f32(got), bits_to_f32(want["ref"])) <= FP8_TOL
+    _fwd_bwd_check(d, k, fmt, tag=f"split/{M}/{K}/{N}/")
+    _saved_codes_check(d, k, fmt, tag=f"split/{M}/{K}/{N}/")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_layer_tiny_workload(fmt):
+    w = synthetic.WORKLOADS[1]
+    _layer_check(synthetic.draw(w), w.k, fmt)
+
+
+@pytest.mark.parametrize("wid", (2, 3, 4))
+def test_layer_token_prefix(wid):
+    """Each workload at its full K and N but a 512-token prefix (exact, full comparison)."""
+    w = synthetic.WORKLOADS[wid]
+    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
+    for li in range(len(w.layers)):
+        _layer_check(synthetic.draw(w, li, M=512), w.k, fmt, tag=f"{w.name}/{li}/")
+
+
+@pytest.mark.parametrize("wid", (1, 2, 3, 4))
+def test_layer_full_size(wid):
+    """Each workload at its full size (the bench's launch configuration), outputs compared on
+    sampled rows; codes and scales compared in full."""
+    w = synthetic.WORKLOADS[wid]
+    fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
+    for li in range(len(w.layers)):
+        _layer_check(synthetic.draw(w, li), w.k, fmt, rows_sample=True, tag=f"{w.name}/{li}/")
+
+
+@pytest.mark.parametrize("fmt_name,k", synthetic.WORKLOADS[5].sweep)
+def test_llama_block_sweep_o_proj(fmt_name, k):
+    """Llama-2-7B block sweep over formats and k on the 4096 -> 4096 projection (8192 tokens)."""
+    w = synthetic.WORKLOADS[5]
+    fmt = oracle.INT8 if fmt_name == "int8" else oracle.FP8_E4M3
+    _layer_check(synthetic.draw(w, 1), k, fmt, rows_sample=True, tag=f"o/{fmt_name}/{k}/")
+
+
+@pytest.mark.parametrize("li", (0, 2, 4))
+def test_llama_block_other_shapes(li):
+    """qkv (4096 -> 12288), gate (4096 -> 11008) and down (11008 -> 4096) at INT8 k=256."""
+    w = synthetic.WORKLOADS[5]
+    _layer_check(synthetic.draw(w, li), 256, oracle.INT8, rows_sample=True, tag=f"{li}/")
