@@ -359,7 +359,7 @@ __device__ __forceinline__ void exchange_rows(float2 (&v)[16], float4* slice, in
 }
 
 template <typename SrcT, int K, int MODE, bool WIDE>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, sizeof(SrcT) == 2 ? 3 : 1)
 fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__ codes,
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
                   unsigned int* __restrict__ status, int reverse) {
@@ -390,12 +390,13 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
     const int64_t last = gw + tw * ((n_units - 1 - gw) / tw);
     const int64_t first = reverse ? last : gw;
     const int64_t step = reverse ? -tw : tw;
-    // two units in flight per thread: the loads of unit u + 2 step go out while u is computed
+    // the loads of unit u + step go out while u is computed (one unit of registers, so that
+    // three CTAs fit per SM)
     auto valid = [&](int64_t u) { return reverse ? u >= 0 : u < n_units; };
     auto body = [&](uint32_t (&raw)[RW], int64_t u) {
       float2 v[16];
       unpack_rows32<SrcT>(raw, v);
-      const int64_t nu = u + 2 * step;
+      const int64_t nu = u + step;
       if (valid(nu)) load_rows32<SrcT, WIDE, QUANT>(src, n, nu * kRowsWarpElems + 32 * lane, raw);
       stages_low<(K < 32 ? K : 32), 16>(v);
       if constexpr (EXCH) {
@@ -439,14 +440,9 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
         }
       }
     };
-    uint32_t raw0[RW], raw1[RW];
-    load_rows32<SrcT, WIDE, QUANT>(src, n, first * kRowsWarpElems + 32 * lane, raw0);
-    if (valid(first + step)) load_rows32<SrcT, WIDE, QUANT>(src, n, (first + step) * kRowsWarpElems + 32 * lane, raw1);
-    for (int64_t u = first; valid(u); u += 2 * step) {
-      body(raw0, u);
-      if (!valid(u + step)) break;
-      body(raw1, u + step);
-    }
+    uint32_t raw[RW];
+    load_rows32<SrcT, WIDE, QUANT>(src, n, first * kRowsWarpElems + 32 * lane, raw);
+    for (int64_t u = first; valid(u); u += step) body(raw, u);
   }
   if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
 }
