@@ -62,6 +62,10 @@ def lib():
         L.hq_oracle_rotate.restype = i32
         L.hq_oracle_quantize.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p]
         L.hq_oracle_quantize.restype = i32
+        L.hq_oracle_rotate_signed.argtypes = [p, i32, i64, i64, i32, i32, p, p]
+        L.hq_oracle_rotate_signed.restype = i32
+        L.hq_oracle_quantize_signed.argtypes = [p, i32, i64, i64, i32, i32, p, i32, p, p]
+        L.hq_oracle_quantize_signed.restype = i32
         L.hq_oracle_quantize_rotated.argtypes = [p, i64, i32, p, p]
         L.hq_oracle_quantize_rotated.restype = i32
         L.hq_oracle_fwht_block.argtypes = [p, i32]
@@ -121,15 +125,27 @@ def norm_const(k: int) -> np.float32:
     return np.float32(lib().hq_oracle_norm_const(k))
 
 
-def rotate(x: np.ndarray, dim: int, k: int) -> np.ndarray:
+def _neg_flags(neg, length: int):
+    if neg is None:
+        return None
+    f = np.ascontiguousarray(np.asarray(neg).astype(np.uint8) != 0, dtype=np.uint8)
+    if f.shape != (length,):
+        raise ValueError(f"sign flags must have one entry per position of the rotated dim ({length})")
+    return f
+
+
+def rotate(x: np.ndarray, dim: int, k: int, neg=None) -> np.ndarray:
     """y = blockdiag(H_k / sqrt(k)) applied along `dim` of x[rows][cols], in fp32.
 
     dim=1: along columns, result [rows][cols].  dim=0: along rows, result [cols][rows]
-    (rotated dimension innermost, i.e. K-major for the GEMM that contracts it)."""
+    (rotated dimension innermost, i.e. K-major for the GEMM that contracts it).
+    neg: optional flags, one per position of the rotated dim; a set flag negates that
+    position before the Hadamard blocks (randomized Hadamard: H_k D x)."""
     x, dt = _src(x)
     rows, cols = x.shape
+    f = _neg_flags(neg, cols if dim == 1 else rows)
     y = np.empty((rows, cols) if dim == 1 else (cols, rows), dtype=np.float32)
-    st = lib().hq_oracle_rotate(_ptr(x), dt, rows, cols, dim, k, _ptr(y))
+    st = lib().hq_oracle_rotate_signed(_ptr(x), dt, rows, cols, dim, k, None if f is None else _ptr(f), _ptr(y))
     if st != OK:
         raise OracleError(st, "rotate")
     return y
@@ -145,15 +161,18 @@ def quantize_rotated(y: np.ndarray, fmt: int):
     return codes, np.float32(scale[0])
 
 
-def quantize(x: np.ndarray, dim: int, k: int, fmt: int):
+def quantize(x: np.ndarray, dim: int, k: int, fmt: int, neg=None):
     """hq_quantize's definition: rotate along `dim`, tensor-wise absmax, RNE codes.
+    neg: optional sign flags of the randomized variant (see rotate).
 
     Returns (codes uint8 with the rotated dim innermost, fp32 scale)."""
     x, dt = _src(x)
     rows, cols = x.shape
+    f = _neg_flags(neg, cols if dim == 1 else rows)
     codes = np.empty((rows, cols) if dim == 1 else (cols, rows), dtype=np.uint8)
     scale = np.zeros(1, dtype=np.float32)
-    st = lib().hq_oracle_quantize(_ptr(x), dt, rows, cols, dim, k, fmt, _ptr(codes), _ptr(scale))
+    st = lib().hq_oracle_quantize_signed(_ptr(x), dt, rows, cols, dim, k, None if f is None else _ptr(f), fmt,
+                                         _ptr(codes), _ptr(scale))
     if st != OK:
         raise OracleError(st, "quantize")
     return codes, np.float32(scale[0])

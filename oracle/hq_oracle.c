@@ -142,12 +142,25 @@ static float load_elem(const void* src, int dtype, int64_t idx) {
     return bf16_bits_to_f32(((const uint16_t*)src)[idx]);
 }
 
+/* Randomized variant (a random sign diagonal D before the Hadamard blocks, t = H_k D x: the
+ * "randomized Hadamard transform" of the neighbouring pages' incoherence processing, e.g. the
+ * QuIP# abstract in the search listing).  neg[p] != 0 negates position p of the rotated
+ * dimension (one flag per position, shared by every block row/column); NULL = no signs.
+ * The negation is exact, so D only permutes signs before the same fp32 butterflies. */
+int hq_oracle_rotate_signed(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
+                            const uint8_t* neg, float* y);
+
 /* Rotate src[rows][cols] (dtype 0 = fp32, 1 = bf16) along `dim` in blocks of k and normalise.
  * dim = 1: along cols, y has shape [rows][cols].
  * dim = 0: along rows, y has shape [cols][rows] (the rotated dimension is made innermost).
  * Returns ORC_OK or an error code. */
 int hq_oracle_rotate(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
                      float* y) {
+    return hq_oracle_rotate_signed(src, dtype, rows, cols, dim, k, NULL, y);
+}
+
+int hq_oracle_rotate_signed(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
+                            const uint8_t* neg, float* y) {
     if (!valid_k(k) || (dtype != 0 && dtype != 1) || (dim != 0 && dim != 1)) return ORC_ERR_ARG;
     if (rows < 0 || cols < 0) return ORC_ERR_ARG;
     int64_t rot = dim == 1 ? cols : rows, other = dim == 1 ? rows : cols;
@@ -159,7 +172,8 @@ int hq_oracle_rotate(const void* src, int dtype, int64_t rows, int64_t cols, int
         for (int64_t b = 0; b < rot; b += k) {
             for (int i = 0; i < k; ++i) {
                 int64_t r = dim == 1 ? o : b + i, cc = dim == 1 ? b + i : o;
-                buf[i] = load_elem(src, dtype, r * cols + cc);
+                float v = load_elem(src, dtype, r * cols + cc);
+                buf[i] = (neg && neg[b + i]) ? -v : v;
             }
             hq_oracle_fwht_block(buf, k);
             for (int i = 0; i < k; ++i) y[o * rot + b + i] = buf[i] * c;
@@ -212,12 +226,21 @@ int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* code
 }
 
 /* Rotate then quantize (hq_quantize's definition).  codes has the rotated dim innermost. */
+int hq_oracle_quantize_signed(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
+                              const uint8_t* neg, int fmt, uint8_t* codes, float* scale);
+
 int hq_oracle_quantize(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
                        int fmt, uint8_t* codes, float* scale) {
+    return hq_oracle_quantize_signed(src, dtype, rows, cols, dim, k, NULL, fmt, codes, scale);
+}
+
+/* Randomized variant: the sign flags neg (see hq_oracle_rotate_signed), then the same. */
+int hq_oracle_quantize_signed(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,
+                              const uint8_t* neg, int fmt, uint8_t* codes, float* scale) {
     int64_t n = rows * cols;
     float* y = (float*)malloc((size_t)(n > 0 ? n : 1) * sizeof(float));
     if (!y) return ORC_ERR_ARG;
-    int st = hq_oracle_rotate(src, dtype, rows, cols, dim, k, y);
+    int st = hq_oracle_rotate_signed(src, dtype, rows, cols, dim, k, neg, y);
     if (st == ORC_OK) st = hq_oracle_quantize_rotated(y, n, fmt, codes, scale);
     free(y);
     return st;

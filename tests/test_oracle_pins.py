@@ -139,6 +139,74 @@ def test_product_preserved(oracle_lib, k):
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-5 * np.abs(want).max())
 
 
+# ------------------------------------------------------------- randomized Hadamard (H_k D)
+
+def _flags(n, seed):
+    return np.random.default_rng(seed).integers(0, 2, size=n).astype(np.uint8)
+
+
+@pytest.mark.parametrize("k", (16, 64, 256))
+def test_signed_rotation_equals_dense_h_times_d(oracle_lib, k):
+    """Integer inputs: the unnormalised signed rotation is exact, so rotate * sqrt(k) equals
+    the dense integer product (x * s) H_k block by block, with s = 1 - 2 * neg."""
+    x = _ints((3, 2 * k), 21, -8, 8)
+    neg = _flags(2 * k, 22)
+    s = 1 - 2 * neg.astype(np.int64)
+    H = scipy.linalg.hadamard(k).astype(np.int64)
+    xs = x.astype(np.int64) * s
+    want = np.concatenate([xs[:, :k] @ H, xs[:, k:] @ H], 1)
+    got = oracle.rotate(x, 1, k, neg=neg).astype(np.float64) / float(oracle.norm_const(k))
+    np.testing.assert_allclose(got, want, rtol=2 ** -22, atol=0)
+
+
+@pytest.mark.parametrize("k", (16, 128))
+def test_signed_rotation_plain_and_all_negated(oracle_lib, k):
+    """No flags is the plain rotation; flipping every position negates the result (H is
+    linear, negation exact); the strided rotation uses the flags of its own positions."""
+    x = synthetic.tiny_random((2 * k, 3 * k), 23)
+    np.testing.assert_array_equal(oracle.rotate(x, 1, k, neg=np.zeros(3 * k)), oracle.rotate(x, 1, k))
+    np.testing.assert_array_equal(oracle.rotate(x, 1, k, neg=np.ones(3 * k)), -oracle.rotate(x, 1, k))
+    neg = _flags(2 * k, 24)
+    np.testing.assert_array_equal(oracle.rotate(x, 0, k, neg=neg),
+                                  oracle.rotate(np.ascontiguousarray(x.T), 1, k, neg=neg))
+
+
+@pytest.mark.parametrize("k", (32, 256))
+def test_signed_product_preserved(oracle_lib, k):
+    """(X D H)(W D H)^T = X D D W^T = X W^T: exact for integer inputs (unnormalised,
+    k X W^T), to fp32 rounding otherwise; with different signs on the two operands it is not."""
+    neg = _flags(2 * k, 25)
+    s = (1 - 2 * neg.astype(np.int64))
+    X = _ints((6, 2 * k), 26, -4, 4)
+    W = _ints((5, 2 * k), 27, -4, 4)
+    def unnorm(A):
+        As = (A.astype(np.int64) * s).astype(np.float32)
+        return np.concatenate([np.stack([oracle.fwht_block(r[b:b + k]) for r in As])
+                               for b in range(0, A.shape[1], k)], 1)
+    np.testing.assert_array_equal(unnorm(X).astype(np.int64) @ unnorm(W).astype(np.int64).T,
+                                  k * (X.astype(np.int64) @ W.astype(np.int64).T))
+    Xf = synthetic.tiny_random((6, 2 * k), 28)
+    Wf = synthetic.tiny_random((5, 2 * k), 29)
+    got = oracle.rotate(Xf, 1, k, neg=neg).astype(np.float64) @ oracle.rotate(Wf, 1, k, neg=neg).astype(np.float64).T
+    want = Xf.astype(np.float64) @ Wf.astype(np.float64).T
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-5 * np.abs(want).max())
+    other = oracle.rotate(Wf, 1, k, neg=_flags(2 * k, 30)).astype(np.float64)
+    assert np.abs(oracle.rotate(Xf, 1, k, neg=neg).astype(np.float64) @ other.T - want).max() > 1e-2 * np.abs(want).max()
+
+
+def test_signed_quantize_matches_rotate_then_quantize(oracle_lib):
+    x = synthetic.tiny_random((64, 128), 31)
+    x[:, 5] *= 40.0
+    neg = _flags(128, 32)
+    for fmt in (oracle.INT8, oracle.FP8_E4M3):
+        codes, scale = oracle.quantize(x, 1, 64, fmt, neg=neg)
+        c2, s2 = oracle.quantize_rotated(oracle.rotate(x, 1, 64, neg=neg), fmt)
+        np.testing.assert_array_equal(codes, c2)
+        assert scale == s2
+    with pytest.raises(ValueError):
+        oracle.quantize(x, 1, 64, oracle.INT8, neg=np.zeros(64))
+
+
 def test_rotate_rejects_bad_shapes(oracle_lib):
     with pytest.raises(oracle.OracleError):
         oracle.rotate(np.zeros((3, 24), np.float32), 1, 16)
