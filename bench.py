@@ -276,29 +276,35 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(device)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    # The step, as pre-marshalled C-ABI calls in the schedule hq_linear_fwd_bwd uses: the
-    # forward operands and GEMM on the main stream, the four rotations only the backward
-    # GEMMs need on a side stream alongside them, joined by events.  CUDA events on each
-    # stream time every group of launches.
+    # The step, as pre-marshalled C-ABI calls in the schedule hq_linear_fwd_bwd uses: X and W
+    # quantized in both rotations and the forward GEMM on the main stream, dY in both
+    # rotations on a side stream alongside them, joined by an event before the backward
+    # GEMMs.  CUDA events on each stream time every group of launches.
     L_ = hq.lib()
     side = torch.cuda.Stream(device)
     sh, sh2 = stream.cuda_stream, side.cuda_stream
     sp = lambda i: scales[i:i + 1].data_ptr()  # noqa: E731
-    part = torch.empty(2 * hq.hq_quantize_workspace_bytes(), dtype=torch.uint8, device=device)
-    pw = hq.hq_quantize_workspace_bytes()
+    pw = hq.hq_quantize_dual_workspace_bytes()
+    part = torch.empty(2 * pw, dtype=torch.uint8, device=device)
     ws_main, ws_side = part.data_ptr(), part.data_ptr() + pw
 
-    def quant(src, dim, codes, si, ws, st):
-        return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt, codes.data_ptr(),
-                sp(si), ws, pw, st)
+    def dual(src, codes_c, si_c, codes_r, si_r, ws, st):
+        return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], k, fmt, codes_c.data_ptr(), sp(si_c),
+                codes_r.data_ptr(), sp(si_r), ws, pw, st)
 
     def gemm(a, ai, b, bi, out):
         return (a.data_ptr(), sp(ai), b.data_ptr(), sp(bi), a.shape[0], b.shape[0], a.shape[1], fmt,
                 hq.HQ_OUT_BF16, out.data_ptr(), sh)
 
-    q_main = [quant(X, 1, qX_K, 0, ws_main, sh), quant(W, 1, qW_K, 2, ws_main, sh)]
-    q_side_dx = [quant(W, 0, qW_N, 3, ws_side, sh2), quant(dY, 1, qdY_N, 4, ws_side, sh2)]
-    q_side_dw = [quant(X, 0, qX_M, 1, ws_side, sh2), quant(dY, 0, qdY_M, 5, ws_side, sh2)]
+    pq = hq.hq_quantize_workspace_bytes()
+
+    def single(src, dim, codes, si, ws, st):
+        return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt, codes.data_ptr(), sp(si),
+                ws, pq, st)
+
+    q_main = [single(X, 1, qX_K, 0, ws_main, sh), single(W, 1, qW_K, 2, ws_main, sh)]
+    q_side_dual = [dual(dY, qdY_N, 4, qdY_M, 5, ws_side, sh2)]
+    q_side = [single(W, 0, qW_N, 3, ws_side, sh2), single(X, 0, qX_M, 1, ws_side, sh2)]
     g_fwd, g_dx, g_dw = gemm(qX_K, 0, qW_K, 2, Y), gemm(qdY_N, 4, qW_N, 3, dX), gemm(qdY_M, 5, qX_M, 1, dW)
 
     def run(calls, fn, what):
@@ -313,27 +319,23 @@ def run_gpu(args):
         fork.record(stream)
         side.wait_event(fork)
         rec(ev_side, 0, side)
-        run(q_side_dx, L_.hq_quantize, "hq_quantize")
-        rec(ev_side, 2, side)
-        j_dx = torch.cuda.Event()
-        j_dx.record(side)
-        run(q_side_dw, L_.hq_quantize, "hq_quantize")
+        run(q_side_dual, L_.hq_quantize_dual, "hq_quantize_dual")
         rec(ev_side, 1, side)
-        j_dw = torch.cuda.Event()
-        j_dw.record(side)
+        run(q_side, L_.hq_quantize, "hq_quantize")
+        rec(ev_side, 2, side)
+        join = torch.cuda.Event()
+        join.record(side)
         rec(ev_main, 0, stream)
         run(q_main, L_.hq_quantize, "hq_quantize")
         rec(ev_main, 1, stream)
         run([g_fwd], L_.hq_gemm, "hq_gemm")
         rec(ev_main, 2, stream)
-        stream.wait_event(j_dx)
+        stream.wait_event(join)
         rec(ev_main, 3, stream)
         run([g_dx], L_.hq_gemm, "hq_gemm")
         rec(ev_main, 4, stream)
-        stream.wait_event(j_dw)
-        rec(ev_main, 5, stream)
         run([g_dw], L_.hq_gemm, "hq_gemm")
-        rec(ev_main, 6, stream)
+        rec(ev_main, 5, stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -343,7 +345,7 @@ def run_gpu(args):
         raise SystemExit("device status error during warm-up")
 
     # ---------------------------------------------------------------- timed region (device)
-    ev_main = [[ev() for _ in range(7)] for _ in range(args.steps)]
+    ev_main = [[ev() for _ in range(6)] for _ in range(args.steps)]
     ev_side = [[ev() for _ in range(3)] for _ in range(args.steps)]
     barrier(world, device)
     torch.cuda.synchronize(device)
@@ -355,44 +357,54 @@ def run_gpu(args):
     barrier(world, device)
     torch.cuda.synchronize(device)
     status = hq.hq_get_error(stream)
-    step_ms_local = sum(e[0].elapsed_time(e[6]) for e in ev_main) / args.steps
-    gemm_ms = sum(e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) + e[5].elapsed_time(e[6]) for e in ev_main)
-    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev_main) + sum(e[0].elapsed_time(e[1]) for e in ev_side)
+    step_ms_local = sum(e[0].elapsed_time(e[5]) for e in ev_main) / args.steps
+    gemm_ms = sum(e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[5]) for e in ev_main)
+    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev_main) + sum(e[0].elapsed_time(e[2]) for e in ev_side)
     def mean_ms(pairs):
         return sum(a.elapsed_time(b) for a, b in pairs) / args.steps
     phases = {
         "main_quant_fwd_operands": mean_ms((e[0], e[1]) for e in ev_main),
         "gemm_fwd": mean_ms((e[1], e[2]) for e in ev_main),
-        "wait_side_dx": mean_ms((e[2], e[3]) for e in ev_main),
+        "wait_side_dy": mean_ms((e[2], e[3]) for e in ev_main),
         "gemm_dx": mean_ms((e[3], e[4]) for e in ev_main),
-        "wait_side_dw": mean_ms((e[4], e[5]) for e in ev_main),
-        "gemm_dw": mean_ms((e[5], e[6]) for e in ev_main),
-        "side_quant_dx_operands": mean_ms((e[0], e[2]) for e in ev_side),
-        "side_quant_dw_operands": mean_ms((e[2], e[1]) for e in ev_side),
+        "gemm_dw": mean_ms((e[4], e[5]) for e in ev_main),
+        "side_quant_dy_both_rotations": mean_ms((e[0], e[1]) for e in ev_side),
+        "side_quant_w_n_x_m": mean_ms((e[1], e[2]) for e in ev_side),
     }
     step_ms = reduce_max(step_ms_local, world, device)
     gemm_ms_launch = reduce_max(gemm_ms / (3 * args.steps), world, device)
     quant_ms_step = reduce_max(quant_ms / args.steps, world, device)
-    launches = 15 * args.steps  # per step: 6 quantizations x 2 kernels + 3 GEMMs
+    launches = 13 * args.steps  # per step: 5 quantization calls x 2 kernels + 3 GEMMs
 
     # ---------------------------------------------------------------- quantizer alone
-    # The six rotations one after another on one stream (nothing overlapping), L2 flushed
-    # before each, to report the quantization kernels' own throughput.
-    alone_ms = 0.0
-    reps = max(3, min(args.steps, 10))
-    for _ in range(reps):
-        for c in q_main + [quant(*(src_args[:4]), ws_main, sh) for src_args in
-                           ((W, 0, qW_N, 3), (dY, 1, qdY_N, 4), (X, 0, qX_M, 1), (dY, 0, qdY_M, 5))]:
+    # The three two-rotation quantizations one after another on one stream (nothing
+    # overlapping), L2 flushed before each, to report the quantization kernels' own throughput;
+    # and, for comparison, the six rotations as single-rotation calls (two reads each).
+    def alone(calls, fn, what):
+        tot = 0.0
+        for c in calls:
             flush.zero_()
             a, b = ev(), ev()
             a.record(stream)
-            st = L_.hq_quantize(*c)
+            st = fn(*c)
             if st:
-                raise hq.HQError(st, "hq_quantize")
+                raise hq.HQError(st, what)
             b.record(stream)
             torch.cuda.synchronize(device)
-            alone_ms += a.elapsed_time(b)
+            tot += a.elapsed_time(b)
+        return tot
+
+    reps = max(3, min(args.steps, 10))
+    single = [(src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt, codes.data_ptr(), sp(si),
+               ws_main, pq, sh)
+              for src, dim, codes, si in ((X, 1, qX_K, 0), (X, 0, qX_M, 1), (W, 1, qW_K, 2), (W, 0, qW_N, 3),
+                                          (dY, 1, qdY_N, 4), (dY, 0, qdY_M, 5))]
+    dual_calls = [dual(X, qX_K, 0, qX_M, 1, ws_main, sh), dual(W, qW_K, 2, qW_N, 3, ws_main, sh),
+                  dual(dY, qdY_N, 4, qdY_M, 5, ws_main, sh)]
+    alone_ms = sum(alone(dual_calls, L_.hq_quantize_dual, "hq_quantize_dual") for _ in range(reps))
     alone_ms_step = reduce_max(alone_ms / reps, world, device)
+    single_ms = sum(alone(single, L_.hq_quantize, "hq_quantize") for _ in range(reps))
+    single_ms_step = reduce_max(single_ms / reps, world, device)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     # Every step copies X, W, dY from pinned host memory, runs hq_linear_fwd_bwd and copies Y,
@@ -475,10 +487,13 @@ def run_gpu(args):
                        "frac": quant_bytes / (alone_ms_step * 1e-3) / 1e9 / peaks["hbm"],
                        "bytes_per_step": quant_bytes, "ms_per_step": alone_ms_step,
                        "in_step_gbs": quant_gbs, "in_step_ms": quant_ms_step,
-                       "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each); achieved: the six rotations timed alone with CUDA events, L2 flushed before each; in_step: summed event time of the same launches inside the overlapped step (sharing the GPU with the GEMMs)"},
+                       "kernel": "fwhtq_dual_kernel (both rotations of X, W, dY from one read per pass)",
+                       "single_rotation_gbs": quant_bytes / (single_ms_step * 1e-3) / 1e9,
+                       "single_rotation_ms": single_ms_step,
+                       "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each); achieved: the three two-rotation quantizations timed alone with CUDA events, L2 flushed before each; in_step: summed event time of the same launches inside the overlapped step (sharing the GPU with the GEMMs); single_rotation: the six rotations as one-rotation calls"},
         "phases_ms": phases,
         "gemm_ms_per_step": gemm_ms_launch * 3,
-        "schedule": "forward operands + GEMM on the main stream; the other four rotations on a side stream overlapping them",
+        "schedule": "X and W along K + forward GEMM on the main stream; dY in both rotations (one read per pass), W along N and X along M on a side stream overlapping them",
         "frac_of_int8_peak_end_to_end": value / world / int8_peak,
         "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": elem * (M * K + N * K + M * N),
@@ -551,12 +566,13 @@ def run_sweep(args):
                 step_ms = timed(lambda: hq.hq_linear_fwd_bwd(X, W, dY, k, fmt, Y=Y, dX=dX, dW=dW, workspace=ws))
                 codes = {}
                 quant_ms = 0.0
-                for name, src, dim in (("XK", X, 1), ("XM", X, 0), ("WK", W, 1), ("WN", W, 0), ("DN", dY, 1), ("DM", dY, 0)):
-                    c_out = torch.empty((src.shape[0], src.shape[1]) if dim == 1 else (src.shape[1], src.shape[0]),
-                                        dtype=torch.uint8, device=dev)
-                    sc = torch.empty(1, dtype=torch.float32, device=dev)
-                    quant_ms += timed(lambda: hq.hq_quantize(src, dim, k, fmt, codes=c_out, scale=sc))
-                    codes[name] = (c_out, sc)
+                for (nc, nr), src in ((("XK", "XM"), X), (("WK", "WN"), W), (("DN", "DM"), dY)):
+                    cc = torch.empty(src.shape[0], src.shape[1], dtype=torch.uint8, device=dev)
+                    cr = torch.empty(src.shape[1], src.shape[0], dtype=torch.uint8, device=dev)
+                    sc, sr = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2))
+                    quant_ms += timed(lambda: hq.hq_quantize_dual(src, k, fmt, codes_c=cc, scale_c=sc,
+                                                                  codes_r=cr, scale_r=sr))
+                    codes[nc], codes[nr] = (cc, sc), (cr, sr)
                 gemm_ms = 0.0
                 for a, b, o in (("XK", "WK", Y), ("DN", "WN", dX), ("DM", "XM", dW)):
                     (ca, sa), (cb, sb) = codes[a], codes[b]
@@ -602,6 +618,10 @@ def run_kernel_case(args):
         out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         for _ in range(2):
             hq.hq_gemm(A, s, B, s, fmt, out=out)
+    elif case == "quant_dual":
+        x = torch.randn(11008, 4096, generator=g, device="cuda").to(torch.bfloat16)
+        for _ in range(2):
+            hq.hq_quantize_dual(x, 256, "int8")
     else:
         rows, cols, dim = (11008, 4096, 1) if case == "quant_rows" else (11008, 4096, 0)
         x = torch.randn(rows, cols, generator=g, device="cuda").to(torch.bfloat16)
@@ -619,7 +639,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
-    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols"),
+    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload (one JSON line per workload/layer/format/k) and exit")

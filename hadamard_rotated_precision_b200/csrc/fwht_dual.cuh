@@ -1,0 +1,395 @@
+// Both rotations of one bf16 matrix from a single read per pass: the block-Hadamard rotation
+// along the columns (codes [rows][cols]) and along the rows (codes written transposed,
+// [cols][rows]), each with its own tensor-wise absmax scale.
+//
+// Method: "Training Transformers with 4-bit Integers", section 3.3 (block-diagonal Hadamard
+// rotation before quantization) and "HALO: Hadamard-Assisted Lower-Precision Optimization
+// for LLMs" (Approach: every operand of the three linear-layer GEMMs is rotated along that
+// GEMM's contraction dimension, so X, W and dY are each needed in two rotations; quantized
+// rotated tensors are stored and reused).  The arithmetic is the same as in fwht_quant.cuh
+// (Sylvester FWHT, index bit 0 first, fp32 round-to-nearest-even adds, normalisation by
+// fp32(1/sqrt(k)), tensor-wise absmax, INT8 / e4m3 codes), so the codes are bit-identical to
+// the single-rotation kernels'.
+//
+// Data movement: the tensor is cut into 256 x 256 tiles (a tile holds whole k-blocks in both
+// directions for every k <= 256).  TMA streams each tile into shared memory as four 32 KB
+// strips of 64 columns x 256 rows, through a 7-strip ring.  Eight warps read every strip
+// twice from shared memory; the warp that is the last to finish with a strip issues the copy
+// that refills its slot:
+//   row role  (rotation along the columns): a thread takes 64 consecutive columns of one row
+//             (one strip row), so in-block index bits 0..5 are register bits and bits 6, 7
+//             are the strip, i.e. lane bits 3, 4;
+//   col role  (rotation along the rows): four ldmatrix.trans x4 gathers per 32 rows give a
+//             thread 64 consecutive rows of one column (bits 0..5 in registers, bits 6, 7 in
+//             lane bits 0, 1).
+// Pass 1 reduces both rotations' absmax into one partial per CTA and role; pass 2 reduces
+// the partials, rotates again and writes both code tensors.  HBM traffic per element and
+// pass is one 2-byte read (plus two 1-byte code writes in pass 2), against two reads when
+// each rotation runs on its own.
+//
+// Shared-memory layout of a strip: the copy is a 3-D box over the view (col, a, b) of the
+// tensor with row = 64a + b, dims ordered (col, a, b), so strip row rho = 4b + a holds tile
+// row 64a + b.  With the 128-byte swizzle (16-byte chunk index XOR rho & 7) the eight rows
+// one ldmatrix matrix reads (a = 0..3, b even/odd) and the eight rows one quarter-warp of
+// the row role reads are in distinct chunks: both gathers are bank-conflict-free.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "fwht_quant.cuh"
+#include "sm100_ptx.cuh"
+
+namespace hq {
+namespace dual {
+
+// Eight warps at up to 255 registers each (no spills, 64 values per thread in flight) measured
+// as fast as sixteen at 128 for k = 256 and faster for smaller k.  The step code also handles
+// sixteen warps (two row steps and two column steps per warp and tile).
+constexpr int kComputeWarps = 8;
+static_assert(kComputeWarps == 8 || kComputeWarps == 16, "8 or 16 warps");
+constexpr int kSteps = 32 / kComputeWarps;    // row steps and column steps per warp and tile
+constexpr int kThreads = 32 * kComputeWarps;
+constexpr int kTile = 256;                          // rows and columns of a tile
+constexpr int kStripCols = 64;                      // 128 bytes of bf16 per strip row
+constexpr int kStripsPerTile = kTile / kStripCols;  // 4
+constexpr uint32_t kStripBytes = uint32_t(kTile) * kStripCols * 2;  // 32 KB
+constexpr int kSlots = 7;                                           // strips in the ring
+constexpr size_t kSmemBytes = 1024 + size_t(kSlots) * kStripBytes + kSlots * 8;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+// Bounded wait: false once another warp raised the abort flag or after kWaitLimitNs (which
+// raises the flag and records HQ_ERR_TIMEOUT).
+__device__ __forceinline__ bool wait_full(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicCAS(status, 0u, 6u /* HQ_ERR_TIMEOUT */);
+      return false;
+    }
+  }
+}
+
+// max(m, fl(|a| + |b|), fl(|c| + |d|)), NaN-propagating.  For a butterfly pair (u, v) the two
+// outputs satisfy max(|fl(u + v)|, |fl(u - v)|) = fl(|u| + |v|) (one of them is the sum of the
+// magnitudes, the other the difference, and rounding is monotone and sign-symmetric), so the
+// absmax pass never forms the last stage's outputs.
+__device__ __forceinline__ float max_abs_sums(float m, float a, float b, float c, float d) {
+  return absmax3(m, __fadd_rn(fabsf(a), fabsf(b)), __fadd_rn(fabsf(c), fabsf(d)));
+}
+
+// Running maxima of the absmax pass: eight independent chains, so consecutive max
+// instructions do not wait on each other.
+constexpr int kAcc = 8;
+
+// Rotation of a thread's 64 values (v[i] = positions 2i, 2i+1 of bits 0..5) for block size K:
+// register stages for bits 0..min(log2 K, 6) - 1, then the lane stages (bit 6: lane xor m6,
+// bit 7: lane xor m7).  ABSMAX: the last stage is folded into the running maxima `am` of the
+// unnormalised |t| instead (v is left partly rotated); otherwise v ends fully rotated.
+template <int K, bool ABSMAX>
+__device__ __forceinline__ void rotate64(float2 (&v)[32], int lane, int m6, int m7, float (&am)[kAcc]) {
+  if constexpr (K <= 64) {
+    if constexpr (ABSMAX) {
+      stages_low<K / 2, 32>(v);
+      constexpr int h2 = K / 4;  // float2 distance of the last stage's pairs
+      int n = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (i & h2) continue;
+        am[n % kAcc] = max_abs_sums(am[n % kAcc], v[i].x, v[i + h2].x, v[i].y, v[i + h2].y);
+        ++n;
+      }
+    } else {
+      stages_low<K, 32>(v);
+    }
+  } else {
+    stages_low<64, 32>(v);
+    if constexpr (K == 256) stage_lanes<32>(v, m6, lane);
+    const int ml = K == 256 ? m7 : m6;
+    if constexpr (ABSMAX) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float px = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, ml);
+        const float py = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, ml);
+        am[i % kAcc] = max_abs_sums(am[i % kAcc], v[i].x, px, v[i].y, py);
+      }
+    } else {
+      stage_lanes<32>(v, ml, lane);
+    }
+  }
+}
+
+// Scaling of a rotated value t to the code grid.  The definition is z = fp32(fp32(t * c) * inv).
+// When c = 1/sqrt(k) is a power of two (k = 16, 64, 256) and inv <= 2^100 this equals
+// fp32(t * ci) with ci = c * inv (exact): if t * c is a normal number it is exact, so one
+// rounding of t * c * inv remains either way; otherwise |z| <= 2^-126 * 2^100 under both forms,
+// which is the zero code for INT8 and e4m3 alike (with the sign of t).
+struct CodeScale {
+  float2 c2, inv2, ci2;
+  bool one_mul;
+};
+
+template <int K>
+__device__ __forceinline__ CodeScale code_scale(float c, float inv) {
+  CodeScale s;
+  s.c2 = make_float2(c, c);
+  s.inv2 = make_float2(inv, inv);
+  const float ci = __fmul_rn(c, inv);
+  s.ci2 = make_float2(ci, ci);
+  s.one_mul = (K == 16 || K == 64 || K == 256) && inv <= 0x1p100f;
+  return s;
+}
+
+__device__ __forceinline__ void st_global_32B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                              uint32_t f, uint32_t g, uint32_t h) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d),
+               "r"(e), "r"(f), "r"(g), "r"(h)
+               : "memory");
+}
+
+// Codes of a thread's 64 rotated values, 64 contiguous bytes at dst (W32: two 32-byte stores,
+// each a whole sector; dst 32-byte aligned).
+template <int MODE, bool W32>
+__device__ __forceinline__ void store_codes64(uint8_t* dst, const float2 (&v)[32], const CodeScale& cs, bool zero) {
+  uint32_t w[16];
+  if (cs.one_mul) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = codes4<MODE>(mul2(v[2 * j], cs.ci2), mul2(v[2 * j + 1], cs.ci2));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      w[j] = codes4<MODE>(mul2(mul2(v[2 * j], cs.c2), cs.inv2), mul2(mul2(v[2 * j + 1], cs.c2), cs.inv2));
+  }
+  if (zero) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = 0u;
+  }
+  if constexpr (W32) {
+    st_global_32B(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_32B(dst + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float2& f) {
+  f = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+template <int K, int MODE, bool W32>
+__global__ void __launch_bounds__(kThreads, 1)
+fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
+                  uint8_t* __restrict__ codes_c, uint8_t* __restrict__ codes_r,
+                  float* __restrict__ part_c, float* __restrict__ part_r, int n_partials,
+                  float* __restrict__ scale_c, float* __restrict__ scale_r,
+                  unsigned int* __restrict__ status, int reverse) {
+  static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  constexpr bool QUANT = MODE != kModeAbsmax;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ float scratch[32];
+  __shared__ float red[2 * kComputeWarps];
+  __shared__ int abort_flag;
+  __shared__ unsigned int released[kSlots];  // warps done with the slot, over all rounds
+  __shared__ int issued_round[kSlots];       // round of the slot's latest copy (-1: none)
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(base);
+  const uint32_t bars = sbase + kSlots * kStripBytes;  // full[kSlots]
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int64_t n_ct = (cols + kTile - 1) / kTile;
+  const int64_t n_tiles = ((rows + kTile - 1) / kTile) * n_ct;
+  const int64_t G = gridDim.x, b = blockIdx.x;
+  const int64_t my_tiles = b < n_tiles ? (n_tiles - 1 - b) / G + 1 : 0;
+  const int64_t n_strips = my_tiles * kStripsPerTile;
+  // alternate passes walk the tiles in opposite orders, so each starts on what the previous
+  // one left in L2
+  auto tile_of = [&](int64_t i) { return reverse ? b + G * (my_tiles - 1 - i) : b + G * i; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      released[s] = 0u;
+      issued_round[s] = -1;
+    }
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto issue = [&](int64_t q) {
+    const int64_t t = tile_of(q / kStripsPerTile);
+    const int s = static_cast<int>(q % kStripsPerTile);
+    const int slot = static_cast<int>(q % kSlots);
+    issued_round[slot] = static_cast<int>(q / kSlots);
+    ptx::mbar_arrive_expect_tx(full_bar(slot), kStripBytes);
+    ptx::tma_load_3d(sbase + slot * kStripBytes, &map, static_cast<int32_t>(kStripCols * (kStripsPerTile * (t % n_ct) + s)),
+                     static_cast<int32_t>(4 * (t / n_ct)), 0, full_bar(slot));
+  };
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&map);
+    for (int64_t q = 0; q < (n_strips < kSlots ? n_strips : kSlots); ++q) issue(q);
+  }
+  // A warp is done with strip q: the sixteenth warp to say so for this round of the slot
+  // refills it with strip q + kSlots.  Each warp's reads of the strip are ordered before its
+  // count (syncwarp, then a CTA fence), and the counting warp's fence orders all of them
+  // before its copy is issued.
+  auto release = [&](int64_t q) {
+    __syncwarp();
+    if (lane == 0) {
+      const int slot = static_cast<int>(q % kSlots);
+      __threadfence_block();
+      const unsigned int done = atomicAdd(&released[slot], 1u) + 1u;
+      if (done == static_cast<unsigned int>(kComputeWarps) * static_cast<unsigned int>(q / kSlots + 1)) {
+        __threadfence_block();
+        ptx::fence_proxy_async_smem();
+        if (q + kSlots < n_strips && !abort_flag) issue(q + kSlots);
+      }
+    }
+  };
+
+  const float c = __frsqrt_rn(static_cast<float>(K));
+  QuantParams qc{0.0f, false, false}, qr{0.0f, false, false};
+  if constexpr (QUANT) {
+    qc = finish_absmax<MODE>(part_c, n_partials, scale_c, scratch, status);
+    qr = finish_absmax<MODE>(part_r, n_partials, scale_r, scratch, status);
+  }
+  const int64_t work_tiles = (qc.abort && qr.abort) ? 0 : my_tiles;
+
+  const CodeScale csc = code_scale<K>(c, qc.inv), csr = code_scale<K>(c, qr.inv);
+  float amc[kAcc], amr[kAcc];
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) amc[j] = amr[j] = 0.0f;
+
+  // row role lane constants: strip sr = lane >> 3, row selector x = lane & 7
+  const int x = lane & 7, sr = lane >> 3;
+  const uint32_t swr = 4u * (x & 1) + (x >> 1);
+  // col role: the tile's 32 (strip, 8-column chunk) pairs p = warp + kComputeWarps * j go to
+  // strip p >> 3, chunk p & 7 (the chunk is warp & 7 for every j); lane constants: matrix row
+  // i = lane & 7 (same swizzle), matrix mm = lane >> 3
+  const int grp = warp >> 3;
+  const uint32_t col_lane_off = (8u * (lane >> 3) + swr) * 128u + ((static_cast<uint32_t>(warp & 7) ^ swr) << 4);
+
+  for (int64_t i = 0; i < work_tiles; ++i) {
+    const int64_t t = tile_of(i);
+    const int64_t row0 = (t / n_ct) * kTile, col0 = (t % n_ct) * kTile;
+    const int64_t q0 = i * kStripsPerTile;
+    const int slot0 = static_cast<int>(q0 % kSlots);
+    auto slot_of = [&](int s) { return slot0 + s < kSlots ? slot0 + s : slot0 + s - kSlots; };
+    bool ok = true;
+#pragma unroll
+    for (int s = 0; s < kStripsPerTile; ++s) {
+      const int64_t q = q0 + s;
+      ok = ok && wait_full(full_bar(slot_of(s)), static_cast<uint32_t>((q / kSlots) & 1), &abort_flag, status);
+    }
+    if (!ok) break;
+
+    // ---- row role: rotation along the columns, kSteps steps of 8 rows x 256 columns per warp
+    const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+#pragma unroll 1
+    for (int st = 0; st < kSteps; ++st) {
+      const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
+      const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+      float2 v[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+        unpack_bf16x2(raw.x, v[4 * j]);
+        unpack_bf16x2(raw.y, v[4 * j + 1]);
+        unpack_bf16x2(raw.z, v[4 * j + 2]);
+        unpack_bf16x2(raw.w, v[4 * j + 3]);
+      }
+      if (kSteps == 2 && st == 1) {
+        // this warp's last reads of the two strips it has no column step on (with 16 warps a
+        // warp's column steps cover strips grp and grp + 2; with 8 warps all four)
+        release(q0 + 1 - grp);
+        release(q0 + 3 - grp);
+      }
+      if constexpr (!QUANT) {
+        rotate64<K, true>(v, lane, 8, 16, amc);
+      } else {
+        rotate64<K, false>(v, lane, 8, 16, amc);
+        const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
+        const int64_t cc = col0 + kStripCols * sr;
+        if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero);
+      }
+    }
+
+    // ---- col role: rotation along the rows, 8 columns of one strip per step
+#pragma unroll 1
+    for (int j2 = 0; j2 < kSteps; ++j2) {
+      const int s = grp + (kComputeWarps / 8) * j2;
+      const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+      float2 v[32];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        uint32_t r4[4];
+        ldmatrix_x4_trans(lbase + 4096u * n, r4);
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) unpack_bf16x2(r4[mm], v[4 * n + mm]);
+      }
+      release(q0 + s);
+      if constexpr (!QUANT) {
+        rotate64<K, true>(v, lane, 1, 2, amr);
+      } else {
+        rotate64<K, false>(v, lane, 1, 2, amr);
+        const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
+        const int64_t gr = row0 + 64 * (lane & 3);
+        if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero);
+      }
+    }
+  }
+
+  // every copy issued has landed before the CTA exits (all are consumed above unless a wait
+  // gave up or both rotations were abandoned)
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      if (issued_round[s] < 0) continue;
+      const uint32_t par = static_cast<uint32_t>(issued_round[s] & 1);
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!ptx::mbar_try_wait(full_bar(s), par)) {
+        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicCAS(status, 0u, 6u);
+          break;
+        }
+      }
+    }
+  }
+  if constexpr (!QUANT) {
+    float mc = amc[0], mr = amr[0];
+#pragma unroll
+    for (int j = 1; j < kAcc; ++j) {
+      mc = absmax3(mc, amc[j], 0.0f);
+      mr = absmax3(mr, amr[j], 0.0f);
+    }
+    mc = mc != mc ? INFINITY : mc;
+    mr = mr != mr ? INFINITY : mr;
+    mc = warp_max(mc);
+    mr = warp_max(mr);
+    if (lane == 0) {
+      red[warp] = mc;
+      red[kComputeWarps + warp] = mr;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < kComputeWarps; ++w) {
+        mc = fmaxf(mc, red[w]);
+        mr = fmaxf(mr, red[kComputeWarps + w]);
+      }
+      mc = fmaxf(mc, red[0]);
+      mr = fmaxf(mr, red[kComputeWarps]);
+      part_c[b] = __fmul_rn(mc, c);
+      part_r[b] = __fmul_rn(mr, c);
+    }
+  }
+}
+
+}  // namespace dual
+}  // namespace hq

@@ -11,6 +11,7 @@
 
 #include "hq.h"
 #include "fwht_quant.cuh"
+#include "fwht_dual.cuh"
 #include "gemm_tcgen05.cuh"
 
 namespace {
@@ -34,6 +35,7 @@ struct DeviceInfo {
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
   unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
+  unsigned dual_attr_set = 0;  // bit per fused two-rotation quantizer instantiation
 };
 
 std::mutex g_mu;
@@ -216,6 +218,94 @@ cudaError_t launch_dual(const void* src_v, int64_t rows, int64_t cols, hq_fmt fm
     if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, d, st, &g);
   }
   return e;
+}
+
+// Both rotations of a bf16 tensor from one read per pass (fwht_dual.cuh).  The tensor is
+// described to TMA as the 3-D view (col, a, b) with row = 64a + b, so it needs rows and
+// cols to be multiples of 64; the caller falls back to launch_dual otherwise.
+bool fused_dual_ok(int64_t rows, int64_t cols) {
+  return rows % 64 == 0 && cols % 64 == 0 && rows / 64 < (int64_t(1) << 31) && cols < (int64_t(1) << 31);
+}
+
+hq_status encode_dual_map(CUtensorMap* map, const void* src, int64_t rows, int64_t cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  hq_status s = tensor_map_encoder(&enc);
+  if (s != HQ_OK) return s;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows / 64), 64};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(64 * cols * 2), static_cast<cuuint64_t>(cols * 2)};
+  const cuuint32_t box[3] = {hq::dual::kStripCols, 4, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(src), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return HQ_OK;
+}
+
+template <int K, int MODE, bool W32>
+cudaError_t dual_smem_attr(DeviceInfo& d) {
+  constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
+  const unsigned bit = 1u << ((kIdx * 3 + MODE) * 2 + (W32 ? 1 : 0));
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (d.dual_attr_set & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(hq::dual::fwhtq_dual_kernel<K, MODE, W32>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(hq::dual::kSmemBytes));
+  if (e == cudaSuccess) d.dual_attr_set |= bit;
+  return e;
+}
+
+// Pass 1 (both absmax partials, tiles in order) then pass 2 (both code tensors, tiles in
+// reverse order), one CTA per SM.  W32: both code buffers are 32-byte aligned, so the code
+// stores are whole 32-byte sectors.
+template <int K, bool W32>
+hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
+                              float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
+                              DeviceInfo& d, cudaStream_t st) {
+  using namespace hq;
+  using namespace hq::dual;
+  const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+  const int g = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(n_tiles, d.sms)));
+  cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32>(d);
+  if (e != cudaSuccess) return cuda_fail(e);
+  fwhtq_dual_kernel<K, kModeAbsmax, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
+                                                                           part_r, 0, scale_c, scale_r, d.status, 0);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  if (fmt == HQ_INT8) {
+    if ((e = dual_smem_attr<K, kModeInt8, W32>(d)) != cudaSuccess) return cuda_fail(e);
+    fwhtq_dual_kernel<K, kModeInt8, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
+                                                                           part_r, g, scale_c, scale_r, d.status, 1);
+  } else {
+    if ((e = dual_smem_attr<K, kModeFp8, W32>(d)) != cudaSuccess) return cuda_fail(e);
+    fwhtq_dual_kernel<K, kModeFp8, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
+                                                                          part_r, g, scale_c, scale_r, d.status, 1);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  return HQ_OK;
+}
+
+template <int K>
+hq_status launch_dual_fused(const CUtensorMap& map, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
+                            float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
+                            DeviceInfo& d, cudaStream_t st) {
+  const bool w32 = ((reinterpret_cast<uintptr_t>(codes_c) | reinterpret_cast<uintptr_t>(codes_r)) & 31u) == 0;
+  return w32 ? launch_dual_fused_w<K, true>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st)
+             : launch_dual_fused_w<K, false>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+}
+
+hq_status launch_dual_fused_k(const void* src, int64_t rows, int64_t cols, int k, hq_fmt fmt, uint8_t* codes_c,
+                              float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
+                              DeviceInfo& d, cudaStream_t st) {
+  CUtensorMap map;
+  hq_status s = encode_dual_map(&map, src, rows, cols);
+  if (s != HQ_OK) return s;
+  switch (k) {
+    case 16: return launch_dual_fused<16>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 32: return launch_dual_fused<32>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 64: return launch_dual_fused<64>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 128: return launch_dual_fused<128>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    default: return launch_dual_fused<256>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+  }
 }
 
 template <typename SrcT>
@@ -643,6 +733,8 @@ hq_status dual_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, in
   }
   uint8_t* cc = static_cast<uint8_t*>(codes_c);
   uint8_t* cr = static_cast<uint8_t*>(codes_r);
+  if (dt == HQ_BF16 && fused_dual_ok(rows, cols))
+    return launch_dual_fused_k(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st);
   cudaError_t e = dt == HQ_BF16
                       ? launch_dual_k<__nv_bfloat16>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st)
                       : launch_dual_k<float>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st);
@@ -677,11 +769,13 @@ hq_status side_stream(SideStream** out) {
   return HQ_OK;
 }
 
-// Workspace of hq_linear_fwd_bwd: six code tensors, six scales, two partial buffers.
+// Workspace of hq_linear_fwd_bwd: six code tensors, six scales, four partial buffers (one
+// pair per stream).
 struct StepWs {
   uint8_t *xq, *xqt, *wq, *wqt, *dyq, *dyqt;
   float* scales;  // x_c, x_r, w_c, w_r, dy_c, dy_r
-  float *part_c, *part_r;
+  float *part_c, *part_r;    // caller's stream
+  float *spart_c, *spart_r;  // side stream
   void* split;  // split-contraction scratch shared by the GEMMs (they run in stream order)
   size_t split_len;
 };
@@ -692,7 +786,7 @@ size_t step_split_bytes(int64_t M, int64_t K, int64_t N) {
 
 size_t step_ws_bytes(int64_t M, int64_t K, int64_t N) {
   return 2 * (align_up(size_t(M * K)) + align_up(size_t(N * K)) + align_up(size_t(M * N))) + kAlign +
-         2 * kPartialBytes + align_up(step_split_bytes(M, K, N));
+         4 * kPartialBytes + align_up(step_split_bytes(M, K, N));
 }
 
 hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t N, StepWs* w) {
@@ -709,6 +803,8 @@ hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t
   w->scales = reinterpret_cast<float*>(take(kAlign));
   w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
   w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  w->spart_c = reinterpret_cast<float*>(take(kPartialBytes));
+  w->spart_r = reinterpret_cast<float*>(take(kPartialBytes));
   w->split_len = step_split_bytes(M, K, N);
   w->split = w->split_len ? take(w->split_len) : nullptr;
   return HQ_OK;
@@ -728,16 +824,18 @@ hq_status check_step_shape(hq_dtype dt, int64_t M, int64_t K, int64_t N, int k, 
 }
 
 // Workspace of hq_linear_fwd_save (X along K, W along K) and hq_linear_bwd (dY along N,
-// W along N, dY along M): up to three code tensors, scales, two partial buffers.
+// W along N, dY along M): up to three code tensors, scales, four partial buffers (one pair
+// per stream).
 size_t codes_ws_bytes(int64_t b0, int64_t b1, int64_t b2, size_t split_bytes) {
-  return align_up(size_t(b0)) + align_up(size_t(b1)) + align_up(size_t(b2)) + kAlign + 2 * kPartialBytes +
+  return align_up(size_t(b0)) + align_up(size_t(b1)) + align_up(size_t(b2)) + kAlign + 4 * kPartialBytes +
          align_up(split_bytes);
 }
 
 struct CodesWs {
   uint8_t* c[3];
   float* scales;
-  float *part_c, *part_r;
+  float *part_c, *part_r;    // caller's stream
+  float *spart_c, *spart_r;  // side stream
   void* split;  // split-contraction scratch of the GEMMs (they run in stream order)
   size_t split_len;
 };
@@ -754,6 +852,8 @@ hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int6
   w->scales = reinterpret_cast<float*>(take(kAlign));
   w->part_c = reinterpret_cast<float*>(take(kPartialBytes));
   w->part_r = reinterpret_cast<float*>(take(kPartialBytes));
+  w->spart_c = reinterpret_cast<float*>(take(kPartialBytes));
+  w->spart_r = reinterpret_cast<float*>(take(kPartialBytes));
   w->split_len = split_bytes;
   w->split = split_bytes ? take(split_bytes) : nullptr;
   return HQ_OK;
@@ -892,25 +992,25 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
   cudaError_t e;
   if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
   if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
-  // side stream: the four rotations the forward GEMM does not need, in the order the
-  // backward GEMMs need them; they run alongside the forward quantizations and GEMM
-  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.part_r, *d, ss->s)) != HQ_OK) return s;
-  if ((s = quantize_impl(dY, dt, M, N, 1, k, fmt, w.dyq, sc + 4, w.part_r, *d, ss->s)) != HQ_OK) return s;
-  if ((e = cudaEventRecord(ss->join_dx, ss->s)) != cudaSuccess) return cuda_fail(e);
-  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.part_r, *d, ss->s)) != HQ_OK) return s;
-  if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, w.dyqt, sc + 5, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  // side stream: the rotations only the backward GEMMs need, alongside the forward operands
+  // and GEMM: dY in both rotations (one read per pass), W along N, X along M
+  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.dyq, sc + 4, w.dyqt, sc + 5, w.spart_c, w.spart_r, *d, ss->s)) !=
+      HQ_OK)
+    return s;
+  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.spart_c, *d, ss->s)) != HQ_OK) return s;
+  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.spart_c, *d, ss->s)) != HQ_OK) return s;
   if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
-  // caller's stream: forward operands, forward GEMM, then the backward GEMMs as their codes land
+  // caller's stream: the forward operands (X and W along K) first, so the forward GEMM starts
+  // as early as possible, then the backward GEMMs once the side stream's codes have landed
   if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.wq, sc + 2, w.part_c, *d, st)) != HQ_OK) return s;
   if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split, w.split_len)) !=
       HQ_OK)
     return s;
-  if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st, w.split,
                      w.split_len)) != HQ_OK)
     return s;
-  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split, w.split_len);
 }
 
@@ -939,17 +1039,17 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
   cudaError_t e;
   if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
   if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
-  // side stream: the codes kept for the weight gradient
-  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, xqt_codes, xqt_scale, w.part_r, *d, ss->s)) != HQ_OK) return s;
+  // side stream: W along K
+  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.c[1], w.scales + 1, w.spart_c, *d, ss->s)) != HQ_OK) return s;
   if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
-  // caller's stream: the forward operands and GEMM
-  if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.c[0], w.scales + 0, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.c[1], w.scales + 1, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split,
-                     w.split_len)) != HQ_OK)
+  // caller's stream: X in both rotations (along K for the forward GEMM, along M kept for the
+  // weight gradient), then the forward GEMM once W's codes have landed
+  if ((s = dual_impl(X, dt, M, K, k, fmt, w.c[0], w.scales + 0, xqt_codes, xqt_scale, w.part_c, w.part_r, *d,
+                     st)) != HQ_OK)
     return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
-  return HQ_OK;
+  return gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split,
+                   w.split_len);
 }
 
 size_t hq_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -980,16 +1080,16 @@ hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, co
   cudaError_t e;
   if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
   if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
-  // side stream: dY along the tokens, for the weight gradient
-  if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, w.c[2], sc + 2, w.part_r, *d, ss->s)) != HQ_OK) return s;
-  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
-  // caller's stream: dX operands and GEMM, then dW once dY's second rotation has landed
-  if ((s = quantize_impl(dY, dt, M, N, 1, k, fmt, w.c[0], sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.c[1], sc + 1, w.part_c, *d, st)) != HQ_OK) return s;
+  // side stream: W along N
+  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.c[1], sc + 1, w.spart_r, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dx, ss->s)) != cudaSuccess) return cuda_fail(e);
+  // caller's stream: dY in both rotations, then dX once W's codes have landed, then dW
+  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.c[0], sc + 0, w.c[2], sc + 2, w.part_c, w.part_r, *d, st)) != HQ_OK)
+    return s;
+  if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
   if ((s = gemm_impl(w.c[0], sc + 0, w.c[1], sc + 1, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st, w.split,
                      w.split_len)) != HQ_OK)
     return s;
-  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split,
                    w.split_len);
 }

@@ -145,9 +145,13 @@ HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, in
  * of its two dimensions).  Results are bit-identical to two hq_quantize calls:
  *   codes_c [rows][cols] + scale_c: rotated along cols  (hq_quantize dim = 1)
  *   codes_r [cols][rows] + scale_r: rotated along rows  (hq_quantize dim = 0)
- * rows and cols must both be multiples of k.  The four passes (two absmax, two code passes)
- * run back to back in alternating directions so that after the first one most source reads
- * are served by L2.  workspace: >= hq_quantize_dual_workspace_bytes() bytes.
+ * rows and cols must both be multiples of k.  For a bf16 source with rows and cols multiples
+ * of 64 one kernel computes both rotations from a single read of each 256 x 256 tile per pass
+ * (2 launches: both absmax partials, then both code tensors); otherwise the four single-
+ * rotation passes run back to back in alternating directions so that after the first one most
+ * source reads are served by L2.  workspace: >= hq_quantize_dual_workspace_bytes() bytes.
+ * Device-side errors as for hq_quantize, per rotation (a rotation whose absmax is not finite
+ * writes no codes and a NaN scale; the other rotation is still written).
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_quantize_dual_workspace_bytes(void);
 HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k,
@@ -158,14 +162,16 @@ HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, in
 /* ------------------------------------------------------------------------------------------
  * hq_linear_fwd_bwd -- the whole layer step: Y = X W^T, dX = dY W and dW = dY^T X, each GEMM
  * on operands rotated along its contraction dimension, every operand rotation computed once
- * (six quantizations + three GEMMs, 15 kernels).  Outputs equal those of hq_linear_fwd,
- * hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
+ * (six rotations in five quantization calls + three GEMMs, 13 kernels).  Outputs equal those
+ * of hq_linear_fwd, hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
  *   X [M][K], W [N][K], dY [M][N] (dtype dt); Y [M][N], dX [M][K], dW [N][K] bf16.
  *   M, K, N: positive multiples of k.  workspace: >= hq_linear_fwd_bwd_workspace_bytes().
- * The four rotations the forward GEMM does not use (W along N, dY along N, X along M, dY
- * along M) run on a per-device side stream that the library creates on first use (with two
- * events) and forks from / joins back to `stream` with events, so they overlap the forward
- * quantizations and GEMM; everything is complete when `stream` reaches the end of the call.
+ * X and W along K and the forward GEMM run on `stream`; the four rotations the forward GEMM
+ * does not use (dY along N and along M together, as in hq_quantize_dual, then W along N and
+ * X along M) run on a per-device side stream that the library creates on first use (with
+ * three events) and forks from / joins back to `stream` with events, so they overlap the
+ * forward quantizations and GEMM; everything is complete when `stream` reaches the end of the
+ * call.
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
 HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt,
@@ -183,13 +189,13 @@ HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY,
  * for hq_linear_bwd; X itself is then not needed after the forward.
  *   X [M][K], W [N][K] (dtype dt); Y [M][N] bf16; M, K, N positive multiples of k.
  *   workspace: >= hq_linear_fwd_save_workspace_bytes(M, K, N) bytes (not preserved).
- * X along M runs on the library's per-device side stream (see hq_linear_fwd_bwd), alongside
- * the forward quantizations and GEMM; all outputs are complete when `stream` reaches the end
- * of the call.
+ * X is quantized in both rotations at once (as in hq_quantize_dual) on `stream` while W along
+ * K runs on the library's per-device side stream (see hq_linear_fwd_bwd); all outputs are
+ * complete when `stream` reaches the end of the call.
  *
  * hq_linear_bwd -- dX = dY W and dW = dY^T X from the saved codes: dY is quantized once in
- * both rotations (along N for dX, along M for dW; the latter on the side stream), W along N,
- * then the two GEMMs.  Outputs equal those of hq_linear_bwd_dx and hq_linear_bwd_dw (the
+ * both rotations (along N for dX, along M for dW, as in hq_quantize_dual) on `stream` while
+ * W along N runs on the side stream, then the two GEMMs.  Outputs equal those of hq_linear_bwd_dx and hq_linear_bwd_dw (the
  * latter given the X the codes came from) bit for bit.
  *   dY [M][N], W [N][K] (dtype dt); xqt_codes [K][M] and xqt_scale from hq_linear_fwd_save
  *   with the same M, K, k and fmt (not checked: the library cannot tell codes apart);

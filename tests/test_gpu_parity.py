@@ -153,6 +153,71 @@ def test_quantize_dual(dtype, k, fmt):
         assert scale.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32)
 
 
+# Shapes for the fused two-rotation kernel (bf16, rows and cols multiples of 64, 256 x 256
+# tiles): ragged last tiles in both directions where k allows it, and a case with more
+# tiles than SMs so that CTAs run several tiles and the strip ring wraps.
+def _fused_shapes(k):
+    small = {16: (1344, 1216), 32: (1344, 1216), 64: (1344, 1216), 128: (1408, 1152), 256: (1536, 1280)}[k]
+    many = (3328, 3328) if k == 256 else (3200, 3200)
+    return (small, many)
+
+
+@pytest.mark.parametrize("k", KS)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_dual_fused_tiles(k, fmt):
+    """The fused kernel's codes and scales equal the oracle's for both rotations."""
+    for rows, cols in _fused_shapes(k):
+        x = _outlier_input(rows, cols, 7 * k + rows, "bf16")
+        cc, sc, cr, sr = hq.hq_quantize_dual(to_device(x), k, fmt)
+        for codes, scale, dim in ((cc, sc, 1), (cr, sr, 0)):
+            want_codes, want_scale = oracle.quantize(x, dim, k, fmt)
+            got = codes.cpu().numpy()
+            mism = np.count_nonzero(got != want_codes)
+            assert mism == 0, f"{rows}x{cols} dim {dim}: {mism} code mismatches"
+            assert scale.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32)
+    assert hq.hq_get_error() == 0
+
+
+@pytest.mark.parametrize("k", (64, 256))
+def test_quantize_dual_fused_matches_single(k):
+    """At a full weight size (11008 x 4096, every CTA several tiles deep) the fused kernel
+    writes the same bytes as the two single-rotation calls."""
+    w = synthetic.WORKLOADS[2]
+    W = to_device(synthetic.draw(w)["W"])
+    for fmt in FMTS:
+        cc, sc, cr, sr = hq.hq_quantize_dual(W, k, fmt)
+        c1, s1 = hq.hq_quantize(W, 1, k, fmt)
+        c0, s0 = hq.hq_quantize(W, 0, k, fmt)
+        assert torch.equal(cc, c1) and torch.equal(sc, s1)
+        assert torch.equal(cr, c0) and torch.equal(sr, s0)
+    assert hq.hq_get_error() == 0
+
+
+def test_quantize_dual_fused_special_values():
+    """Zero tensor (scale 1, zero codes); a NaN (both rotations flagged); two near-maximal
+    values in one row block, which overflow the rotation along the columns only: that
+    rotation is flagged and the other is still written, equal to the oracle's."""
+    z = torch.zeros(256, 512, dtype=torch.bfloat16, device="cuda")
+    cc, sc, cr, sr = hq.hq_quantize_dual(z, 64, "int8")
+    assert sc.item() == 1.0 and sr.item() == 1.0
+    assert int(cc.count_nonzero()) == 0 and int(cr.count_nonzero()) == 0
+    x = torch.randn(256, 512, device="cuda").to(torch.bfloat16)
+    x[100, 300] = float("nan")
+    assert hq.hq_get_error() == 0
+    hq.hq_quantize_dual(x, 128, "fp8")
+    assert hq.hq_get_error() == 5
+    xb = _outlier_input(512, 512, 11, "bf16")
+    big = np.uint16(0x7F7F)  # largest finite bf16, about 3.39e38
+    xb[40, 0] = big
+    xb[40, 1] = big
+    cc, sc, cr, sr = hq.hq_quantize_dual(to_device(xb), 64, "int8")
+    assert hq.hq_get_error() == 5
+    assert not np.isfinite(sc.cpu().numpy()[0])
+    want_codes, want_scale = oracle.quantize(xb, 0, 64, oracle.INT8)
+    assert np.array_equal(cr.cpu().numpy(), want_codes)
+    assert sr.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32)
+
+
 # ------------------------------------------------------------------------------ GEMM
 
 def _rand_codes(shape, fmt, seed):
