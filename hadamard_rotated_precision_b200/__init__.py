@@ -31,6 +31,7 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_fwd_bwd_workspace_bytes", "hq_linear_fwd_bwd",
            "hq_linear_fwd_save_workspace_bytes", "hq_linear_fwd_save",
            "hq_linear_bwd_workspace_bytes", "hq_linear_bwd", "hq_selftest_gemm_timeout",
+           "hq_quantize_rht", "hq_quantize_dual_rht", "hq_linear_fwd_bwd_rht",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -64,6 +65,12 @@ def lib() -> ctypes.CDLL:
         L.hq_quantize.restype = i32
         L.hq_quantize_noalloc.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p]
         L.hq_quantize_noalloc.restype = i32
+        L.hq_quantize_rht.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p, p, sz, p]
+        L.hq_quantize_rht.restype = i32
+        L.hq_quantize_dual_rht.argtypes = [p, i32, i64, i64, i32, i32, p, p, p, p, p, p, p, sz, p]
+        L.hq_quantize_dual_rht.restype = i32
+        L.hq_linear_fwd_bwd_rht.argtypes = [p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, p, p, p, sz, p]
+        L.hq_linear_fwd_bwd_rht.restype = i32
         L.hq_quantize_dual_workspace_bytes.argtypes = []
         L.hq_quantize_dual_workspace_bytes.restype = sz
         L.hq_quantize_dual.argtypes = [p, i32, i64, i64, i32, i32, p, p, p, p, p, sz, p]
@@ -187,6 +194,71 @@ def hq_quantize(src, dim: int, k: int, fmt, codes=None, scale=None, workspace=No
     return codes, scale
 
 
+def _sign_flags(neg, length: int, name: str):
+    """Device uint8 flags (bit 0 = negate), one per position of a rotated dimension; None = plain."""
+    if neg is None:
+        return None
+    _dev_tensor(neg, name)
+    torch = _torch()
+    if neg.dtype != torch.uint8 or neg.dim() != 1 or neg.numel() != length or not neg.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous uint8 CUDA tensor of {length} flags")
+    return neg
+
+
+def _ptr_or_none(t):
+    return None if t is None else t.data_ptr()
+
+
+def hq_quantize_rht(src, dim: int, k: int, fmt, neg, codes=None, scale=None, workspace=None, stream=None):
+    """hq_quantize with the randomized Hadamard's sign flags `neg` (uint8 CUDA tensor, one per
+    position of the rotated dimension, bit 0 = negate before the blocks; None = plain)."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    neg = _sign_flags(neg, cols if dim == 1 else rows, "neg")
+    shape = (rows, cols) if dim == 1 else (cols, rows)
+    codes = torch.empty(shape, dtype=torch.uint8, device=src.device) if codes is None else codes
+    scale = torch.empty(1, dtype=torch.float32, device=src.device) if scale is None else scale
+    _dev_tensor(codes, "codes")
+    _dev_tensor(scale, "scale")
+    ws = _workspace(hq_quantize_workspace_bytes(), src.device, workspace)
+    st = lib().hq_quantize_rht(src.data_ptr(), dt, rows, cols, dim, k, _fmt(fmt), _ptr_or_none(neg),
+                               codes.data_ptr(), scale.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                               _stream_handle(stream))
+    _check(st, "hq_quantize_rht")
+    return codes, scale
+
+
+def hq_quantize_dual_rht(src, k: int, fmt, neg_c, neg_r, codes_c=None, scale_c=None, codes_r=None,
+                         scale_r=None, workspace=None, stream=None):
+    """hq_quantize_dual with sign flags neg_c over the columns and neg_r over the rows."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    neg_c = _sign_flags(neg_c, cols, "neg_c")
+    neg_r = _sign_flags(neg_r, rows, "neg_r")
+    dev = src.device
+    codes_c = torch.empty((rows, cols), dtype=torch.uint8, device=dev) if codes_c is None else codes_c
+    codes_r = torch.empty((cols, rows), dtype=torch.uint8, device=dev) if codes_r is None else codes_r
+    scale_c = torch.empty(1, dtype=torch.float32, device=dev) if scale_c is None else scale_c
+    scale_r = torch.empty(1, dtype=torch.float32, device=dev) if scale_r is None else scale_r
+    for t, n in ((codes_c, "codes_c"), (codes_r, "codes_r"), (scale_c, "scale_c"), (scale_r, "scale_r")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_quantize_dual_workspace_bytes(), dev, workspace)
+    st = lib().hq_quantize_dual_rht(src.data_ptr(), dt, rows, cols, k, _fmt(fmt), _ptr_or_none(neg_c),
+                                    _ptr_or_none(neg_r), codes_c.data_ptr(), scale_c.data_ptr(), codes_r.data_ptr(),
+                                    scale_r.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                    _stream_handle(stream))
+    _check(st, "hq_quantize_dual_rht")
+    return codes_c, scale_c, codes_r, scale_r
+
+
 def hq_quantize_dual_workspace_bytes() -> int:
     return int(lib().hq_quantize_dual_workspace_bytes())
 
@@ -242,6 +314,34 @@ def hq_linear_fwd_bwd(X, W, dY, k: int, fmt, Y=None, dX=None, dW=None, workspace
                                  Y.data_ptr(), dX.data_ptr(), dW.data_ptr(), ws.data_ptr(),
                                  ws.numel() * ws.element_size(), _stream_handle(stream))
     _check(st, "hq_linear_fwd_bwd")
+    return Y, dX, dW
+
+
+def hq_linear_fwd_bwd_rht(X, W, dY, k: int, fmt, neg_k, neg_n, neg_m, Y=None, dX=None, dW=None, workspace=None,
+                          stream=None):
+    """hq_linear_fwd_bwd with the randomized Hadamard's sign flags per contraction dimension:
+    neg_k [K] (forward), neg_n [N] (dX), neg_m [M] (dW); None = plain for that dimension."""
+    torch = _torch()
+    for t, n in ((X, "X"), (W, "W"), (dY, "dY")):
+        _dev_tensor(t, n)
+    dt = _src_dtype(X, "X")
+    if _src_dtype(W, "W") != dt or _src_dtype(dY, "dY") != dt:
+        raise TypeError("X, W and dY must have the same dtype")
+    M, K = X.shape
+    N = W.shape[0]
+    neg_k, neg_n, neg_m = _sign_flags(neg_k, K, "neg_k"), _sign_flags(neg_n, N, "neg_n"), _sign_flags(neg_m, M, "neg_m")
+    dev = X.device
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if Y is None else Y
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if dW is None else dW
+    for t, n in ((Y, "Y"), (dX, "dX"), (dW, "dW")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_fwd_bwd_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_fwd_bwd_rht(X.data_ptr(), W.data_ptr(), dY.data_ptr(), dt, M, K, N, k, _fmt(fmt),
+                                     _ptr_or_none(neg_k), _ptr_or_none(neg_n), _ptr_or_none(neg_m), Y.data_ptr(),
+                                     dX.data_ptr(), dW.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                     _stream_handle(stream))
+    _check(st, "hq_linear_fwd_bwd_rht")
     return Y, dX, dW
 
 

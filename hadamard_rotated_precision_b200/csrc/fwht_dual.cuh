@@ -182,13 +182,15 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float2& f) {
   f = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-template <int K, int MODE, bool W32>
+template <int K, int MODE, bool W32, bool SIGNED>
 __global__ void __launch_bounds__(kThreads, 1)
 fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes_c, uint8_t* __restrict__ codes_r,
                   float* __restrict__ part_c, float* __restrict__ part_r, int n_partials,
                   float* __restrict__ scale_c, float* __restrict__ scale_r,
-                  unsigned int* __restrict__ status, int reverse) {
+                  unsigned int* __restrict__ status, int reverse,
+                  const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r) {
+  // SIGNED: sign flags per column (neg_c) and per row (neg_r); either may be null (all clear)
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   extern __shared__ uint8_t dsmem[];
@@ -296,10 +298,30 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
     for (int st = 0; st < kSteps; ++st) {
       const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
       const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+      // sign flags of the thread's 64 columns (the randomized variant; cols is a multiple of 64,
+      // so they are all inside the tensor or all past its end)
+      uint32_t sm[SIGNED ? 32 : 1];
+      if constexpr (SIGNED) {
+        const int64_t c0 = col0 + kStripCols * sr;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t m8[8];
+          sign_masks_bf16x16(neg_c != nullptr && c0 < cols ? __ldg(reinterpret_cast<const uint4*>(neg_c + c0 + 16 * c))
+                                                           : make_uint4(0u, 0u, 0u, 0u), m8);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+        }
+      }
       float2 v[32];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+        uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+        if constexpr (SIGNED) {
+          raw.x ^= sm[(4 * j) % (SIGNED ? 32 : 1)];
+          raw.y ^= sm[(4 * j + 1) % (SIGNED ? 32 : 1)];
+          raw.z ^= sm[(4 * j + 2) % (SIGNED ? 32 : 1)];
+          raw.w ^= sm[(4 * j + 3) % (SIGNED ? 32 : 1)];
+        }
         unpack_bf16x2(raw.x, v[4 * j]);
         unpack_bf16x2(raw.y, v[4 * j + 1]);
         unpack_bf16x2(raw.z, v[4 * j + 2]);
@@ -326,13 +348,27 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
     for (int j2 = 0; j2 < kSteps; ++j2) {
       const int s = grp + (kComputeWarps / 8) * j2;
       const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+      // sign flags of the thread's 64 rows (rows is a multiple of 64)
+      uint32_t sm[SIGNED ? 32 : 1];
+      if constexpr (SIGNED) {
+        const int64_t r0t = row0 + 64 * (lane & 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t m8[8];
+          sign_masks_bf16x16(neg_r != nullptr && r0t < rows ? __ldg(reinterpret_cast<const uint4*>(neg_r + r0t + 16 * c))
+                                                            : make_uint4(0u, 0u, 0u, 0u), m8);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+        }
+      }
       float2 v[32];
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
         uint32_t r4[4];
         ldmatrix_x4_trans(lbase + 4096u * n, r4);
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) unpack_bf16x2(r4[mm], v[4 * n + mm]);
+        for (int mm = 0; mm < 4; ++mm)
+          unpack_bf16x2(SIGNED ? r4[mm] ^ sm[(4 * n + mm) % (SIGNED ? 32 : 1)] : r4[mm], v[4 * n + mm]);
       }
       release(q0 + s);
       if constexpr (!QUANT) {

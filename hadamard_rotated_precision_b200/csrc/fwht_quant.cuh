@@ -272,6 +272,32 @@ __device__ __forceinline__ uint32_t codes4(float2 z0, float2 z1) {
   }
 }
 
+// ------------------------------------------------------------------ sign flags
+
+// Randomized variant (a sign diagonal D before the blocks, t = H_k D x): `neg` holds one byte
+// per position of the rotated dimension, bit 0 set negating that position.  The flip is an
+// exact change of the source's sign bit before the butterflies, applied as an XOR mask to the
+// raw words.
+
+// Masks for 16 consecutive bf16 positions held as 8 bf16x2 words (word j: positions 2j in the
+// low half, 2j + 1 in the high half); f = the 16 flag bytes.
+__device__ __forceinline__ void sign_masks_bf16x16(uint4 f, uint32_t (&m)[8]) {
+  const uint32_t w[4] = {f.x & 0x01010101u, f.y & 0x01010101u, f.z & 0x01010101u, f.w & 0x01010101u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[2 * i] = __byte_perm(w[i], 0u, 0x1404) << 7;      // flag bytes 0, 1 -> bits 15, 31
+    m[2 * i + 1] = __byte_perm(w[i], 0u, 0x3424) << 7;  // flag bytes 2, 3 -> bits 15, 31
+  }
+}
+
+// Masks for 4 consecutive fp32 positions (one word each) from 4 flag bytes.
+__device__ __forceinline__ void sign_masks_f32x4(uint32_t f, uint32_t (&m)[4]) {
+  m[0] = (f << 31) & 0x80000000u;
+  m[1] = (f << 23) & 0x80000000u;
+  m[2] = (f << 15) & 0x80000000u;
+  m[3] = (f << 7) & 0x80000000u;
+}
+
 // ------------------------------------------------------------------ dim = 1 (contiguous)
 
 // Each thread owns 32 consecutive elements (one warp step = 1024 elements), so in-block index
@@ -358,11 +384,12 @@ __device__ __forceinline__ void exchange_rows(float2 (&v)[16], float4* slice, in
   __syncwarp();
 }
 
-template <typename SrcT, int K, int MODE, bool WIDE>
+template <typename SrcT, int K, int MODE, bool WIDE, bool SIGNED>
 __global__ void __launch_bounds__(kQuantThreads, sizeof(SrcT) == 2 ? 3 : 1)
 fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__ codes,
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
-                  unsigned int* __restrict__ status, int reverse) {
+                  unsigned int* __restrict__ status, int reverse, const uint8_t* __restrict__ neg,
+                  int64_t cols) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr bool EXCH = K >= 64;
@@ -393,7 +420,38 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
     // the loads of unit u + step go out while u is computed (one unit of registers, so that
     // three CTAs fit per SM)
     auto valid = [&](int64_t u) { return reverse ? u >= 0 : u < n_units; };
+    // column of this thread's first element in the current unit (sign flags only): tracked
+    // incrementally, the units of a thread being `step` apart
+    int64_t col = 0, dcol = 0;
+    if constexpr (SIGNED) {
+      col = (first * kRowsWarpElems + 32 * lane) % cols;
+      dcol = ((step * kRowsWarpElems) % cols + cols) % cols;
+    }
     auto body = [&](uint32_t (&raw)[RW], int64_t u) {
+      if constexpr (SIGNED) {
+        // each 16-element half lies in one row (cols is a multiple of 16)
+        const int64_t c1 = col + 16 >= cols ? col + 16 - cols : col + 16;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 f = __ldg(reinterpret_cast<const uint4*>(neg + (h == 0 ? col : c1)));
+          if constexpr (sizeof(SrcT) == 2) {
+            uint32_t m[8];
+            sign_masks_bf16x16(f, m);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) raw[8 * h + j] ^= m[j];
+          } else {
+            const uint32_t fw[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t m[4];
+              sign_masks_f32x4(fw[q], m);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) raw[16 * h + 4 * q + j] ^= m[j];
+            }
+          }
+        }
+        col = col + dcol >= cols ? col + dcol - cols : col + dcol;
+      }
       float2 v[16];
       unpack_rows32<SrcT>(raw, v);
       const int64_t nu = u + step;
@@ -476,11 +534,12 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
 
-template <int K, int MODE>
+template <int K, int MODE, bool SIGNED>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols,
                        uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
-                       float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse) {
+                       float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
+                       const uint8_t* __restrict__ neg) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   extern __shared__ __align__(128) uint4 tiles[];  // [3][256 rows][8 chunks]
@@ -539,6 +598,21 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
       // gather: 8 x (ldmatrix.x4.trans) -> 64 consecutive rows of one column per thread
       float2 v[32];
       {
+        // sign flags of the thread's rows r0t + 0..63 (16-row chunks wholly inside or outside
+        // the tensor: rows is a multiple of 16); rows past the end stay unflipped zeros
+        uint32_t sm[SIGNED ? 32 : 1];
+        if constexpr (SIGNED) {
+          const int64_t r0t = (t / n_ct) * kColsTileRows2 + 64 * (lane & 3);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t m8[8];
+            const uint4 f = r0t + 16 * c < rows ? __ldg(reinterpret_cast<const uint4*>(neg + r0t + 16 * c))
+                                                : make_uint4(0u, 0u, 0u, 0u);
+            sign_masks_bf16x16(f, m8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+          }
+        }
         const int m = lane >> 3, q = lane & 7;
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
@@ -546,8 +620,10 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
           uint32_t r[4];
           ldmatrix_x4_trans(ptx::smem_u32(&tiles[(buf * kColsTileRows2 + rho) * 8 + (warp ^ cols_swz(rho))]), r);
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm)
-            v[4 * kc + mm] = make_float2(__uint_as_float(r[mm] << 16), __uint_as_float(r[mm] & 0xFFFF0000u));
+          for (int mm = 0; mm < 4; ++mm) {
+            const uint32_t rw = SIGNED ? r[mm] ^ sm[(4 * kc + mm) % (SIGNED ? 32 : 1)] : r[mm];
+            v[4 * kc + mm] = make_float2(__uint_as_float(rw << 16), __uint_as_float(rw & 0xFFFF0000u));
+          }
         }
       }
       __syncthreads();  // buffer free before the copies issued next iteration reuse it
@@ -588,12 +664,14 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
 constexpr int kColsTileRows = 256;   // rows per tile: 32 lanes x 8 registers
 constexpr int kColsTileBytes = 128;  // bytes of each source row per tile (8 x 16-byte chunks)
 
-template <typename SrcT, int K, int MODE>
+template <typename SrcT, int K, int MODE, bool SIGNED>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
-                  float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse) {
+                  float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
+                  const uint8_t* __restrict__ neg) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  static_assert(!SIGNED || sizeof(SrcT) == 4, "sign masks of this kernel are for fp32 words");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr int CPC = 16 / static_cast<int>(sizeof(SrcT));  // columns per 16-byte chunk
   constexpr int TCOLS = 8 * CPC;                            // columns per tile
@@ -636,9 +714,27 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
       __syncthreads();
       // thread (warp w, lane l): rows 8l..8l+7 of the w-th 16-byte column chunk
       float v[8][CPC];
+      uint32_t sm[8];  // sign masks of the 8 rows (8-row groups are wholly inside or outside)
+      if constexpr (SIGNED) {
+        const int64_t r8 = r0 + 8 * lane;
+        const uint2 f = r8 < rows ? __ldg(reinterpret_cast<const uint2*>(neg + r8)) : make_uint2(0u, 0u);
+        uint32_t m4[4];
+        sign_masks_f32x4(f.x, m4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm[i] = m4[i];
+        sign_masks_f32x4(f.y, m4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm[4 + i] = m4[i];
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint4 raw = tile[8 * lane + i][warp ^ (lane & 7)];
+        uint4 raw = tile[8 * lane + i][warp ^ (lane & 7)];
+        if constexpr (SIGNED) {
+          raw.x ^= sm[i];
+          raw.y ^= sm[i];
+          raw.z ^= sm[i];
+          raw.w ^= sm[i];
+        }
         if constexpr (CPC == 8) {
           float t8[8];
           unpack_bf16x8(raw, t8);

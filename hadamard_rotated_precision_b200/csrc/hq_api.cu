@@ -33,9 +33,9 @@ struct DeviceInfo {
   int sms = 0;
   unsigned int* status = nullptr;
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
-  unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation
+  unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation (30 used)
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
-  unsigned dual_attr_set = 0;  // bit per fused two-rotation quantizer instantiation
+  uint64_t dual_attr_set = 0;  // bit per fused two-rotation quantizer instantiation (60 used)
 };
 
 std::mutex g_mu;
@@ -132,13 +132,13 @@ int blocks_per_sm(const void* fn, size_t smem) {
   return b;
 }
 
-template <int K, int MODE>
+template <int K, int MODE, bool SIGNED>
 cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
   constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
-  const unsigned bit = 1u << (kIdx * 3 + MODE);
+  const unsigned bit = 1u << ((kIdx * 3 + MODE) * 2 + (SIGNED ? 1 : 0));
   std::lock_guard<std::mutex> lock(g_mu);
   if (d.cols_attr_set & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(hq::fwhtq_cols_bf16_kernel<K, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(hq::fwhtq_cols_bf16_kernel<K, MODE, SIGNED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(hq::kColsSmemBytes2));
   if (e == cudaSuccess) d.cols_attr_set |= bit;
@@ -146,11 +146,11 @@ cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
 }
 
 // Launch one pass; returns its grid through *grid (the absmax pass's grid is the number of
-// partials the code pass reduces).
-template <typename SrcT, int K, int MODE>
-cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes,
-                        float* scale, float* partials, int n_partials, int reverse, DeviceInfo& d,
-                        cudaStream_t st, int* grid) {
+// partials the code pass reduces).  SIGNED: the randomized variant with sign flags `neg`.
+template <typename SrcT, int K, int MODE, bool SIGNED>
+cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes,
+                          float* scale, float* partials, int n_partials, int reverse, const uint8_t* neg,
+                          DeviceInfo& d, cudaStream_t st, int* grid) {
   using namespace hq;
   const int64_t units = quant_units(sizeof(SrcT) == 2 ? HQ_BF16 : HQ_F32, rows, cols, dim);
   auto grid_for = [&](const void* fn, size_t smem) {
@@ -161,41 +161,55 @@ cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, ui
   if (dim == 1) {
     const int64_t n = rows * cols;
     if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0) {
-      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, true>;
+      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, true, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
-      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
+                                      reverse, neg, cols);
     } else {
-      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, false>;
+      auto fn = fwhtq_rows_kernel<SrcT, K, MODE, false, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
-      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
+                                      reverse, neg, cols);
     }
   } else if constexpr (sizeof(SrcT) == 2) {
-    cudaError_t e = cols_bf16_smem_attr<K, MODE>(d);
+    cudaError_t e = cols_bf16_smem_attr<K, MODE, SIGNED>(d);
     if (e != cudaSuccess) return e;
-    auto fn = fwhtq_cols_bf16_kernel<K, MODE>;
+    auto fn = fwhtq_cols_bf16_kernel<K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), kColsSmemBytes2);
-    fn<<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+    fn<<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials,
+                                                  scale, d.status, reverse, neg);
   } else {
-    auto fn = fwhtq_cols_f32_kernel<SrcT, K, MODE>;
+    auto fn = fwhtq_cols_f32_kernel<SrcT, K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), 0);
-    fn<<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse);
+    fn<<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale,
+                                    d.status, reverse, neg);
   }
   *grid = g;
   return cudaGetLastError();
 }
 
+template <typename SrcT, int K, int MODE>
+cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes, float* scale,
+                        float* partials, int n_partials, int reverse, const uint8_t* neg, DeviceInfo& d,
+                        cudaStream_t st, int* grid) {
+  return neg ? launch_pass_s<SrcT, K, MODE, true>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse,
+                                                  neg, d, st, grid)
+             : launch_pass_s<SrcT, K, MODE, false>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse,
+                                                   nullptr, d, st, grid);
+}
+
 // One operand, one rotation: absmax pass forward, code pass backward.
 template <typename SrcT, int K>
 cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim, hq_fmt fmt,
-                         uint8_t* codes, float* scale, float* partials, DeviceInfo& d,
+                         uint8_t* codes, float* scale, float* partials, const uint8_t* neg, DeviceInfo& d,
                          cudaStream_t st) {
   const SrcT* src = static_cast<const SrcT*>(src_v);
   using namespace hq;
   int g1 = 0, g2 = 0;
-  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, 0, 0, d, st, &g1);
+  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, 0, 0, neg, d, st, &g1);
   if (e != cudaSuccess) return e;
-  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g1, 1, d, st, &g2);
-  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g1, 1, d, st, &g2);
+  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g1, 1, neg, d, st, &g2);
+  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g1, 1, neg, d, st, &g2);
 }
 
 // One operand, both rotations: the four passes run back to back, alternating direction, so
@@ -203,19 +217,19 @@ cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim,
 template <typename SrcT, int K>
 cudaError_t launch_dual(const void* src_v, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
                         float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
-                        DeviceInfo& d, cudaStream_t st) {
+                        const uint8_t* neg_c, const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st) {
   const SrcT* src = static_cast<const SrcT*>(src_v);
   using namespace hq;
   int gc = 0, gr = 0, g = 0;
-  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 1, codes_c, scale_c, part_c, 0, 0, d, st, &gc);
-  if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 0, codes_r, scale_r, part_r, 0, 1, d, st, &gr);
+  cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 1, codes_c, scale_c, part_c, 0, 0, neg_c, d, st, &gc);
+  if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 0, codes_r, scale_r, part_r, 0, 1, neg_r, d, st, &gr);
   if (e != cudaSuccess) return e;
   if (fmt == HQ_INT8) {
-    e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, d, st, &g);
-    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, d, st, &g);
+    e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, neg_c, d, st, &g);
+    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, neg_r, d, st, &g);
   } else {
-    e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, d, st, &g);
-    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, d, st, &g);
+    e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, neg_c, d, st, &g);
+    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, neg_r, d, st, &g);
   }
   return e;
 }
@@ -242,13 +256,13 @@ hq_status encode_dual_map(CUtensorMap* map, const void* src, int64_t rows, int64
   return HQ_OK;
 }
 
-template <int K, int MODE, bool W32>
+template <int K, int MODE, bool W32, bool SIGNED>
 cudaError_t dual_smem_attr(DeviceInfo& d) {
   constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
-  const unsigned bit = 1u << ((kIdx * 3 + MODE) * 2 + (W32 ? 1 : 0));
+  const uint64_t bit = uint64_t(1) << (((kIdx * 3 + MODE) * 2 + (W32 ? 1 : 0)) * 2 + (SIGNED ? 1 : 0));
   std::lock_guard<std::mutex> lock(g_mu);
   if (d.dual_attr_set & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(hq::dual::fwhtq_dual_kernel<K, MODE, W32>,
+  cudaError_t e = cudaFuncSetAttribute(hq::dual::fwhtq_dual_kernel<K, MODE, W32, SIGNED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(hq::dual::kSmemBytes));
   if (e == cudaSuccess) d.dual_attr_set |= bit;
@@ -257,28 +271,29 @@ cudaError_t dual_smem_attr(DeviceInfo& d) {
 
 // Pass 1 (both absmax partials, tiles in order) then pass 2 (both code tensors, tiles in
 // reverse order), one CTA per SM.  W32: both code buffers are 32-byte aligned, so the code
-// stores are whole 32-byte sectors.
-template <int K, bool W32>
+// stores are whole 32-byte sectors.  SIGNED: the randomized variant (neg_c per column for the
+// rotation along the columns, neg_r per row for the rotation along the rows).
+template <int K, bool W32, bool SIGNED>
 hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
                               float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
-                              DeviceInfo& d, cudaStream_t st) {
+                              const uint8_t* neg_c, const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st) {
   using namespace hq;
   using namespace hq::dual;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
   const int g = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(n_tiles, d.sms)));
-  cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32>(d);
+  cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32, SIGNED>(d);
   if (e != cudaSuccess) return cuda_fail(e);
-  fwhtq_dual_kernel<K, kModeAbsmax, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
-                                                                           part_r, 0, scale_c, scale_r, d.status, 0);
+  fwhtq_dual_kernel<K, kModeAbsmax, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
+      map, rows, cols, codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (fmt == HQ_INT8) {
-    if ((e = dual_smem_attr<K, kModeInt8, W32>(d)) != cudaSuccess) return cuda_fail(e);
-    fwhtq_dual_kernel<K, kModeInt8, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
-                                                                           part_r, g, scale_c, scale_r, d.status, 1);
+    if ((e = dual_smem_attr<K, kModeInt8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
+    fwhtq_dual_kernel<K, kModeInt8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
+        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r);
   } else {
-    if ((e = dual_smem_attr<K, kModeFp8, W32>(d)) != cudaSuccess) return cuda_fail(e);
-    fwhtq_dual_kernel<K, kModeFp8, W32><<<g, kThreads, kSmemBytes, st>>>(map, rows, cols, codes_c, codes_r, part_c,
-                                                                          part_r, g, scale_c, scale_r, d.status, 1);
+    if ((e = dual_smem_attr<K, kModeFp8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
+    fwhtq_dual_kernel<K, kModeFp8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
+        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   return HQ_OK;
@@ -287,50 +302,58 @@ hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols
 template <int K>
 hq_status launch_dual_fused(const CUtensorMap& map, int64_t rows, int64_t cols, hq_fmt fmt, uint8_t* codes_c,
                             float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
-                            DeviceInfo& d, cudaStream_t st) {
+                            const uint8_t* neg_c, const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st) {
   const bool w32 = ((reinterpret_cast<uintptr_t>(codes_c) | reinterpret_cast<uintptr_t>(codes_r)) & 31u) == 0;
-  return w32 ? launch_dual_fused_w<K, true>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st)
-             : launch_dual_fused_w<K, false>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+  if (neg_c || neg_r) {
+    return w32 ? launch_dual_fused_w<K, true, true>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                     part_r, neg_c, neg_r, d, st)
+               : launch_dual_fused_w<K, false, true>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                      part_r, neg_c, neg_r, d, st);
+  }
+  return w32 ? launch_dual_fused_w<K, true, false>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                    part_r, nullptr, nullptr, d, st)
+             : launch_dual_fused_w<K, false, false>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                     part_r, nullptr, nullptr, d, st);
 }
 
 hq_status launch_dual_fused_k(const void* src, int64_t rows, int64_t cols, int k, hq_fmt fmt, uint8_t* codes_c,
                               float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
-                              DeviceInfo& d, cudaStream_t st) {
+                              const uint8_t* neg_c, const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st) {
   CUtensorMap map;
   hq_status s = encode_dual_map(&map, src, rows, cols);
   if (s != HQ_OK) return s;
   switch (k) {
-    case 16: return launch_dual_fused<16>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 32: return launch_dual_fused<32>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 64: return launch_dual_fused<64>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 128: return launch_dual_fused<128>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    default: return launch_dual_fused<256>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 16: return launch_dual_fused<16>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 32: return launch_dual_fused<32>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 64: return launch_dual_fused<64>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 128: return launch_dual_fused<128>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    default: return launch_dual_fused<256>(map, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
   }
 }
 
 template <typename SrcT>
 cudaError_t launch_dual_k(const void* src, int64_t rows, int64_t cols, int k, hq_fmt fmt, uint8_t* codes_c,
                           float* scale_c, uint8_t* codes_r, float* scale_r, float* part_c, float* part_r,
-                          DeviceInfo& d, cudaStream_t st) {
+                          const uint8_t* neg_c, const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st) {
   switch (k) {
-    case 16: return launch_dual<SrcT, 16>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 32: return launch_dual<SrcT, 32>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 64: return launch_dual<SrcT, 64>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    case 128: return launch_dual<SrcT, 128>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
-    default: return launch_dual<SrcT, 256>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, d, st);
+    case 16: return launch_dual<SrcT, 16>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 32: return launch_dual<SrcT, 32>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 64: return launch_dual<SrcT, 64>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    case 128: return launch_dual<SrcT, 128>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
+    default: return launch_dual<SrcT, 256>(src, rows, cols, fmt, codes_c, scale_c, codes_r, scale_r, part_c, part_r, neg_c, neg_r, d, st);
   }
 }
 
 template <typename SrcT>
 cudaError_t launch_quant_k(const void* src, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
-                           uint8_t* codes, float* scale, float* partials, DeviceInfo& d,
+                           uint8_t* codes, float* scale, float* partials, const uint8_t* neg, DeviceInfo& d,
                            cudaStream_t st) {
   switch (k) {
-    case 16: return launch_quant<SrcT, 16>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
-    case 32: return launch_quant<SrcT, 32>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
-    case 64: return launch_quant<SrcT, 64>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
-    case 128: return launch_quant<SrcT, 128>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
-    default: return launch_quant<SrcT, 256>(src, rows, cols, dim, fmt, codes, scale, partials, d, st);
+    case 16: return launch_quant<SrcT, 16>(src, rows, cols, dim, fmt, codes, scale, partials, neg, d, st);
+    case 32: return launch_quant<SrcT, 32>(src, rows, cols, dim, fmt, codes, scale, partials, neg, d, st);
+    case 64: return launch_quant<SrcT, 64>(src, rows, cols, dim, fmt, codes, scale, partials, neg, d, st);
+    case 128: return launch_quant<SrcT, 128>(src, rows, cols, dim, fmt, codes, scale, partials, neg, d, st);
+    default: return launch_quant<SrcT, 256>(src, rows, cols, dim, fmt, codes, scale, partials, neg, d, st);
   }
 }
 
@@ -352,15 +375,15 @@ hq_status check_quant_args(const void* src, hq_dtype dt, int64_t rows, int64_t c
 
 hq_status quantize_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
                         hq_fmt fmt, void* codes, float* scale, float* partials, DeviceInfo& d,
-                        cudaStream_t st) {
+                        cudaStream_t st, const uint8_t* neg = nullptr) {
   if (rows == 0 || cols == 0) {
     set_scale_one_kernel<<<1, 1, 0, st>>>(scale);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? HQ_OK : cuda_fail(e);
   }
   cudaError_t e = (dt == HQ_BF16)
-                      ? launch_quant_k<__nv_bfloat16>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, d, st)
-                      : launch_quant_k<float>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, d, st);
+                      ? launch_quant_k<__nv_bfloat16>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, neg, d, st)
+                      : launch_quant_k<float>(src, rows, cols, dim, k, fmt, static_cast<uint8_t*>(codes), scale, partials, neg, d, st);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -724,7 +747,7 @@ hq_status check_dual_args(const void* src, hq_dtype dt, int64_t rows, int64_t co
 
 hq_status dual_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt, void* codes_c,
                     float* scale_c, void* codes_r, float* scale_r, float* part_c, float* part_r, DeviceInfo& d,
-                    cudaStream_t st) {
+                    cudaStream_t st, const uint8_t* neg_c = nullptr, const uint8_t* neg_r = nullptr) {
   if (rows == 0 || cols == 0) {
     set_scale_one_kernel<<<1, 1, 0, st>>>(scale_c);
     set_scale_one_kernel<<<1, 1, 0, st>>>(scale_r);
@@ -734,10 +757,10 @@ hq_status dual_impl(const void* src, hq_dtype dt, int64_t rows, int64_t cols, in
   uint8_t* cc = static_cast<uint8_t*>(codes_c);
   uint8_t* cr = static_cast<uint8_t*>(codes_r);
   if (dt == HQ_BF16 && fused_dual_ok(rows, cols))
-    return launch_dual_fused_k(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st);
+    return launch_dual_fused_k(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, neg_c, neg_r, d, st);
   cudaError_t e = dt == HQ_BF16
-                      ? launch_dual_k<__nv_bfloat16>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st)
-                      : launch_dual_k<float>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, d, st);
+                      ? launch_dual_k<__nv_bfloat16>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, neg_c, neg_r, d, st)
+                      : launch_dual_k<float>(src, rows, cols, k, fmt, cc, scale_c, cr, scale_r, part_c, part_r, neg_c, neg_r, d, st);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -897,11 +920,12 @@ extern "C" {
 
 size_t hq_quantize_workspace_bytes(void) { return kPartialBytes; }
 
-hq_status hq_quantize(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
-                      hq_fmt fmt, void* codes, float* scale, void* workspace, size_t ws_bytes,
-                      hq_stream_t stream) {
+hq_status hq_quantize_rht(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
+                          const uint8_t* neg, void* codes, float* scale, void* workspace, size_t ws_bytes,
+                          hq_stream_t stream) {
   hq_status s = check_quant_args(src, dt, rows, cols, dim, k, fmt, codes, scale);
   if (s != HQ_OK) return s;
+  if (neg && !aligned16(neg)) return HQ_ERR_ALIGN;
   if (rows > 0 && cols > 0) {
     if (!workspace || ws_bytes < kPartialBytes) return HQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return HQ_ERR_ALIGN;
@@ -909,7 +933,13 @@ hq_status hq_quantize(const void* src, hq_dtype dt, int64_t rows, int64_t cols, 
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   return quantize_impl(src, dt, rows, cols, dim, k, fmt, codes, scale, static_cast<float*>(workspace), *d,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       reinterpret_cast<cudaStream_t>(stream), neg);
+}
+
+hq_status hq_quantize(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                      hq_fmt fmt, void* codes, float* scale, void* workspace, size_t ws_bytes,
+                      hq_stream_t stream) {
+  return hq_quantize_rht(src, dt, rows, cols, dim, k, fmt, nullptr, codes, scale, workspace, ws_bytes, stream);
 }
 
 hq_status hq_gemm(const void* A, const float* scale_a, const void* B, const float* scale_b, int64_t M,
@@ -950,11 +980,13 @@ hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, int64_t M
 
 size_t hq_quantize_dual_workspace_bytes(void) { return 2 * kPartialBytes; }
 
-hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
-                           void* codes_c, float* scale_c, void* codes_r, float* scale_r, void* workspace,
-                           size_t ws_bytes, hq_stream_t stream) {
+hq_status hq_quantize_dual_rht(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
+                               const uint8_t* neg_c, const uint8_t* neg_r, void* codes_c, float* scale_c,
+                               void* codes_r, float* scale_r, void* workspace, size_t ws_bytes,
+                               hq_stream_t stream) {
   hq_status s = check_dual_args(src, dt, rows, cols, k, fmt, codes_c, scale_c, codes_r, scale_r);
   if (s != HQ_OK) return s;
+  if ((neg_c && !aligned16(neg_c)) || (neg_r && !aligned16(neg_r))) return HQ_ERR_ALIGN;
   if (rows > 0 && cols > 0) {
     if (!workspace || ws_bytes < 2 * kPartialBytes) return HQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return HQ_ERR_ALIGN;
@@ -963,7 +995,14 @@ hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t c
   if ((s = device_info(&d)) != HQ_OK) return s;
   float* part = static_cast<float*>(workspace);
   return dual_impl(src, dt, rows, cols, k, fmt, codes_c, scale_c, codes_r, scale_r, part, part + kMaxPartials,
-                   *d, reinterpret_cast<cudaStream_t>(stream));
+                   *d, reinterpret_cast<cudaStream_t>(stream), neg_c, neg_r);
+}
+
+hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
+                           void* codes_c, float* scale_c, void* codes_r, float* scale_r, void* workspace,
+                           size_t ws_bytes, hq_stream_t stream) {
+  return hq_quantize_dual_rht(src, dt, rows, cols, k, fmt, nullptr, nullptr, codes_c, scale_c, codes_r, scale_r,
+                              workspace, ws_bytes, stream);
 }
 
 size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -971,11 +1010,14 @@ size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   return step_ws_bytes(M, K, N);
 }
 
-hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt, int64_t M, int64_t K,
-                            int64_t N, int k, hq_fmt fmt, void* Y, void* dX, void* dW, void* workspace,
-                            size_t ws_bytes, hq_stream_t stream) {
+hq_status hq_linear_fwd_bwd_rht(const void* X, const void* W, const void* dY, hq_dtype dt, int64_t M, int64_t K,
+                                int64_t N, int k, hq_fmt fmt, const uint8_t* neg_k, const uint8_t* neg_n,
+                                const uint8_t* neg_m, void* Y, void* dX, void* dW, void* workspace,
+                                size_t ws_bytes, hq_stream_t stream) {
   hq_status s = check_step_shape(dt, M, K, N, k, fmt);
   if (s != HQ_OK) return s;
+  if ((neg_k && !aligned16(neg_k)) || (neg_n && !aligned16(neg_n)) || (neg_m && !aligned16(neg_m)))
+    return HQ_ERR_ALIGN;
   if (!X || !W || !dY || !Y || !dX || !dW) return HQ_ERR_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || !aligned16(Y) || !aligned16(dX) || !aligned16(dW))
     return HQ_ERR_ALIGN;
@@ -994,16 +1036,16 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
   if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
   // side stream: the rotations only the backward GEMMs need, alongside the forward operands
   // and GEMM: dY in both rotations (one read per pass), W along N, X along M
-  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.dyq, sc + 4, w.dyqt, sc + 5, w.spart_c, w.spart_r, *d, ss->s)) !=
-      HQ_OK)
+  if ((s = dual_impl(dY, dt, M, N, k, fmt, w.dyq, sc + 4, w.dyqt, sc + 5, w.spart_c, w.spart_r, *d, ss->s, neg_n,
+                     neg_m)) != HQ_OK)
     return s;
-  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.spart_c, *d, ss->s)) != HQ_OK) return s;
-  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.spart_c, *d, ss->s)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.spart_c, *d, ss->s, neg_n)) != HQ_OK) return s;
+  if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.spart_c, *d, ss->s, neg_m)) != HQ_OK) return s;
   if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
   // caller's stream: the forward operands (X and W along K) first, so the forward GEMM starts
   // as early as possible, then the backward GEMMs once the side stream's codes have landed
-  if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st)) != HQ_OK) return s;
-  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.wq, sc + 2, w.part_c, *d, st)) != HQ_OK) return s;
+  if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st, neg_k)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.wq, sc + 2, w.part_c, *d, st, neg_k)) != HQ_OK) return s;
   if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split, w.split_len)) !=
       HQ_OK)
     return s;
@@ -1012,6 +1054,13 @@ hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dty
                      w.split_len)) != HQ_OK)
     return s;
   return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split, w.split_len);
+}
+
+hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt, int64_t M, int64_t K,
+                            int64_t N, int k, hq_fmt fmt, void* Y, void* dX, void* dW, void* workspace,
+                            size_t ws_bytes, hq_stream_t stream) {
+  return hq_linear_fwd_bwd_rht(X, W, dY, dt, M, K, N, k, fmt, nullptr, nullptr, nullptr, Y, dX, dW, workspace,
+                               ws_bytes, stream);
 }
 
 size_t hq_linear_fwd_save_workspace_bytes(int64_t M, int64_t K, int64_t N) {

@@ -141,5 +141,12 @@ def tiny_random(shape, seed: int, dist: str = "normal", scale: float = 1.0) -> n
     return v.astype(np.float32)
 
 
+def sign_flags(n: int, seed: int) -> np.ndarray:
+    """Seeded random sign flags for the randomized Hadamard variant: n bytes, each 0 or 1 with
+    probability 1/2 (a Rademacher diagonal D = diag(1 - 2 * flags))."""
+    r = np.random.default_rng(np.random.SeedSequence([seed, 1 << 20, n]))
+    return r.integers(0, 2, size=n).astype(np.uint8)
+
+
 def layer_list(w: Workload) -> List[Layer]:
     return list(w.layers)

@@ -180,6 +180,39 @@ HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY,
                                    hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Randomized Hadamard variant: a sign diagonal D applied before the blocks, t = H_k D x
+ * (the randomized Hadamard transform of the neighbouring methods listed beside the pages'
+ * subject, e.g. QuIP#'s incoherence processing; the two source pages use plain H).  D is
+ * given per rotated dimension as device arrays of one byte per position, bit 0 set = that
+ * position is negated (an exact sign flip of the source before the same fp32 butterflies).
+ * Both operands of a GEMM must use the same D along its contraction dimension; D^2 = I then
+ * cancels in the product exactly like H.  The flags are the caller's random draws (the
+ * library draws nothing).  A NULL vector is the plain rotation (all flags clear).
+ *   neg arrays: 16-byte aligned (HQ_ERR_ALIGN), length = the rotated dimension (not checked).
+ *
+ * hq_quantize_rht      -- hq_quantize with flags `neg` over the rotated dimension (cols for
+ *                         dim = 1, rows for dim = 0).
+ * hq_quantize_dual_rht -- hq_quantize_dual with flags neg_c over the columns (for codes_c)
+ *                         and neg_r over the rows (for codes_r).
+ * hq_linear_fwd_bwd_rht -- hq_linear_fwd_bwd with one sign vector per contraction dimension:
+ *                         neg_k [K] (X and W for the forward GEMM), neg_n [N] (dY and W for
+ *                         dX), neg_m [M] (dY and X for dW).
+ * Errors, workspaces and launches as for the plain calls.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_quantize_rht(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim,
+                                 int k, hq_fmt fmt, const uint8_t* neg, void* codes, float* scale,
+                                 void* workspace, size_t ws_bytes, hq_stream_t stream);
+HQ_API hq_status hq_quantize_dual_rht(const void* src, hq_dtype dt, int64_t rows, int64_t cols,
+                                      int k, hq_fmt fmt, const uint8_t* neg_c, const uint8_t* neg_r,
+                                      void* codes_c, float* scale_c, void* codes_r, float* scale_r,
+                                      void* workspace, size_t ws_bytes, hq_stream_t stream);
+HQ_API hq_status hq_linear_fwd_bwd_rht(const void* X, const void* W, const void* dY, hq_dtype dt,
+                                       int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt,
+                                       const uint8_t* neg_k, const uint8_t* neg_n,
+                                       const uint8_t* neg_m, void* Y, void* dX, void* dW,
+                                       void* workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Training flow with saved codes ("HALO" Approach: the quantized rotated tensors are kept for
  * the backward pass instead of the bf16 activation, which halves the activation memory).
  *

@@ -257,24 +257,29 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 # ------------------------------------------------------------------------------- the layer
 
-def _gemm_layer(a_src, a_dim, b_src, b_dim, k, fmt, rows=None):
-    qa, sa = quantize(a_src, a_dim, k, fmt)
-    qb, sb = quantize(b_src, b_dim, k, fmt)
+def _gemm_layer(a_src, a_dim, b_src, b_dim, k, fmt, rows=None, neg=None):
+    # neg: optional sign flags of the randomized variant over the contraction dimension, the
+    # same D for both operands (D^2 = I cancels in the product like H)
+    qa, sa = quantize(a_src, a_dim, k, fmt, neg=neg)
+    qb, sb = quantize(b_src, b_dim, k, fmt, neg=neg)
     acc = gemm(qa, qb, fmt, rows)
     ref, fast = epilogue(acc, sa, sb)
     return dict(qa=qa, sa=sa, qb=qb, sb=sb, acc=acc, ref=ref, fast=fast)
 
 
-def linear_fwd(X, W, k, fmt, rows=None):
-    """Y[M][N] = (X H)(W H)^T, both operands rotated along K (HALO right-hand rotation)."""
-    return _gemm_layer(X, 1, W, 1, k, fmt, rows)
+def linear_fwd(X, W, k, fmt, rows=None, neg=None):
+    """Y[M][N] = (X H)(W H)^T, both operands rotated along K (HALO right-hand rotation).
+    neg: optional sign flags over K (randomized variant, (X D H)(W D H)^T)."""
+    return _gemm_layer(X, 1, W, 1, k, fmt, rows, neg)
 
 
-def linear_bwd_dx(dY, W, k, fmt, rows=None):
-    """dX[M][K] = dY W: dY rotated along N (its columns), W rotated along N (its rows)."""
-    return _gemm_layer(dY, 1, W, 0, k, fmt, rows)
+def linear_bwd_dx(dY, W, k, fmt, rows=None, neg=None):
+    """dX[M][K] = dY W: dY rotated along N (its columns), W rotated along N (its rows).
+    neg: optional sign flags over N."""
+    return _gemm_layer(dY, 1, W, 0, k, fmt, rows, neg)
 
 
-def linear_bwd_dw(dY, X, k, fmt, rows=None):
-    """dW[N][K] = dY^T X: both rotated along the token dimension M (HALO-2 left-hand)."""
-    return _gemm_layer(dY, 0, X, 0, k, fmt, rows)
+def linear_bwd_dw(dY, X, k, fmt, rows=None, neg=None):
+    """dW[N][K] = dY^T X: both rotated along the token dimension M (HALO-2 left-hand).
+    neg: optional sign flags over M."""
+    return _gemm_layer(dY, 0, X, 0, k, fmt, rows, neg)

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import hadamard_rotated_precision_b200 as hq
@@ -201,3 +202,35 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(hq, "LIB_PATH", str(tmp_path / "libhq.so"))
     with pytest.raises(ImportError):
         hq.lib()
+
+
+def test_rht_argument_errors(L):
+    """The randomized variant's entry points: the plain checks, plus 16-byte-aligned flags."""
+    q = lambda **kw: L.hq_quantize_rht(kw.get("src", FAKE), hq.HQ_BF16, 256, 256, kw.get("dim", 1), 64, 0,
+                                       kw.get("neg", FAKE), FAKE, FAKE, FAKE, 1 << 20, None)
+    assert q(neg=FAKE_MIS) == 4
+    assert q(dim=2) == 1
+    assert q(src=None) == 1
+    dq = lambda **kw: L.hq_quantize_dual_rht(FAKE, hq.HQ_BF16, 256, kw.get("cols", 256), 64, 0,
+                                             kw.get("nc", FAKE), kw.get("nr", FAKE), FAKE, FAKE, FAKE, FAKE,
+                                             FAKE, 1 << 20, None)
+    assert dq(nc=FAKE_MIS) == 4
+    assert dq(nr=FAKE_MIS) == 4
+    assert dq(cols=96) == 2
+    f = lambda **kw: L.hq_linear_fwd_bwd_rht(FAKE, FAKE, FAKE, hq.HQ_BF16, 256, 512, 256, 64, 0,
+                                             kw.get("nk", FAKE), kw.get("nn", FAKE), kw.get("nm", FAKE),
+                                             FAKE, FAKE, FAKE, FAKE, kw.get("wsb", 1 << 34), None)
+    assert f(nk=FAKE_MIS) == 4
+    assert f(nn=FAKE_MIS) == 4
+    assert f(nm=FAKE_MIS) == 4
+    assert f(wsb=1000) == 8
+
+
+def test_sign_flag_draws():
+    """The randomized variant's flags are seeded draws of 0/1 (about half set), reproducible."""
+    from hadamard_rotated_precision_b200 import synthetic
+    a = synthetic.sign_flags(4096, 9)
+    assert a.dtype == np.uint8 and set(np.unique(a)) <= {0, 1}
+    assert 0.45 < a.mean() < 0.55
+    assert np.array_equal(a, synthetic.sign_flags(4096, 9))
+    assert not np.array_equal(a, synthetic.sign_flags(4096, 10))

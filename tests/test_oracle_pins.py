@@ -485,3 +485,25 @@ def test_synthetic_prefix_and_reproducible():
     assert len(full["outlier_cols"]) == 4   # 0.5% of 768
     assert len(synthetic.draw_fp32(w, 1, M=4)["outlier_cols"]) == 15   # 0.5% of 3072
     assert len(synthetic.draw_fp32(synthetic.WORKLOADS[1])["outlier_cols"]) == 4
+
+
+def test_signed_layer_wiring(oracle_lib):
+    """The layer with sign flags over each contraction dimension still tracks the unquantized
+    product (the same D on both operands cancels); giving the two operands different flags
+    does not."""
+    from hadamard_rotated_precision_b200 import synthetic
+    w = synthetic.WORKLOADS[1]
+    d = synthetic.draw_fp32(w)
+    X, W, dY = d["X"].astype(np.float64), d["W"].astype(np.float64), d["dY"].astype(np.float64)
+    k = w.k
+    for name, fn, a, b, want, n in (("fwd", oracle.linear_fwd, d["X"], d["W"], X @ W.T, X.shape[1]),
+                                    ("dx", oracle.linear_bwd_dx, d["dY"], d["W"], dY @ W, W.shape[0]),
+                                    ("dw", oracle.linear_bwd_dw, d["dY"], d["X"], dY.T @ X, X.shape[0])):
+        neg = synthetic.sign_flags(n, 3)
+        got = oracle.bf16_bits_to_f32(fn(a, b, k, oracle.INT8, neg=neg)["ref"]).astype(np.float64)
+        assert np.linalg.norm(got - want) / np.linalg.norm(want) < 0.1, name
+    neg = synthetic.sign_flags(X.shape[1], 3)
+    qa, sa = oracle.quantize(d["X"], 1, k, oracle.INT8, neg=neg)
+    qb, sb = oracle.quantize(d["W"], 1, k, oracle.INT8, neg=1 - neg)
+    acc = oracle.gemm(qa, qb, oracle.INT8).astype(np.float64) * float(sa) * float(sb)
+    assert np.linalg.norm(acc - X @ W.T) / np.linalg.norm(X @ W.T) > 0.5
