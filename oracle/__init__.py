@@ -34,6 +34,8 @@ _SRC = os.path.join(_HERE, "hq_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libhq_oracle.so")
 
 INT8, FP8_E4M3 = 0, 1
+FP6_E3M2, FP6_E2M3, FP4_E2M1 = 2, 3, 4  # minifloats below FP8 (one code per byte, low bits)
+MINIFLOATS = (FP6_E3M2, FP6_E2M3, FP4_E2M1)
 F32, BF16 = 0, 1
 
 OK, ERR_ARG, ERR_SHAPE, ERR_NONFINITE = 0, 1, 2, 5
@@ -84,6 +86,14 @@ def lib():
         L.hq_oracle_gemm_i8.restype = None
         L.hq_oracle_gemm_f8.argtypes = [p, p, i64, i64, i64, p, i64, p]
         L.hq_oracle_gemm_f8.restype = None
+        L.hq_oracle_gemm_fp.argtypes = [i32, p, p, i64, i64, i64, p, i64, p]
+        L.hq_oracle_gemm_fp.restype = None
+        L.hq_oracle_minifloat_max.argtypes = [i32]
+        L.hq_oracle_minifloat_max.restype = ctypes.c_double
+        L.hq_oracle_minifloat_decode.argtypes = [i32, ctypes.c_uint8]
+        L.hq_oracle_minifloat_decode.restype = ctypes.c_double
+        L.hq_oracle_minifloat_encode.argtypes = [i32, ctypes.c_float]
+        L.hq_oracle_minifloat_encode.restype = ctypes.c_uint8
         L.hq_oracle_epilogue.argtypes = [p, i32, i64, ctypes.c_float, ctypes.c_float, p, p]
         L.hq_oracle_epilogue.restype = None
         L.hq_oracle_threads.argtypes = []
@@ -178,6 +188,23 @@ def quantize(x: np.ndarray, dim: int, k: int, fmt: int, neg=None):
     return codes, np.float32(scale[0])
 
 
+def minifloat_max(fmt: int) -> float:
+    return lib().hq_oracle_minifloat_max(fmt)
+
+
+def minifloat_decode(fmt: int, code: int) -> float:
+    return lib().hq_oracle_minifloat_decode(fmt, code)
+
+
+def minifloat_encode(fmt: int, x: float) -> int:
+    return lib().hq_oracle_minifloat_encode(fmt, float(x))
+
+
+def minifloat_bits(fmt: int) -> int:
+    """Bits of a code of the format (sign included): 6 for FP6, 4 for FP4."""
+    return 4 if fmt == FP4_E2M1 else 6
+
+
 def e4m3_decode(code: int) -> float:
     return lib().hq_oracle_e4m3_decode(code)
 
@@ -208,7 +235,8 @@ def bf16_from_f32(v: float) -> int:
 def gemm(A: np.ndarray, B: np.ndarray, fmt: int, rows=None) -> np.ndarray:
     """C[i][j] = sum_l A[i][l] B[j][l] over codes (both operands contraction-innermost).
 
-    INT8: int32 accumulators.  FP8: exact fp64 accumulators.  `rows` selects rows of A."""
+    INT8: int32 accumulators.  FP8 / FP6 / FP4: exact fp64 accumulators.  `rows` selects
+    rows of A."""
     A = np.ascontiguousarray(A)
     B = np.ascontiguousarray(B)
     M, K = A.shape
@@ -226,7 +254,7 @@ def gemm(A: np.ndarray, B: np.ndarray, fmt: int, rows=None) -> np.ndarray:
                                 R, _ptr(C))
     else:
         C = np.empty((R, N), dtype=np.float64)
-        lib().hq_oracle_gemm_f8(_ptr(A.view(np.uint8)), _ptr(B.view(np.uint8)), M, N, K, rp,
+        lib().hq_oracle_gemm_fp(int(fmt), _ptr(A.view(np.uint8)), _ptr(B.view(np.uint8)), M, N, K, rp,
                                 R, _ptr(C))
     return C
 

@@ -25,6 +25,11 @@
  *  - INT8: inv = fp32(127/a), q = clamp(rne(fp32(y*inv)), -127, 127), scale = fp32(a/127).
  *  - FP8 e4m3 (E4M3FN, bias 7, max 448, no infinities): inv = fp32(448/a),
  *    q = e4m3 nearest-even of fp32(y*inv) saturated to +-448, scale = fp32(a/448).
+ *  - FP6 / FP4 (the formats HALO names below FP8; the pages give no bit layout): the
+ *    minifloats e3m2 (bias 3, max 28), e2m3 (bias 1, max 7.5) and e2m1 (bias 1, max 6),
+ *    sign-magnitude, subnormals, no infinities or NaN; inv = fp32(max/a), q = nearest-even
+ *    of fp32(y*inv) saturated to +-max, scale = fp32(a/max); one code per byte, value in the
+ *    low 6 (4) bits.
  *  - a = 0 gives scale 1 and all-zero codes; a non-finite a is an error.
  *  - Codes are stored with the rotated dimension innermost (K-major for the GEMM).
  *
@@ -117,6 +122,57 @@ uint8_t hq_oracle_e4m3_encode(float x) {
     return sign | (uint8_t)(((lead + 7) << 3) | m);
 }
 
+/* ---------------------------------------------------------------- FP6 / FP4 minifloats */
+
+/* Format parameters by code: fmt 2 = e3m2, 3 = e2m3, 4 = e2m1 (exponent bits, mantissa bits,
+ * bias).  Returns 0 for any other fmt. */
+static int minifloat_params(int fmt, int* ebits, int* mbits, int* bias) {
+    switch (fmt) {
+        case 2: *ebits = 3; *mbits = 2; *bias = 3; return 1;
+        case 3: *ebits = 2; *mbits = 3; *bias = 1; return 1;
+        case 4: *ebits = 2; *mbits = 1; *bias = 1; return 1;
+        default: return 0;
+    }
+}
+
+/* Largest finite value: all exponent and mantissa bits set (there are no infinities). */
+double hq_oracle_minifloat_max(int fmt) {
+    int eb, mb, bias;
+    if (!minifloat_params(fmt, &eb, &mb, &bias)) return NAN;
+    return ldexp(2.0 - ldexp(1.0, -mb), (1 << eb) - 1 - bias);
+}
+
+/* Decode from the bit definition: s | e (eb bits) | m (mb bits); e = 0 is subnormal,
+ * m * 2^(1 - bias - mb); otherwise (1 + m / 2^mb) * 2^(e - bias).  Bits above the sign are
+ * ignored. */
+double hq_oracle_minifloat_decode(int fmt, uint8_t c) {
+    int eb, mb, bias;
+    if (!minifloat_params(fmt, &eb, &mb, &bias)) return NAN;
+    int s = (c >> (eb + mb)) & 1, e = (c >> mb) & ((1 << eb) - 1), m = c & ((1 << mb) - 1);
+    double v = e == 0 ? ldexp((double)m, 1 - bias - mb) : ldexp(1.0 + ldexp((double)m, -mb), e - bias);
+    return s ? -v : v;
+}
+
+/* fp32 -> code, nearest with ties to even, saturating to +-max; the sign of zero is kept. */
+uint8_t hq_oracle_minifloat_encode(int fmt, float x) {
+    int eb, mb, bias;
+    if (!minifloat_params(fmt, &eb, &mb, &bias)) return 0;
+    const uint8_t sign = (x < 0 || (x == 0 && signbit(x))) ? (uint8_t)(1u << (eb + mb)) : 0;
+    const uint8_t maxcode = (uint8_t)((1u << (eb + mb)) - 1);
+    const double mx = hq_oracle_minifloat_max(fmt), emin = 1 - bias;
+    double a = fabs((double)x);
+    if (a >= mx) return sign | maxcode;
+    double r = round_to_format(a, mb + 1, (int)emin);
+    if (r >= mx) return sign | maxcode;
+    if (r == 0.0) return sign;
+    int e;
+    frexp(r, &e);
+    int lead = e - 1;
+    if (lead < emin) return sign | (uint8_t)(int)ldexp(r, bias - 1 + mb); /* subnormal */
+    int m = (int)ldexp(ldexp(r, -lead) - 1.0, mb);
+    return sign | (uint8_t)(((lead + bias) << mb) | m);
+}
+
 /* ---------------------------------------------------------------- Hadamard */
 
 /* In-place Sylvester FWHT of one block of length k: for h = 1, 2, ..., k/2, every pair
@@ -194,10 +250,11 @@ static float absmax(const float* y, int64_t n) {
     return bad ? INFINITY : a;
 }
 
-/* Quantize already-rotated values y[n] tensor-wise.  fmt 0 = INT8, 1 = FP8 e4m3.
- * Writes n one-byte codes and the fp32 dequantization scale. */
+/* Quantize already-rotated values y[n] tensor-wise.  fmt 0 = INT8, 1 = FP8 e4m3,
+ * 2 = FP6 e3m2, 3 = FP6 e2m3, 4 = FP4 e2m1.  Writes n one-byte codes and the fp32
+ * dequantization scale. */
 int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* codes, float* scale) {
-    if (fmt != 0 && fmt != 1) return ORC_ERR_ARG;
+    if (fmt < 0 || fmt > 4) return ORC_ERR_ARG;
     float a = absmax(y, n);
     if (!isfinite(a)) {
         *scale = NAN;
@@ -208,7 +265,7 @@ int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* code
         *scale = 1.0f;
         return ORC_OK;
     }
-    float qmax = fmt == 0 ? 127.0f : 448.0f;
+    float qmax = fmt == 0 ? 127.0f : fmt == 1 ? 448.0f : (float)hq_oracle_minifloat_max(fmt);
     float inv = qmax / a;
     *scale = a / qmax;
     for (int64_t i = 0; i < n; ++i) {
@@ -218,8 +275,10 @@ int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* code
             if (r > 127.0f) r = 127.0f;
             if (r < -127.0f) r = -127.0f;
             codes[i] = (uint8_t)(int8_t)(int)r;
-        } else {
+        } else if (fmt == 1) {
             codes[i] = hq_oracle_e4m3_encode(z);
+        } else {
+            codes[i] = hq_oracle_minifloat_encode(fmt, z);
         }
     }
     return ORC_OK;
@@ -265,11 +324,13 @@ void hq_oracle_gemm_i8(const int8_t* A, const int8_t* B, int64_t M, int64_t N, i
     }
 }
 
-/* Same contraction for e4m3 codes, each decoded exactly to double, fp64 accumulation. */
-void hq_oracle_gemm_f8(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K,
+/* Same contraction for floating-point codes (fmt 1 = e4m3, 2..4 = FP6 / FP4), each decoded
+ * exactly to double, fp64 accumulation (exact for these formats at the sizes tested). */
+void hq_oracle_gemm_fp(int fmt, const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K,
                        const int64_t* rows, int64_t nrows, double* C) {
     double lut[256];
-    for (int c = 0; c < 256; ++c) lut[c] = hq_oracle_e4m3_decode((uint8_t)c);
+    for (int c = 0; c < 256; ++c)
+        lut[c] = fmt == 1 ? hq_oracle_e4m3_decode((uint8_t)c) : hq_oracle_minifloat_decode(fmt, (uint8_t)c);
     int64_t R = rows ? nrows : M;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < R; ++r) {
@@ -281,6 +342,11 @@ void hq_oracle_gemm_f8(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N,
             C[r * N + j] = s;
         }
     }
+}
+
+void hq_oracle_gemm_f8(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K,
+                       const int64_t* rows, int64_t nrows, double* C) {
+    hq_oracle_gemm_fp(1, A, B, M, N, K, rows, nrows, C);
 }
 
 /* ---------------------------------------------------------------- dequantization epilogue */

@@ -357,6 +357,112 @@ def test_fp8_quantizer_absmax_maps_to_448(oracle_lib):
     assert rel.max() <= 2 ** -4 * (1 + 1e-6)   # half of e4m3's 2^-3 relative spacing
 
 
+# ------------------------------------------------------------------------- FP6 / FP4
+
+# (fmt, exponent bits, mantissa bits): the minifloats below FP8 that HALO names (FP6) plus
+# FP4; sign-magnitude with subnormals and no infinities or NaN.
+MINIS = [(oracle.FP6_E3M2, 3, 2), (oracle.FP6_E2M3, 2, 3), (oracle.FP4_E2M1, 2, 1)]
+
+
+def _mini_table(fmt):
+    return [oracle.minifloat_decode(fmt, c) for c in range(1 << oracle.minifloat_bits(fmt))]
+
+
+@pytest.mark.parametrize("fmt,eb,mb", MINIS)
+def test_minifloat_value_structure(oracle_lib, fmt, eb, mb):
+    """Positive codes decode strictly increasing from 0; the sign bit negates; the spacing is
+    constant within each binade of 2^mb values and doubles from one binade to the next (the
+    subnormals share the first normal binade's spacing)."""
+    t = _mini_table(fmt)
+    half = len(t) // 2
+    pos = t[:half]
+    assert pos[0] == 0.0 and all(b > a for a, b in zip(pos, pos[1:]))
+    for c in range(half):
+        assert t[c + half] == -t[c]
+    steps = [b - a for a, b in zip(pos, pos[1:])]
+    n = 1 << mb
+    for i, st in enumerate(steps):  # step from code i to i + 1
+        assert st == steps[0] * 2 ** max(0, i // n - 1), (fmt, i)
+    assert oracle.minifloat_max(fmt) == pos[-1]
+
+
+def test_minifloat_spec_points(oracle_lib):
+    """Closed forms: e2m1 is exactly {0, 0.5, 1, 1.5, 2, 3, 4, 6}; e2m3 tops out at 7.5 with
+    smallest subnormal 1/8; e3m2 tops out at 28 with smallest subnormal 1/16."""
+    assert _mini_table(oracle.FP4_E2M1)[:8] == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    t = _mini_table(oracle.FP6_E2M3)
+    assert (t[1], t[31], t[8]) == (0.125, 7.5, 1.0)
+    t = _mini_table(oracle.FP6_E3M2)
+    assert (t[1], t[31], t[4]) == (0.0625, 28.0, 0.25)
+
+
+def _mini_nearest_even(x, fmt):
+    t = _mini_table(fmt)
+    half = len(t) // 2
+    a = abs(x)
+    best = min(range(half), key=lambda c: abs(t[c] - a))
+    d = abs(t[best] - a)
+    ties = [c for c in range(half) if abs(t[c] - a) == d]
+    if len(ties) > 1:
+        best = [c for c in ties if c % 2 == 0][0]
+    if a > t[half - 1]:
+        best = half - 1
+    sign = half if (x < 0 or (x == 0 and math.copysign(1, x) < 0)) else 0
+    return best | sign
+
+
+@pytest.mark.parametrize("fmt,eb,mb", MINIS)
+def test_minifloat_encode_bruteforce_and_ties(oracle_lib, fmt, eb, mb):
+    """Encode = brute-force nearest over every code, ties to the even code, at every code
+    value, every midpoint (exact ties), just beside each midpoint, random values and beyond
+    the maximum (saturation)."""
+    t = _mini_table(fmt)
+    pos = t[: len(t) // 2]
+    vals = list(pos) + [(a + b) / 2 for a, b in zip(pos, pos[1:])]
+    vals += [np.nextafter(np.float32(v), np.float32(100)) for v in vals] + [np.nextafter(np.float32(v), np.float32(-1)) for v in vals]
+    mx = pos[-1]
+    vals += list(np.random.default_rng(41).uniform(0, 1.3 * mx, 300).astype(np.float32)) + [mx * 1.01, mx * 5, 1e30]
+    vals = [float(np.float32(v)) for v in vals]
+    vals += [-v for v in vals] + [-0.0]
+    for v in vals:
+        assert oracle.minifloat_encode(fmt, v) == _mini_nearest_even(v, fmt), (fmt, v)
+
+
+@pytest.mark.parametrize("fmt,eb,mb", MINIS)
+def test_minifloat_quantizer_absmax_and_roundtrip(oracle_lib, fmt, eb, mb):
+    """The absmax element maps to the largest code; every element decodes back to within half
+    a step of its binade (relative 2^-(mb+1), or the subnormal step near zero)."""
+    y = synthetic.tiny_random((48, 40), 7 + fmt, scale=3.0)
+    codes, s = oracle.quantize_rotated(y, fmt)
+    mx = np.float32(oracle.minifloat_max(fmt))
+    a = np.float32(np.abs(y).max())
+    assert s == np.float32(a / mx)
+    i = np.unravel_index(np.abs(y).argmax(), y.shape)
+    half = 1 << (eb + mb)
+    assert codes[i] & (half - 1) == half - 1
+    t = np.array(_mini_table(fmt))
+    dec = t[codes] * float(s)
+    sub_step = t[1] * float(s)
+    err = np.abs(dec - y.astype(np.float64))
+    bound = np.maximum(np.abs(y) * 2.0 ** -(mb + 1), sub_step / 2) * (1 + 1e-6)
+    assert (err <= bound).all()
+    assert (codes < 2 * half).all()
+
+
+@pytest.mark.parametrize("fmt,eb,mb", MINIS)
+def test_gemm_minifloat_exact_rational(oracle_lib, fmt, eb, mb):
+    r = np.random.default_rng(43 + fmt)
+    n = 1 << oracle.minifloat_bits(fmt)
+    A = r.integers(0, n, size=(4, 40)).astype(np.uint8)
+    B = r.integers(0, n, size=(3, 40)).astype(np.uint8)
+    t = _mini_table(fmt)
+    C = oracle.gemm(A, B, fmt)
+    for i in range(4):
+        for j in range(3):
+            exact = sum(Fraction(t[A[i, l]]) * Fraction(t[B[j, l]]) for l in range(40))
+            assert Fraction(C[i, j]) == exact
+
+
 # ------------------------------------------------------------------------- GEMMs
 
 def test_gemm_i8_triple_loop_and_numpy(oracle_lib):
