@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libhq.so")
 
 HQ_OK = 0
 HQ_INT8, HQ_FP8_E4M3 = 0, 1
+HQ_FP6_E3M2, HQ_FP6_E2M3, HQ_FP4_E2M1 = 2, 3, 4
 HQ_F32, HQ_BF16 = 0, 1
 HQ_OUT_BF16, HQ_OUT_ACC = 0, 1
 HQ_MAX_K_INT8 = 133143
@@ -144,10 +145,12 @@ def _src_dtype(t, name: str) -> int:
 
 
 def _fmt(fmt) -> int:
-    if fmt in (HQ_INT8, "int8"):
-        return HQ_INT8
-    if fmt in (HQ_FP8_E4M3, "fp8", "fp8_e4m3"):
-        return HQ_FP8_E4M3
+    names = {"int8": HQ_INT8, "fp8": HQ_FP8_E4M3, "fp8_e4m3": HQ_FP8_E4M3, "fp6_e3m2": HQ_FP6_E3M2,
+             "fp6_e2m3": HQ_FP6_E2M3, "fp4_e2m1": HQ_FP4_E2M1}
+    if isinstance(fmt, str) and fmt in names:
+        return names[fmt]
+    if fmt in (HQ_INT8, HQ_FP8_E4M3, HQ_FP6_E3M2, HQ_FP6_E2M3, HQ_FP4_E2M1):
+        return int(fmt)
     raise ValueError(f"unknown format {fmt!r}")
 
 

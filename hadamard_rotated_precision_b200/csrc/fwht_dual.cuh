@@ -154,21 +154,35 @@ __device__ __forceinline__ void st_global_32B(void* p, uint32_t a, uint32_t b, u
 // Codes of a thread's 64 rotated values, 64 contiguous bytes at dst (W32: two 32-byte stores,
 // each a whole sector; dst 32-byte aligned).
 template <int MODE, bool W32>
-__device__ __forceinline__ void store_codes64(uint8_t* dst, const float2 (&v)[32], const CodeScale& cs, bool zero) {
+__device__ __forceinline__ void store_codes64(uint8_t* dst, const float2 (&v)[32], const CodeScale& cs, bool zero,
+                                              int lp_fmt) {
   uint32_t w[16];
   if (cs.one_mul) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) w[j] = codes4<MODE>(mul2(v[2 * j], cs.ci2), mul2(v[2 * j + 1], cs.ci2));
+    for (int j = 0; j < 16; ++j) w[j] = codes4x<MODE>(mul2(v[2 * j], cs.ci2), mul2(v[2 * j + 1], cs.ci2), lp_fmt);
   } else {
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      w[j] = codes4<MODE>(mul2(mul2(v[2 * j], cs.c2), cs.inv2), mul2(mul2(v[2 * j + 1], cs.c2), cs.inv2));
+      w[j] = codes4x<MODE>(mul2(mul2(v[2 * j], cs.c2), cs.inv2), mul2(mul2(v[2 * j + 1], cs.c2), cs.inv2), lp_fmt);
   }
   if (zero) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) w[j] = 0u;
   }
-  if constexpr (W32) {
+  if constexpr (MODE == kModeLowp) {
+    // minifloats: four 16-code groups, each packed into its 16-byte chunk
+    uint4 ch[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ch[q] = lowp_pack16(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], lp_fmt);
+    if constexpr (W32) {
+      st_global_32B(dst, ch[0].x, ch[0].y, ch[0].z, ch[0].w, ch[1].x, ch[1].y, ch[1].z, ch[1].w);
+      st_global_32B(dst + 32, ch[2].x, ch[2].y, ch[2].z, ch[2].w, ch[3].x, ch[3].y, ch[3].z, ch[3].w);
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) o[q] = ch[q];
+    }
+  } else if constexpr (W32) {
     st_global_32B(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
     st_global_32B(dst + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
   } else {
@@ -189,7 +203,7 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
                   float* __restrict__ part_c, float* __restrict__ part_r, int n_partials,
                   float* __restrict__ scale_c, float* __restrict__ scale_r,
                   unsigned int* __restrict__ status, int reverse,
-                  const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r) {
+                  const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r, int lp_fmt) {
   // SIGNED: sign flags per column (neg_c) and per row (neg_r); either may be null (all clear)
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
@@ -259,8 +273,8 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
   const float c = __frsqrt_rn(static_cast<float>(K));
   QuantParams qc{0.0f, false, false}, qr{0.0f, false, false};
   if constexpr (QUANT) {
-    qc = finish_absmax<MODE>(part_c, n_partials, scale_c, scratch, status);
-    qr = finish_absmax<MODE>(part_r, n_partials, scale_r, scratch, status);
+    qc = finish_absmax<MODE>(part_c, n_partials, scale_c, scratch, status, lp_fmt);
+    qr = finish_absmax<MODE>(part_r, n_partials, scale_r, scratch, status, lp_fmt);
   }
   const int64_t work_tiles = (qc.abort && qr.abort) ? 0 : my_tiles;
 
@@ -339,7 +353,7 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
         rotate64<K, false>(v, lane, 8, 16, amc);
         const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
         const int64_t cc = col0 + kStripCols * sr;
-        if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero);
+        if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero, lp_fmt);
       }
     }
 
@@ -377,7 +391,7 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
         rotate64<K, false>(v, lane, 1, 2, amr);
         const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
         const int64_t gr = row0 + 64 * (lane & 3);
-        if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero);
+        if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero, lp_fmt);
       }
     }
   }

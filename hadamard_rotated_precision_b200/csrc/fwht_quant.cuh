@@ -29,13 +29,20 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+#include <cuda_fp6.h>
+#include <cuda_fp4.h>
 #include "sm100_ptx.cuh"
 #include <cfloat>
 #include <cstdint>
 
 namespace hq {
 
-enum QuantMode : int { kModeAbsmax = 0, kModeInt8 = 1, kModeFp8 = 2 };
+// kModeLowp: the FP6 / FP4 minifloats, the format (2 = e3m2, 3 = e2m3, 4 = e2m1, as the
+// library's format enum) passed at run time as `lp_fmt`.
+enum QuantMode : int { kModeAbsmax = 0, kModeInt8 = 1, kModeFp8 = 2, kModeLowp = 3 };
+
+// Largest finite value of a minifloat format (the QMAX its codes are scaled to).
+__device__ __forceinline__ float lowp_max(int lp_fmt) { return lp_fmt == 2 ? 28.0f : lp_fmt == 3 ? 7.5f : 6.0f; }
 
 constexpr int kQuantThreads = 256;
 
@@ -122,12 +129,21 @@ __device__ __forceinline__ uint32_t code_fp8(float y, float inv) {
   return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fmul_rn(y, inv), __NV_SATFINITE, __NV_E4M3));
 }
 
+// One minifloat code (nearest-even, saturating), value in the low bits of the byte.
+__device__ __forceinline__ uint32_t code_lowp_z(float z, int lp_fmt) {
+  if (lp_fmt == 4) return static_cast<uint32_t>(__nv_cvt_float_to_fp4(z, __NV_E2M1, cudaRoundNearest)) & 0xFu;
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp6(z, lp_fmt == 2 ? __NV_E3M2 : __NV_E2M3, cudaRoundNearest));
+}
+
 template <int MODE>
-__device__ __forceinline__ uint2 codes8(const float (&y)[8], float inv, bool zero) {
+__device__ __forceinline__ uint2 codes8(const float (&y)[8], float inv, bool zero, int lp_fmt = 0) {
   uint32_t b[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    b[i] = zero ? 0u : (MODE == kModeInt8 ? code_int8(y[i], inv) : code_fp8(y[i], inv));
+    b[i] = zero ? 0u
+                : (MODE == kModeInt8 ? code_int8(y[i], inv)
+                   : MODE == kModeFp8 ? code_fp8(y[i], inv)
+                                      : code_lowp_z(__fmul_rn(y[i], inv), lp_fmt));
   return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
                     b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
 }
@@ -168,11 +184,11 @@ struct QuantParams {
 template <int MODE>
 __device__ __forceinline__ QuantParams finish_absmax(const float* partials, int n_partials,
                                                      float* scale_out, float* scratch,
-                                                     unsigned int* status) {
+                                                     unsigned int* status, int lp_fmt = 0) {
   float m = 0.0f;
   for (int i = threadIdx.x; i < n_partials; i += blockDim.x) m = fmaxf(m, partials[i]);
   const float a = block_max(m, scratch);
-  constexpr float QMAX = MODE == kModeInt8 ? 127.0f : 448.0f;
+  const float QMAX = MODE == kModeInt8 ? 127.0f : MODE == kModeFp8 ? 448.0f : lowp_max(lp_fmt);
   QuantParams p;
   p.abort = !(a <= FLT_MAX);
   p.zero = (a == 0.0f);
@@ -270,6 +286,49 @@ __device__ __forceinline__ uint32_t codes4(float2 z0, float2 z1) {
     const uint32_t hi = __nv_cvt_float2_to_fp8x2(z1, __NV_SATFINITE, __NV_E4M3);
     return lo | (hi << 16);
   }
+}
+
+// Codes of 4 consecutive elements for any mode (the minifloats' format at run time).
+template <int MODE>
+__device__ __forceinline__ uint32_t codes4x(float2 z0, float2 z1, int lp_fmt) {
+  if constexpr (MODE != kModeLowp) {
+    return codes4<MODE>(z0, z1);
+  } else {
+    if (lp_fmt == 4) {
+      // two codes per byte from the conversion, one per byte in the layout
+      const uint32_t a = __nv_cvt_float2_to_fp4x2(z0, __NV_E2M1, cudaRoundNearest);
+      const uint32_t b = __nv_cvt_float2_to_fp4x2(z1, __NV_E2M1, cudaRoundNearest);
+      return (a & 0xFu) | ((a & 0xF0u) << 4) | ((b & 0xFu) << 16) | ((b & 0xF0u) << 20);
+    }
+    const __nv_fp6_interpretation_t f = lp_fmt == 2 ? __NV_E3M2 : __NV_E2M3;
+    const uint32_t lo = __nv_cvt_float2_to_fp6x2(z0, f, cudaRoundNearest);
+    const uint32_t hi = __nv_cvt_float2_to_fp6x2(z1, f, cudaRoundNearest);
+    return (lo & 0xFFFFu) | (hi << 16);
+  }
+}
+
+// Tensor-core operand layout of the minifloat codes: each group of 16 consecutive codes along
+// the rotated dimension fills one 16-byte chunk, packed LSB-first (code i in bits
+// [b*i, b*i + b), b = 6 or 4) from byte 0, the rest of the chunk zero; kind::f8f6f4 reads FP6 /
+// FP4 operands from shared memory in this form.
+
+// Codes of 4 consecutive elements (one per byte, low bits) compressed to 24 (FP6) or 16 (FP4)
+// bits, code 0 lowest.
+__device__ __forceinline__ uint32_t lowp_compress4(uint32_t w, int lp_fmt) {
+  if (lp_fmt == 4) return (w & 0xFu) | ((w >> 4) & 0xF0u) | ((w >> 8) & 0xF00u) | ((w >> 12) & 0xF000u);
+  return (w & 0x3Fu) | ((w >> 2) & 0xFC0u) | ((w >> 4) & 0x3F000u) | ((w >> 6) & 0xFC0000u);
+}
+
+// One 16-byte chunk from the compressed codes of 4 consecutive 4-element pieces.
+__device__ __forceinline__ uint4 lowp_chunk(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3, int lp_fmt) {
+  if (lp_fmt == 4) return make_uint4(p0 | (p1 << 16), p2 | (p3 << 16), 0u, 0u);
+  return make_uint4(p0 | (p1 << 24), (p1 >> 8) | (p2 << 16), (p2 >> 16) | (p3 << 8), 0u);
+}
+
+// 16 codes (one per byte in w0..w3) -> their chunk.
+__device__ __forceinline__ uint4 lowp_pack16(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, int lp_fmt) {
+  return lowp_chunk(lowp_compress4(w0, lp_fmt), lowp_compress4(w1, lp_fmt), lowp_compress4(w2, lp_fmt),
+                    lowp_compress4(w3, lp_fmt), lp_fmt);
 }
 
 // ------------------------------------------------------------------ sign flags
@@ -389,7 +448,7 @@ __global__ void __launch_bounds__(kQuantThreads, sizeof(SrcT) == 2 ? 3 : 1)
 fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__ codes,
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
                   unsigned int* __restrict__ status, int reverse, const uint8_t* __restrict__ neg,
-                  int64_t cols) {
+                  int64_t cols, int lp_fmt) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr bool EXCH = K >= 64;
@@ -401,7 +460,7 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
 
   QuantParams qp{0.0f, false, false};
   if (QUANT) {
-    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status);
+    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status, lp_fmt);
     if (qp.abort) return;
   }
   const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
@@ -479,9 +538,30 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          w[j] = qp.zero ? 0u : codes4<MODE>(mul2(mul2(v[2 * j], c2), inv2), mul2(mul2(v[2 * j + 1], c2), inv2));
+          w[j] = qp.zero ? 0u : codes4x<MODE>(mul2(mul2(v[2 * j], c2), inv2), mul2(mul2(v[2 * j + 1], c2), inv2), lp_fmt);
         const bool full = ub + kRowsWarpElems <= n;  // all but a ragged last unit
-        if constexpr (!EXCH) {
+        if constexpr (MODE == kModeLowp) {
+          // minifloats: 16-code groups packed into 16-byte chunks (n is a multiple of 16)
+          if constexpr (!EXCH) {
+            const int64_t e = ub + 32 * lane;
+            if (full || e < n) *reinterpret_cast<uint4*>(codes + e) = lowp_pack16(w[0], w[1], w[2], w[3], lp_fmt);
+            if (full || e + 16 < n)
+              *reinterpret_cast<uint4*>(codes + e + 16) = lowp_pack16(w[4], w[5], w[6], w[7], lp_fmt);
+          } else {
+            // word b of lane l holds codes e0 + 32b + 0..3 with e0 = 4 (l & 7) + ...: a group's
+            // four words sit in lanes 4g .. 4g + 3, gathered into the first of them
+            const int64_t e0 = ub + 256 * (lane >> 3) + 4 * (lane & 7);
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              const uint32_t p = lowp_compress4(w[b], lp_fmt);
+              const uint32_t p1 = __shfl_down_sync(0xFFFFFFFFu, p, 1);
+              const uint32_t p2 = __shfl_down_sync(0xFFFFFFFFu, p, 2);
+              const uint32_t p3 = __shfl_down_sync(0xFFFFFFFFu, p, 3);
+              if ((lane & 3) == 0 && (full || e0 + 32 * b < n))
+                *reinterpret_cast<uint4*>(codes + e0 + 32 * b) = lowp_chunk(p, p1, p2, p3, lp_fmt);
+            }
+          }
+        } else if constexpr (!EXCH) {
           const int64_t e = ub + 32 * lane;
           if (full || e < n) *reinterpret_cast<uint4*>(codes + e) = make_uint4(w[0], w[1], w[2], w[3]);
           if (full || e + 16 < n) *reinterpret_cast<uint4*>(codes + e + 16) = make_uint4(w[4], w[5], w[6], w[7]);
@@ -539,7 +619,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols,
                        uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
                        float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
-                       const uint8_t* __restrict__ neg) {
+                       const uint8_t* __restrict__ neg, int lp_fmt) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   extern __shared__ __align__(128) uint4 tiles[];  // [3][256 rows][8 chunks]
@@ -549,7 +629,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
 
   QuantParams qp{0.0f, false, false};
   if (QUANT) {
-    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status);
+    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status, lp_fmt);
     if (qp.abort) return;
   }
   const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
@@ -646,9 +726,10 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int i = 8 * j + 2 * e;
-                w[e] = qp.zero ? 0u : codes4<MODE>(mul2(mul2(v[i], c2), inv2), mul2(mul2(v[i + 1], c2), inv2));
+                w[e] = qp.zero ? 0u : codes4x<MODE>(mul2(mul2(v[i], c2), inv2), mul2(mul2(v[i + 1], c2), inv2), lp_fmt);
               }
-              *reinterpret_cast<uint4*>(o + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<uint4*>(o + 16 * j) =
+                  MODE == kModeLowp ? lowp_pack16(w[0], w[1], w[2], w[3], lp_fmt) : make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
@@ -669,7 +750,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
                   float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
-                  const uint8_t* __restrict__ neg) {
+                  const uint8_t* __restrict__ neg, int lp_fmt) {
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   static_assert(!SIGNED || sizeof(SrcT) == 4, "sign masks of this kernel are for fp32 words");
   constexpr bool QUANT = MODE != kModeAbsmax;
@@ -682,7 +763,7 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
 
   QuantParams qp{0.0f, false, false};
   if (QUANT) {
-    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status);
+    qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status, lp_fmt);
     if (qp.abort) return;
   }
 
@@ -785,6 +866,22 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
             bad |= !(ay <= FLT_MAX);
             amax = fmaxf(amax, ay);
           }
+      } else if constexpr (MODE == kModeLowp) {
+        // minifloats: lanes 2m and 2m + 1 hold rows 16m .. 16m + 15 of a column, one 16-byte chunk
+        // (rows is a multiple of 16, so both lanes are inside the tensor or both past its end)
+        const int64_t row = r0 + 8 * lane;
+#pragma unroll
+        for (int j = 0; j < CPC; ++j) {
+          const int64_t col = c0 + warp * CPC + j;
+          float y8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y8[i] = v[i][j];
+          const uint2 c8 = codes8<MODE>(y8, qp.inv, qp.zero, lp_fmt);
+          const uint32_t px = lowp_compress4(c8.x, lp_fmt), py = lowp_compress4(c8.y, lp_fmt);
+          const uint32_t qx = __shfl_down_sync(0xFFFFFFFFu, px, 1), qy = __shfl_down_sync(0xFFFFFFFFu, py, 1);
+          if ((lane & 1) == 0 && row < rows && col < cols)
+            __stcs(reinterpret_cast<uint4*>(codes + col * rows + row), lowp_chunk(px, py, qx, qy, lp_fmt));
+        }
       } else {
         const int64_t row = r0 + 8 * lane;
         if (row < rows) {
@@ -795,7 +892,7 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
               float y8[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) y8[i] = v[i][j];
-              __stcs(reinterpret_cast<uint2*>(codes + col * rows + row), codes8<MODE>(y8, qp.inv, qp.zero));
+              __stcs(reinterpret_cast<uint2*>(codes + col * rows + row), codes8<MODE>(y8, qp.inv, qp.zero, lp_fmt));
             }
           }
         }

@@ -158,7 +158,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
             const float* __restrict__ scale_a, const float* __restrict__ scale_b, void* __restrict__ out,
-            int M, int N, int K, unsigned int* __restrict__ status, int skip_first_load) {
+            int M, int N, int K, unsigned int* __restrict__ status, int skip_first_load, uint32_t ab_code) {
   extern __shared__ uint8_t smem_raw[];
   const Shared sh = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,7 +231,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc<FMT>();
+      // ab_code: the A and B element format of kind::f8f6f4 (e4m3 0, e2m3 3, e3m2 4, e2m1 5)
+      const uint32_t idesc = instr_desc<FMT>() | (ab_code << 7) | (ab_code << 10);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -373,7 +374,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
                  unsigned int* __restrict__ status, int splits, uint32_t* __restrict__ part_ws,
-                 int* __restrict__ counters) {
+                 int* __restrict__ counters, uint32_t ab_code) {
   using G = Geo<BN_, SHORT_K>;
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
@@ -458,7 +459,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (CTA 0)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = instr_desc<FMT, BN_>();
+      // ab_code: the A and B element format of kind::f8f6f4 (e4m3 0, e2m3 3, e3m2 4, e2m1 5)
+      const uint32_t idesc = instr_desc<FMT, BN_>() | (ab_code << 7) | (ab_code << 10);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;

@@ -33,9 +33,9 @@ struct DeviceInfo {
   int sms = 0;
   unsigned int* status = nullptr;
   unsigned gemm_attr_set = 0;  // bit per GEMM instantiation
-  unsigned cols_attr_set = 0;  // bit per strided bf16 quantizer instantiation (30 used)
+  bool cols_attr[5][4][2] = {};  // strided bf16 quantizer instantiations prepared [k][mode][signed]
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
-  uint64_t dual_attr_set = 0;  // bit per fused two-rotation quantizer instantiation (60 used)
+  bool dual_attr[5][4][2][2] = {};  // fused two-rotation instantiations prepared [k][mode][w32][signed]
 };
 
 std::mutex g_mu;
@@ -87,6 +87,18 @@ hq_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 }
 
 bool valid_k(int k) { return k == 16 || k == 32 || k == 64 || k == 128 || k == 256; }
+bool valid_fmt(int fmt) {
+  return fmt == HQ_INT8 || fmt == HQ_FP8_E4M3 || fmt == HQ_FP6_E3M2 || fmt == HQ_FP6_E2M3 || fmt == HQ_FP4_E2M1;
+}
+// A/B element format field of the kind::f8f6f4 instruction descriptor (0 for INT8's kind::i8).
+uint32_t ab_format_code(int fmt) {
+  switch (fmt) {
+    case HQ_FP6_E2M3: return 3;
+    case HQ_FP6_E3M2: return 4;
+    case HQ_FP4_E2M1: return 5;
+    default: return 0;
+  }
+}
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -135,13 +147,13 @@ int blocks_per_sm(const void* fn, size_t smem) {
 template <int K, int MODE, bool SIGNED>
 cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
   constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
-  const unsigned bit = 1u << ((kIdx * 3 + MODE) * 2 + (SIGNED ? 1 : 0));
   std::lock_guard<std::mutex> lock(g_mu);
-  if (d.cols_attr_set & bit) return cudaSuccess;
+  bool& done = d.cols_attr[kIdx][MODE][SIGNED ? 1 : 0];
+  if (done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(hq::fwhtq_cols_bf16_kernel<K, MODE, SIGNED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(hq::kColsSmemBytes2));
-  if (e == cudaSuccess) d.cols_attr_set |= bit;
+  if (e == cudaSuccess) done = true;
   return e;
 }
 
@@ -150,7 +162,7 @@ cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
 template <typename SrcT, int K, int MODE, bool SIGNED>
 cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes,
                           float* scale, float* partials, int n_partials, int reverse, const uint8_t* neg,
-                          DeviceInfo& d, cudaStream_t st, int* grid) {
+                          int lp_fmt, DeviceInfo& d, cudaStream_t st, int* grid) {
   using namespace hq;
   const int64_t units = quant_units(sizeof(SrcT) == 2 ? HQ_BF16 : HQ_F32, rows, cols, dim);
   auto grid_for = [&](const void* fn, size_t smem) {
@@ -164,12 +176,12 @@ cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, 
       auto fn = fwhtq_rows_kernel<SrcT, K, MODE, true, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
       fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
-                                      reverse, neg, cols);
+                                      reverse, neg, cols, lp_fmt);
     } else {
       auto fn = fwhtq_rows_kernel<SrcT, K, MODE, false, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
       fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
-                                      reverse, neg, cols);
+                                      reverse, neg, cols, lp_fmt);
     }
   } else if constexpr (sizeof(SrcT) == 2) {
     cudaError_t e = cols_bf16_smem_attr<K, MODE, SIGNED>(d);
@@ -177,12 +189,12 @@ cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, 
     auto fn = fwhtq_cols_bf16_kernel<K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), kColsSmemBytes2);
     fn<<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials,
-                                                  scale, d.status, reverse, neg);
+                                                  scale, d.status, reverse, neg, lp_fmt);
   } else {
     auto fn = fwhtq_cols_f32_kernel<SrcT, K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), 0);
     fn<<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale,
-                                    d.status, reverse, neg);
+                                    d.status, reverse, neg, lp_fmt);
   }
   *grid = g;
   return cudaGetLastError();
@@ -191,11 +203,29 @@ cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, 
 template <typename SrcT, int K, int MODE>
 cudaError_t launch_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, uint8_t* codes, float* scale,
                         float* partials, int n_partials, int reverse, const uint8_t* neg, DeviceInfo& d,
-                        cudaStream_t st, int* grid) {
+                        cudaStream_t st, int* grid, int lp_fmt = 0) {
   return neg ? launch_pass_s<SrcT, K, MODE, true>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse,
-                                                  neg, d, st, grid)
+                                                  neg, lp_fmt, d, st, grid)
              : launch_pass_s<SrcT, K, MODE, false>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse,
-                                                   nullptr, d, st, grid);
+                                                   nullptr, lp_fmt, d, st, grid);
+}
+
+// Code pass of a format: INT8 and FP8 have their own instantiations, the FP6 / FP4
+// minifloats share one that takes the format at run time.
+template <typename SrcT, int K>
+cudaError_t launch_code_pass(const SrcT* src, int64_t rows, int64_t cols, int dim, hq_fmt fmt, uint8_t* codes,
+                             float* scale, float* partials, int n_partials, int reverse, const uint8_t* neg,
+                             DeviceInfo& d, cudaStream_t st) {
+  using namespace hq;
+  int g = 0;
+  if (fmt == HQ_INT8)
+    return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse, neg, d,
+                                           st, &g);
+  if (fmt == HQ_FP8_E4M3)
+    return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse, neg, d,
+                                          st, &g);
+  return launch_pass<SrcT, K, kModeLowp>(src, rows, cols, dim, codes, scale, partials, n_partials, reverse, neg, d,
+                                         st, &g, static_cast<int>(fmt));
 }
 
 // One operand, one rotation: absmax pass forward, code pass backward.
@@ -208,8 +238,8 @@ cudaError_t launch_quant(const void* src_v, int64_t rows, int64_t cols, int dim,
   int g1 = 0, g2 = 0;
   cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, dim, codes, scale, partials, 0, 0, neg, d, st, &g1);
   if (e != cudaSuccess) return e;
-  if (fmt == HQ_INT8) return launch_pass<SrcT, K, kModeInt8>(src, rows, cols, dim, codes, scale, partials, g1, 1, neg, d, st, &g2);
-  return launch_pass<SrcT, K, kModeFp8>(src, rows, cols, dim, codes, scale, partials, g1, 1, neg, d, st, &g2);
+  (void)g2;
+  return launch_code_pass<SrcT, K>(src, rows, cols, dim, fmt, codes, scale, partials, g1, 1, neg, d, st);
 }
 
 // One operand, both rotations: the four passes run back to back, alternating direction, so
@@ -224,13 +254,9 @@ cudaError_t launch_dual(const void* src_v, int64_t rows, int64_t cols, hq_fmt fm
   cudaError_t e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 1, codes_c, scale_c, part_c, 0, 0, neg_c, d, st, &gc);
   if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeAbsmax>(src, rows, cols, 0, codes_r, scale_r, part_r, 0, 1, neg_r, d, st, &gr);
   if (e != cudaSuccess) return e;
-  if (fmt == HQ_INT8) {
-    e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, neg_c, d, st, &g);
-    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeInt8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, neg_r, d, st, &g);
-  } else {
-    e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 1, codes_c, scale_c, part_c, gc, 0, neg_c, d, st, &g);
-    if (e == cudaSuccess) e = launch_pass<SrcT, K, kModeFp8>(src, rows, cols, 0, codes_r, scale_r, part_r, gr, 1, neg_r, d, st, &g);
-  }
+  (void)g;
+  e = launch_code_pass<SrcT, K>(src, rows, cols, 1, fmt, codes_c, scale_c, part_c, gc, 0, neg_c, d, st);
+  if (e == cudaSuccess) e = launch_code_pass<SrcT, K>(src, rows, cols, 0, fmt, codes_r, scale_r, part_r, gr, 1, neg_r, d, st);
   return e;
 }
 
@@ -259,13 +285,13 @@ hq_status encode_dual_map(CUtensorMap* map, const void* src, int64_t rows, int64
 template <int K, int MODE, bool W32, bool SIGNED>
 cudaError_t dual_smem_attr(DeviceInfo& d) {
   constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
-  const uint64_t bit = uint64_t(1) << (((kIdx * 3 + MODE) * 2 + (W32 ? 1 : 0)) * 2 + (SIGNED ? 1 : 0));
   std::lock_guard<std::mutex> lock(g_mu);
-  if (d.dual_attr_set & bit) return cudaSuccess;
+  bool& done = d.dual_attr[kIdx][MODE][W32 ? 1 : 0][SIGNED ? 1 : 0];
+  if (done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(hq::dual::fwhtq_dual_kernel<K, MODE, W32, SIGNED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(hq::dual::kSmemBytes));
-  if (e == cudaSuccess) d.dual_attr_set |= bit;
+  if (e == cudaSuccess) done = true;
   return e;
 }
 
@@ -284,16 +310,21 @@ hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols
   cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32, SIGNED>(d);
   if (e != cudaSuccess) return cuda_fail(e);
   fwhtq_dual_kernel<K, kModeAbsmax, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-      map, rows, cols, codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r);
+      map, rows, cols, codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r, 0);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (fmt == HQ_INT8) {
     if ((e = dual_smem_attr<K, kModeInt8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
     fwhtq_dual_kernel<K, kModeInt8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r);
-  } else {
+        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+  } else if (fmt == HQ_FP8_E4M3) {
     if ((e = dual_smem_attr<K, kModeFp8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
     fwhtq_dual_kernel<K, kModeFp8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r);
+        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+  } else {
+    if ((e = dual_smem_attr<K, kModeLowp, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
+    fwhtq_dual_kernel<K, kModeLowp, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
+        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r,
+        static_cast<int>(fmt));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   return HQ_OK;
@@ -362,7 +393,7 @@ __global__ void set_scale_one_kernel(float* scale) { *scale = 1.0f; }
 hq_status check_quant_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
                            hq_fmt fmt, const void* codes, const float* scale) {
   if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if ((dim != 0 && dim != 1) || !valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if ((dim != 0 && dim != 1) || !valid_k(k) || !valid_fmt(fmt)) return HQ_ERR_ARG;
   if (rows < 0 || cols < 0 || !scale) return HQ_ERR_ARG;
   if (rows == 0 || cols == 0) return HQ_OK;
   if (!src || !codes) return HQ_ERR_ARG;
@@ -423,7 +454,7 @@ hq_status encode_out_map(CUtensorMap* map, void* base, int64_t rows, int64_t col
 
 template <int FMT, int OUT>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const float* sa, const float* sb,
-                        void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st,
+                        void* out, int M, int N, int K, DeviceInfo& d, cudaStream_t st, uint32_t ab_code,
                         int skip_first_load = 0) {
   auto kernel = hq::gemm::gemm_kernel<FMT, OUT>;
   const unsigned bit = 1u << (FMT * 2 + OUT);
@@ -439,13 +470,13 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const floa
   const int tiles = ((M + hq::gemm::BM - 1) / hq::gemm::BM) * ((N + hq::gemm::BN - 1) / hq::gemm::BN);
   const int grid = std::max(1, std::min(tiles, d.sms));
   kernel<<<grid, hq::gemm::NUM_THREADS, hq::gemm::SMEM_BYTES, st>>>(ta, tb, sa, sb, out, M, N, K, d.status,
-                                                                     skip_first_load);
+                                                                     skip_first_load, ab_code);
   return cudaGetLastError();
 }
 
 hq_status check_gemm_args(const void* A, const float* sa, const void* B, const float* sb, int64_t M,
                           int64_t N, int64_t K, hq_fmt fmt, hq_out ok, const void* out) {
-  if ((fmt != HQ_INT8 && fmt != HQ_FP8_E4M3) || (ok != HQ_OUT_BF16 && ok != HQ_OUT_ACC)) return HQ_ERR_ARG;
+  if (!valid_fmt(fmt) || (ok != HQ_OUT_BF16 && ok != HQ_OUT_ACC)) return HQ_ERR_ARG;
   if (M < 0 || N < 0 || K < 0) return HQ_ERR_ARG;
   if (M == 0 || N == 0) return HQ_OK;
   if (!out) return HQ_ERR_ARG;
@@ -495,7 +526,7 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
 template <int FMT, int OUT, int BN, bool SK>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
                              const float* sb, void* out, int M, int N, int K, int clusters, int splits,
-                             uint32_t* part_ws, int* counters, DeviceInfo& d, cudaStream_t st) {
+                             uint32_t* part_ws, int* counters, uint32_t ab_code, DeviceInfo& d, cudaStream_t st) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN, SK>;
   auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK>;
@@ -514,7 +545,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   (void)d;
-  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, splits, part_ws, counters);
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, splits, part_ws, counters,
+                            ab_code);
 }
 
 // Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
@@ -592,6 +624,7 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
   }
   const bool pair = M >= kPairMinRows;
   const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
+  const uint32_t ab = ab_format_code(fmt);
   using namespace hq::gemm;
   cudaError_t e;
   int bn = 256, clusters = 0;
@@ -639,9 +672,9 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     if (ok == HQ_OUT_BF16 && (s = encode_out_map(&to, out, M, N)) != HQ_OK) return s;
 #define HQ_PAIR_LAUNCH(F, O, SKV)                                                                       \
   (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
-                                                counters, d, st)                                             \
+                                                counters, ab, d, st)                                         \
              : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
-                                                counters, d, st))
+                                                counters, ab, d, st))
     if (fmt == HQ_INT8)
       e = ok == HQ_OUT_ACC ? HQ_PAIR_LAUNCH(kInt8, kOutAcc, false)
           : sk             ? HQ_PAIR_LAUNCH(kInt8, kOutBf16, true)
@@ -653,11 +686,11 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
 #undef HQ_PAIR_LAUNCH
   } else {
     if (fmt == HQ_INT8)
-      e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                            : launch_gemm<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+      e = ok == HQ_OUT_BF16 ? launch_gemm<kInt8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st, 0)
+                            : launch_gemm<kInt8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st, 0);
     else
-      e = ok == HQ_OUT_BF16 ? launch_gemm<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st)
-                            : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st);
+      e = ok == HQ_OUT_BF16 ? launch_gemm<kFp8, kOutBf16>(ta, tb, sa, sb, out, m, n, kk, d, st, ab)
+                            : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st, ab);
   }
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
@@ -707,7 +740,7 @@ struct Operand {
 hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, hq_dtype dt, int k,
                       hq_fmt fmt, void* out, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (!valid_k(k) || !valid_fmt(fmt)) return HQ_ERR_ARG;
   if (gm < 0 || gn < 0 || gk < 0) return HQ_ERR_ARG;
   if (gm % k || gn % k || gk % k) return HQ_ERR_SHAPE;
   if (gm == 0 || gn == 0) return HQ_OK;
@@ -734,7 +767,7 @@ hq_status linear_gemm(Operand a, Operand b, int64_t gm, int64_t gn, int64_t gk, 
 hq_status check_dual_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int k, hq_fmt fmt,
                           const void* codes_c, const float* scale_c, const void* codes_r, const float* scale_r) {
   if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (!valid_k(k) || !valid_fmt(fmt)) return HQ_ERR_ARG;
   if (rows < 0 || cols < 0 || !scale_c || !scale_r) return HQ_ERR_ARG;
   if (rows == 0 || cols == 0) return HQ_OK;
   if (!src || !codes_c || !codes_r) return HQ_ERR_ARG;
@@ -837,7 +870,7 @@ hq_status carve_step_ws(void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t
 // contraction length of one of the layer's GEMMs and a rotated dimension).
 hq_status check_step_shape(hq_dtype dt, int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt) {
   if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (!valid_k(k) || !valid_fmt(fmt)) return HQ_ERR_ARG;
   if (M < 0 || K < 0 || N < 0) return HQ_ERR_ARG;
   if (M % k || K % k || N % k) return HQ_ERR_SHAPE;
   if (M == 0 || K == 0 || N == 0) return HQ_ERR_SHAPE;
@@ -1168,7 +1201,8 @@ hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int6
   if ((s = encode_codes_map(&ta, A, M, K, hq::gemm::BM)) != HQ_OK) return s;
   if ((s = encode_codes_map(&tb, B, N, K, hq::gemm::BN)) != HQ_OK) return s;
   cudaError_t e = launch_gemm<hq::gemm::kInt8, hq::gemm::kOutAcc>(ta, tb, nullptr, nullptr, out, int(M), int(N),
-                                                                  int(K), *d, reinterpret_cast<cudaStream_t>(stream), 1);
+                                                                  int(K), *d, reinterpret_cast<cudaStream_t>(stream), 0,
+                                                                  1);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 

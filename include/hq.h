@@ -67,7 +67,23 @@ typedef enum {
   HQ_ERR_UNSUPPORTED = 9  /* the current device is not sm_100 */
 } hq_status;
 
-typedef enum { HQ_INT8 = 0, HQ_FP8_E4M3 = 1 } hq_fmt;
+/* Code formats.  Every code is one byte; the scale is fp32(a / max) with a the tensor's absmax.
+ *   HQ_INT8      symmetric integers -127..127 (max 127), GEMM on kind::i8, int32 accumulators
+ *   HQ_FP8_E4M3  E4M3FN (max 448), kind::f8f6f4, fp32 accumulators
+ *   HQ_FP6_E3M2  FP6 sign | 3 exponent (bias 3) | 2 mantissa, max 28, value in bits 5..0
+ *   HQ_FP6_E2M3  FP6 sign | 2 exponent (bias 1) | 3 mantissa, max 7.5, value in bits 5..0
+ *   HQ_FP4_E2M1  FP4 sign | 2 exponent (bias 1) | 1 mantissa, max 6, value in bits 3..0
+ * FP6 and FP4 are the formats HALO names below FP8 (its GPUs had no FP6 matmul, so it
+ * lower-bounded them with FP8); B200's kind::f8f6f4 multiplies them directly, one code per
+ * byte in shared memory.  The minifloats have subnormals and no infinities or NaN; codes are
+ * nearest-even with saturation to +-max, the upper bits of each byte zero. */
+typedef enum {
+  HQ_INT8 = 0,
+  HQ_FP8_E4M3 = 1,
+  HQ_FP6_E3M2 = 2,
+  HQ_FP6_E2M3 = 3,
+  HQ_FP4_E2M1 = 4
+} hq_fmt;
 typedef enum { HQ_F32 = 0, HQ_BF16 = 1 } hq_dtype;
 typedef enum {
   HQ_OUT_BF16 = 0, /* dequantized bf16 */

@@ -205,6 +205,36 @@ def minifloat_bits(fmt: int) -> int:
     return 4 if fmt == FP4_E2M1 else 6
 
 
+def device_codes(codes: np.ndarray, fmt: int) -> np.ndarray:
+    """The library's storage layout of a code tensor (rotated dimension innermost): INT8 and
+    FP8 one code per byte as they are; FP6 / FP4 in the tensor cores' operand form, each group
+    of 16 consecutive codes along the last axis packed LSB-first (code i at bits b*i .. b*i+b-1,
+    b = 6 or 4, of the little-endian chunk) into the leading 12 or 8 bytes of one 16-byte
+    chunk, the rest zero.  Plain integer bit packing, no arithmetic of the method."""
+    if fmt not in MINIFLOATS:
+        return codes
+    b = minifloat_bits(fmt)
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, n = c.reshape(-1, c.shape[-1]).shape
+    if n % 16:
+        raise ValueError("the packed layout needs the rotated dimension to be a multiple of 16")
+    g = c.reshape(rows, n // 16, 16).astype(np.uint64)
+    lo = np.zeros((rows, n // 16), dtype=np.uint64)  # bits 0..63 of each chunk
+    hi = np.zeros((rows, n // 16), dtype=np.uint64)  # bits 64..127
+    for i in range(16):
+        sh = b * i
+        v = g[:, :, i] & np.uint64((1 << b) - 1)
+        if sh + b <= 64:
+            lo |= v << np.uint64(sh)
+        elif sh >= 64:
+            hi |= v << np.uint64(sh - 64)
+        else:  # straddles bit 64
+            lo |= (v << np.uint64(sh)) & np.uint64(0xFFFFFFFFFFFFFFFF)
+            hi |= v >> np.uint64(64 - sh)
+    out = np.concatenate([lo[..., None], hi[..., None]], axis=-1).view(np.uint8)
+    return out.reshape(c.shape)
+
+
 def e4m3_decode(code: int) -> float:
     return lib().hq_oracle_e4m3_decode(code)
 

@@ -62,7 +62,10 @@ def test_quantize_argument_errors(L):
     assert _q(L, k=24) == 1
     assert _q(L, k=512) == 1
     assert _q(L, dim=2) == 1
-    assert _q(L, fmt=3) == 1
+    assert _q(L, fmt=5) == 1
+    assert _q(L, fmt=-1) == 1
+    for f in (2, 3, 4):  # FP6 e3m2 / e2m3 and FP4 e2m1 pass the format check: a misaligned
+        assert _q(L, fmt=f, codes=FAKE_MIS) == 4  # codes pointer is what fails (no launch)
     assert _q(L, rows=-1) == 1
     assert _q(L, scale=None) == 1
     assert _q(L, src=None) == 1
@@ -81,7 +84,7 @@ def _g(L, A=FAKE, sa=FAKE, B=FAKE, sb=FAKE, M=128, N=256, K=128, fmt=0, out_kind
 
 
 def test_gemm_argument_errors(L):
-    assert _g(L, fmt=2) == 1
+    assert _g(L, fmt=6) == 1
     assert _g(L, out_kind=2) == 1
     assert _g(L, M=-1) == 1
     assert _g(L, out=None) == 1
@@ -173,7 +176,7 @@ def test_saved_codes_flow_argument_errors(L):
                                      kw.get("dX", FAKE), kw.get("dW", FAKE), kw.get("ws", FAKE),
                                      kw.get("wsb", 1 << 34), None)
     assert b(dt=3) == 3
-    assert b(fmt=4) == 1
+    assert b(fmt=9) == 1
     assert b(K=80) == 2
     assert b(M=133248, K=128, N=128, fmt=0) == 2   # INT8 contraction bound on the dW GEMM
     assert b(xqt=None) == 1

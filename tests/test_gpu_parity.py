@@ -37,6 +37,7 @@ def _setup(oracle_lib):
 def _quant_check(x_np, dim, k, fmt):
     codes, scale = hq.hq_quantize(to_device(x_np), dim, k, fmt)
     want_codes, want_scale = oracle.quantize(x_np, dim, k, fmt)
+    want_codes = oracle.device_codes(want_codes, fmt)
     got = codes.cpu().numpy()
     assert got.shape == want_codes.shape
     mism = np.count_nonzero(got != want_codes)
@@ -324,8 +325,8 @@ def _layer_check(d, k, fmt, rows_sample=None, tag=""):
         # codes and scales of both operands, bit-exact
         qa, sa = hq.hq_quantize(to_device(a_src), a_dim, k, fmt)
         qb, sb = hq.hq_quantize(to_device(b_src), b_dim, k, fmt)
-        assert np.array_equal(qa.cpu().numpy(), want["qa"]), f"{tag}{name}: A codes"
-        assert np.array_equal(qb.cpu().numpy(), want["qb"]), f"{tag}{name}: B codes"
+        assert np.array_equal(qa.cpu().numpy(), oracle.device_codes(want["qa"], fmt)), f"{tag}{name}: A codes"
+        assert np.array_equal(qb.cpu().numpy(), oracle.device_codes(want["qb"], fmt)), f"{tag}{name}: B codes"
         assert sa.cpu().numpy()[0] == want["sa"] and sb.cpu().numpy()[0] == want["sb"], f"{tag}{name}: scales"
         got = bf16_bits(out)
         if rows is not None:
@@ -363,7 +364,7 @@ def _saved_codes_check(d, k, fmt, tag=""):
     Xd, Wd, dYd = to_device(X), to_device(d["W"]), to_device(d["dY"])
     Y, xqt, sx = hq.hq_linear_fwd_save(Xd, Wd, k, fmt)
     want_codes, want_scale = oracle.quantize(X, 0, k, fmt)
-    assert np.array_equal(xqt.cpu().numpy(), want_codes), f"{tag}saved codes"
+    assert np.array_equal(xqt.cpu().numpy(), oracle.device_codes(want_codes, fmt)), f"{tag}saved codes"
     assert sx.cpu().numpy()[0].view(np.uint32) == np.float32(want_scale).view(np.uint32), f"{tag}saved scale"
     dX, dW = hq.hq_linear_bwd(dYd, Wd, xqt, sx, k, fmt)
     sep = (hq.hq_linear_fwd(Xd, Wd, k, fmt), hq.hq_linear_bwd_dx(dYd, Wd, k, fmt),
