@@ -546,9 +546,12 @@ def run_sweep(args):
         return tot / reps
 
     out_lines = []
-    for wid in sorted(synthetic.WORKLOADS):
+    wids = [WORKLOAD_ID] if args.formats else sorted(synthetic.WORKLOADS)
+    for wid in wids:
         w = synthetic.WORKLOADS[wid]
         points = list(w.sweep) if w.sweep else [(w.fmt, w.k)]
+        if args.formats:  # the bench workload's layer in every code format at its k
+            points = [(f, w.k) for f in ("int8", "fp8", "fp6_e3m2", "fp6_e2m3", "fp4_e2m1")]
         for li, Lr in enumerate(w.layers):
             d = synthetic.draw(w, li)
             def dev_t(a):
@@ -562,7 +565,7 @@ def run_sweep(args):
             dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
             dW = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
             for fmt_name, k in points:
-                fmt = hq.HQ_INT8 if fmt_name == "int8" else hq.HQ_FP8_E4M3
+                fmt = hq._fmt(fmt_name)
                 step_ms = timed(lambda: hq.hq_linear_fwd_bwd(X, W, dY, k, fmt, Y=Y, dX=dX, dW=dW, workspace=ws))
                 codes = {}
                 quant_ms = 0.0
@@ -641,6 +644,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
     ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
+    ap.add_argument("--formats", action="store_true",
+                    help="with --sweep: the bench workload's layer in every code format (INT8, FP8, FP6, FP4)")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload (one JSON line per workload/layer/format/k) and exit")
     args = ap.parse_args(argv)
