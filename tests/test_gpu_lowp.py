@@ -9,7 +9,8 @@ import oracle
 import hadamard_rotated_precision_b200 as hq
 from hadamard_rotated_precision_b200 import synthetic
 from _helpers import to_device, bf16_bits, bits_to_f32, rel_fro
-from test_gpu_parity import _quant_check, _outlier_input, _layer_check, _fwd_bwd_check, _fused_shapes
+from test_gpu_parity import (_quant_check, _outlier_input, _layer_check, _fwd_bwd_check, _fused_shapes,
+                             _saved_codes_check)
 
 pytestmark = pytest.mark.gpu
 
@@ -90,3 +91,36 @@ def test_layer_lowp_token_prefix(fmt):
     d = synthetic.draw(w, 0, M=512)
     _layer_check(d, w.k, fmt, tag=f"llama512/{fmt}/")
     _fwd_bwd_check(d, w.k, fmt, tag=f"llama512/{fmt}/")
+
+
+@pytest.mark.parametrize("fmt", LOWP)
+def test_layer_lowp_saved_codes(fmt):
+    """Training flow with saved codes in FP6 / FP4: the kept token-rotated codes equal the
+    oracle's (packed layout) and the backward from them equals the separate entry points."""
+    w = synthetic.WORKLOADS[1]
+    d = synthetic.draw(w)
+    _saved_codes_check(d, w.k, fmt, tag=f"tiny/{fmt}/")
+    d = synthetic.draw(synthetic.WORKLOADS[4], 0, M=512)
+    _saved_codes_check(d, 64, fmt, tag=f"vit512/{fmt}/")
+
+
+@pytest.mark.parametrize("fmt", LOWP)
+@pytest.mark.parametrize("dtype", ("f32", "bf16"))
+def test_quantize_rht_lowp(fmt, dtype):
+    """The randomized variant's sign flags with minifloat codes: single rotations in both
+    directions and both rotations at once (fused kernel for the bf16 source)."""
+    k = 64
+    rows, cols = (1344, 1216) if dtype == "bf16" else (512 + 2 * k, 3 * k)
+    x = _outlier_input(rows, cols, 21 + fmt, dtype)
+    nc, nr = synthetic.sign_flags(cols, 30 + fmt), synthetic.sign_flags(rows, 40 + fmt)
+    f = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    for dim, neg in ((1, nc), (0, nr)):
+        codes, scale = hq.hq_quantize_rht(to_device(x), dim, k, fmt, f(neg))
+        want, ws = oracle.quantize(x, dim, k, fmt, neg=neg)
+        assert np.array_equal(codes.cpu().numpy(), oracle.device_codes(want, fmt)), f"dim {dim}"
+        assert scale.cpu().numpy()[0].view(np.uint32) == np.float32(ws).view(np.uint32)
+    cc, sc, cr, sr = hq.hq_quantize_dual_rht(to_device(x), k, fmt, f(nc), f(nr))
+    for codes, scale, dim, neg in ((cc, sc, 1, nc), (cr, sr, 0, nr)):
+        want, ws = oracle.quantize(x, dim, k, fmt, neg=neg)
+        assert np.array_equal(codes.cpu().numpy(), oracle.device_codes(want, fmt)), f"dual dim {dim}"
+        assert scale.cpu().numpy()[0].view(np.uint32) == np.float32(ws).view(np.uint32)
