@@ -33,6 +33,7 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_fwd_save_workspace_bytes", "hq_linear_fwd_save",
            "hq_linear_bwd_workspace_bytes", "hq_linear_bwd", "hq_selftest_gemm_timeout",
            "hq_quantize_rht", "hq_quantize_dual_rht", "hq_linear_fwd_bwd_rht",
+           "hq_quantize_absmax", "hq_quantize_codes",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -72,6 +73,10 @@ def lib() -> ctypes.CDLL:
         L.hq_quantize_dual_rht.restype = i32
         L.hq_linear_fwd_bwd_rht.argtypes = [p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, p, p, p, sz, p]
         L.hq_linear_fwd_bwd_rht.restype = i32
+        L.hq_quantize_absmax.argtypes = [p, i32, i64, i64, i32, i32, p, p, p, sz, p]
+        L.hq_quantize_absmax.restype = i32
+        L.hq_quantize_codes.argtypes = [p, i32, i64, i64, i32, i32, i32, p, p, p, p, p]
+        L.hq_quantize_codes.restype = i32
         L.hq_quantize_dual_workspace_bytes.argtypes = []
         L.hq_quantize_dual_workspace_bytes.restype = sz
         L.hq_quantize_dual.argtypes = [p, i32, i64, i64, i32, i32, p, p, p, p, p, sz, p]
@@ -260,6 +265,86 @@ def hq_quantize_dual_rht(src, k: int, fmt, neg_c, neg_r, codes_c=None, scale_c=N
                                     _stream_handle(stream))
     _check(st, "hq_quantize_dual_rht")
     return codes_c, scale_c, codes_r, scale_r
+
+
+def hq_quantize_absmax(src, dim: int, k: int, neg=None, absmax=None, workspace=None, stream=None):
+    """Pass 1 alone: max |y| of the rotation of `src` along `dim`, as a float32[1] CUDA tensor."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    neg = _sign_flags(neg, cols if dim == 1 else rows, "neg")
+    absmax = torch.empty(1, dtype=torch.float32, device=src.device) if absmax is None else absmax
+    _dev_tensor(absmax, "absmax")
+    ws = _workspace(hq_quantize_workspace_bytes(), src.device, workspace)
+    st = lib().hq_quantize_absmax(src.data_ptr(), dt, rows, cols, dim, k, _ptr_or_none(neg), absmax.data_ptr(),
+                                  ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_quantize_absmax")
+    return absmax
+
+
+def hq_quantize_codes(src, dim: int, k: int, fmt, absmax, neg=None, codes=None, scale=None, stream=None):
+    """Pass 2 from a given absmax (float32[1] CUDA tensor): codes and scale of `src` as the
+    slice of a tensor whose absmax that is."""
+    torch = _torch()
+    _dev_tensor(src, "src")
+    if src.dim() != 2:
+        raise ValueError("src must be 2-D")
+    _dev_tensor(absmax, "absmax")
+    dt = _src_dtype(src, "src")
+    rows, cols = src.shape
+    neg = _sign_flags(neg, cols if dim == 1 else rows, "neg")
+    shape = (rows, cols) if dim == 1 else (cols, rows)
+    codes = torch.empty(shape, dtype=torch.uint8, device=src.device) if codes is None else codes
+    scale = torch.empty(1, dtype=torch.float32, device=src.device) if scale is None else scale
+    _dev_tensor(codes, "codes")
+    _dev_tensor(scale, "scale")
+    st = lib().hq_quantize_codes(src.data_ptr(), dt, rows, cols, dim, k, _fmt(fmt), _ptr_or_none(neg),
+                                 absmax.data_ptr(), codes.data_ptr(), scale.data_ptr(), _stream_handle(stream))
+    _check(st, "hq_quantize_codes")
+    return codes, scale
+
+
+def sharded_quantize_flow(absmax_pass, reduce_max, codes_pass):
+    """The sharded quantization of quantized FSDP communication: this rank's absmax, the maximum
+    over ranks, then this rank's codes scaled by the whole tensor's absmax.  The passes and the
+    collective are arguments so the same flow runs on the library's kernels with NCCL and, in the
+    CPU tests, on other implementations with gloo."""
+    a = absmax_pass()
+    a = reduce_max(a)
+    return codes_pass(a)
+
+
+def hq_quantize_sharded(shard, dim: int, k: int, fmt, group=None, neg=None, stream=None):
+    """This rank's slice `shard` of a tensor distributed over the ranks of `group`, quantized
+    with the whole tensor's tensor-wise scale (slices along the non-rotated dimension, or along
+    the rotated one in multiples of k).  Returns (codes of the slice, scale)."""
+    import torch.distributed as dist
+
+    def reduce_max(a):
+        if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+            dist.all_reduce(a, op=dist.ReduceOp.MAX, group=group)
+        return a
+
+    return sharded_quantize_flow(lambda: hq_quantize_absmax(shard, dim, k, neg=neg, stream=stream), reduce_max,
+                                 lambda a: hq_quantize_codes(shard, dim, k, fmt, a, neg=neg, stream=stream))
+
+
+def hq_fsdp_all_gather(w_shard, k: int, fmt, group=None, neg=None):
+    """Quantized weight all-gather: this rank holds rows [r*n, (r+1)*n) of W [N][K]; every rank
+    gets the codes of the whole W rotated along K (1 byte per element on the wire instead of 2)
+    and its scale, equal to hq_quantize(W, dim=1) bit for bit."""
+    import torch.distributed as dist
+    torch = _torch()
+    codes, scale = hq_quantize_sharded(w_shard, 1, k, fmt, group=group, neg=neg)
+    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+    if world == 1:
+        return codes, scale
+    full = torch.empty((world * codes.shape[0], codes.shape[1]), dtype=torch.uint8, device=codes.device)
+    dist.all_gather_into_tensor(full, codes, group=group)
+    return full, scale
 
 
 def hq_quantize_dual_workspace_bytes() -> int:

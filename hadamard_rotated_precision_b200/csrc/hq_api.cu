@@ -389,18 +389,73 @@ cudaError_t launch_quant_k(const void* src, int64_t rows, int64_t cols, int dim,
 }
 
 __global__ void set_scale_one_kernel(float* scale) { *scale = 1.0f; }
+__global__ void set_zero_kernel(float* v) { *v = 0.0f; }
+
+// Maximum of the absmax pass's per-CTA partials into one device scalar (a non-finite rotated
+// value is already +inf in its partial).
+__global__ void reduce_partials_kernel(const float* __restrict__ partials, int n, float* __restrict__ out) {
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partials[i]);
+  __shared__ float scratch[32];
+  m = hq::block_max(m, scratch);
+  if (threadIdx.x == 0) *out = m;
+}
+
+// Split passes for sharded tensors: the absmax pass alone into a device scalar, and the code
+// pass from a given absmax (one "partial", e.g. the maximum over ranks).
+template <typename SrcT, int K>
+cudaError_t launch_absmax_only(const void* src_v, int64_t rows, int64_t cols, int dim, float* partials,
+                               const uint8_t* neg, float* absmax, DeviceInfo& d, cudaStream_t st) {
+  int g = 0;
+  cudaError_t e = launch_pass<SrcT, K, hq::kModeAbsmax>(static_cast<const SrcT*>(src_v), rows, cols, dim, nullptr,
+                                                        nullptr, partials, 0, 0, neg, d, st, &g);
+  if (e != cudaSuccess) return e;
+  reduce_partials_kernel<<<1, 256, 0, st>>>(partials, g, absmax);
+  return cudaGetLastError();
+}
+
+template <typename SrcT>
+cudaError_t split_pass_k(bool codes_pass, const void* src, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
+                         const uint8_t* neg, float* partials, float* absmax, uint8_t* codes, float* scale,
+                         DeviceInfo& d, cudaStream_t st) {
+  const SrcT* sp = static_cast<const SrcT*>(src);
+#define HQ_SPLIT_CASE(KK)                                                                                     \
+  case KK:                                                                                                    \
+    return codes_pass ? launch_code_pass<SrcT, KK>(sp, rows, cols, dim, fmt, codes, scale, absmax, 1, 1, neg, d, st) \
+                      : launch_absmax_only<SrcT, KK>(src, rows, cols, dim, partials, neg, absmax, d, st);
+  switch (k) {
+    HQ_SPLIT_CASE(16)
+    HQ_SPLIT_CASE(32)
+    HQ_SPLIT_CASE(64)
+    HQ_SPLIT_CASE(128)
+    default: HQ_SPLIT_CASE(256)
+  }
+#undef HQ_SPLIT_CASE
+}
+
+// The source side of a quantization: dtype, dim, k, sizes, the rotated dim's divisibility.
+// `out` is the scalar the call writes (scale or absmax): non-null, 4-byte aligned.
+hq_status check_src_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k, const float* out) {
+  if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
+  if ((dim != 0 && dim != 1) || !valid_k(k)) return HQ_ERR_ARG;
+  if (rows < 0 || cols < 0 || !out) return HQ_ERR_ARG;
+  if (rows == 0 || cols == 0) return HQ_OK;
+  if (!src) return HQ_ERR_ARG;
+  if (dim == 1 && cols % k != 0) return HQ_ERR_SHAPE;
+  if (dim == 0 && (rows % k != 0 || cols % 16 != 0)) return HQ_ERR_SHAPE;
+  if (rows > (int64_t(1) << 40) / cols) return HQ_ERR_SHAPE;
+  if (!aligned16(src) || (reinterpret_cast<uintptr_t>(out) & 3u)) return HQ_ERR_ALIGN;
+  return HQ_OK;
+}
 
 hq_status check_quant_args(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
                            hq_fmt fmt, const void* codes, const float* scale) {
   if (dt != HQ_F32 && dt != HQ_BF16) return HQ_ERR_DTYPE;
-  if ((dim != 0 && dim != 1) || !valid_k(k) || !valid_fmt(fmt)) return HQ_ERR_ARG;
-  if (rows < 0 || cols < 0 || !scale) return HQ_ERR_ARG;
-  if (rows == 0 || cols == 0) return HQ_OK;
-  if (!src || !codes) return HQ_ERR_ARG;
-  if (dim == 1 && cols % k != 0) return HQ_ERR_SHAPE;
-  if (dim == 0 && (rows % k != 0 || cols % 16 != 0)) return HQ_ERR_SHAPE;
-  if (rows > (int64_t(1) << 40) / cols) return HQ_ERR_SHAPE;
-  if (!aligned16(src) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scale) & 3u)) return HQ_ERR_ALIGN;
+  if (!valid_fmt(fmt)) return HQ_ERR_ARG;
+  hq_status s = check_src_args(src, dt, rows, cols, dim, k, scale);
+  if (s != HQ_OK || rows == 0 || cols == 0) return s;
+  if (!codes) return HQ_ERR_ARG;
+  if (!aligned16(codes)) return HQ_ERR_ALIGN;
   return HQ_OK;
 }
 
@@ -1188,6 +1243,53 @@ hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_
     return HQ_ERR_WORKSPACE;
   return quantize_impl(src, dt, rows, cols, dim, k, fmt, codes, scale, partials, *d,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_quantize_absmax(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,
+                             const uint8_t* neg, float* absmax, void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_src_args(src, dt, rows, cols, dim, k, absmax);
+  if (s != HQ_OK) return s;
+  if (neg && !aligned16(neg)) return HQ_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0 || cols == 0) {
+    set_zero_kernel<<<1, 1, 0, st>>>(absmax);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  if (!workspace || ws_bytes < kPartialBytes) return HQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  float* part = static_cast<float*>(workspace);
+  cudaError_t e = dt == HQ_BF16
+                      ? split_pass_k<__nv_bfloat16>(false, src, rows, cols, dim, k, HQ_INT8, neg, part, absmax, nullptr,
+                                                    nullptr, *d, st)
+                      : split_pass_k<float>(false, src, rows, cols, dim, k, HQ_INT8, neg, part, absmax, nullptr, nullptr,
+                                            *d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+hq_status hq_quantize_codes(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k, hq_fmt fmt,
+                            const uint8_t* neg, const float* absmax, void* codes, float* scale, hq_stream_t stream) {
+  hq_status s = check_quant_args(src, dt, rows, cols, dim, k, fmt, codes, scale);
+  if (s != HQ_OK) return s;
+  if (!absmax) return HQ_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(absmax) & 3u) || (neg && !aligned16(neg))) return HQ_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0 || cols == 0) {
+    set_scale_one_kernel<<<1, 1, 0, st>>>(scale);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  float* a = const_cast<float*>(absmax);  // read only: the code pass reduces it as one partial
+  cudaError_t e = dt == HQ_BF16
+                      ? split_pass_k<__nv_bfloat16>(true, src, rows, cols, dim, k, fmt, neg, nullptr, a,
+                                                    static_cast<uint8_t*>(codes), scale, *d, st)
+                      : split_pass_k<float>(true, src, rows, cols, dim, k, fmt, neg, nullptr, a,
+                                            static_cast<uint8_t*>(codes), scale, *d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
 hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int64_t M, int64_t N, int64_t K,

@@ -229,6 +229,31 @@ HQ_API hq_status hq_linear_fwd_bwd_rht(const void* X, const void* W, const void*
                                        void* workspace, size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Sharded quantization (quantized FSDP weight communication, "HALO" HQ-FSDP): each rank holds
+ * a slice of a tensor and must quantize it with the tensor-wise scale of the WHOLE tensor,
+ * then all-gather 1-byte codes instead of 2-byte bf16 values.  The two passes of hq_quantize
+ * are split so that the absmax can be reduced across ranks in between (e.g. an NCCL
+ * all-reduce MAX on the device scalar):
+ *
+ * hq_quantize_absmax -- pass 1 only: *absmax = max |y| of the rotation of src (device fp32
+ *   scalar; +inf if a rotated value is not finite).  Slices along the non-rotated dimension,
+ *   or along the rotated one in multiples of k, have whole blocks each: the maximum of their
+ *   absmax values is the whole tensor's.  workspace >= hq_quantize_workspace_bytes().
+ * hq_quantize_codes -- pass 2 from a given absmax (device scalar, read only): codes and
+ *   scale equal to hq_quantize of the whole tensor restricted to this slice, bit for bit.
+ *   A non-finite absmax sets HQ_ERR_NONFINITE and writes no codes (scale NaN), an absmax of 0
+ *   gives zero codes and scale 1.
+ * neg: optional sign flags of the randomized variant (as hq_quantize_rht), NULL = plain.
+ * Both calls enqueue on `stream`; argument errors as for hq_quantize.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_quantize_absmax(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim,
+                                    int k, const uint8_t* neg, float* absmax, void* workspace,
+                                    size_t ws_bytes, hq_stream_t stream);
+HQ_API hq_status hq_quantize_codes(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim,
+                                   int k, hq_fmt fmt, const uint8_t* neg, const float* absmax,
+                                   void* codes, float* scale, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Training flow with saved codes ("HALO" Approach: the quantized rotated tensors are kept for
  * the backward pass instead of the bf16 activation, which halves the activation memory).
  *

@@ -70,6 +70,10 @@ def lib():
         L.hq_oracle_quantize_signed.restype = i32
         L.hq_oracle_quantize_rotated.argtypes = [p, i64, i32, p, p]
         L.hq_oracle_quantize_rotated.restype = i32
+        L.hq_oracle_quantize_rotated_given.argtypes = [p, i64, i32, ctypes.c_float, p, p]
+        L.hq_oracle_quantize_rotated_given.restype = i32
+        L.hq_oracle_absmax.argtypes = [p, i64]
+        L.hq_oracle_absmax.restype = ctypes.c_float
         L.hq_oracle_fwht_block.argtypes = [p, i32]
         L.hq_oracle_fwht_block.restype = None
         L.hq_oracle_norm_const.argtypes = [i32]
@@ -161,10 +165,24 @@ def rotate(x: np.ndarray, dim: int, k: int, neg=None) -> np.ndarray:
     return y
 
 
-def quantize_rotated(y: np.ndarray, fmt: int):
+def absmax(y: np.ndarray) -> np.float32:
+    """max |y| of rotated values (+inf if any is not finite)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    return np.float32(lib().hq_oracle_absmax(_ptr(y), y.size))
+
+
+def quantize_rotated(y: np.ndarray, fmt: int, absmax_of_whole=None):
+    """Tensor-wise quantization of rotated values; absmax_of_whole: the absmax of the tensor
+    y is a slice of (sharded quantization), else y's own."""
     y = np.ascontiguousarray(y, dtype=np.float32)
     codes = np.empty(y.shape, dtype=np.uint8)
     scale = np.zeros(1, dtype=np.float32)
+    if absmax_of_whole is not None:
+        st = lib().hq_oracle_quantize_rotated_given(_ptr(y), y.size, fmt, float(absmax_of_whole), _ptr(codes),
+                                                    _ptr(scale))
+        if st != OK:
+            raise OracleError(st, "quantize")
+        return codes, np.float32(scale[0])
     st = lib().hq_oracle_quantize_rotated(_ptr(y), y.size, fmt, _ptr(codes), _ptr(scale))
     if st != OK:
         raise OracleError(st, "quantize")

@@ -253,9 +253,17 @@ static float absmax(const float* y, int64_t n) {
 /* Quantize already-rotated values y[n] tensor-wise.  fmt 0 = INT8, 1 = FP8 e4m3,
  * 2 = FP6 e3m2, 3 = FP6 e2m3, 4 = FP4 e2m1.  Writes n one-byte codes and the fp32
  * dequantization scale. */
+int hq_oracle_quantize_rotated_given(const float* y, int64_t n, int fmt, float a, uint8_t* codes, float* scale);
+
 int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* codes, float* scale) {
     if (fmt < 0 || fmt > 4) return ORC_ERR_ARG;
-    float a = absmax(y, n);
+    return hq_oracle_quantize_rotated_given(y, n, fmt, absmax(y, n), codes, scale);
+}
+
+/* The same quantizer with the tensor-wise absmax a supplied: for a slice of a larger tensor,
+ * a is the whole tensor's (sharded quantization). */
+int hq_oracle_quantize_rotated_given(const float* y, int64_t n, int fmt, float a, uint8_t* codes, float* scale) {
+    if (fmt < 0 || fmt > 4) return ORC_ERR_ARG;
     if (!isfinite(a)) {
         *scale = NAN;
         return ORC_ERR_NONFINITE;
@@ -283,6 +291,9 @@ int hq_oracle_quantize_rotated(const float* y, int64_t n, int fmt, uint8_t* code
     }
     return ORC_OK;
 }
+
+/* max |y[i]| (exact; +inf if any element is not finite). */
+float hq_oracle_absmax(const float* y, int64_t n) { return absmax(y, n); }
 
 /* Rotate then quantize (hq_quantize's definition).  codes has the rotated dim innermost. */
 int hq_oracle_quantize_signed(const void* src, int dtype, int64_t rows, int64_t cols, int dim, int k,

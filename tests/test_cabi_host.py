@@ -237,3 +237,22 @@ def test_sign_flag_draws():
     assert 0.45 < a.mean() < 0.55
     assert np.array_equal(a, synthetic.sign_flags(4096, 9))
     assert not np.array_equal(a, synthetic.sign_flags(4096, 10))
+
+
+def test_split_pass_argument_errors(L):
+    """hq_quantize_absmax / hq_quantize_codes: the source checks of hq_quantize, a non-null
+    4-byte-aligned absmax scalar, 16-byte-aligned flags (all rejected before any launch)."""
+    a = lambda **kw: L.hq_quantize_absmax(kw.get("src", FAKE), hq.HQ_BF16, 256, 256, kw.get("dim", 1),
+                                          kw.get("k", 64), kw.get("neg", None), kw.get("am", FAKE), FAKE,
+                                          1 << 20, None)
+    assert a(am=None) == 1
+    assert a(am=FAKE + 2) == 4
+    assert a(k=48) == 1
+    assert a(neg=FAKE_MIS) == 4
+    assert a(src=FAKE_MIS) == 4
+    c = lambda **kw: L.hq_quantize_codes(FAKE, hq.HQ_BF16, 256, 256, 1, 64, kw.get("fmt", 0), None,
+                                         kw.get("am", FAKE), kw.get("codes", FAKE), FAKE, None)
+    assert c(am=None) == 1
+    assert c(am=FAKE + 2) == 4
+    assert c(fmt=7) == 1
+    assert c(codes=FAKE_MIS) == 4
