@@ -123,27 +123,6 @@ __device__ __forceinline__ void rotate64(float2 (&v)[32], int lane, int m6, int 
   }
 }
 
-// Scaling of a rotated value t to the code grid.  The definition is z = fp32(fp32(t * c) * inv).
-// When c = 1/sqrt(k) is a power of two (k = 16, 64, 256) and inv <= 2^100 this equals
-// fp32(t * ci) with ci = c * inv (exact): if t * c is a normal number it is exact, so one
-// rounding of t * c * inv remains either way; otherwise |z| <= 2^-126 * 2^100 under both forms,
-// which is the zero code for INT8 and e4m3 alike (with the sign of t).
-struct CodeScale {
-  float2 c2, inv2, ci2;
-  bool one_mul;
-};
-
-template <int K>
-__device__ __forceinline__ CodeScale code_scale(float c, float inv) {
-  CodeScale s;
-  s.c2 = make_float2(c, c);
-  s.inv2 = make_float2(inv, inv);
-  const float ci = __fmul_rn(c, inv);
-  s.ci2 = make_float2(ci, ci);
-  s.one_mul = (K == 16 || K == 64 || K == 256) && inv <= 0x1p100f;
-  return s;
-}
-
 __device__ __forceinline__ void st_global_32B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
                                               uint32_t f, uint32_t g, uint32_t h) {
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d),

@@ -288,6 +288,31 @@ __device__ __forceinline__ uint32_t codes4(float2 z0, float2 z1) {
   }
 }
 
+// Scaling of a rotated value t to the code grid.  The definition is z = fp32(fp32(t * c) * inv).
+// When c = 1/sqrt(k) is a power of two (k = 16, 64, 256) and inv <= 2^100 this equals
+// fp32(t * ci) with ci = c * inv (exact): if t * c is a normal number it is exact, so one
+// rounding of t * c * inv remains either way; otherwise |z| <= 2^-126 * 2^100 under both forms,
+// which is the zero code for INT8 and e4m3 alike (with the sign of t).
+struct CodeScale {
+  float2 c2, inv2, ci2;
+  bool one_mul;
+};
+
+template <int K>
+__device__ __forceinline__ CodeScale code_scale(float c, float inv) {
+  CodeScale s;
+  s.c2 = make_float2(c, c);
+  s.inv2 = make_float2(inv, inv);
+  const float ci = __fmul_rn(c, inv);
+  s.ci2 = make_float2(ci, ci);
+  s.one_mul = (K == 16 || K == 64 || K == 256) && inv <= 0x1p100f;
+  return s;
+}
+
+// Codes of 4 consecutive rotated values (t0.x, t0.y, t1.x, t1.y) at the scale of cs.
+template <int MODE>
+__device__ __forceinline__ uint32_t scaled_codes4(float2 t0, float2 t1, const CodeScale& cs, int lp_fmt);
+
 // Codes of 4 consecutive elements for any mode (the minifloats' format at run time).
 template <int MODE>
 __device__ __forceinline__ uint32_t codes4x(float2 z0, float2 z1, int lp_fmt) {
@@ -305,6 +330,12 @@ __device__ __forceinline__ uint32_t codes4x(float2 z0, float2 z1, int lp_fmt) {
     const uint32_t hi = __nv_cvt_float2_to_fp6x2(z1, f, cudaRoundNearest);
     return (lo & 0xFFFFu) | (hi << 16);
   }
+}
+
+template <int MODE>
+__device__ __forceinline__ uint32_t scaled_codes4(float2 t0, float2 t1, const CodeScale& cs, int lp_fmt) {
+  return cs.one_mul ? codes4x<MODE>(mul2(t0, cs.ci2), mul2(t1, cs.ci2), lp_fmt)
+                    : codes4x<MODE>(mul2(mul2(t0, cs.c2), cs.inv2), mul2(mul2(t1, cs.c2), cs.inv2), lp_fmt);
 }
 
 // Tensor-core operand layout of the minifloat codes: each group of 16 consecutive codes along
@@ -463,7 +494,7 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
     qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status, lp_fmt);
     if (qp.abort) return;
   }
-  const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
+  const CodeScale cs = code_scale<K>(c, qp.inv);
 
   const int64_t wpc = kQuantThreads / 32;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * wpc + warp;
@@ -536,9 +567,18 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
       } else {
         const int64_t ub = u * kRowsWarpElems;
         uint32_t w[8];
+        if (cs.one_mul) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          w[j] = qp.zero ? 0u : codes4x<MODE>(mul2(mul2(v[2 * j], c2), inv2), mul2(mul2(v[2 * j + 1], c2), inv2), lp_fmt);
+          for (int j = 0; j < 8; ++j) w[j] = codes4x<MODE>(mul2(v[2 * j], cs.ci2), mul2(v[2 * j + 1], cs.ci2), lp_fmt);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            w[j] = codes4x<MODE>(mul2(mul2(v[2 * j], cs.c2), cs.inv2), mul2(mul2(v[2 * j + 1], cs.c2), cs.inv2), lp_fmt);
+        }
+        if (qp.zero) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[j] = 0u;
+        }
         const bool full = ub + kRowsWarpElems <= n;  // all but a ragged last unit
         if constexpr (MODE == kModeLowp) {
           // minifloats: 16-code groups packed into 16-byte chunks (n is a multiple of 16)
@@ -632,7 +672,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
     qp = finish_absmax<MODE>(partials, n_partials, scale_out, scratch, status, lp_fmt);
     if (qp.abort) return;
   }
-  const float2 c2 = make_float2(c, c), inv2 = make_float2(qp.inv, qp.inv);
+  const CodeScale cs = code_scale<K>(c, qp.inv);
 
   const int64_t n_rt = (rows + kColsTileRows2 - 1) / kColsTileRows2;
   const int64_t n_ct = (cols + kColsTileCols2 - 1) / kColsTileCols2;
@@ -726,7 +766,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int i = 8 * j + 2 * e;
-                w[e] = qp.zero ? 0u : codes4x<MODE>(mul2(mul2(v[i], c2), inv2), mul2(mul2(v[i + 1], c2), inv2), lp_fmt);
+                w[e] = qp.zero ? 0u : scaled_codes4<MODE>(v[i], v[i + 1], cs, lp_fmt);
               }
               *reinterpret_cast<uint4*>(o + 16 * j) =
                   MODE == kModeLowp ? lowp_pack16(w[0], w[1], w[2], w[3], lp_fmt) : make_uint4(w[0], w[1], w[2], w[3]);
