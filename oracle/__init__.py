@@ -20,6 +20,10 @@ Every rotation runs along the contraction dimension of its GEMM:
     forward   Y  = X  W^T   contraction over K (d_in):  X along K, W along K
     backward  dX = dY W     contraction over N (d_out): dY along N, W along N
     backward  dW = dY^T X   contraction over M (tokens): dY along M, X along M  (left-hand)
+
+A second placement reuses the forward's codes (``linear_bwd_reuse``): dY is rotated along M
+only, dX multiplies its codes with the forward's K-rotated weight codes and undoes both
+rotations on the GEMM output.
 """
 from __future__ import annotations
 
@@ -100,6 +104,10 @@ def lib():
         L.hq_oracle_minifloat_encode.restype = ctypes.c_uint8
         L.hq_oracle_epilogue.argtypes = [p, i32, i64, ctypes.c_float, ctypes.c_float, p, p]
         L.hq_oracle_epilogue.restype = None
+        L.hq_oracle_dequant_f32.argtypes = [p, i32, i64, ctypes.c_float, ctypes.c_float, p]
+        L.hq_oracle_dequant_f32.restype = None
+        L.hq_oracle_f32_to_bf16.argtypes = [p, i64, p]
+        L.hq_oracle_f32_to_bf16.restype = None
         L.hq_oracle_threads.argtypes = []
         L.hq_oracle_threads.restype = i32
         _lib = L
@@ -359,3 +367,77 @@ def linear_bwd_dw(dY, X, k, fmt, rows=None, neg=None):
     """dW[N][K] = dY^T X: both rotated along the token dimension M (HALO-2 left-hand).
     neg: optional sign flags over M."""
     return _gemm_layer(dY, 0, X, 0, k, fmt, rows, neg)
+
+
+# ------------------------------------------------- rotated-output placement (forward codes reused)
+#
+# "HALO: Hadamard-Assisted Lower-Precision Optimization for LLMs", Approach: the quantized
+# rotated tensors of the forward pass are reused, and the backward pass puts a left-hand
+# Hadamard on the output gradient; "Training Transformers with 4-bit Integers", section 4: the
+# backward GEMMs quantize only the output gradient and reuse the forward's quantized activations
+# and weights.  With Wq = Q(W H) kept from the forward (rotated along K, [N][K]) and dY rotated
+# along the tokens M once (G = Q(H dY), stored [N][M] as for dW):
+#
+#     dX = dY W = H (H dY) (W H) H      (H symmetric and orthonormal: H H = I)
+#        ~ H [ s_g s_w * G^T Wq ] H     GEMM contraction over N, then both rotations undone on
+#                                       the output: along its columns (K), then its rows (M).
+#
+# Reading: the de-rotation runs on the fp32 dequantized accumulators (the epilogue's
+# fp32(acc) * fp32(s_g * s_w)), as two rotations like `rotate` (butterflies bit 0 first, then
+# x fp32(1/sqrt(k))), columns first; the result is rounded to bf16 once at the end.
+
+
+def dequant_f32(acc: np.ndarray, sa: float, sb: float) -> np.ndarray:
+    """fp32(acc) * fp32(sa * sb) elementwise, fp32 (the epilogue before its bf16 rounding)."""
+    acc = np.ascontiguousarray(acc)
+    kind = 0 if acc.dtype == np.int32 else 1
+    if kind == 1:
+        acc = acc.astype(np.float64, copy=False)
+    z = np.empty(acc.shape, dtype=np.float32)
+    lib().hq_oracle_dequant_f32(_ptr(acc), kind, acc.size, float(sa), float(sb), _ptr(z))
+    return z
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) of fp32 values, round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().hq_oracle_f32_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def derotate_output(Z: np.ndarray, k: int) -> np.ndarray:
+    """blockdiag(H_k/sqrt k) applied to Z[rows][cols] on both sides, in fp32: along the columns
+    (each row's k-blocks) first, then along the rows.  Both dims must be multiples of k."""
+    Z1 = rotate(np.ascontiguousarray(Z, dtype=np.float32), 1, k)  # [rows][cols]
+    return np.ascontiguousarray(rotate(Z1, 0, k).T)                # rotate gives [cols][rows]
+
+
+def linear_bwd_dx_reuse(g_codes, s_g, wq_codes, s_w, k, fmt, rows=None):
+    """dX[M][K] from dY's token-rotated codes g_codes[N][M] (scale s_g) and the forward's
+    weight codes wq_codes[N][K] (rotated along K, scale s_w):
+    bf16( H [fp32(G^T Wq) scaled] H ).
+
+    rows: optional first row of each k-row block to evaluate (sampling whole blocks, since the
+    rows of a block mix); returns the rows of those blocks in order.
+
+    Returns dict(acc, z, out): accumulators, fp32 de-rotated values, bf16 bits."""
+    A = np.ascontiguousarray(np.asarray(g_codes).T)   # [M][N]
+    B = np.ascontiguousarray(np.asarray(wq_codes).T)  # [K][N]
+    sel = None
+    if rows is not None:
+        sel = np.concatenate([np.arange(r, r + k) for r in np.asarray(rows, dtype=np.int64)])
+    acc = gemm(A, B, fmt, sel)
+    z = derotate_output(dequant_f32(acc, s_g, s_w), k)
+    return dict(acc=acc, z=z, out=f32_to_bf16(z))
+
+
+def linear_bwd_reuse(dY, xqt_codes, s_x, wq_codes, s_w, k, fmt):
+    """Backward of the reuse placement: dY is quantized once, rotated along M ([N][M]); dW uses
+    it with the saved token-rotated X codes (as linear_bwd_dw), dX with the forward's weight
+    codes (linear_bwd_dx_reuse).  Returns dict(g, s_g, dw, dx) with bf16 bits."""
+    g, s_g = quantize(dY, 0, k, fmt)
+    dw_acc = gemm(g, np.asarray(xqt_codes), fmt)
+    _, dw = epilogue(dw_acc, s_g, s_x)
+    dx = linear_bwd_dx_reuse(g, s_g, wq_codes, s_w, k, fmt)
+    return dict(g=g, s_g=s_g, dw=dw, dx=dx["out"], dx_z=dx["z"])

@@ -380,3 +380,21 @@ void hq_oracle_epilogue(const void* acc, int acc_kind, int64_t n, float sa, floa
         }
     }
 }
+
+/* ---------------------------------------------------------------- rotated-output placement */
+
+/* The accumulators scaled to fp32 without the bf16 rounding: z = fp32(acc) * fp32(s_a * s_b),
+ * every step fp32 RNE (the "fast" epilogue formula above, stopped before bf16).  Used where
+ * the GEMM's output is still rotated and is de-rotated in fp32 before it is rounded. */
+void hq_oracle_dequant_f32(const void* acc, int acc_kind, int64_t n, float sa, float sb, float* z) {
+    float sab = sa * sb;
+    for (int64_t i = 0; i < n; ++i) {
+        float af = acc_kind == 0 ? (float)((const int32_t*)acc)[i] : (float)((const double*)acc)[i];
+        z[i] = af * sab;
+    }
+}
+
+/* bf16 bit patterns of n fp32 values, each rounded to nearest even. */
+void hq_oracle_f32_to_bf16(const float* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = hq_oracle_bf16_from_f32(x[i]);
+}

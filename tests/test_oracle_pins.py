@@ -613,3 +613,105 @@ def test_signed_layer_wiring(oracle_lib):
     qb, sb = oracle.quantize(d["W"], 1, k, oracle.INT8, neg=1 - neg)
     acc = oracle.gemm(qa, qb, oracle.INT8).astype(np.float64) * float(sa) * float(sb)
     assert np.linalg.norm(acc - X @ W.T) / np.linalg.norm(X @ W.T) > 0.5
+
+
+# ------------------------------------------------- rotated-output placement (forward codes reused)
+
+def _blockdiag_h(n, k):
+    """fp64 blockdiag(H_k) of size n (scipy's Sylvester construction), unnormalised."""
+    return scipy.linalg.block_diag(*([scipy.linalg.hadamard(k).astype(np.float64)] * (n // k)))
+
+
+@pytest.mark.parametrize("k", KS)
+def test_derotate_output_one_hot_closed_form(oracle_lib, k):
+    """E_ij -> c^2 h_i h_j^T on the (row block of i) x (column block of j): every butterfly is
+    exact for a one-hot input, so the value is fp32(c * c) with the Sylvester sign
+    (-1)^(popcount(i' & a) + popcount(j' & b)), zero outside the two blocks."""
+    c = oracle.norm_const(k)
+    mag = np.float32(c) * np.float32(c)
+    H = scipy.linalg.hadamard(k)
+    for (i, j) in ((0, 0), (k + 3 % k, 1), (2 * k - 1, k // 2), (5 % k, 2 * k - 1)):
+        Z = np.zeros((2 * k, 3 * k), dtype=np.float32)
+        Z[i, j] = 1.0
+        got = oracle.derotate_output(Z, k)
+        want = np.zeros_like(Z)
+        r0, c0 = (i // k) * k, (j // k) * k
+        want[r0:r0 + k, c0:c0 + k] = mag * np.outer(H[i % k], H[j % k]).astype(np.float32)
+        np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("k", KS)
+def test_derotate_output_close_to_dense(oracle_lib, k):
+    """Against the fp64 product H Z H / k with scipy's block-diagonal Hadamard matrices: equal
+    up to fp32 rounding of log2(k) butterfly stages per side."""
+    rng = np.random.default_rng(k)
+    Z = rng.standard_normal((2 * k, 3 * k)).astype(np.float32)
+    want = _blockdiag_h(2 * k, k) @ Z.astype(np.float64) @ _blockdiag_h(3 * k, k) / k
+    got = oracle.derotate_output(Z, k).astype(np.float64)
+    assert np.abs(got - want).max() < 1e-4
+
+
+@pytest.mark.parametrize("k", (16, 128))
+def test_derotate_output_involution(oracle_lib, k):
+    rng = np.random.default_rng(7)
+    Z = rng.standard_normal((k, 2 * k)).astype(np.float32)
+    back = oracle.derotate_output(oracle.derotate_output(Z, k), k)
+    assert np.abs(back - Z).max() < 1e-5
+
+
+def test_dequant_f32_and_bf16_rounding(oracle_lib):
+    """dequant_f32 is the fp32 product with the fp32 product of the scales (numpy's IEEE
+    single arithmetic), f32_to_bf16 agrees with torch's round-to-nearest-even conversion."""
+    rng = np.random.default_rng(3)
+    acc = rng.integers(-2**24, 2**24, size=1000).astype(np.int32)
+    sa, sb = np.float32(0.0123), np.float32(3.7e-3)
+    np.testing.assert_array_equal(oracle.dequant_f32(acc, sa, sb), acc.astype(np.float32) * (sa * sb))
+    x = (rng.standard_normal(4096) * 10.0 ** rng.integers(-30, 30, 4096)).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.f32_to_bf16(x), want)
+
+
+def _reuse_case(fmt):
+    w = synthetic.WORKLOADS[1]
+    d = synthetic.draw(w)
+    k = w.k
+    wq, sw = oracle.quantize(d["W"], 1, k, fmt)    # forward's W codes, rotated along K
+    xq, sx = oracle.quantize(d["X"], 0, k, fmt)    # saved X codes, rotated along M
+    return w, d, k, wq, sw, xq, sx
+
+
+@pytest.mark.parametrize("fmt", (oracle.INT8, oracle.FP8_E4M3))
+def test_reuse_backward_tracks_unquantized_products(oracle_lib, fmt):
+    """dX from dY's token-rotated codes and the forward's K-rotated weight codes approximates
+    dY W once both rotations are undone on the output; leaving out either de-rotation (a
+    mistake planted here, on the CPU) or transposing the weight codes gives errors near 1."""
+    w, d, k, wq, sw, xq, sx = _reuse_case(fmt)
+    X, W, dY = (d[n].astype(np.float64) for n in ("X", "W", "dY"))
+    f = oracle.bf16_bits_to_f32
+    r = oracle.linear_bwd_reuse(d["dY"], xq, sx, wq, sw, k, fmt)
+    assert r["dx"].shape == (64, 256) and r["dw"].shape == (128, 256)
+    assert _rel_fro(f(r["dx"]), dY @ W) < 0.1
+    assert _rel_fro(f(r["dw"]), dY.T @ X) < 0.1
+    acc = oracle.gemm(np.ascontiguousarray(r["g"].T), np.ascontiguousarray(wq.T), fmt)
+    z = oracle.dequant_f32(acc, r["s_g"], sw)
+    only_cols = oracle.rotate(z, 1, k)
+    only_rows = np.ascontiguousarray(oracle.rotate(z, 0, k).T)
+    for bad in (z, only_cols, only_rows):
+        assert _rel_fro(bad.astype(np.float64), dY @ W) > 0.5
+    wrong = oracle.linear_bwd_dx_reuse(r["g"], r["s_g"], np.ascontiguousarray(np.flip(wq, 0)), sw, k, fmt)
+    assert _rel_fro(f(wrong["out"]), dY @ W) > 0.5
+
+
+def test_reuse_dw_is_the_standard_dw(oracle_lib):
+    """The reuse placement's dW is the HALO-2 dW: same dY codes along M, same X codes."""
+    w, d, k, wq, sw, xq, sx = _reuse_case(oracle.INT8)
+    r = oracle.linear_bwd_reuse(d["dY"], xq, sx, wq, sw, k, oracle.INT8)
+    np.testing.assert_array_equal(r["dw"], oracle.linear_bwd_dw(d["dY"], d["X"], k, oracle.INT8)["fast"])
+
+
+def test_reuse_dx_row_block_sampling(oracle_lib):
+    """Sampling whole k-row blocks gives exactly those rows of the full result."""
+    w, d, k, wq, sw, xq, sx = _reuse_case(oracle.INT8)
+    r = oracle.linear_bwd_reuse(d["dY"], xq, sx, wq, sw, k, oracle.INT8)
+    part = oracle.linear_bwd_dx_reuse(r["g"], r["s_g"], wq, sw, k, oracle.INT8, rows=[2 * k, 0])
+    np.testing.assert_array_equal(part["out"], np.concatenate([r["dx"][2 * k:3 * k], r["dx"][:k]]))
