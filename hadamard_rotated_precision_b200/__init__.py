@@ -34,6 +34,9 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_bwd_workspace_bytes", "hq_linear_bwd", "hq_selftest_gemm_timeout",
            "hq_quantize_rht", "hq_quantize_dual_rht", "hq_linear_fwd_bwd_rht",
            "hq_quantize_absmax", "hq_quantize_codes",
+           "hq_linear_fwd_keep_workspace_bytes", "hq_linear_fwd_keep",
+           "hq_linear_bwd_dx_reuse_workspace_bytes", "hq_linear_bwd_dx_reuse",
+           "hq_linear_bwd_reuse_workspace_bytes", "hq_linear_bwd_reuse",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -92,6 +95,16 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_fwd_save.restype = i32
         L.hq_linear_bwd.argtypes = [p, p, p, p, i32, i64, i64, i64, i32, i32, p, p, p, sz, p]
         L.hq_linear_bwd.restype = i32
+        for name in ("hq_linear_fwd_keep_workspace_bytes", "hq_linear_bwd_dx_reuse_workspace_bytes",
+                     "hq_linear_bwd_reuse_workspace_bytes"):
+            getattr(L, name).argtypes = [i64, i64, i64]
+            getattr(L, name).restype = sz
+        L.hq_linear_fwd_keep.argtypes = [p, p, i32, i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, p]
+        L.hq_linear_fwd_keep.restype = i32
+        L.hq_linear_bwd_dx_reuse.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p, sz, p]
+        L.hq_linear_bwd_dx_reuse.restype = i32
+        L.hq_linear_bwd_reuse.argtypes = [p, i32, p, p, p, p, i64, i64, i64, i32, i32, p, p, p, sz, p]
+        L.hq_linear_bwd_reuse.restype = i32
         L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm.restype = i32
         L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]
@@ -488,6 +501,93 @@ def hq_linear_bwd(dY, W, xqt, xqt_scale, k: int, fmt, dX=None, dW=None, workspac
                              _fmt(fmt), dX.data_ptr(), dW.data_ptr(), ws.data_ptr(),
                              ws.numel() * ws.element_size(), _stream_handle(stream))
     _check(st, "hq_linear_bwd")
+    return dX, dW
+
+
+def hq_linear_fwd_keep_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_fwd_keep_workspace_bytes(M, K, N))
+
+
+def hq_linear_fwd_keep(X, W, k: int, fmt, Y=None, xqt=None, xqt_scale=None, wq=None, wq_scale=None,
+                       workspace=None, stream=None):
+    """hq_linear_fwd_save that also returns W's K-rotated codes (wq [N][K] uint8 + device scale)
+    for hq_linear_bwd_reuse.  Returns (Y, xqt, xqt_scale, wq, wq_scale)."""
+    torch = _torch()
+    _dev_tensor(X, "X")
+    _dev_tensor(W, "W")
+    dt = _src_dtype(X, "X")
+    if _src_dtype(W, "W") != dt:
+        raise TypeError("X and W must have the same dtype")
+    M, K = X.shape
+    N = W.shape[0]
+    dev = X.device
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if Y is None else Y
+    xqt = torch.empty((K, M), dtype=torch.uint8, device=dev) if xqt is None else xqt
+    xqt_scale = torch.empty((1,), dtype=torch.float32, device=dev) if xqt_scale is None else xqt_scale
+    wq = torch.empty((N, K), dtype=torch.uint8, device=dev) if wq is None else wq
+    wq_scale = torch.empty((1,), dtype=torch.float32, device=dev) if wq_scale is None else wq_scale
+    for t, n in ((Y, "Y"), (xqt, "xqt"), (xqt_scale, "xqt_scale"), (wq, "wq"), (wq_scale, "wq_scale")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_fwd_keep_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_fwd_keep(X.data_ptr(), W.data_ptr(), dt, M, K, N, k, _fmt(fmt), Y.data_ptr(),
+                                  xqt.data_ptr(), xqt_scale.data_ptr(), wq.data_ptr(), wq_scale.data_ptr(),
+                                  ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_linear_fwd_keep")
+    return Y, xqt, xqt_scale, wq, wq_scale
+
+
+def hq_linear_bwd_dx_reuse_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N))
+
+
+def hq_linear_bwd_dx_reuse(g, g_scale, wq, wq_scale, k: int, fmt, dX=None, workspace=None, stream=None):
+    """dX [M][K] bf16 = H [G^T-contraction with Wq, dequantized in fp32] H from dY's token-rotated
+    codes g [N][M] and the forward's K-rotated weight codes wq [N][K]."""
+    torch = _torch()
+    for t, n in ((g, "g"), (g_scale, "g_scale"), (wq, "wq"), (wq_scale, "wq_scale")):
+        _dev_tensor(t, n)
+    N, M = g.shape
+    if wq.shape[0] != N:
+        raise ValueError("g and wq must share their first (contraction) dimension")
+    K = wq.shape[1]
+    dev = g.device
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    _dev_tensor(dX, "dX")
+    ws = _workspace(hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_bwd_dx_reuse(g.data_ptr(), g_scale.data_ptr(), wq.data_ptr(), wq_scale.data_ptr(), M, K, N,
+                                      k, _fmt(fmt), dX.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                      _stream_handle(stream))
+    _check(st, "hq_linear_bwd_dx_reuse")
+    return dX
+
+
+def hq_linear_bwd_reuse_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().hq_linear_bwd_reuse_workspace_bytes(M, K, N))
+
+
+def hq_linear_bwd_reuse(dY, xqt, xqt_scale, wq, wq_scale, k: int, fmt, dX=None, dW=None, workspace=None,
+                        stream=None):
+    """(dX, dW) of one layer from dY and the codes hq_linear_fwd_keep kept: dY quantized once
+    along the tokens, dW from the saved X codes, dX from the weight codes with both rotations
+    undone on the output."""
+    torch = _torch()
+    for t, n in ((dY, "dY"), (xqt, "xqt"), (xqt_scale, "xqt_scale"), (wq, "wq"), (wq_scale, "wq_scale")):
+        _dev_tensor(t, n)
+    dt = _src_dtype(dY, "dY")
+    M, N = dY.shape
+    K = wq.shape[1]
+    if tuple(xqt.shape) != (K, M) or wq.shape[0] != N:
+        raise ValueError(f"xqt must be [K][M] = [{K}][{M}] and wq [N][K] = [{N}][{K}]")
+    dev = dY.device
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if dW is None else dW
+    for t, n in ((dX, "dX"), (dW, "dW")):
+        _dev_tensor(t, n)
+    ws = _workspace(hq_linear_bwd_reuse_workspace_bytes(M, K, N), dev, workspace)
+    st = lib().hq_linear_bwd_reuse(dY.data_ptr(), dt, xqt.data_ptr(), xqt_scale.data_ptr(), wq.data_ptr(),
+                                   wq_scale.data_ptr(), M, K, N, k, _fmt(fmt), dX.data_ptr(), dW.data_ptr(),
+                                   ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_linear_bwd_reuse")
     return dX, dW
 
 

@@ -43,7 +43,9 @@ constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + NUM_BARS * 8
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s per wait
 
 enum Fmt : int { kInt8 = 0, kFp8 = 1 };
-enum Out : int { kOutBf16 = 0, kOutAcc = 1 };
+// kOutF32: the dequantized value fp32(acc) * fp32(s_a * s_b) without the bf16 rounding (for an
+// output that is still rotated and is de-rotated in fp32 afterwards).
+enum Out : int { kOutBf16 = 0, kOutAcc = 1, kOutF32 = 2 };
 
 // Instruction descriptor: dense, D = s32 (int8) / f32 (fp8), A = B = s8 / e4m3, both K-major,
 // N = 256, M = 128.
@@ -143,6 +145,19 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], void* out, 
         pk[e] = *reinterpret_cast<const uint32_t*>(&h);
       }
       *reinterpret_cast<uint4*>(o + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  } else if (OUT == kOutF32) {
+    float* o = reinterpret_cast<float*>(out) + row * N + col0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (col0 + 4 * q + 4 > N) break;
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t u = r[4 * q + e];
+        x[e] = __fmul_rn(FMT == kInt8 ? __int2float_rn(static_cast<int>(u)) : __uint_as_float(u), sab);
+      }
+      *reinterpret_cast<float4*>(o + 4 * q) = make_float4(x[0], x[1], x[2], x[3]);
     }
   } else {
     uint32_t* o = reinterpret_cast<uint32_t*>(out) + row * N + col0;
@@ -368,7 +383,12 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
   return s;
 }
 
-template <int FMT, int OUT, int BN_, bool SHORT_K>
+// MN: both operands MN-major, i.e. stored contraction-outermost (A as [K][M], B as [K][N]; the
+// kind::i8 and e4m3 inputs allow it).  A TMA box is then 128 contraction rows of 128 bytes
+// along M (or N): one 128-byte swizzle atom wide, so the smem descriptor keeps its 1024-byte
+// stride between 8-row groups (now groups along the contraction), and one MMA's 32-deep slice
+// starts 32 rows = 4096 bytes further on.  Needs BN_ = 256 (128 B rows per CTA).
+template <int FMT, int OUT, int BN_, bool SHORT_K, bool MN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
@@ -376,6 +396,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                  unsigned int* __restrict__ status, int splits, uint32_t* __restrict__ part_ws,
                  int* __restrict__ counters, uint32_t ab_code) {
   using G = Geo<BN_, SHORT_K>;
+  static_assert(!MN || (BN_ == 256 && !SHORT_K && OUT != kOutBf16), "MN-major operands: 256-wide tiles, direct stores");
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -441,10 +462,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
           const uint32_t fb = ptx::mapa_shared(full_bar(stage), 0);
           if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          ptx::tma_load_2d_pair(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, kb * BK,
-                                m_blk * BM + int(rank) * HALF, fb);
-          ptx::tma_load_2d_pair(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, kb * BK,
-                                n_blk * BN + int(rank) * G::B_ROWS, fb);
+          const int a_mn = m_blk * BM + int(rank) * HALF, b_mn = n_blk * BN + int(rank) * G::B_ROWS;
+          ptx::tma_load_2d_pair(ptx::smem_u32(sh.a + stage * A_STAGE_BYTES), &tmap_a, MN ? a_mn : kb * BK,
+                                MN ? kb * BK : a_mn, fb);
+          ptx::tma_load_2d_pair(ptx::smem_u32(sh.b + stage * B_STAGE_BYTES), &tmap_b, MN ? b_mn : kb * BK,
+                                MN ? kb * BK : b_mn, fb);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -460,7 +482,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     // ---------------------------------------------------------------- MMA issuer (CTA 0)
     if (lane == 0 && leader) {
       // ab_code: the A and B element format of kind::f8f6f4 (e4m3 0, e2m3 3, e3m2 4, e2m1 5)
-      const uint32_t idesc = instr_desc<FMT, BN_>() | (ab_code << 7) | (ab_code << 10);
+      // bits 15 / 16: A / B MN-major
+      const uint32_t idesc = instr_desc<FMT, BN_>() | (ab_code << 7) | (ab_code << 10) | (MN ? (3u << 15) : 0u);
+      constexpr uint32_t kk_step = MN ? UMMA_K * 128 : UMMA_K;  // bytes between consecutive MMAs' slices
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -479,8 +503,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           const uint32_t b_addr = ptx::smem_u32(sh.b + stage * B_STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a_addr + kk * UMMA_K);
-            const uint64_t bd = smem_desc_sw128(b_addr + kk * UMMA_K);
+            const uint64_t ad = smem_desc_sw128(a_addr + kk * kk_step);
+            const uint64_t bd = smem_desc_sw128(b_addr + kk * kk_step);
             const uint32_t accumulate = (kb > kb_begin || kk > 0) ? 1u : 0u;
             if (FMT == kInt8) ptx::mma_i8_pair(d_tmem, ad, bd, idesc, accumulate);
             else ptx::mma_f8_pair(d_tmem, ad, bd, idesc, accumulate);
@@ -498,7 +522,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int quarter = warp & 3;
-    const float sab = (OUT == kOutBf16) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
+    const float sab = (OUT != kOutAcc) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
     // bf16 output: chunk j (64 columns) of this warp's 32 rows goes TMEM -> registers -> a
     // swizzled 32 x 64 box in shared memory -> TMA store (asynchronous).  Box b of the warp's
     // NB boxes is rewritten only once the store that last used it has read it.

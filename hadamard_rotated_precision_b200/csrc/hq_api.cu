@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -13,6 +14,7 @@
 #include "fwht_quant.cuh"
 #include "fwht_dual.cuh"
 #include "gemm_tcgen05.cuh"
+#include "rotate_out.cuh"
 
 namespace {
 
@@ -36,6 +38,7 @@ struct DeviceInfo {
   bool cols_attr[5][4][2] = {};  // strided bf16 quantizer instantiations prepared [k][mode][signed]
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
   bool dual_attr[5][4][2][2] = {};  // fused two-rotation instantiations prepared [k][mode][w32][signed]
+  bool mn_attr[2] = {};             // MN-major pair GEMM (fp32 output) prepared [int8 / fp8]
 };
 
 std::mutex g_mu;
@@ -578,13 +581,13 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
   return c;
 }
 
-template <int FMT, int OUT, int BN, bool SK>
+template <int FMT, int OUT, int BN, bool SK, bool MN = false>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
                              const float* sb, void* out, int M, int N, int K, int clusters, int splits,
                              uint32_t* part_ws, int* counters, uint32_t ab_code, DeviceInfo& d, cudaStream_t st) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN, SK>;
-  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK>;
+  auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK, MN>;
   const int items = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN) * splits;
   const int pairs = std::max(1, std::min(items, clusters));
   cudaLaunchConfig_t cfg = {};
@@ -748,6 +751,92 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
                             : launch_gemm<kFp8, kOutAcc>(ta, tb, sa, sb, out, m, n, kk, d, st, ab);
   }
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------ rotated-output placement
+
+// out[M][N] fp32 = fp32(sum_l A[l][i] B[l][j]) * fp32(s_a * s_b) with both operands stored
+// contraction-outermost: A as [K][M], B as [K][N] (the token-rotated output-gradient codes and
+// the forward's K-rotated weight codes); CTA pairs, 256 x 256 tiles.
+hq_status gemm_mn_f32_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
+                           int64_t K, hq_fmt fmt, float* out, DeviceInfo& d, cudaStream_t st) {
+  namespace gp = hq::gemm::pair;
+  using G = gp::Geo<256, false>;
+  const int f = fmt == HQ_INT8 ? 0 : 1;
+  const void* kernel = f == 0 ? reinterpret_cast<const void*>(gp::gemm_pair_kernel<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false, true>)
+                              : reinterpret_cast<const void*>(gp::gemm_pair_kernel<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false, true>);
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d.mn_attr[f]) {
+      if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(G::SMEM_BYTES))) != cudaSuccess)
+        return cuda_fail(e);
+      d.mn_attr[f] = true;
+    }
+  }
+  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms);
+  CUtensorMap ta, tb, to;
+  std::memset(&to, 0, sizeof(to));
+  // boxes of 128 contraction rows x 128 bytes along M (N): the K-major map with the roles of
+  // its two dimensions exchanged
+  hq_status s = encode_codes_map(&ta, A, K, M, gp::HALF);
+  if (s != HQ_OK) return s;
+  if ((s = encode_codes_map(&tb, B, K, N, G::B_ROWS)) != HQ_OK) return s;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
+  e = f == 0 ? launch_gemm_pair<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false, true>(
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st)
+             : launch_gemm_pair<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false, true>(
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+template <int K>
+cudaError_t launch_derotate_k(float* z, int64_t rows, int64_t cols, __nv_bfloat16* out, DeviceInfo& d,
+                              cudaStream_t st) {
+  const float c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(K)));  // fp32(1/sqrt(k)), one rounding
+  const int64_t n8 = rows * cols / 8;
+  const int64_t blocks_c = std::min<int64_t>((n8 + hq::rot::kThreads - 1) / hq::rot::kThreads, int64_t(d.sms) * 8);
+  hq::rot::rot_cols_f32_kernel<K><<<static_cast<unsigned>(std::max<int64_t>(1, blocks_c)), hq::rot::kThreads, 0, st>>>(z, n8, c);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t blocks_r = ((rows + 255) / 256) * ((cols + 31) / 32);
+  hq::rot::rot_rows_f32_bf16_kernel<K><<<static_cast<unsigned>(blocks_r), hq::rot::kThreads, 0, st>>>(z, rows, cols, c, out);
+  return cudaGetLastError();
+}
+
+// out = bf16(H Z H): Z's columns rotated in place, then its rows into out.
+hq_status derotate_impl(float* z, int64_t rows, int64_t cols, int k, void* out, DeviceInfo& d, cudaStream_t st) {
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  cudaError_t e;
+  switch (k) {
+    case 16: e = launch_derotate_k<16>(z, rows, cols, o, d, st); break;
+    case 32: e = launch_derotate_k<32>(z, rows, cols, o, d, st); break;
+    case 64: e = launch_derotate_k<64>(z, rows, cols, o, d, st); break;
+    case 128: e = launch_derotate_k<128>(z, rows, cols, o, d, st); break;
+    default: e = launch_derotate_k<256>(z, rows, cols, o, d, st); break;
+  }
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// Shape rules of the reuse placement's dX: M and K are rotated (multiples of k and below 2^31),
+// N is the contraction.
+hq_status check_dx_reuse_shape(int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt) {
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0) return HQ_ERR_ARG;
+  if (M == 0 || K == 0 || N == 0) return HQ_ERR_SHAPE;
+  if (M % k || K % k) return HQ_ERR_SHAPE;
+  if (fmt == HQ_INT8 && N > HQ_MAX_K_INT8) return HQ_ERR_SHAPE;
+  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return HQ_ERR_SHAPE;
+  return HQ_OK;
+}
+
+hq_status dx_reuse_impl(const void* g_codes, const float* g_scale, const void* wq_codes, const float* wq_scale,
+                        int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt, void* dX, float* z, DeviceInfo& d,
+                        cudaStream_t st) {
+  hq_status s = gemm_mn_f32_impl(g_codes, g_scale, wq_codes, wq_scale, M, K, N, fmt, z, d, st);
+  if (s != HQ_OK) return s;
+  return derotate_impl(z, M, K, k, dX, d, st);
 }
 
 // ------------------------------------------------------------------ the linear layer
@@ -1156,17 +1245,27 @@ size_t hq_linear_fwd_save_workspace_bytes(int64_t M, int64_t K, int64_t N) {
   return codes_ws_bytes(M * K, N * K, 0, split_ws_bytes(M, N, K));
 }
 
-hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
-                             hq_fmt fmt, void* Y, void* xqt_codes, float* xqt_scale, void* workspace,
-                             size_t ws_bytes, hq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// hq_linear_fwd_save, and with wq_codes / wq_scale non-null hq_linear_fwd_keep (W's K-rotated
+// codes and scale go to the caller's buffers instead of the workspace).
+hq_status fwd_save_impl(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                        hq_fmt fmt, void* Y, void* xqt_codes, float* xqt_scale, void* wq_codes, float* wq_scale,
+                        void* workspace, size_t ws_bytes, hq_stream_t stream) {
   hq_status s = check_step_shape(dt, M, K, N, k, fmt);
   if (s != HQ_OK) return s;
   if (!X || !W || !Y || !xqt_codes || !xqt_scale) return HQ_ERR_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || !aligned16(xqt_codes) ||
       (reinterpret_cast<uintptr_t>(xqt_scale) & 3u))
     return HQ_ERR_ALIGN;
+  if (wq_codes && (!aligned16(wq_codes) || (reinterpret_cast<uintptr_t>(wq_scale) & 3u))) return HQ_ERR_ALIGN;
   CodesWs w;
-  if ((s = carve_codes_ws(workspace, ws_bytes, M * K, N * K, 0, split_ws_bytes(M, N, K), &w)) != HQ_OK) return s;
+  if ((s = carve_codes_ws(workspace, ws_bytes, M * K, wq_codes ? 0 : N * K, 0, split_ws_bytes(M, N, K), &w)) != HQ_OK)
+    return s;
+  uint8_t* wc = wq_codes ? static_cast<uint8_t*>(wq_codes) : w.c[1];
+  float* ws_ = wq_codes ? wq_scale : w.scales + 1;
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1177,7 +1276,7 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
   if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
   if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
   // side stream: W along K
-  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, w.c[1], w.scales + 1, w.spart_c, *d, ss->s)) != HQ_OK) return s;
+  if ((s = quantize_impl(W, dt, N, K, 1, k, fmt, wc, ws_, w.spart_c, *d, ss->s)) != HQ_OK) return s;
   if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
   // caller's stream: X in both rotations (along K for the forward GEMM, along M kept for the
   // weight gradient), then the forward GEMM once W's codes have landed
@@ -1185,8 +1284,31 @@ hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t 
                      st)) != HQ_OK)
     return s;
   if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
-  return gemm_impl(w.c[0], w.scales + 0, w.c[1], w.scales + 1, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split,
-                   w.split_len);
+  return gemm_impl(w.c[0], w.scales + 0, wc, ws_, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split, w.split_len);
+}
+
+}  // namespace
+
+extern "C" {
+
+hq_status hq_linear_fwd_save(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                             hq_fmt fmt, void* Y, void* xqt_codes, float* xqt_scale, void* workspace,
+                             size_t ws_bytes, hq_stream_t stream) {
+  return fwd_save_impl(X, W, dt, M, K, N, k, fmt, Y, xqt_codes, xqt_scale, nullptr, nullptr, workspace, ws_bytes,
+                       stream);
+}
+
+size_t hq_linear_fwd_keep_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  return codes_ws_bytes(M * K, 0, 0, split_ws_bytes(M, N, K));
+}
+
+hq_status hq_linear_fwd_keep(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K, int64_t N, int k,
+                             hq_fmt fmt, void* Y, void* xqt_codes, float* xqt_scale, void* wq_codes, float* wq_scale,
+                             void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  if (!wq_codes || !wq_scale) return HQ_ERR_ARG;
+  return fwd_save_impl(X, W, dt, M, K, N, k, fmt, Y, xqt_codes, xqt_scale, wq_codes, wq_scale, workspace, ws_bytes,
+                       stream);
 }
 
 size_t hq_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N) {
@@ -1229,6 +1351,66 @@ hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, co
     return s;
   return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split,
                    w.split_len);
+}
+
+size_t hq_linear_bwd_dx_reuse_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  (void)N;
+  if (M < 0 || K < 0) return 0;
+  return align_up(size_t(M) * size_t(K) * 4);
+}
+
+hq_status hq_linear_bwd_dx_reuse(const void* g_codes, const float* g_scale, const void* wq_codes,
+                                 const float* wq_scale, int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt, void* dX,
+                                 void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_dx_reuse_shape(M, K, N, k, fmt);
+  if (s != HQ_OK) return s;
+  if (!g_codes || !g_scale || !wq_codes || !wq_scale || !dX) return HQ_ERR_ARG;
+  if (!aligned16(g_codes) || !aligned16(wq_codes) || !aligned16(dX) ||
+      (reinterpret_cast<uintptr_t>(g_scale) & 3u) || (reinterpret_cast<uintptr_t>(wq_scale) & 3u))
+    return HQ_ERR_ALIGN;
+  if (!workspace || ws_bytes < hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  return dx_reuse_impl(g_codes, g_scale, wq_codes, wq_scale, M, K, N, k, fmt, dX, static_cast<float*>(workspace), *d,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_linear_bwd_reuse_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  return align_up(size_t(N) * size_t(M)) + kAlign + kPartialBytes + align_up(size_t(M) * size_t(K) * 4) +
+         align_up(split_ws_bytes(N, K, M));
+}
+
+hq_status hq_linear_bwd_reuse(const void* dY, hq_dtype dt, const void* xqt_codes, const float* xqt_scale,
+                              const void* wq_codes, const float* wq_scale, int64_t M, int64_t K, int64_t N, int k,
+                              hq_fmt fmt, void* dX, void* dW, void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  hq_status s = check_step_shape(dt, M, K, N, k, fmt);
+  if (s != HQ_OK) return s;
+  if ((s = check_dx_reuse_shape(M, K, N, k, fmt)) != HQ_OK) return s;
+  if (!dY || !xqt_codes || !xqt_scale || !wq_codes || !wq_scale || !dX || !dW) return HQ_ERR_ARG;
+  if (!aligned16(dY) || !aligned16(xqt_codes) || !aligned16(wq_codes) || !aligned16(dX) || !aligned16(dW) ||
+      (reinterpret_cast<uintptr_t>(xqt_scale) & 3u) || (reinterpret_cast<uintptr_t>(wq_scale) & 3u))
+    return HQ_ERR_ALIGN;
+  if (!workspace || ws_bytes < hq_linear_bwd_reuse_workspace_bytes(M, K, N)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  auto take = [&](size_t n) { uint8_t* r = p; p += align_up(n); return r; };
+  uint8_t* g = take(size_t(N) * size_t(M));
+  float* g_scale = reinterpret_cast<float*>(take(kAlign));
+  float* partials = reinterpret_cast<float*>(take(kPartialBytes));
+  float* z = reinterpret_cast<float*>(take(size_t(M) * size_t(K) * 4));
+  const size_t split_len = split_ws_bytes(N, K, M);
+  void* split = split_len ? take(split_len) : nullptr;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // dY once, rotated along the tokens: [N][M], the weight gradient's operand as it is and the
+  // input gradient's MN-major operand
+  if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, g, g_scale, partials, *d, st)) != HQ_OK) return s;
+  if ((s = gemm_impl(g, g_scale, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, split, split_len)) != HQ_OK)
+    return s;
+  return dx_reuse_impl(g, g_scale, wq_codes, wq_scale, M, K, N, k, fmt, dX, z, *d, st);
 }
 
 hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,

@@ -1,0 +1,146 @@
+// De-rotation of a GEMM output that is still rotated on both sides: out = bf16(H Z H), H =
+// blockdiag(H_k / sqrt(k)), Z fp32 [rows][cols] (the dequantized accumulators).
+//
+// Method: "HALO: Hadamard-Assisted Lower-Precision Optimization for LLMs", Approach (the
+// quantized rotated tensors of the forward pass are reused in the backward pass, which puts a
+// left-hand Hadamard on the output gradient): the input gradient then comes out of its GEMM
+// rotated along the tokens (rows) and along K (columns), and both rotations are undone here.
+//
+// Numerics, as the library's rotation: Sylvester butterflies h = 1, 2, ..., k/2 (index bit 0
+// first), every add / sub fp32 round-to-nearest-even, then one multiply by fp32(1/sqrt(k));
+// the columns' rotation (each row's k-blocks) runs first, in place in fp32, then the rows',
+// which rounds to bf16 once at the end.
+//
+// Both kernels stream: 4 bytes read and written per element (columns), 4 read and 2 written
+// (rows).
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace hq {
+namespace rot {
+
+constexpr int kThreads = 256;
+
+// Along the columns, in place.  A thread holds 8 consecutive elements (index bits 0-2 in
+// registers), the k/8 lanes of one k-block hold the rest (bits 3.. across lanes); a warp
+// covers 256 consecutive elements, so a block never straddles warps (cols % k == 0).
+template <int K>
+__global__ void __launch_bounds__(kThreads) rot_cols_f32_kernel(float* __restrict__ z, int64_t n8, float c) {
+  static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = int64_t(blockIdx.x) * kThreads; base < n8; base += int64_t(gridDim.x) * kThreads) {
+    const int64_t i = base + threadIdx.x;
+    const bool valid = i < n8;
+    float v[8];
+    if (valid) {
+      const float4 a = *reinterpret_cast<const float4*>(z + 8 * i);
+      const float4 b = *reinterpret_cast<const float4*>(z + 8 * i + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j & h) continue;
+        const float u = v[j], w = v[j + h];
+        v[j] = __fadd_rn(u, w);
+        v[j + h] = __fsub_rn(u, w);
+      }
+    }
+    // bit 3 + s lives in lane bit s: the lower lane keeps u + w, the upper one u - w
+#pragma unroll
+    for (int m = 1; m < K / 8; m <<= 1) {
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float p = __shfl_xor_sync(0xFFFFFFFFu, v[j], m);
+        v[j] = upper ? __fsub_rn(p, v[j]) : __fadd_rn(v[j], p);
+      }
+    }
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], c);
+      *reinterpret_cast<float4*>(z + 8 * i) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(z + 8 * i + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
+// Along the rows, fp32 in, bf16 out.  A CTA takes a tile of 256 rows x 32 columns (whole
+// k-blocks of rows, since rows % k == 0 and k divides 256):
+//   phase 1: thread (warp w, lane l) holds column l, rows 32w .. 32w+31 (bits 0-4 of the row
+//            in registers) and runs the stages h = 1 .. 16;
+//   phase 2 (k >= 64): through shared memory, the thread holds rows r + 32j (j = 0..7) for
+//            r = 4w .. 4w+3 (bits 5-7 in registers) and runs the stages h = 32 .. k/2.
+// Both phases read and write shared memory along a row (lanes = columns): conflict-free.
+template <int K>
+__global__ void __launch_bounds__(kThreads) rot_rows_f32_bf16_kernel(const float* __restrict__ z, int64_t rows,
+                                                                     int64_t cols, float c,
+                                                                     __nv_bfloat16* __restrict__ out) {
+  static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  constexpr int kTileRows = 256, kTileCols = 32;
+  __shared__ float tile[K >= 64 ? kTileRows : 1][kTileCols];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t col_tiles = (cols + kTileCols - 1) / kTileCols;
+  const int64_t row0 = (int64_t(blockIdx.x) / col_tiles) * kTileRows;
+  const int64_t col = (int64_t(blockIdx.x) % col_tiles) * kTileCols + lane;
+  const bool col_ok = col < cols;
+
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int64_t r = row0 + 32 * warp + i;
+    v[i] = (col_ok && r < rows) ? z[r * cols + col] : 0.0f;
+  }
+  constexpr int H1 = K < 32 ? K : 32;  // phase 1 covers h < H1
+#pragma unroll
+  for (int h = 1; h < H1; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i & h) continue;
+      const float u = v[i], w = v[i + h];
+      v[i] = __fadd_rn(u, w);
+      v[i + h] = __fsub_rn(u, w);
+    }
+  }
+  if constexpr (K <= 32) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t r = row0 + 32 * warp + i;
+      if (col_ok && r < rows) out[r * cols + col] = __float2bfloat16_rn(__fmul_rn(v[i], c));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) tile[32 * warp + i][lane] = v[i];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float u8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u8[j] = tile[4 * warp + q + 32 * j][lane];
+#pragma unroll
+      for (int h = 1; h < K / 32; h <<= 1) {  // register bit s of j is row bit 5 + s
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j & h) continue;
+          const float a = u8[j], b = u8[j + h];
+          u8[j] = __fadd_rn(a, b);
+          u8[j + h] = __fsub_rn(a, b);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t r = row0 + 4 * warp + q + 32 * j;
+        if (col_ok && r < rows) out[r * cols + col] = __float2bfloat16_rn(__fmul_rn(u8[j], c));
+      }
+    }
+  }
+}
+
+}  // namespace rot
+}  // namespace hq

@@ -288,6 +288,59 @@ HQ_API hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_co
                                size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Backward placement that reuses the forward's codes ("HALO: Hadamard-Assisted Lower-Precision
+ * Optimization for LLMs", Approach: quantized rotated tensors of the forward pass are reused,
+ * and the output gradient gets a left-hand Hadamard; "Training Transformers with 4-bit
+ * Integers", section 4: the backward GEMMs quantize only the output gradient and reuse the
+ * forward's quantized activations and weights).
+ *
+ * With Wq = Q(W H) from the forward (rotated along K) and G = Q(H dY) (dY rotated along the
+ * tokens M, quantized once), H symmetric and orthonormal:
+ *   dW = G^T-contraction with the saved X codes (as hq_linear_bwd's dW, rotation along M);
+ *   dX = dY W = H (H dY)(W H) H  ~  H [ fp32(sum_n G[n][m] Wq[n][j]) * fp32(s_g * s_w) ] H,
+ * the GEMM reading both code tensors as stored (contraction outermost), then both rotations
+ * undone on the fp32 output: along its columns (K) in k-blocks, then along its rows (M), each
+ * as the library's rotation (butterflies, then x fp32(1/sqrt(k))), one bf16 rounding at the
+ * end.  One quantization of dY and none of W in the backward: four rotations per layer step
+ * instead of six.  Formats: HQ_INT8 and HQ_FP8_E4M3 only (the tensor cores read operands with
+ * the contraction outermost only for 8-bit formats); others are HQ_ERR_ARG.
+ *
+ * hq_linear_fwd_keep -- hq_linear_fwd_save that also hands back W's codes along K:
+ *   wq_codes [N][K] (1 byte per element) and the device scalar *wq_scale, exactly what
+ *   hq_quantize(W, dim = 1) gives.  workspace: >= hq_linear_fwd_keep_workspace_bytes(M, K, N).
+ *   Errors: as hq_linear_fwd_save; a null wq_codes or wq_scale is HQ_ERR_ARG.
+ *
+ * hq_linear_bwd_dx_reuse -- dX [M][K] bf16 from g_codes [N][M] (dY rotated along M, as
+ *   hq_quantize(dY, dim = 0) writes them) with scale *g_scale, and wq_codes [N][K] with
+ *   *wq_scale.  M and K multiples of k; N (the contraction) >= 1, at most HQ_MAX_K_INT8 for
+ *   INT8.  workspace: >= hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N) bytes (the fp32
+ *   output before its de-rotation, 4 M K bytes; not preserved).  Three kernels on `stream`.
+ *
+ * hq_linear_bwd_reuse -- dX and dW of one layer from dY [M][N] (dtype dt), the saved
+ *   xqt_codes [K][M] / *xqt_scale of hq_linear_fwd_save / _keep and the kept wq_codes [N][K] /
+ *   *wq_scale: dY quantized once along M, the dW GEMM, then hq_linear_bwd_dx_reuse, all on
+ *   `stream`.  Shape rules as hq_linear_fwd_bwd.  workspace: >=
+ *   hq_linear_bwd_reuse_workspace_bytes(M, K, N).  dW equals hq_linear_bwd's bit for bit.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API size_t hq_linear_fwd_keep_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_fwd_keep(const void* X, const void* W, hq_dtype dt, int64_t M,
+                                    int64_t K, int64_t N, int k, hq_fmt fmt, void* Y,
+                                    void* xqt_codes, float* xqt_scale, void* wq_codes,
+                                    float* wq_scale, void* workspace, size_t ws_bytes,
+                                    hq_stream_t stream);
+HQ_API size_t hq_linear_bwd_dx_reuse_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_bwd_dx_reuse(const void* g_codes, const float* g_scale,
+                                        const void* wq_codes, const float* wq_scale, int64_t M,
+                                        int64_t K, int64_t N, int k, hq_fmt fmt, void* dX,
+                                        void* workspace, size_t ws_bytes, hq_stream_t stream);
+HQ_API size_t hq_linear_bwd_reuse_workspace_bytes(int64_t M, int64_t K, int64_t N);
+HQ_API hq_status hq_linear_bwd_reuse(const void* dY, hq_dtype dt, const void* xqt_codes,
+                                     const float* xqt_scale, const void* wq_codes,
+                                     const float* wq_scale, int64_t M, int64_t K, int64_t N,
+                                     int k, hq_fmt fmt, void* dX, void* dW, void* workspace,
+                                     size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * hq_quantize_noalloc -- hq_quantize for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this call: it exists for integration only.  Some callers

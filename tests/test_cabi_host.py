@@ -256,3 +256,56 @@ def test_split_pass_argument_errors(L):
     assert c(am=FAKE + 2) == 4
     assert c(fmt=7) == 1
     assert c(codes=FAKE_MIS) == 4
+
+
+def test_reuse_flow_argument_errors(L):
+    """The forward that keeps W's codes and the backward that reuses them reject bad arguments
+    before any launch; the reuse GEMM takes 8-bit formats only (FP6 / FP4 are HQ_ERR_ARG)."""
+    fk = lambda **kw: L.hq_linear_fwd_keep(FAKE, FAKE, hq.HQ_BF16, kw.get("M", 256), kw.get("K", 512),
+                                           kw.get("N", 256), kw.get("k", 64), kw.get("fmt", 0), FAKE, FAKE, FAKE,
+                                           kw.get("wq", FAKE), kw.get("sw", FAKE), kw.get("ws", FAKE),
+                                           kw.get("wsb", 1 << 34), None)
+    assert fk(wq=None) == 1
+    assert fk(sw=None) == 1
+    assert fk(wq=FAKE_MIS) == 4
+    assert fk(sw=FAKE + 1) == 4
+    assert fk(M=96) == 2
+    assert fk(ws=None) == 8
+    assert fk(wsb=16) == 8
+    dx = lambda **kw: L.hq_linear_bwd_dx_reuse(kw.get("g", FAKE), kw.get("sg", FAKE), kw.get("wq", FAKE), FAKE,
+                                               kw.get("M", 256), kw.get("K", 512), kw.get("N", 200),
+                                               kw.get("k", 64), kw.get("fmt", 0), kw.get("dX", FAKE),
+                                               kw.get("ws", FAKE), kw.get("wsb", 1 << 34), None)
+    for fmt in (2, 3, 4, 7):
+        assert dx(fmt=fmt) == 1
+    assert dx(k=48) == 1
+    assert dx(M=96) == 2          # M rotated: multiple of k
+    assert dx(K=32) == 2          # K rotated: multiple of k
+    assert dx(N=0) == 2
+    assert dx(N=133200) == 2      # INT8 contraction bound
+    assert dx(g=None) == 1
+    assert dx(dX=None) == 1
+    assert dx(wq=FAKE_MIS) == 4
+    assert dx(sg=FAKE + 2) == 4
+    assert dx(ws=None) == 8
+    assert dx(wsb=256 * 512 * 4 - 1) == 8
+    assert dx(ws=FAKE_MIS) == 4
+    br = lambda **kw: L.hq_linear_bwd_reuse(FAKE, kw.get("dt", hq.HQ_BF16), kw.get("xqt", FAKE), FAKE,
+                                            kw.get("wq", FAKE), kw.get("sw", FAKE), kw.get("M", 256),
+                                            kw.get("K", 512), kw.get("N", 256), 64, kw.get("fmt", 1),
+                                            kw.get("dX", FAKE), kw.get("dW", FAKE), kw.get("ws", FAKE),
+                                            kw.get("wsb", 1 << 34), None)
+    assert br(dt=5) == 3
+    assert br(fmt=2) == 1
+    assert br(N=200) == 2         # the layer calls keep every dimension a multiple of k
+    assert br(wq=None) == 1
+    assert br(dW=None) == 1
+    assert br(sw=FAKE + 2) == 4
+    assert br(ws=None) == 8
+    assert br(wsb=4096) == 8
+    M, K, N = 4096, 4096, 11008
+    assert hq.hq_linear_fwd_keep_workspace_bytes(M, K, N) >= M * K
+    assert hq.hq_linear_fwd_keep_workspace_bytes(M, K, N) < hq.hq_linear_fwd_save_workspace_bytes(M, K, N)
+    assert hq.hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N) >= 4 * M * K
+    assert hq.hq_linear_bwd_reuse_workspace_bytes(M, K, N) >= N * M + 4 * M * K
+    assert hq.hq_linear_bwd_reuse_workspace_bytes(-1, 1, 1) == 0
