@@ -598,6 +598,92 @@ def run_sweep(args):
     return 0 if all(l["status"] == 0 for l in out_lines) else 1
 
 
+def run_reuse(args):
+    """The backward placement that reuses the forward's codes against the HALO-2 saved-codes
+    flow, per workload and layer (INT8 / FP8 at the workload's k): hq_linear_fwd_keep +
+    hq_linear_bwd_reuse (four rotations, the contraction-outermost dX GEMM, the output's
+    de-rotation) against hq_linear_fwd_save + hq_linear_bwd (six rotations), each timed whole
+    with CUDA events, L2 flushed before each; the reuse dX alone (GEMM + de-rotation) beside
+    the HALO-2 dX GEMM alone.  One JSON line per point."""
+    import torch
+    import hadamard_rotated_precision_b200 as hq
+    from hadamard_rotated_precision_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    int8_peak = peaks["bf16"] * INT8_OVER_BF16
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    reps = max(3, args.steps)
+
+    def timed(fn):
+        for _ in range(2):
+            flush.zero_()
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / reps
+
+    def dev_t(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    out_lines = []
+    for wid in (2, 3, 4, 5):
+        w = synthetic.WORKLOADS[wid]
+        for li, Lr in enumerate(w.layers):
+            d = synthetic.draw(w, li)
+            X, W, dY = dev_t(d["X"]), dev_t(d["W"]), dev_t(d["dY"])
+            M, K, N = Lr.M, Lr.K, Lr.N
+            fmt, k = hq._fmt(w.fmt), w.k
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+            dW = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+            xqt = torch.empty(K, M, dtype=torch.uint8, device=dev)
+            wq = torch.empty(N, K, dtype=torch.uint8, device=dev)
+            sx, sw = (torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2))
+            ws = torch.empty(max(hq.hq_linear_fwd_save_workspace_bytes(M, K, N), hq.hq_linear_bwd_workspace_bytes(M, K, N),
+                                 hq.hq_linear_fwd_keep_workspace_bytes(M, K, N),
+                                 hq.hq_linear_bwd_reuse_workspace_bytes(M, K, N)), dtype=torch.uint8, device=dev)
+
+            def halo2():
+                hq.hq_linear_fwd_save(X, W, k, fmt, Y=Y, xqt=xqt, xqt_scale=sx, workspace=ws)
+                hq.hq_linear_bwd(dY, W, xqt, sx, k, fmt, dX=dX, dW=dW, workspace=ws)
+
+            def reuse():
+                hq.hq_linear_fwd_keep(X, W, k, fmt, Y=Y, xqt=xqt, xqt_scale=sx, wq=wq, wq_scale=sw, workspace=ws)
+                hq.hq_linear_bwd_reuse(dY, xqt, sx, wq, sw, k, fmt, dX=dX, dW=dW, workspace=ws)
+
+            halo2_ms = timed(halo2)
+            reuse_ms = timed(reuse)
+            g, sg = hq.hq_quantize(dY, 0, k, fmt)
+            dx_reuse_ms = timed(lambda: hq.hq_linear_bwd_dx_reuse(g, sg, wq, sw, k, fmt, dX=dX, workspace=ws))
+            gn, sgn = hq.hq_quantize(dY, 1, k, fmt)
+            wn, swn = hq.hq_quantize(W, 0, k, fmt)
+            dx_gemm_ms = timed(lambda: hq.hq_gemm(gn, sgn, wn, swn, fmt, out=dX))
+            ops = 6.0 * M * N * K
+            line = {"workload": w.name, "layer": Lr.name, "M": M, "K": K, "N": N, "fmt": w.fmt, "k": k,
+                    "halo2_step_ms": halo2_ms, "halo2_step_tops": ops / (halo2_ms * 1e-3) / 1e12,
+                    "reuse_step_ms": reuse_ms, "reuse_step_tops": ops / (reuse_ms * 1e-3) / 1e12,
+                    "reuse_frac_of_peak": ops / (reuse_ms * 1e-3) / 1e12 / int8_peak,
+                    "dx_reuse_ms": dx_reuse_ms, "dx_halo2_gemm_ms": dx_gemm_ms,
+                    "derotate_bytes": 14 * M * K,
+                    "status": hq.hq_get_error()}
+            out_lines.append(line)
+            print(json.dumps(line), flush=True)
+            del X, W, dY, Y, dX, dW, xqt, wq, ws
+            torch.cuda.empty_cache()
+    return 0 if all(l["status"] == 0 for l in out_lines) else 1
+
+
 def run_kernel_case(args):
     """One small standalone invocation of a hot kernel, for profiler captures: a warm-up
     call, then the captured call(s).  Inputs exceed L2 (126 MB) but stay near 200 MB."""
@@ -621,6 +707,15 @@ def run_kernel_case(args):
         out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         for _ in range(2):
             hq.hq_gemm(A, s, B, s, fmt, out=out)
+    elif case == "dx_reuse":
+        # a dX of the reuse placement at 4096 tokens, K = 4096, contraction 8192 (codes 2 x 32 MB,
+        # fp32 output 64 MB + bf16 32 MB: more than L2)
+        M, K, N = 4096, 4096, 8192
+        gq = torch.randint(-127, 128, (N, M), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        wq = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        s = torch.full((1,), 0.01, device="cuda")
+        for _ in range(2):
+            hq.hq_linear_bwd_dx_reuse(gq, s, wq, s, 128, "int8")
     elif case == "quant_dual":
         x = torch.randn(11008, 4096, generator=g, device="cuda").to(torch.bfloat16)
         for _ in range(2):
@@ -642,10 +737,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
-    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual"),
+    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual",
+                                              "dx_reuse"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
     ap.add_argument("--formats", action="store_true",
                     help="with --sweep: the bench workload's layer in every code format (INT8, FP8, FP6, FP4)")
+    ap.add_argument("--reuse", action="store_true",
+                    help="time the backward placement that reuses the forward's codes against HALO-2, every workload, and exit")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload (one JSON line per workload/layer/format/k) and exit")
     args = ap.parse_args(argv)
@@ -653,6 +751,8 @@ def main(argv=None):
         return run_kernel_case(args)
     if args.sweep:
         return run_sweep(args)
+    if args.reuse:
+        return run_reuse(args)
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
