@@ -39,6 +39,7 @@ struct DeviceInfo {
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
   bool dual_attr[5][4][2][2] = {};  // fused two-rotation instantiations prepared [k][mode][w32][signed]
   bool mn_attr[2] = {};             // MN-major pair GEMM (fp32 output) prepared [int8 / fp8]
+  bool rot_attr[3] = {};            // row de-rotation with its 64 KB tile prepared [k = 64, 128, 256]
 };
 
 std::mutex g_mu;
@@ -800,8 +801,20 @@ cudaError_t launch_derotate_k(float* z, int64_t rows, int64_t cols, __nv_bfloat1
   hq::rot::rot_cols_f32_kernel<K><<<static_cast<unsigned>(std::max<int64_t>(1, blocks_c)), hq::rot::kThreads, 0, st>>>(z, n8, c);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t blocks_r = ((rows + 255) / 256) * ((cols + 31) / 32);
-  hq::rot::rot_rows_f32_bf16_kernel<K><<<static_cast<unsigned>(blocks_r), hq::rot::kThreads, 0, st>>>(z, rows, cols, c, out);
+  namespace hr = hq::rot;
+  const size_t smem = K >= 64 ? hr::kRowsSmemBytes : 0;
+  if (K >= 64) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    const int ki = K == 64 ? 0 : K == 128 ? 1 : 2;
+    if (!d.rot_attr[ki]) {
+      if ((e = cudaFuncSetAttribute(hr::rot_rows_f32_bf16_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem))) != cudaSuccess)
+        return e;
+      d.rot_attr[ki] = true;
+    }
+  }
+  const int64_t blocks_r = ((rows + hr::kRowTile - 1) / hr::kRowTile) * ((cols + hr::kColTile - 1) / hr::kColTile);
+  hr::rot_rows_f32_bf16_kernel<K><<<static_cast<unsigned>(blocks_r), hr::kThreads, smem, st>>>(z, rows, cols, c, out);
   return cudaGetLastError();
 }
 
