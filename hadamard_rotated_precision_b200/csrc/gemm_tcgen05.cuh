@@ -321,6 +321,110 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
 }
 
 
+// ---------------------------------------------------------------- output rotation in the epilogue
+//
+// For the fp32 output (kOutF32) the epilogue can apply blockdiag(H_k / sqrt(k)) along the
+// output's columns before storing: an epilogue thread owns one output row of the tile in TMEM,
+// so a k-block of columns is in its registers.  Arithmetic as the library's rotation:
+// z = fp32(acc) * sab, Sylvester butterflies h = 1 .. k/2 (index bit 0 first, fp32 RNE), then
+// one multiply by fp32(1/sqrt(k)).
+
+// Dequantized fp32 values of 32 consecutive accumulator columns of this thread's row.
+template <int FMT>
+__device__ __forceinline__ void load_dequant32(uint32_t taddr, float sab, float* v) {
+  uint32_t r[32];
+  ptx::tmem_ld_32x32b_x32(taddr, r);
+  ptx::tmem_ld_wait(r);
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    v[i] = __fmul_rn(FMT == kInt8 ? __int2float_rn(static_cast<int>(r[i])) : __uint_as_float(r[i]), sab);
+}
+
+// Butterfly stages h = 1 .. H/2 over NV consecutive values (blocks of H).
+template <int NV, int H>
+__device__ __forceinline__ void butterflies(float* v) {
+#pragma unroll
+  for (int h = 1; h < H; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if (i & h) continue;
+      const float u = v[i], w = v[i + h];
+      v[i] = __fadd_rn(u, w);
+      v[i + h] = __fsub_rn(u, w);
+    }
+  }
+}
+
+// o[0 .. n) = v * c for the first n of NV values (n a multiple of 4; unrolled, so v stays in
+// registers).
+template <int NV>
+__device__ __forceinline__ void store_f32_scaled(float* o, const float* v, int n, float c) {
+#pragma unroll
+  for (int q = 0; q < NV; q += 4)
+    if (q < n)
+      *reinterpret_cast<float4*>(o + q) =
+          make_float4(__fmul_rn(v[q], c), __fmul_rn(v[q + 1], c), __fmul_rn(v[q + 2], c), __fmul_rn(v[q + 3], c));
+}
+
+// k <= 128: chunks of max(k, 32) columns, each rotated in registers and stored.
+template <int FMT, int RK, int TILE_N>
+__device__ __forceinline__ void epi_rot_cols(uint32_t t_row, float sab, float c, float* out_row, int col_base,
+                                             bool row_ok, int N) {
+  constexpr int W = RK < 32 ? 32 : RK;
+#pragma unroll 1
+  for (int b = 0; b < TILE_N / W; ++b) {
+    float v[W];
+#pragma unroll
+    for (int q = 0; q < W / 32; ++q) load_dequant32<FMT>(t_row + uint32_t(b * W + 32 * q), sab, v + 32 * q);
+    butterflies<W, RK>(v);
+    const int col0 = col_base + b * W;
+    // N % k == 0: whole blocks (a 32-column chunk of k = 16 blocks may end at N after one)
+    if (row_ok && col0 < N) store_f32_scaled<W>(out_row + col0, v, N - col0, c);
+  }
+}
+
+// k = 256 (the tile's whole width): stages h = 1 .. 64 on each 128-column half, written back to
+// the accumulator as fp32 bits, then the last stage pairs column j with j + 128.
+template <int FMT, int TILE_N>
+__device__ __forceinline__ void epi_rot_cols256(uint32_t t_row, float sab, float c, float* out_row, int col_base,
+                                                bool row_ok, int N) {
+  static_assert(TILE_N == 256, "k = 256 spans the whole tile");
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {
+    float v[128];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) load_dequant32<FMT>(t_row + uint32_t(128 * hf + 32 * q), sab, v + 32 * q);
+    butterflies<128, 128>(v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[32 * q + i]);
+      ptx::tmem_st_32x32b_x32(t_row + uint32_t(128 * hf + 32 * q), r);
+    }
+  }
+  ptx::tmem_st_wait();
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a[32], b[32];
+    ptx::tmem_ld_32x32b_x32(t_row + uint32_t(32 * q), a);
+    ptx::tmem_ld_32x32b_x32(t_row + uint32_t(128 + 32 * q), b);
+    ptx::tmem_ld_wait(a);
+    ptx::reg_fence(b);
+    float lo[32], hi[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float u = __uint_as_float(a[i]), w = __uint_as_float(b[i]);
+      lo[i] = __fadd_rn(u, w);
+      hi[i] = __fsub_rn(u, w);
+    }
+    if (row_ok && col_base < N) {
+      store_f32_scaled<32>(out_row + col_base + 32 * q, lo, 32, c);
+      store_f32_scaled<32>(out_row + col_base + 128 + 32 * q, hi, 32, c);
+    }
+  }
+}
+
 // ====================================================================== CTA-pair variant
 //
 // A cluster of two CTAs on the two SMs of a TPC computes a 256 x 256 output tile with
@@ -394,7 +498,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
                  unsigned int* __restrict__ status, int splits, uint32_t* __restrict__ part_ws,
-                 int* __restrict__ counters, uint32_t ab_code) {
+                 int* __restrict__ counters, uint32_t ab_code, int rot_k) {
+  // rot_k (kOutF32 only; 0 = none): rotate the output along its columns in blocks of rot_k
+  // before storing (see epi_rot_cols)
   using G = Geo<BN_, SHORT_K>;
   static_assert(!MN || (BN_ == 256 && !SHORT_K && OUT != kOutBf16), "MN-major operands: 256-wide tiles, direct stores");
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
@@ -646,13 +752,32 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         if (peer && lane == 0) *slab_counter = 0;  // both halves counted: ready for the next launch
       } else {
         const int64_t row = int64_t(row0) + lane;
+        bool done = false;
+        if constexpr (OUT == kOutF32 && BN_ == 256) {
+          if (rot_k != 0) {
+            const float c = __frsqrt_rn(static_cast<float>(rot_k));  // fp32(1/sqrt(k)), correctly rounded
+            float* orow = reinterpret_cast<float*>(out) + row * N;
+            const int cb = n_blk * BN;
+            const bool rok = row < M;
+            switch (rot_k) {
+              case 16: epi_rot_cols<FMT, 16, BN_>(t_row, sab, c, orow, cb, rok, N); break;
+              case 32: epi_rot_cols<FMT, 32, BN_>(t_row, sab, c, orow, cb, rok, N); break;
+              case 64: epi_rot_cols<FMT, 64, BN_>(t_row, sab, c, orow, cb, rok, N); break;
+              case 128: epi_rot_cols<FMT, 128, BN_>(t_row, sab, c, orow, cb, rok, N); break;
+              default: epi_rot_cols256<FMT, BN_>(t_row, sab, c, orow, cb, rok, N); break;
+            }
+            done = true;
+          }
+        }
+        if (!done) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
-          ptx::tmem_ld_wait();
-          const int col0 = n_blk * BN + c * 32;
-          if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
+            ptx::tmem_ld_wait();
+            const int col0 = n_blk * BN + c * 32;
+            if (row < M && col0 < N) store_chunk<FMT, OUT>(r, out, row, col0, N, sab);
+          }
         }
         ptx::tc_fence_before_sync();
         __syncwarp();

@@ -585,7 +585,8 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
 template <int FMT, int OUT, int BN, bool SK, bool MN = false>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
                              const float* sb, void* out, int M, int N, int K, int clusters, int splits,
-                             uint32_t* part_ws, int* counters, uint32_t ab_code, DeviceInfo& d, cudaStream_t st) {
+                             uint32_t* part_ws, int* counters, uint32_t ab_code, DeviceInfo& d, cudaStream_t st,
+                             int rot_k = 0) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN, SK>;
   auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK, MN>;
@@ -605,7 +606,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.numAttrs = 1;
   (void)d;
   return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, splits, part_ws, counters,
-                            ab_code);
+                            ab_code, rot_k);
 }
 
 // Dynamic shared memory of every pair-GEMM instantiation enabled once per device.
@@ -758,9 +759,10 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
 
 // out[M][N] fp32 = fp32(sum_l A[l][i] B[l][j]) * fp32(s_a * s_b) with both operands stored
 // contraction-outermost: A as [K][M], B as [K][N] (the token-rotated output-gradient codes and
-// the forward's K-rotated weight codes); CTA pairs, 256 x 256 tiles.
+// the forward's K-rotated weight codes); CTA pairs, 256 x 256 tiles.  rot_k != 0: the output
+// leaves the epilogue rotated along its columns in blocks of rot_k (N % rot_k == 0).
 hq_status gemm_mn_f32_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
-                           int64_t K, hq_fmt fmt, float* out, DeviceInfo& d, cudaStream_t st) {
+                           int64_t K, hq_fmt fmt, float* out, DeviceInfo& d, cudaStream_t st, int rot_k) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<256, false>;
   const int f = fmt == HQ_INT8 ? 0 : 1;
@@ -786,9 +788,9 @@ hq_status gemm_mn_f32_impl(const void* A, const float* sa, const void* B, const 
   if ((s = encode_codes_map(&tb, B, K, N, G::B_ROWS)) != HQ_OK) return s;
   const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
   e = f == 0 ? launch_gemm_pair<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false, true>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st)
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, rot_k)
              : launch_gemm_pair<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false, true>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st);
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, rot_k);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -796,11 +798,7 @@ template <int K>
 cudaError_t launch_derotate_k(float* z, int64_t rows, int64_t cols, __nv_bfloat16* out, DeviceInfo& d,
                               cudaStream_t st) {
   const float c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(K)));  // fp32(1/sqrt(k)), one rounding
-  const int64_t n8 = rows * cols / 8;
-  const int64_t blocks_c = std::min<int64_t>((n8 + hq::rot::kThreads - 1) / hq::rot::kThreads, int64_t(d.sms) * 8);
-  hq::rot::rot_cols_f32_kernel<K><<<static_cast<unsigned>(std::max<int64_t>(1, blocks_c)), hq::rot::kThreads, 0, st>>>(z, n8, c);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   namespace hr = hq::rot;
   const size_t smem = K >= 64 ? hr::kRowsSmemBytes : 0;
   if (K >= 64) {
@@ -818,7 +816,8 @@ cudaError_t launch_derotate_k(float* z, int64_t rows, int64_t cols, __nv_bfloat1
   return cudaGetLastError();
 }
 
-// out = bf16(H Z H): Z's columns rotated in place, then its rows into out.
+// out = bf16(H Z) for Z already rotated along its columns (by the GEMM's epilogue): the rows'
+// rotation, rounded to bf16.
 hq_status derotate_impl(float* z, int64_t rows, int64_t cols, int k, void* out, DeviceInfo& d, cudaStream_t st) {
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   cudaError_t e;
@@ -847,7 +846,7 @@ hq_status check_dx_reuse_shape(int64_t M, int64_t K, int64_t N, int k, hq_fmt fm
 hq_status dx_reuse_impl(const void* g_codes, const float* g_scale, const void* wq_codes, const float* wq_scale,
                         int64_t M, int64_t K, int64_t N, int k, hq_fmt fmt, void* dX, float* z, DeviceInfo& d,
                         cudaStream_t st) {
-  hq_status s = gemm_mn_f32_impl(g_codes, g_scale, wq_codes, wq_scale, M, K, N, fmt, z, d, st);
+  hq_status s = gemm_mn_f32_impl(g_codes, g_scale, wq_codes, wq_scale, M, K, N, fmt, z, d, st, k);
   if (s != HQ_OK) return s;
   return derotate_impl(z, M, K, k, dX, d, st);
 }

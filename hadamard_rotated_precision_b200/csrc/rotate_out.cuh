@@ -1,5 +1,7 @@
 // De-rotation of a GEMM output that is still rotated on both sides: out = bf16(H Z H), H =
-// blockdiag(H_k / sqrt(k)), Z fp32 [rows][cols] (the dequantized accumulators).
+// blockdiag(H_k / sqrt(k)), Z fp32 [rows][cols] (the dequantized accumulators).  The rotation
+// along the columns runs in the GEMM's epilogue (an epilogue thread owns an output row); this
+// kernel does the one along the rows.
 //
 // Method: "HALO: Hadamard-Assisted Lower-Precision Optimization for LLMs", Approach (the
 // quantized rotated tensors of the forward pass are reused in the backward pass, which puts a
@@ -8,11 +10,11 @@
 //
 // Numerics, as the library's rotation: Sylvester butterflies h = 1, 2, ..., k/2 (index bit 0
 // first), every add / sub fp32 round-to-nearest-even, then one multiply by fp32(1/sqrt(k));
-// the columns' rotation (each row's k-blocks) runs first, in place in fp32, then the rows',
-// which rounds to bf16 once at the end.
+// the columns' rotation (each row's k-blocks) runs first, in fp32, then the rows', which
+// rounds to bf16 once at the end.
 //
-// Both kernels stream: 4 bytes read and written per element (columns), 4 read and 2 written
-// (rows).  Requires cols % k == 0 and rows % k == 0 (so both are even and whole blocks).
+// Streams 4 bytes read and 2 written per element.  Requires cols % k == 0 and rows % k == 0
+// (so both are even and whole blocks).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -21,55 +23,6 @@ namespace hq {
 namespace rot {
 
 constexpr int kThreads = 256;
-
-// Along the columns, in place.  A thread holds 8 consecutive elements (index bits 0-2 in
-// registers), the k/8 lanes of one k-block hold the rest (bits 3.. across lanes); a warp
-// covers 256 consecutive elements, so a block never straddles warps (cols % k == 0).
-template <int K>
-__global__ void __launch_bounds__(kThreads) rot_cols_f32_kernel(float* __restrict__ z, int64_t n8, float c) {
-  static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
-  const int lane = threadIdx.x & 31;
-  for (int64_t base = int64_t(blockIdx.x) * kThreads; base < n8; base += int64_t(gridDim.x) * kThreads) {
-    const int64_t i = base + threadIdx.x;
-    const bool valid = i < n8;
-    float v[8];
-    if (valid) {
-      const float4 a = *reinterpret_cast<const float4*>(z + 8 * i);
-      const float4 b = *reinterpret_cast<const float4*>(z + 8 * i + 4);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-    }
-#pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j & h) continue;
-        const float u = v[j], w = v[j + h];
-        v[j] = __fadd_rn(u, w);
-        v[j + h] = __fsub_rn(u, w);
-      }
-    }
-    // bit 3 + s lives in lane bit s: the lower lane keeps u + w, the upper one u - w
-#pragma unroll
-    for (int m = 1; m < K / 8; m <<= 1) {
-      const bool upper = (lane & m) != 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float p = __shfl_xor_sync(0xFFFFFFFFu, v[j], m);
-        v[j] = upper ? __fsub_rn(p, v[j]) : __fadd_rn(v[j], p);
-      }
-    }
-    if (valid) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(v[j], c);
-      *reinterpret_cast<float4*>(z + 8 * i) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(z + 8 * i + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    }
-  }
-}
 
 // Along the rows, fp32 in, bf16 out.  A CTA takes a tile of 256 rows x 64 columns (whole
 // k-blocks of rows, since rows % k == 0 and k divides 256); a thread holds two adjacent
