@@ -441,3 +441,17 @@ def linear_bwd_reuse(dY, xqt_codes, s_x, wq_codes, s_w, k, fmt):
     _, dw = epilogue(dw_acc, s_g, s_x)
     dx = linear_bwd_dx_reuse(g, s_g, wq_codes, s_w, k, fmt)
     return dict(g=g, s_g=s_g, dw=dw, dx=dx["out"], dx_z=dx["z"])
+
+
+# ------------------------------------------------- next layer's rotation in the GEMM's epilogue
+#
+# "Training Transformers with 4-bit Integers", section 3.3 (the Hadamard blocks are applied to
+# an operand before it is quantized): when a GEMM's output is the next GEMM's operand along its
+# columns, the producing GEMM can apply that rotation to its fp32 dequantized output, and the
+# next operand is then only quantized (quantize_rotated).  Reading: the rotation acts on the
+# fp32 values fp32(acc) * fp32(s_a * s_b), as `rotate` does (butterflies, then x c_k).
+
+
+def gemm_rotout(A, B, sa, sb, fmt: int, k: int, rows=None) -> np.ndarray:
+    """fp32 [M][N]: blockdiag(H_k/sqrt k) along the columns of the dequantized A B^T."""
+    return rotate(dequant_f32(gemm(A, B, fmt, rows), sa, sb), 1, k)

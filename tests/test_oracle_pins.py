@@ -715,3 +715,42 @@ def test_reuse_dx_row_block_sampling(oracle_lib):
     r = oracle.linear_bwd_reuse(d["dY"], xq, sx, wq, sw, k, oracle.INT8)
     part = oracle.linear_bwd_dx_reuse(r["g"], r["s_g"], wq, sw, k, oracle.INT8, rows=[2 * k, 0])
     np.testing.assert_array_equal(part["out"], np.concatenate([r["dx"][2 * k:3 * k], r["dx"][:k]]))
+
+
+# ------------------------------------------------- next layer's rotation in the GEMM's epilogue
+
+@pytest.mark.parametrize("k", (16, 128))
+def test_gemm_rotout_close_to_dense(oracle_lib, k):
+    """The dequantized product rotated along its columns equals the fp64 dense product
+    (A B^T s_a s_b) blockdiag(H_k) / sqrt(k) up to fp32 rounding."""
+    rng = np.random.default_rng(k)
+    A = rng.integers(-127, 128, size=(48, 96)).astype(np.int8).view(np.uint8)
+    B = rng.integers(-127, 128, size=(2 * k, 96)).astype(np.int8).view(np.uint8)
+    sa, sb = np.float32(0.013), np.float32(0.0021)
+    want = (A.view(np.int8).astype(np.float64) @ B.view(np.int8).astype(np.float64).T) * float(sa * sb)
+    want = want @ _blockdiag_h(2 * k, k) / math.sqrt(k)
+    got = oracle.gemm_rotout(A, B, sa, sb, oracle.INT8, k).astype(np.float64)
+    assert np.abs(got - want).max() <= 1e-5 * np.abs(want).max()
+
+
+def test_next_layer_flow_tracks_two_layer_product(oracle_lib):
+    """Layer 1's output rotated in its epilogue and quantized as it is, times layer 2's weight
+    codes rotated along the same dimension, approximates X W1^T W2^T; leaving out the epilogue
+    rotation (a planted mistake) does not."""
+    w = synthetic.WORKLOADS[1]
+    d = synthetic.draw_fp32(w)
+    X, W1 = d["X"], d["W"]                                       # [64][256], [128][256]
+    W2 = synthetic.tiny_random((96, 128), 4, scale=0.05)          # the next layer, 128 -> 96
+    k = 16
+    qx, sx = oracle.quantize(X, 1, k, oracle.INT8)
+    qw1, sw1 = oracle.quantize(W1, 1, k, oracle.INT8)
+    y_rot = oracle.gemm_rotout(qx, qw1, sx, sw1, oracle.INT8, k)   # [64][128], rotated along N
+    qy, sy = oracle.quantize_rotated(y_rot, oracle.INT8)
+    qw2, sw2 = oracle.quantize(W2, 1, k, oracle.INT8)
+    _, fast = oracle.epilogue(oracle.gemm(qy, qw2, oracle.INT8), sy, sw2)
+    want = X.astype(np.float64) @ W1.astype(np.float64).T @ W2.astype(np.float64).T
+    assert _rel_fro(oracle.bf16_bits_to_f32(fast).astype(np.float64), want) < 0.1
+    y_plain = oracle.dequant_f32(oracle.gemm(qx, qw1, oracle.INT8), sx, sw1)
+    qp, sp = oracle.quantize_rotated(y_plain, oracle.INT8)
+    bad = oracle.gemm(qp, qw2, oracle.INT8).astype(np.float64) * float(sp) * float(sw2)
+    assert _rel_fro(bad, want) > 0.5
