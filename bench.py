@@ -681,6 +681,36 @@ def run_reuse(args):
             print(json.dumps(line), flush=True)
             del X, W, dY, Y, dX, dW, xqt, wq, ws
             torch.cuda.empty_cache()
+    # the next layer's rotation in the epilogue, on the bench layer's forward GEMM: the GEMM
+    # writing its output rotated along N in fp32 plus the quantization of that output as it is,
+    # against the bf16 GEMM plus the rotating quantization of its output along N
+    w = synthetic.WORKLOADS[WORKLOAD_ID]
+    Lr = w.layers[0]
+    M, K, N = Lr.M, Lr.K, Lr.N
+    fmt, k = hq._fmt(w.fmt), w.k
+    g = torch.Generator(device="cuda").manual_seed(1)
+    qa = torch.randint(-127, 128, (M, K), generator=g, device=dev, dtype=torch.int32).to(torch.int8).view(torch.uint8)
+    qb = torch.randint(-127, 128, (N, K), generator=g, device=dev, dtype=torch.int32).to(torch.int8).view(torch.uint8)
+    s1 = torch.full((1,), 1e-3, device=dev)
+    yr = torch.empty(M, N, dtype=torch.float32, device=dev)
+    yb = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    codes = torch.empty(M, N, dtype=torch.uint8, device=dev)
+    sc = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(hq.hq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+    rot_gemm_ms = timed(lambda: hq.hq_gemm_rotout(qa, s1, qb, s1, k, fmt, out=yr))
+    prerot_ms = timed(lambda: hq.hq_quantize_prerotated(yr, fmt, codes=codes, scale=sc, workspace=ws))
+    plain_gemm_ms = timed(lambda: hq.hq_gemm(qa, s1, qb, s1, fmt, out=yb))
+    plain_quant_ms = timed(lambda: hq.hq_quantize(yb, 1, k, fmt, codes=codes, scale=sc, workspace=ws))
+    line = {"case": "next_layer_rotation_in_epilogue", "workload": w.name, "M": M, "K": K, "N": N, "fmt": w.fmt,
+            "k": k, "gemm_rotout_ms": rot_gemm_ms, "gemm_rotout_tops": 2.0 * M * N * K / (rot_gemm_ms * 1e-3) / 1e12,
+            "quantize_prerotated_ms": prerot_ms,
+            # two passes reading 4 B and one 1-byte code per element
+            "quantize_prerotated_gbs": 9.0 * M * N / (prerot_ms * 1e-3) / 1e9,
+            "gemm_bf16_ms": plain_gemm_ms, "quantize_rotating_ms": plain_quant_ms,
+            "fused_ms": rot_gemm_ms + prerot_ms, "unfused_ms": plain_gemm_ms + plain_quant_ms,
+            "status": hq.hq_get_error()}
+    out_lines.append(line)
+    print(json.dumps(line), flush=True)
     return 0 if all(l["status"] == 0 for l in out_lines) else 1
 
 

@@ -37,6 +37,7 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_fwd_keep_workspace_bytes", "hq_linear_fwd_keep",
            "hq_linear_bwd_dx_reuse_workspace_bytes", "hq_linear_bwd_dx_reuse",
            "hq_linear_bwd_reuse_workspace_bytes", "hq_linear_bwd_reuse",
+           "hq_gemm_rotout", "hq_quantize_prerotated_workspace_bytes", "hq_quantize_prerotated",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -105,6 +106,12 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_bwd_dx_reuse.restype = i32
         L.hq_linear_bwd_reuse.argtypes = [p, i32, p, p, p, p, i64, i64, i64, i32, i32, p, p, p, sz, p]
         L.hq_linear_bwd_reuse.restype = i32
+        L.hq_gemm_rotout.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
+        L.hq_gemm_rotout.restype = i32
+        L.hq_quantize_prerotated_workspace_bytes.argtypes = []
+        L.hq_quantize_prerotated_workspace_bytes.restype = sz
+        L.hq_quantize_prerotated.argtypes = [p, i64, i64, i32, p, p, p, sz, p]
+        L.hq_quantize_prerotated.restype = i32
         L.hq_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm.restype = i32
         L.hq_linear_workspace_bytes.argtypes = [i64, i64, i64]
@@ -589,6 +596,43 @@ def hq_linear_bwd_reuse(dY, xqt, xqt_scale, wq, wq_scale, k: int, fmt, dX=None, 
                                    ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
     _check(st, "hq_linear_bwd_reuse")
     return dX, dW
+
+
+def hq_gemm_rotout(A, scale_a, B, scale_b, k: int, fmt, out=None, stream=None):
+    """out [M][N] fp32: the dequantized A B^T rotated along its columns in blocks of k (the next
+    layer's rotation applied in the GEMM's epilogue)."""
+    torch = _torch()
+    for t, n in ((A, "A"), (scale_a, "scale_a"), (B, "B"), (scale_b, "scale_b")):
+        _dev_tensor(t, n)
+    M, K = A.shape
+    N = B.shape[0]
+    out = torch.empty((M, N), dtype=torch.float32, device=A.device) if out is None else out
+    _dev_tensor(out, "out")
+    st = lib().hq_gemm_rotout(A.data_ptr(), scale_a.data_ptr(), B.data_ptr(), scale_b.data_ptr(), M, N, K, k,
+                              _fmt(fmt), out.data_ptr(), _stream_handle(stream))
+    _check(st, "hq_gemm_rotout")
+    return out
+
+
+def hq_quantize_prerotated_workspace_bytes() -> int:
+    return int(lib().hq_quantize_prerotated_workspace_bytes())
+
+
+def hq_quantize_prerotated(y, fmt, codes=None, scale=None, workspace=None, stream=None):
+    """Tensor-wise codes of already-rotated fp32 values y [rows][cols] (no transform).
+    Returns (codes uint8 [rows][cols], scale)."""
+    torch = _torch()
+    _dev_tensor(y, "y")
+    if y.dtype != torch.float32:
+        raise TypeError("y must be float32")
+    rows, cols = y.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=y.device) if codes is None else codes
+    scale = torch.empty((1,), dtype=torch.float32, device=y.device) if scale is None else scale
+    ws = _workspace(hq_quantize_prerotated_workspace_bytes(), y.device, workspace)
+    st = lib().hq_quantize_prerotated(y.data_ptr(), rows, cols, _fmt(fmt), codes.data_ptr(), scale.data_ptr(),
+                                      ws.data_ptr(), ws.numel() * ws.element_size(), _stream_handle(stream))
+    _check(st, "hq_quantize_prerotated")
+    return codes, scale
 
 
 def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None):

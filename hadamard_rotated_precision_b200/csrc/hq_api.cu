@@ -15,6 +15,7 @@
 #include "fwht_dual.cuh"
 #include "gemm_tcgen05.cuh"
 #include "rotate_out.cuh"
+#include "prerot_quant.cuh"
 
 namespace {
 
@@ -40,6 +41,7 @@ struct DeviceInfo {
   bool dual_attr[5][4][2][2] = {};  // fused two-rotation instantiations prepared [k][mode][w32][signed]
   bool mn_attr[2] = {};             // MN-major pair GEMM (fp32 output) prepared [int8 / fp8]
   bool rot_attr[3] = {};            // row de-rotation with its 64 KB tile prepared [k = 64, 128, 256]
+  bool rotout_attr[2] = {};         // K-major pair GEMM with fp32 rotated output prepared [int8 / fp8]
 };
 
 std::mutex g_mu;
@@ -851,6 +853,60 @@ hq_status dx_reuse_impl(const void* g_codes, const float* g_scale, const void* w
   return derotate_impl(z, M, K, k, dX, d, st);
 }
 
+// ------------------------------------------------------------------ next layer's rotation in the epilogue
+
+// out[M][N] fp32 = blockdiag(H_k / sqrt(k)) applied along the columns of
+// fp32(sum_l A[i][l] B[j][l]) * fp32(s_a * s_b): both operands K-major, CTA pairs, 256-wide tiles.
+hq_status gemm_rotout_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
+                           int64_t K, int k, hq_fmt fmt, float* out, DeviceInfo& d, cudaStream_t st) {
+  namespace gp = hq::gemm::pair;
+  using G = gp::Geo<256, false>;
+  const int f = fmt == HQ_INT8 ? 0 : 1;
+  const void* kernel = f == 0 ? reinterpret_cast<const void*>(gp::gemm_pair_kernel<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false, false>)
+                              : reinterpret_cast<const void*>(gp::gemm_pair_kernel<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false, false>);
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d.rotout_attr[f]) {
+      if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(G::SMEM_BYTES))) != cudaSuccess)
+        return cuda_fail(e);
+      d.rotout_attr[f] = true;
+    }
+  }
+  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms);
+  CUtensorMap ta, tb, to;
+  std::memset(&to, 0, sizeof(to));
+  hq_status s = encode_codes_map(&ta, A, M, K, gp::HALF);
+  if (s != HQ_OK) return s;
+  if ((s = encode_codes_map(&tb, B, N, K, G::B_ROWS)) != HQ_OK) return s;
+  const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
+  e = f == 0 ? launch_gemm_pair<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false>(
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, k)
+             : launch_gemm_pair<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false>(
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, k);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+// Tensor-wise INT8 / e4m3 codes of n already-rotated fp32 values (n % 4 == 0, n > 0).
+hq_status prerot_quant_impl(const float* y, int64_t n, hq_fmt fmt, void* codes, float* scale, float* partials,
+                            DeviceInfo& d, cudaStream_t st) {
+  namespace pr = hq::prerot;
+  const int64_t n4 = n / 4;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n4 + pr::kThreads - 1) / pr::kThreads,
+                                                                           int64_t(d.sms) * 4)));
+  uint8_t* c = static_cast<uint8_t*>(codes);
+  pr::prerot_quant_kernel<hq::kModeAbsmax><<<grid, pr::kThreads, 0, st>>>(y, n4, c, partials, grid, scale, d.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (fmt == HQ_INT8)
+    pr::prerot_quant_kernel<hq::kModeInt8><<<grid, pr::kThreads, 0, st>>>(y, n4, c, partials, grid, scale, d.status);
+  else
+    pr::prerot_quant_kernel<hq::kModeFp8><<<grid, pr::kThreads, 0, st>>>(y, n4, c, partials, grid, scale, d.status);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------------ the linear layer
 
 struct LinearWs {
@@ -1363,6 +1419,49 @@ hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_codes, co
     return s;
   return gemm_impl(w.c[2], sc + 2, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split,
                    w.split_len);
+}
+
+hq_status hq_gemm_rotout(const void* A, const float* scale_a, const void* B, const float* scale_b, int64_t M,
+                         int64_t N, int64_t K, int k, hq_fmt fmt, float* out, hq_stream_t stream) {
+  if (!valid_k(k) || (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3)) return HQ_ERR_ARG;
+  hq_status s = check_gemm_args(A, scale_a, B, scale_b, M, N, K, fmt, HQ_OUT_BF16, out);
+  if (s != HQ_OK) return s;
+  if (N % k) return HQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    cudaError_t e = cudaMemsetAsync(out, 0, size_t(M) * size_t(N) * 4, st);
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  return gemm_rotout_impl(A, scale_a, B, scale_b, M, N, K, k, fmt, out, *d, st);
+}
+
+size_t hq_quantize_prerotated_workspace_bytes(void) { return kPartialBytes; }
+
+hq_status hq_quantize_prerotated(const float* y, int64_t rows, int64_t cols, hq_fmt fmt, void* codes, float* scale,
+                                 void* workspace, size_t ws_bytes, hq_stream_t stream) {
+  if (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3) return HQ_ERR_ARG;
+  if (rows < 0 || cols < 0) return HQ_ERR_ARG;
+  if (!scale) return HQ_ERR_ARG;
+  if (cols % 16) return HQ_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(scale) & 3u) return HQ_ERR_ALIGN;
+  const bool empty = rows == 0 || cols == 0;
+  if (!empty && (!y || !codes)) return HQ_ERR_ARG;
+  if (!empty && (!aligned16(y) || !aligned16(codes))) return HQ_ERR_ALIGN;
+  if (!workspace || ws_bytes < kPartialBytes) return HQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HQ_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  hq_status s = device_info(&d);
+  if (s != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (empty) {
+    set_scale_one_kernel<<<1, 1, 0, st>>>(scale);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+  }
+  return prerot_quant_impl(y, rows * cols, fmt, codes, scale, static_cast<float*>(workspace), *d, st);
 }
 
 size_t hq_linear_bwd_dx_reuse_workspace_bytes(int64_t M, int64_t K, int64_t N) {

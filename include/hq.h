@@ -341,6 +341,34 @@ HQ_API hq_status hq_linear_bwd_reuse(const void* dY, hq_dtype dt, const void* xq
                                      size_t ws_bytes, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * The next layer's rotation in this GEMM's epilogue ("Training Transformers with 4-bit
+ * Integers", section 3.3: the Hadamard blocks come before quantization; "HALO: Hadamard-Assisted
+ * Lower-Precision Optimization for LLMs", Approach).  When a GEMM's output is the next
+ * GEMM's operand along its columns (a linear map with nothing nonlinear in between), the
+ * producing GEMM can apply that rotation while its accumulators are in registers, and the
+ * next operand is then only quantized.
+ *
+ * hq_gemm_rotout -- out [M][N] fp32 = blockdiag(H_k / sqrt(k)) along the columns of
+ *   fp32(sum_l A[i][l] B[j][l]) * fp32(scale_a * scale_b).  A [M][K], B [N][K] codes (both
+ *   contraction-innermost, as hq_gemm), device scales; N % k == 0.  Arithmetic as the
+ *   library's rotation: butterflies h = 1 .. k/2 (index bit 0 first), then x fp32(1/sqrt(k)).
+ *   Formats HQ_INT8 and HQ_FP8_E4M3 (others HQ_ERR_ARG).  Errors as hq_gemm.
+ *
+ * hq_quantize_prerotated -- tensor-wise codes of rotated values y [rows][cols] fp32 (no
+ *   transform): a = max |y|, codes RNE(fp32(y * fp32(QMAX / a))), *scale = fp32(a / QMAX),
+ *   exactly the steps hq_quantize takes after its rotation.  cols % 16 == 0.  Formats HQ_INT8
+ *   and HQ_FP8_E4M3.  workspace: >= hq_quantize_prerotated_workspace_bytes() bytes.  A
+ *   non-finite a sets HQ_ERR_NONFINITE in the status word and writes no codes.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_gemm_rotout(const void* A, const float* scale_a, const void* B,
+                                const float* scale_b, int64_t M, int64_t N, int64_t K, int k,
+                                hq_fmt fmt, float* out, hq_stream_t stream);
+HQ_API size_t hq_quantize_prerotated_workspace_bytes(void);
+HQ_API hq_status hq_quantize_prerotated(const float* y, int64_t rows, int64_t cols, hq_fmt fmt,
+                                        void* codes, float* scale, void* workspace,
+                                        size_t ws_bytes, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * hq_quantize_noalloc -- hq_quantize for callers that cannot allocate device memory.
  *
  * The pages have no counterpart to this call: it exists for integration only.  Some callers

@@ -309,3 +309,31 @@ def test_reuse_flow_argument_errors(L):
     assert hq.hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N) >= 4 * M * K
     assert hq.hq_linear_bwd_reuse_workspace_bytes(M, K, N) >= N * M + 4 * M * K
     assert hq.hq_linear_bwd_reuse_workspace_bytes(-1, 1, 1) == 0
+
+
+def test_rotout_and_prerotated_argument_errors(L):
+    g = lambda **kw: L.hq_gemm_rotout(kw.get("A", FAKE), kw.get("sa", FAKE), FAKE, FAKE, kw.get("M", 256),
+                                      kw.get("N", 512), kw.get("K", 256), kw.get("k", 128), kw.get("fmt", 0),
+                                      kw.get("out", FAKE), None)
+    for fmt in (2, 3, 4, 9):
+        assert g(fmt=fmt) == 1
+    assert g(k=100) == 1
+    assert g(N=384, k=256) == 2     # N not a multiple of k
+    assert g(K=24) == 2             # contraction not a multiple of 16
+    assert g(sa=None) == 1          # the dequantized output needs both scales
+    assert g(out=None) == 1
+    assert g(A=FAKE_MIS) == 4
+    assert g(M=0) == 0 and g(N=0) == 0
+    q = lambda **kw: L.hq_quantize_prerotated(kw.get("y", FAKE), kw.get("rows", 64), kw.get("cols", 256),
+                                              kw.get("fmt", 1), kw.get("codes", FAKE), kw.get("scale", FAKE),
+                                              kw.get("ws", FAKE), kw.get("wsb", 1 << 20), None)
+    assert q(fmt=3) == 1
+    assert q(rows=-1) == 1
+    assert q(cols=24) == 2
+    assert q(y=None) == 1
+    assert q(scale=None) == 1
+    assert q(codes=FAKE_MIS) == 4
+    assert q(scale=FAKE + 2) == 4
+    assert q(ws=None) == 8
+    assert q(wsb=16) == 8
+    assert hq.hq_quantize_prerotated_workspace_bytes() == hq.hq_quantize_workspace_bytes()
