@@ -292,9 +292,14 @@ def run_gpu(args):
         return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], k, fmt, codes_c.data_ptr(), sp(si_c),
                 codes_r.data_ptr(), sp(si_r), ws, pw, st)
 
+    # the GEMMs run one after another on the main stream and share one split scratch
+    gws_len = max(hq.hq_gemm_workspace_bytes(M, N, K), hq.hq_gemm_workspace_bytes(M, K, N),
+                  hq.hq_gemm_workspace_bytes(N, K, M))
+    gws = torch.empty(max(gws_len, 16), dtype=torch.uint8, device=device)
+
     def gemm(a, ai, b, bi, out):
         return (a.data_ptr(), sp(ai), b.data_ptr(), sp(bi), a.shape[0], b.shape[0], a.shape[1], fmt,
-                hq.HQ_OUT_BF16, out.data_ptr(), sh)
+                hq.HQ_OUT_BF16, out.data_ptr(), gws.data_ptr(), gws_len, sh)
 
     pq = hq.hq_quantize_workspace_bytes()
 
@@ -328,13 +333,13 @@ def run_gpu(args):
         rec(ev_main, 0, stream)
         run(q_main, L_.hq_quantize, "hq_quantize")
         rec(ev_main, 1, stream)
-        run([g_fwd], L_.hq_gemm, "hq_gemm")
+        run([g_fwd], L_.hq_gemm_ws, "hq_gemm_ws")
         rec(ev_main, 2, stream)
         stream.wait_event(join)
         rec(ev_main, 3, stream)
-        run([g_dx], L_.hq_gemm, "hq_gemm")
+        run([g_dx], L_.hq_gemm_ws, "hq_gemm_ws")
         rec(ev_main, 4, stream)
-        run([g_dw], L_.hq_gemm, "hq_gemm")
+        run([g_dw], L_.hq_gemm_ws, "hq_gemm_ws")
         rec(ev_main, 5, stream)
 
     for _ in range(args.warmup):
@@ -579,7 +584,9 @@ def run_sweep(args):
                 gemm_ms = 0.0
                 for a, b, o in (("XK", "WK", Y), ("DN", "WN", dX), ("DM", "XM", dW)):
                     (ca, sa), (cb, sb) = codes[a], codes[b]
-                    gemm_ms += timed(lambda: hq.hq_gemm(ca, sa, cb, sb, fmt, out=o))
+                    gws = torch.empty(max(16, hq.hq_gemm_workspace_bytes(ca.shape[0], cb.shape[0], ca.shape[1])),
+                                      dtype=torch.uint8, device=dev)
+                    gemm_ms += timed(lambda: hq.hq_gemm(ca, sa, cb, sb, fmt, out=o, workspace=gws))
                 elem = X.element_size()
                 qbytes = (elem + 1) * 2 * (M * K + N * K + M * N)
                 ops = 6.0 * M * N * K

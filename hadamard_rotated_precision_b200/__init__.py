@@ -38,6 +38,7 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_bwd_dx_reuse_workspace_bytes", "hq_linear_bwd_dx_reuse",
            "hq_linear_bwd_reuse_workspace_bytes", "hq_linear_bwd_reuse",
            "hq_gemm_rotout", "hq_quantize_prerotated_workspace_bytes", "hq_quantize_prerotated",
+           "hq_gemm_workspace_bytes", "hq_gemm_ws",
            "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
@@ -106,6 +107,10 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_bwd_dx_reuse.restype = i32
         L.hq_linear_bwd_reuse.argtypes = [p, i32, p, p, p, p, i64, i64, i64, i32, i32, p, p, p, sz, p]
         L.hq_linear_bwd_reuse.restype = i32
+        L.hq_gemm_workspace_bytes.argtypes = [i64, i64, i64]
+        L.hq_gemm_workspace_bytes.restype = sz
+        L.hq_gemm_ws.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p, sz, p]
+        L.hq_gemm_ws.restype = i32
         L.hq_gemm_rotout.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
         L.hq_gemm_rotout.restype = i32
         L.hq_quantize_prerotated_workspace_bytes.argtypes = []
@@ -635,9 +640,14 @@ def hq_quantize_prerotated(y, fmt, codes=None, scale=None, workspace=None, strea
     return codes, scale
 
 
-def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None):
+def hq_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().hq_gemm_workspace_bytes(M, N, K))
+
+
+def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, stream=None, workspace=None):
     """out[M][N] = sum_l A[i][l] B[j][l] on codes (both contraction-innermost), dequantized
-    to bf16 by scale_a*scale_b (HQ_OUT_BF16) or raw int32/fp32 accumulators (HQ_OUT_ACC)."""
+    to bf16 by scale_a*scale_b (HQ_OUT_BF16) or raw int32/fp32 accumulators (HQ_OUT_ACC).
+    workspace: optional device scratch (hq_gemm_ws) that lets the last wave's tiles split."""
     torch = _torch()
     _dev_tensor(A, "A")
     _dev_tensor(B, "B")
@@ -655,8 +665,14 @@ def hq_gemm(A, scale_a, B, scale_b, fmt, out_kind: int = HQ_OUT_BF16, out=None, 
     _dev_tensor(out, "out")
     sa = scale_a.data_ptr() if scale_a is not None else None
     sb = scale_b.data_ptr() if scale_b is not None else None
-    st = lib().hq_gemm(A.data_ptr(), sa, B.data_ptr(), sb, M, N, K, f, out_kind, out.data_ptr(),
-                       _stream_handle(stream))
+    if workspace is None:
+        st = lib().hq_gemm(A.data_ptr(), sa, B.data_ptr(), sb, M, N, K, f, out_kind, out.data_ptr(),
+                           _stream_handle(stream))
+    else:
+        _dev_tensor(workspace, "workspace")
+        st = lib().hq_gemm_ws(A.data_ptr(), sa, B.data_ptr(), sb, M, N, K, f, out_kind, out.data_ptr(),
+                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream))
     _check(st, "hq_gemm")
     return out
 

@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
-                 unsigned int* __restrict__ status, int splits, uint32_t* __restrict__ part_ws,
+                 unsigned int* __restrict__ status, int split_from, uint32_t* __restrict__ part_ws,
                  int* __restrict__ counters, uint32_t ab_code, int rot_k) {
   // rot_k (kOutF32 only; 0 = none): rotate the output along its columns in blocks of rot_k
   // before storing (see epi_rot_cols)
@@ -514,11 +514,31 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
-  // Work item i: tile i % num_tiles, k-block range of split i / num_tiles (splits = 1: the
-  // whole contraction).  With splits = 2 each half writes its partial accumulator to part_ws;
-  // the warp slab that finishes second adds the other half and writes the output.
-  const int num_items = num_tiles * splits;
-  const int kb_per = (num_kb + splits - 1) / splits;
+  // Work items: tiles below split_from whole (items 0 .. F-1, tile = item), the tiles from
+  // split_from on in two halves of the k-blocks (item F + j: tile F + j % T, half j / T, so both
+  // halves of a tile run in the same wave).  split_from >= num_tiles: no split; 0: every tile
+  // split; in between: only the last, partial wave's tiles, so that it takes half a tile-time.
+  // A half writes its partial accumulator to part_ws; the warp slab that finishes second adds
+  // the other half and writes the output (bf16 output only).
+  const int split_f = min(split_from, num_tiles);
+  const int split_t = num_tiles - split_f;
+  const int num_items = split_f + 2 * split_t;
+  const int kb_half = (num_kb + 1) / 2;
+  struct Item { int tile, half, kb_begin, kb_end; bool part; };
+  auto item_at = [&](int item) {
+    Item it;
+    if (item < split_f) {
+      it.tile = item; it.half = 0; it.kb_begin = 0; it.kb_end = num_kb; it.part = false;
+    } else {
+      const int j = item - split_f;
+      it.tile = split_f + j % split_t;
+      it.half = j / split_t;
+      it.kb_begin = it.half ? kb_half : 0;
+      it.kb_end = it.half ? num_kb : kb_half;
+      it.part = true;
+    }
+    return it;
+  };
 
   auto bar = [&](int i) { return ptx::smem_u32(sh.bars + i); };
   auto full_bar = [&](int s) { return bar(s); };
@@ -561,10 +581,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int item = pair_id; item < num_items && ok; item += num_pairs) {
-        const int tile = item % num_tiles, split = item / num_tiles;
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
-        const int kb_end = min(num_kb, (split + 1) * kb_per);
-        for (int kb = split * kb_per; kb < kb_end; ++kb) {
+        const Item it = item_at(item);
+        const int m_blk = it.tile % num_m, n_blk = it.tile / num_m;
+        for (int kb = it.kb_begin; kb < it.kb_end; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
           const uint32_t fb = ptx::mapa_shared(full_bar(stage), 0);
           if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
@@ -597,8 +616,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int item = pair_id; item < num_items && ok; item += num_pairs) {
-        const int split = item / num_tiles;
-        const int kb_begin = split * kb_per, kb_end = min(num_kb, kb_begin + kb_per);
+        const Item it = item_at(item);
+        const int kb_begin = it.kb_begin, kb_end = it.kb_end;
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, sh.abort_flag, status)) break;
         ptx::tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
@@ -640,8 +659,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int item = pair_id; item < num_items; item += num_pairs) {
-      const int tile = item % num_tiles, split = item / num_tiles;
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const Item it = item_at(item);
+      const int m_blk = it.tile % num_m, n_blk = it.tile / num_m;
       int ok = 0;
       if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, sh.abort_flag, status) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -656,10 +675,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         const uint32_t* peer = nullptr;
         int* slab_counter = nullptr;
         bool emit = true;
-        if (splits > 1) {
+        if (it.part) {
           const size_t slab_words = size_t(32) * BN;
-          const size_t slab = size_t(tile) * 8 + size_t(rank) * 4 + quarter;  // [tile][rank][quarter]
-          uint32_t* mine = part_ws + (size_t(split) * num_tiles * 8 + slab) * slab_words;
+          // [split tile][rank][quarter], the split tiles counted from split_from
+          const size_t slab = size_t(it.tile - split_f) * 8 + size_t(rank) * 4 + quarter;
+          uint32_t* mine = part_ws + (size_t(it.half) * split_t * 8 + slab) * slab_words;
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t r[32];
@@ -676,10 +696,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           int prev = 0;
           if (lane == 0) prev = atomicAdd(slab_counter, 1);
           prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-          emit = prev == splits - 1;
+          emit = prev == 1;
           if (emit) {
             __threadfence();  // the other half's partial is visible
-            peer = part_ws + (size_t(1 - split) * num_tiles * 8 + slab) * slab_words;
+            peer = part_ws + (size_t(1 - it.half) * split_t * 8 + slab) * slab_words;
           } else {  // the accumulator has been read: the MMA may reuse it
             ptx::tc_fence_before_sync();
             __syncwarp();

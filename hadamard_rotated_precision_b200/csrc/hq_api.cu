@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -586,13 +587,15 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
 
 template <int FMT, int OUT, int BN, bool SK, bool MN = false>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const float* sa,
-                             const float* sb, void* out, int M, int N, int K, int clusters, int splits,
+                             const float* sb, void* out, int M, int N, int K, int clusters, int split_from,
                              uint32_t* part_ws, int* counters, uint32_t ab_code, DeviceInfo& d, cudaStream_t st,
                              int rot_k = 0) {
   namespace gp = hq::gemm::pair;
   using G = gp::Geo<BN, SK>;
   auto kernel = gp::gemm_pair_kernel<FMT, OUT, BN, SK, MN>;
-  const int items = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN) * splits;
+  const int tiles = ((M + gp::BM - 1) / gp::BM) * ((N + BN - 1) / BN);
+  const int f = std::min(split_from, tiles);
+  const int items = f + 2 * (tiles - f);  // whole tiles, then both halves of each split one
   const int pairs = std::max(1, std::min(items, clusters));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
@@ -607,7 +610,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   (void)d;
-  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, splits, part_ws, counters,
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, split_from, part_ws, counters,
                             ab_code, rot_k);
 }
 
@@ -662,17 +665,39 @@ int pick_splits(int64_t M, int64_t N, int64_t K, int clusters) {
   return double(w2) * 0.5 <= 0.7 * double(w1) ? 2 : 1;
 }
 
-size_t split_part_bytes(int64_t M, int64_t N) {
-  return size_t(2) * size_t((M + 255) / 256) * size_t((N + 255) / 256) * 256 * 256 * 4;
+// The first tile split in two along the contraction (the pair kernel's split_from; the
+// number of 256 x 256 tiles when none is):
+//  - every tile, when pick_splits says so;
+//  - otherwise the tiles of the last, partial wave, when they fill at most half the clusters,
+//    there are at most three full waves before them and the contraction has 64 or more
+//    k-blocks. The halves then all run in one wave of half a tile-time.
+// The exchange of partials and the counter reset cost about 8 us. Measured with INT8 on a
+// B200 (74 clusters), plain -> split:
+//   4096 x 4096 x 11008 (3.46 waves):  121.2 -> 116.6 us;
+//   4096 x 4096 x 4096 (3.46 waves):    53.5 -> 57.3 us;
+//   4096 x 11008 x 4096 (9.3 waves):   116.0 -> 118.9 us.
+// Hence the limits above.
+int64_t pick_split_from(int64_t M, int64_t N, int64_t K, int clusters) {
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  if (M < kPairMinRows || clusters <= 0) return tiles;
+  if (pick_splits(M, N, K, clusters) == 2) return 0;
+  const int64_t num_kb = (K + hq::gemm::BK - 1) / hq::gemm::BK;
+  if (num_kb < 64) return tiles;
+  const int64_t full = tiles / clusters, tail = tiles - full * clusters;
+  return (full >= 1 && full <= 3 && tail > 0 && 2 * tail <= clusters) ? tiles - tail : tiles;
 }
-size_t split_counter_bytes(int64_t M, int64_t N) {
-  return align_up(size_t((M + 255) / 256) * size_t((N + 255) / 256) * 8 * sizeof(int));
-}
+
+// Partial accumulators of t split tiles (both halves, fp32 / int32) and their arrival
+// counters (one per 32-row slab).
+size_t split_part_bytes(int64_t t) { return size_t(2) * size_t(t) * 256 * 256 * 4; }
+size_t split_counter_bytes(int64_t t) { return align_up(size_t(t) * 8 * sizeof(int)); }
 
 // Workspace a GEMM of the layer may use for a split contraction (0 when it never splits).
 size_t split_ws_bytes(int64_t M, int64_t N, int64_t K) {
-  if (pick_splits(M, N, K, kRefClusters) < 2) return 0;
-  return split_part_bytes(M, N) + split_counter_bytes(M, N);
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t t = tiles - pick_split_from(M, N, K, kRefClusters);
+  if (t <= 0) return 0;
+  return split_part_bytes(t) + split_counter_bytes(t);
 }
 
 hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* sb, int64_t M, int64_t N,
@@ -712,17 +737,20 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     if (e != cudaSuccess) return cuda_fail(e);
     bn = pick_pair_bn(m, n, clusters);
   }
-  int splits = 1;
+  const int64_t tiles256 = ((M + 255) / 256) * ((N + 255) / 256);
+  int split_from = INT_MAX;  // no split
   uint32_t* part_ws = nullptr;
   int* counters = nullptr;
-  if (pair && !sk && ok == HQ_OUT_BF16 && split_ws && pick_splits(M, N, K, clusters) == 2 &&
-      split_ws_len >= split_part_bytes(M, N) + split_counter_bytes(M, N)) {
-    splits = 2;
-    bn = 256;
-    counters = static_cast<int*>(split_ws);
-    part_ws = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(split_ws) + split_counter_bytes(M, N));
-    e = cudaMemsetAsync(counters, 0, split_counter_bytes(M, N), st);
-    if (e != cudaSuccess) return cuda_fail(e);
+  if (pair && !sk && ok == HQ_OUT_BF16 && split_ws) {
+    const int64_t f = pick_split_from(M, N, K, clusters), t = tiles256 - f;
+    if (t > 0 && split_ws_len >= split_part_bytes(t) + split_counter_bytes(t)) {
+      split_from = static_cast<int>(f);
+      bn = 256;
+      counters = static_cast<int*>(split_ws);
+      part_ws = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(split_ws) + split_counter_bytes(t));
+      e = cudaMemsetAsync(counters, 0, split_counter_bytes(t), st);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
   }
   CUtensorMap ta, tb;
   hq_status s = encode_codes_map(&ta, A, M, K, pair ? hq::gemm::pair::HALF : hq::gemm::BM);
@@ -733,9 +761,9 @@ hq_status gemm_impl(const void* A, const float* sa, const void* B, const float* 
     std::memset(&to, 0, sizeof(to));
     if (ok == HQ_OUT_BF16 && (s = encode_out_map(&to, out, M, N)) != HQ_OK) return s;
 #define HQ_PAIR_LAUNCH(F, O, SKV)                                                                       \
-  (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
+  (bn == 256 ? launch_gemm_pair<F, O, 256, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, split_from, part_ws, \
                                                 counters, ab, d, st)                                         \
-             : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, splits, part_ws, \
+             : launch_gemm_pair<F, O, 128, SKV>(ta, tb, to, sa, sb, out, m, n, kk, clusters, split_from, part_ws, \
                                                 counters, ab, d, st))
     if (fmt == HQ_INT8)
       e = ok == HQ_OUT_ACC ? HQ_PAIR_LAUNCH(kInt8, kOutAcc, false)
@@ -790,9 +818,9 @@ hq_status gemm_mn_f32_impl(const void* A, const float* sa, const void* B, const 
   if ((s = encode_codes_map(&tb, B, K, N, G::B_ROWS)) != HQ_OK) return s;
   const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
   e = f == 0 ? launch_gemm_pair<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false, true>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, rot_k)
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, INT_MAX, nullptr, nullptr, 0u, d, st, rot_k)
              : launch_gemm_pair<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false, true>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, rot_k);
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, INT_MAX, nullptr, nullptr, 0u, d, st, rot_k);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -882,9 +910,9 @@ hq_status gemm_rotout_impl(const void* A, const float* sa, const void* B, const 
   if ((s = encode_codes_map(&tb, B, N, K, G::B_ROWS)) != HQ_OK) return s;
   const int m = static_cast<int>(M), n = static_cast<int>(N), kk = static_cast<int>(K);
   e = f == 0 ? launch_gemm_pair<hq::gemm::kInt8, hq::gemm::kOutF32, 256, false>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, k)
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, INT_MAX, nullptr, nullptr, 0u, d, st, k)
              : launch_gemm_pair<hq::gemm::kFp8, hq::gemm::kOutF32, 256, false>(
-                   ta, tb, to, sa, sb, out, m, n, kk, clusters, 1, nullptr, nullptr, 0u, d, st, k);
+                   ta, tb, to, sa, sb, out, m, n, kk, clusters, INT_MAX, nullptr, nullptr, 0u, d, st, k);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 
@@ -1194,6 +1222,23 @@ hq_status hq_gemm(const void* A, const float* scale_a, const void* B, const floa
   DeviceInfo* d = nullptr;
   if ((s = device_info(&d)) != HQ_OK) return s;
   return gemm_impl(A, scale_a, B, scale_b, M, N, K, fmt, out_kind, out, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return split_ws_bytes(M, N, K);
+}
+
+hq_status hq_gemm_ws(const void* A, const float* scale_a, const void* B, const float* scale_b, int64_t M, int64_t N,
+                     int64_t K, hq_fmt fmt, hq_out out_kind, void* out, void* workspace, size_t ws_bytes,
+                     hq_stream_t stream) {
+  hq_status s = check_gemm_args(A, scale_a, B, scale_b, M, N, K, fmt, out_kind, out);
+  if (s != HQ_OK || M == 0 || N == 0) return s;
+  if (workspace && !aligned16(workspace)) return HQ_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  if ((s = device_info(&d)) != HQ_OK) return s;
+  return gemm_impl(A, scale_a, B, scale_b, M, N, K, fmt, out_kind, out, *d, reinterpret_cast<cudaStream_t>(stream),
+                   workspace, workspace ? ws_bytes : 0);
 }
 
 size_t hq_linear_workspace_bytes(int64_t M, int64_t K, int64_t N) {

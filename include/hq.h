@@ -128,6 +128,18 @@ HQ_API hq_status hq_gemm(const void* A, const float* scale_a, const void* B, con
                   int64_t M, int64_t N, int64_t K, hq_fmt fmt, hq_out out_kind, void* out,
                   hq_stream_t stream);
 
+/* hq_gemm_ws -- hq_gemm with device scratch for splitting tiles along the contraction (the
+ * layer calls use the same).  With at least hq_gemm_workspace_bytes(M, N, K) bytes (16-byte
+ * aligned; contents need no initialisation and are not preserved) a bf16-output GEMM whose
+ * last wave of 256 x 256 tiles fills at most half the CTA pairs splits those tiles in two
+ * halves of the k-blocks, and one with too few tiles for the pairs splits all of them; each
+ * half's fp32 / int32 partial is added to the other's once (INT8 results are unchanged, FP8
+ * ones round once more).  A NULL workspace, or a smaller one, runs hq_gemm. */
+HQ_API size_t hq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+HQ_API hq_status hq_gemm_ws(const void* A, const float* scale_a, const void* B, const float* scale_b,
+                            int64_t M, int64_t N, int64_t K, hq_fmt fmt, hq_out out_kind, void* out,
+                            void* workspace, size_t ws_bytes, hq_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * The three GEMMs of one linear layer Y = X W^T with M tokens, K = d_in, N = d_out, each
  * with both operands rotated along its contraction dimension and quantized tensor-wise

@@ -337,3 +337,16 @@ def test_rotout_and_prerotated_argument_errors(L):
     assert q(ws=None) == 8
     assert q(wsb=16) == 8
     assert hq.hq_quantize_prerotated_workspace_bytes() == hq.hq_quantize_workspace_bytes()
+
+
+def test_gemm_ws_arguments_and_sizes(L):
+    g = lambda **kw: L.hq_gemm_ws(FAKE, FAKE, FAKE, FAKE, 256, 256, kw.get("K", 256), kw.get("fmt", 0), 0,
+                                  kw.get("out", FAKE), kw.get("ws", FAKE), 1 << 20, None)
+    assert g(fmt=7) == 1
+    assert g(K=24) == 2
+    assert g(out=None) == 1
+    assert g(ws=FAKE_MIS) == 4
+    # the Llama up-projection's dX GEMM splits its last wave, its forward GEMM does not
+    assert hq.hq_gemm_workspace_bytes(4096, 4096, 11008) >= 2 * 34 * 256 * 256 * 4
+    assert hq.hq_gemm_workspace_bytes(4096, 11008, 4096) == 0
+    assert hq.hq_gemm_workspace_bytes(-1, 1, 1) == 0
