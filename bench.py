@@ -309,7 +309,8 @@ def run_gpu(args):
 
     q_main = [single(X, 1, qX_K, 0, ws_main, sh), single(W, 1, qW_K, 2, ws_main, sh)]
     q_side_dual = [dual(dY, qdY_N, 4, qdY_M, 5, ws_side, sh2)]
-    q_side = [single(W, 0, qW_N, 3, ws_side, sh2), single(X, 0, qX_M, 1, ws_side, sh2)]
+    q_side_wn = [single(W, 0, qW_N, 3, ws_side, sh2)]
+    q_side_xm = [single(X, 0, qX_M, 1, ws_side, sh2)]
     g_fwd, g_dx, g_dw = gemm(qX_K, 0, qW_K, 2, Y), gemm(qdY_N, 4, qW_N, 3, dX), gemm(qdY_M, 5, qX_M, 1, dW)
 
     def run(calls, fn, what):
@@ -326,7 +327,10 @@ def run_gpu(args):
         rec(ev_side, 0, side)
         run(q_side_dual, L_.hq_quantize_dual, "hq_quantize_dual")
         rec(ev_side, 1, side)
-        run(q_side, L_.hq_quantize, "hq_quantize")
+        run(q_side_wn, L_.hq_quantize, "hq_quantize")
+        join_dx = torch.cuda.Event()
+        join_dx.record(side)
+        run(q_side_xm, L_.hq_quantize, "hq_quantize")
         rec(ev_side, 2, side)
         join = torch.cuda.Event()
         join.record(side)
@@ -335,9 +339,10 @@ def run_gpu(args):
         rec(ev_main, 1, stream)
         run([g_fwd], L_.hq_gemm_ws, "hq_gemm_ws")
         rec(ev_main, 2, stream)
-        stream.wait_event(join)
+        stream.wait_event(join_dx)
         rec(ev_main, 3, stream)
         run([g_dx], L_.hq_gemm_ws, "hq_gemm_ws")
+        stream.wait_event(join)  # X along M, the weight gradient's operand
         rec(ev_main, 4, stream)
         run([g_dw], L_.hq_gemm_ws, "hq_gemm_ws")
         rec(ev_main, 5, stream)

@@ -1330,8 +1330,9 @@ hq_status hq_linear_fwd_bwd_rht(const void* X, const void* W, const void* dY, hq
                      neg_m)) != HQ_OK)
     return s;
   if ((s = quantize_impl(W, dt, N, K, 0, k, fmt, w.wqt, sc + 3, w.spart_c, *d, ss->s, neg_n)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dx, ss->s)) != cudaSuccess) return cuda_fail(e);  // dX's operands
   if ((s = quantize_impl(X, dt, M, K, 0, k, fmt, w.xqt, sc + 1, w.spart_c, *d, ss->s, neg_m)) != HQ_OK) return s;
-  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaEventRecord(ss->join_dw, ss->s)) != cudaSuccess) return cuda_fail(e);  // dW's
   // caller's stream: the forward operands (X and W along K) first, so the forward GEMM starts
   // as early as possible, then the backward GEMMs once the side stream's codes have landed
   if ((s = quantize_impl(X, dt, M, K, 1, k, fmt, w.xq, sc + 0, w.part_c, *d, st, neg_k)) != HQ_OK) return s;
@@ -1339,10 +1340,12 @@ hq_status hq_linear_fwd_bwd_rht(const void* X, const void* W, const void* dY, hq
   if ((s = gemm_impl(w.xq, sc + 0, w.wq, sc + 2, M, N, K, fmt, HQ_OUT_BF16, Y, *d, st, w.split, w.split_len)) !=
       HQ_OK)
     return s;
-  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
   if ((s = gemm_impl(w.dyq, sc + 4, w.wqt, sc + 3, M, K, N, fmt, HQ_OUT_BF16, dX, *d, st, w.split,
                      w.split_len)) != HQ_OK)
     return s;
+  // X along M lands while the dX GEMM runs
+  if ((e = cudaStreamWaitEvent(st, ss->join_dw, 0)) != cudaSuccess) return cuda_fail(e);
   return gemm_impl(w.dyqt, sc + 5, w.xqt, sc + 1, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, w.split, w.split_len);
 }
 

@@ -198,8 +198,9 @@ HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, in
  * does not use (dY along N and along M together, as in hq_quantize_dual, then W along N and
  * X along M) run on a per-device side stream that the library creates on first use (with
  * three events) and forks from / joins back to `stream` with events, so they overlap the
- * forward quantizations and GEMM; everything is complete when `stream` reaches the end of the
- * call.
+ * forward quantizations and GEMM.  The dX GEMM waits only for dY along N and W along N; X
+ * along M lands while it runs and the dW GEMM waits for it.  Everything is complete when
+ * `stream` reaches the end of the call.
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
 HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt,
