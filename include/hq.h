@@ -12,6 +12,11 @@
  *    output gradient is rotated on the left (along tokens) for the weight gradient (HALO-2);
  *    tensor-wise scales; INT8 or FP8 operands ("Key results", "Limitations").
  *
+ * Besides the three rotated GEMMs of a layer: a backward placement that reuses the forward's
+ * codes (hq_linear_fwd_keep / hq_linear_bwd_reuse), the next layer's rotation in a GEMM's
+ * epilogue (hq_gemm_rotout / hq_quantize_prerotated), the randomized Hadamard variant (*_rht)
+ * and the split quantization passes of quantized weight communication.
+ *
  * Readings taken where the pages are silent (all implemented identically by the test oracle):
  *  - H_k is Sylvester's natural-order Hadamard matrix, normalised by fp32(1/sqrt(k)); the
  *    transform is an fp32 FWHT with stages h = 1, 2, ..., k/2, no fused multiply-add.
@@ -24,13 +29,16 @@
  *
  * Conventions for every call:
  *  - All tensors are dense row-major device buffers owned by the caller; the library never
- *    allocates or frees memory and keeps no state except a per-device status word.
+ *    allocates or frees memory.  Its only state, per device: the status word, the side
+ *    stream and three events the multi-kernel layer calls fork to (created on first use),
+ *    and hq_quantize_noalloc's fixed scratch array.
  *  - Every device pointer must be 16-byte aligned (else HQ_ERR_ALIGN).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).
  *    Argument errors are returned synchronously before anything is launched.  Errors found
  *    on the device (non-finite operand, an internal wait that expired) are recorded in the
  *    status word and returned by hq_get_error(); outputs are unspecified after an error.
- *  - Codes are 1 byte each (int8 two's complement, or e4m3 bits) stored with the rotated
+ *  - Codes take 1 byte per element (int8 two's complement, e4m3 bits, or the FP6 / FP4
+ *    minifloats in the tensor cores' packed layout, see hq_fmt) and are stored with the rotated
  *    (contraction) dimension innermost.  Scales are one fp32 each, in device memory.
  *  - k is one of 16, 32, 64, 128, 256.
  */
