@@ -86,37 +86,6 @@ __device__ __forceinline__ void load8<float, true>(const float* p, float (&v)[8]
   v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y); v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
 }
 
-// ------------------------------------------------------------------ butterflies
-
-// Stages h = 1, 2, 4 over the 8 register-resident elements (in-block index bits 0..2).
-__device__ __forceinline__ void butterfly_regs8(float (&v)[8]) {
-#pragma unroll
-  for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i & h) continue;
-      const float u = v[i], w = v[i + h];
-      v[i] = __fadd_rn(u, w);
-      v[i + h] = __fsub_rn(u, w);
-    }
-  }
-}
-
-// Stages h = 8, 16, ..., K/2: the partner element sits in the lane whose index differs in
-// bit log2(h/8).  The lower-index holder keeps u + v, the upper one u - v.
-template <int K, int NV>
-__device__ __forceinline__ void butterfly_lanes(float (&v)[NV], int lane) {
-#pragma unroll
-  for (int m = 1; m < K / 8; m <<= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], m);
-      v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ quantizers
 
 __device__ __forceinline__ uint32_t code_int8(float y, float inv) {
