@@ -37,9 +37,9 @@ def _worker(rank, world, port, out):
 def test_reduce_max_over_two_gloo_ranks():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    ctx = mp.get_context("spawn")  # no fork of this (multi-threaded) process anywhere
+    mgr = ctx.Manager()
     out = mgr.dict()
-    ctx = mp.get_context("spawn")
     procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
     for p in procs:
         p.start()
