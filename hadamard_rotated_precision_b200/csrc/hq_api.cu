@@ -1567,9 +1567,21 @@ hq_status hq_linear_bwd_reuse(const void* dY, hq_dtype dt, const void* xqt_codes
   // dY once, rotated along the tokens: [N][M], the weight gradient's operand as it is and the
   // input gradient's MN-major operand
   if ((s = quantize_impl(dY, dt, M, N, 0, k, fmt, g, g_scale, partials, *d, st)) != HQ_OK) return s;
+  // the dX GEMM first (its output rotated along the columns, fp32), then its row de-rotation
+  // (HBM-bound) on the side stream while the dW GEMM (tensor-bound) runs on `stream`
+  if ((s = gemm_mn_f32_impl(g, g_scale, wq_codes, wq_scale, M, K, N, fmt, z, *d, st, k)) != HQ_OK) return s;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  if ((s = side_stream(&ss)) != HQ_OK) return s;
+  cudaError_t e;
+  if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return cuda_fail(e);
+  if ((s = derotate_impl(z, M, K, k, dX, *d, ss->s)) != HQ_OK) return s;
+  if ((e = cudaEventRecord(ss->join_dx, ss->s)) != cudaSuccess) return cuda_fail(e);
   if ((s = gemm_impl(g, g_scale, xqt_codes, xqt_scale, N, K, M, fmt, HQ_OUT_BF16, dW, *d, st, split, split_len)) != HQ_OK)
     return s;
-  return dx_reuse_impl(g, g_scale, wq_codes, wq_scale, M, K, N, k, fmt, dX, z, *d, st);
+  if ((e = cudaStreamWaitEvent(st, ss->join_dx, 0)) != cudaSuccess) return cuda_fail(e);
+  return HQ_OK;
 }
 
 hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows, int64_t cols, int dim, int k,

@@ -339,9 +339,11 @@ HQ_API hq_status hq_linear_bwd(const void* dY, const void* W, const void* xqt_co
  *
  * hq_linear_bwd_reuse -- dX and dW of one layer from dY [M][N] (dtype dt), the saved
  *   xqt_codes [K][M] / *xqt_scale of hq_linear_fwd_save / _keep and the kept wq_codes [N][K] /
- *   *wq_scale: dY quantized once along M, the dW GEMM, then hq_linear_bwd_dx_reuse, all on
- *   `stream`.  Shape rules as hq_linear_fwd_bwd.  workspace: >=
- *   hq_linear_bwd_reuse_workspace_bytes(M, K, N).  dW equals hq_linear_bwd's bit for bit.
+ *   *wq_scale: dY quantized once along M, the dX GEMM, then the dW GEMM on `stream` while the
+ *   de-rotation of dX's rows runs on the library's side stream (see hq_linear_fwd_bwd); all
+ *   outputs are complete when `stream` reaches the end of the call.  Shape rules as
+ *   hq_linear_fwd_bwd.  workspace: >= hq_linear_bwd_reuse_workspace_bytes(M, K, N).  dW equals
+ *   hq_linear_bwd's bit for bit, dX hq_linear_bwd_dx_reuse's.
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_fwd_keep_workspace_bytes(int64_t M, int64_t K, int64_t N);
 HQ_API hq_status hq_linear_fwd_keep(const void* X, const void* W, hq_dtype dt, int64_t M,
