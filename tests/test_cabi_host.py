@@ -350,3 +350,20 @@ def test_gemm_ws_arguments_and_sizes(L):
     assert hq.hq_gemm_workspace_bytes(4096, 4096, 11008) >= 2 * 34 * 256 * 256 * 4
     assert hq.hq_gemm_workspace_bytes(4096, 11008, 4096) == 0
     assert hq.hq_gemm_workspace_bytes(-1, 1, 1) == 0
+
+
+def test_split_rule_through_workspace_sizes(L):
+    """The GEMM's split choice, seen through the scratch it asks for (74 CTA pairs, 256 x 256
+    tiles): a last wave at most half full after at most three full waves, with 64 or more
+    128-deep k-blocks, splits only its own tiles; a GEMM with too few tiles splits all of them;
+    everything else needs no scratch."""
+    tile_half = 256 * 256 * 4  # one half's fp32 / int32 partial of one tile
+    ws = hq.hq_gemm_workspace_bytes
+    # 4096 x 4096 x 11008: 256 tiles = 3 waves + 34, 86 k-blocks -> the 34 tail tiles split
+    assert 2 * 34 * tile_half <= ws(4096, 4096, 11008) < 2 * 35 * tile_half + 4096
+    assert ws(4096, 4096, 4096) == 0       # 32 k-blocks: the split would cost more than it saves
+    assert ws(4096, 11008, 4096) == 0      # 688 tiles = 9 full waves + 22: not split
+    assert ws(8192, 4096, 4096) == 0       # 512 tiles: the last wave is 68 of 74, more than half
+    # 3072 x 768 x 12608: 36 tiles for 74 pairs -> every tile split in two
+    assert ws(3072, 768, 12608) >= 2 * 36 * tile_half
+    assert ws(128, 4096, 11008) == 0       # fewer than 256 rows: single-CTA kernel, no split
