@@ -231,8 +231,8 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
     ptx::prefetch_tmap(&map);
     for (int64_t q = 0; q < (n_strips < kSlots ? n_strips : kSlots); ++q) issue(q);
   }
-  // A warp is done with strip q: the sixteenth warp to say so for this round of the slot
-  // refills it with strip q + kSlots.  Each warp's reads of the strip are ordered before its
+  // A warp is done with strip q: the last of the kComputeWarps warps to say so for this use of
+  // the slot refills it with strip q + kSlots.  Each warp's reads of the strip are ordered before its
   // count (syncwarp, then a CTA fence), and the counting warp's fence orders all of them
   // before its copy is issued.
   auto release = [&](int64_t q) {
