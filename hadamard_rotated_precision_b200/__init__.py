@@ -1,5 +1,5 @@
-"""Python binding of libhq.so: Hadamard-rotated, tensor-wise quantized INT8/FP8 linear layer
-for B200 (sm_100a).
+"""Python binding of libhq.so: Hadamard-rotated, tensor-wise quantized linear layer (INT8, FP8
+e4m3, FP6 e3m2 / e2m3 and FP4 e2m1 codes) for B200 (sm_100a).
 
 Argument marshalling only: every step of the computation runs in the library's CUDA
 kernels; PyTorch provides device memory and streams.  The functions carry the names of the
