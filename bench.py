@@ -503,7 +503,7 @@ def run_gpu(args):
                        "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each); achieved: the three two-rotation quantizations timed alone with CUDA events, L2 flushed before each; in_step: summed event time of the same launches inside the overlapped step (sharing the GPU with the GEMMs); single_rotation: the six rotations as one-rotation calls"},
         "phases_ms": phases,
         "gemm_ms_per_step": gemm_ms_launch * 3,
-        "schedule": "X and W along K + forward GEMM on the main stream; dY in both rotations (one read per pass), W along N and X along M on a side stream overlapping them",
+        "schedule": "X and W along K + forward GEMM on the main stream; dY in both rotations (one read per pass), W along N and X along M on a side stream overlapping them; the dX GEMM waits for W along N, the dW GEMM for X along M",
         "frac_of_int8_peak_end_to_end": value / world / int8_peak,
         "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": elem * (M * K + N * K + M * N),
