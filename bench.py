@@ -1,16 +1,20 @@
 #!/usr/bin/env python
-"""Benchmark: one HALO-2 linear layer, forward + both backward GEMMs, on B200.
+"""Benchmark: the HALO-2 linear layers of a Llama-2-7B-shaped decoder block, forward + both
+backward GEMMs, on B200.
 
-A step is the whole hot path over one batch: the six Hadamard-rotate + quantize passes
-(X along K and M, W along K and N, dY along N and M) and the three tcgen05 GEMMs with the
-dequantizing epilogue (Y = X W^T, dX = dY W, dW = dY^T X).  Workload: Llama-style MLP
-up-projection, 4096 tokens (batch 4 x seq 1024), d_in 4096 -> d_out 11008, bf16 inputs,
-INT8 codes, k = 256, synthetic seeded inputs (N(0,1) activations with 1% outlier channels
-x U[30,100], N(0,0.02) weights, Student-t(3) x 1e-3 output gradients).
+A step is the whole hot path over one batch for every linear layer of the block (qkv 4096 ->
+12288, o 4096 -> 4096, gate and up 4096 -> 11008, down 11008 -> 4096; 8192 tokens): per
+layer the six Hadamard-rotate + quantize passes (X along K and M, W along K and N, dY along N
+and M) and the three tcgen05 GEMMs with the dequantizing epilogue (Y = X W^T, dX = dY W,
+dW = dY^T X), each layer through the library's own entry point hq_linear_fwd_bwd.  INT8
+codes, k = 256, bf16 inputs drawn seeded (N(0,1) activations with 1% outlier channels x
+U[30,100], N(0,0.02) weights, Student-t(3) x 1e-3 output gradients).
 
-Prints one JSON line (rank 0).  `value` = 6*M*N*K / device time per step (TOPS), inputs
-resident in HBM; `e2e` = the same metric through the public API with the inputs copied
-from pinned host memory and the three outputs copied back inside the timed region.
+Prints one JSON line (rank 0).  `value` = sum over layers of 6*M*N*K / device time per step
+(TOPS), inputs resident in HBM; `e2e` = the same metric through the same entry point with the
+inputs copied from pinned host memory and the three outputs of every layer copied back inside
+the timed region.  The dense INT8 / FP8 tensor peaks are measured in the same run
+(hq_mma_peak: MMA-only, operands in shared memory).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -37,15 +41,18 @@ if ROOT not in sys.path:
 
 from hadamard_rotated_precision_b200 import synthetic  # noqa: E402
 
-WORKLOAD_ID = 2
+WORKLOAD_ID = 5        # the Llama-2-7B block at 8192 tokens (INT8, k = 256 for the headline step)
+LAYER_WORKLOAD_ID = 2  # the Llama up-projection layer at 4096 tokens (an extra key of the line)
 METRIC = "HALO-2 linear fwd+bwd TOPS, % of INT8/FP8 tensor peak; FWHT+quant HBM GB/s"
 UNIT = "TOPS"
-INT8_OVER_BF16 = 2.0  # nominal dense INT8 / bf16 tensor throughput ratio on B200 (4.5 / 2.25)
+NOMINAL_INT8_TOPS = 4500.0  # B200 dense INT8 / FP8, nominal (context only)
 GEMM_SRC = os.path.join(ROOT, "hadamard_rotated_precision_b200", "csrc", "gemm_tcgen05.cuh")
-QUANT_SRC = os.path.join(ROOT, "hadamard_rotated_precision_b200", "csrc", "fwht_quant.cuh")
+QUANT_SRC = os.path.join(ROOT, "hadamard_rotated_precision_b200", "csrc", "fwht_dual.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-CPU_SAMPLE_TOKENS = 512
-REF_STEP_TOKENS = 256
+CPU_SAMPLE_TOKENS = 256   # cpu_baseline: every layer of the block at this many tokens
+REF_STEP_TOKENS = 256     # --impl reference: one layer of the block per step (in turn), this many tokens
+# (token samples are multiples of k: the weight gradient's operands are rotated along the tokens)
+MMA_OPS = 2 * 256 * 256 * 32  # operations of one CTA-pair MMA instruction of the peak probe
 
 
 # ----------------------------------------------------------------------------- distributed
@@ -180,28 +187,69 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def draw_block(w, tokens=None):
+    """Every layer's inputs (seeded, numpy), drawn in parallel worker processes started with
+    spawn before any CUDA call of this process."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    n = len(w.layers)
+    with ProcessPoolExecutor(max_workers=max(1, min(n, os.cpu_count() or 1)),
+                             mp_context=mp.get_context("spawn")) as ex:
+        futs = [ex.submit(synthetic.draw, w, li, tokens) for li in range(n)]
+        return [f.result() for f in futs]
+
+
+def block_ops(w, tokens=None) -> float:
+    return sum(6.0 * (L.M if tokens is None else tokens) * L.N * L.K for L in w.layers)
+
+
+def measure_mma_peaks(hq, torch, sustained: bool = True):
+    """Dense tensor-core peaks of this GPU, measured with the MMA-only probe (operands in
+    shared memory, accumulator in TMEM, no global traffic): burst = best of ten ~1 ms runs,
+    sustained = one run of about a quarter second (under the power cap)."""
+    def run(fmt, n_blocks, reps):
+        best, pairs = 0.0, 0
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            pairs = hq.hq_mma_peak(fmt, n_blocks)
+            b.record()
+            torch.cuda.synchronize()
+            best = max(best, pairs * n_blocks * 4 * MMA_OPS / (a.elapsed_time(b) * 1e-3) / 1e12)
+        return best
+    out = {}
+    for name in ("int8", "fp8"):
+        run(name, 256, 2)
+        out[name] = run(name, 4096, 10)
+        if sustained and name == "int8":
+            out["int8_sustained"] = run(name, 1000000, 1)
+    if hq.hq_get_error() != 0:
+        raise SystemExit("tensor-core peak probe reported a device error")
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU (oracle)
 
-def oracle_layer_seconds(d, k: int, fmt: int) -> float:
+def oracle_block_seconds(ds, w, fmt: int) -> float:
     import oracle
     t0 = time.perf_counter()
-    oracle.linear_fwd(d["X"], d["W"], k, fmt)
-    oracle.linear_bwd_dx(d["dY"], d["W"], k, fmt)
-    oracle.linear_bwd_dw(d["dY"], d["X"], k, fmt)
+    for d in ds:
+        oracle.linear_fwd(d["X"], d["W"], w.k, fmt)
+        oracle.linear_bwd_dx(d["dY"], d["W"], w.k, fmt)
+        oracle.linear_bwd_dw(d["dY"], d["X"], w.k, fmt)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, tokens: int):
-    """The oracle, untuned, on a token-prefix sample of the workload (full K, N, k, format)."""
+def cpu_baseline(w, ds_sample, tokens: int):
+    """The oracle, untuned, on a token-prefix sample of every layer of the block (full K, N,
+    k, format)."""
     import oracle
-    L = w.layers[0]
-    d = synthetic.draw(w, 0, M=tokens)
     fmt = 0 if w.fmt == "int8" else 1
-    secs = oracle_layer_seconds(d, w.k, fmt)
-    ops = 6.0 * tokens * L.K * L.N
+    secs = oracle_block_seconds(ds_sample, w, fmt)
+    ops = block_ops(w, tokens)
     return {"value": ops / secs / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{L.name} layer fwd+dX+dW at {tokens} of {L.M} tokens (K={L.K}, N={L.N}, "
-                      f"k={w.k}, {w.fmt}), {secs:.2f} s"}
+            "sample": f"all {len(w.layers)} layers of {w.name} (fwd+dX+dW) at {tokens} of {w.layers[0].M} tokens "
+                      f"(full K, N, k={w.k}, {w.fmt}), {secs:.2f} s"}
 
 
 def run_reference(args):
@@ -211,25 +259,37 @@ def run_reference(args):
     import oracle
     oracle.build()
     w = synthetic.WORKLOADS[WORKLOAD_ID]
-    L = w.layers[0]
-    d = synthetic.draw(w, 0, M=REF_STEP_TOKENS)
+    ds = draw_block(w, REF_STEP_TOKENS)
     fmt = 0 if w.fmt == "int8" else 1
-    for _ in range(args.warmup):
-        oracle_layer_seconds(d, w.k, fmt)
-    total = 0.0
-    for _ in range(args.steps):
-        total += oracle_layer_seconds(d, w.k, fmt)
-    ops = 6.0 * REF_STEP_TOKENS * L.K * L.N
-    value = ops * args.steps / total / 1e12
+    n = len(w.layers)
+
+    def layer_step(i):
+        d, L = ds[i % n], w.layers[i % n]
+        t0 = time.perf_counter()
+        oracle.linear_fwd(d["X"], d["W"], w.k, fmt)
+        oracle.linear_bwd_dx(d["dY"], d["W"], w.k, fmt)
+        oracle.linear_bwd_dw(d["dY"], d["X"], w.k, fmt)
+        return time.perf_counter() - t0, 6.0 * REF_STEP_TOKENS * L.N * L.K
+
+    for i in range(args.warmup):
+        layer_step(i)
+    total, ops = 0.0, 0.0
+    for i in range(args.steps):
+        t, o = layer_step(i)
+        total += t
+        ops += o
+    value = ops / total / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: M={L.M} K={L.K} N={L.N} k={w.k} {w.fmt} bf16 inputs",
+        "config": {"workload": f"{w.name}: Llama-2-7B block linears (qkv, o, gate, up, down) at "
+                               f"{w.layers[0].M} tokens, k={w.k} {w.fmt}, bf16 inputs",
                    "step_sample_tokens": REF_STEP_TOKENS, "parallelism": "rank 0 only (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                         "sample": f"each step: fwd+dX+dW at {REF_STEP_TOKENS} of {L.M} tokens"},
+                         "sample": f"step i: layer i mod {n} of the block, fwd+dX+dW at {REF_STEP_TOKENS} of "
+                                   f"{w.layers[0].M} tokens (full K, N)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -239,11 +299,16 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- GPU
 
 def run_gpu(args):
+    world, rank, local = dist_env()
+    w = synthetic.WORKLOADS[WORKLOAD_ID]
+    # host-side draws first: the worker pool starts (spawn) before this process touches CUDA
+    inputs = draw_block(w)
+    cpu_sample = draw_block(w, CPU_SAMPLE_TOKENS) if (rank == 0 and world == 1) else None
+
     import torch
     import hadamard_rotated_precision_b200 as hq
     from hadamard_rotated_precision_b200 import build
 
-    world, rank, local = dist_env()
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             raise SystemExit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
@@ -252,100 +317,38 @@ def run_gpu(args):
     init_dist(world, "nccl")
     build.build()
     hq.lib()
-
-    w = synthetic.WORKLOADS[WORKLOAD_ID]
-    L = w.layers[0]
-    M, K, N, k = L.M, L.K, L.N, w.k
+    k = w.k
     fmt = hq.HQ_INT8 if w.fmt == "int8" else hq.HQ_FP8_E4M3
-    d = synthetic.draw(w, 0)
+
     def dev(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
-    X, W, dY = dev(d["X"]), dev(d["W"]), dev(d["dY"])
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=device)
-    dW = torch.empty(N, K, dtype=torch.bfloat16, device=device)
-    qX_K = torch.empty(M, K, dtype=torch.uint8, device=device)
-    qX_M = torch.empty(K, M, dtype=torch.uint8, device=device)
-    qW_K = torch.empty(N, K, dtype=torch.uint8, device=device)
-    qW_N = torch.empty(K, N, dtype=torch.uint8, device=device)
-    qdY_N = torch.empty(M, N, dtype=torch.uint8, device=device)
-    qdY_M = torch.empty(N, M, dtype=torch.uint8, device=device)
-    scales = torch.empty(8, dtype=torch.float32, device=device)
-    lws = torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N), dtype=torch.uint8, device=device)
+
+    layers = []
+    for L, d in zip(w.layers, inputs):
+        M, K, N = L.M, L.K, L.N
+        layers.append(dict(
+            L=L, X=dev(d["X"]), W=dev(d["W"]), dY=dev(d["dY"]),
+            Y=torch.empty(M, N, dtype=torch.bfloat16, device=device),
+            dX=torch.empty(M, K, dtype=torch.bfloat16, device=device),
+            dW=torch.empty(N, K, dtype=torch.bfloat16, device=device),
+            ws=torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N), dtype=torch.uint8, device=device)))
+    del inputs
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    peaks_file = load_peaks()
+    mma = measure_mma_peaks(hq, torch)
+    int8_peak = mma["int8"]
 
-    # The step, as pre-marshalled C-ABI calls in the schedule hq_linear_fwd_bwd uses: X and W
-    # quantized in both rotations and the forward GEMM on the main stream, dY in both
-    # rotations on a side stream alongside them, joined by an event before the backward
-    # GEMMs.  CUDA events on each stream time every group of launches.
-    L_ = hq.lib()
-    side = torch.cuda.Stream(device)
-    sh, sh2 = stream.cuda_stream, side.cuda_stream
-    sp = lambda i: scales[i:i + 1].data_ptr()  # noqa: E731
-    pw = hq.hq_quantize_dual_workspace_bytes()
-    part = torch.empty(2 * pw, dtype=torch.uint8, device=device)
-    ws_main, ws_side = part.data_ptr(), part.data_ptr() + pw
-
-    def dual(src, codes_c, si_c, codes_r, si_r, ws, st):
-        return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], k, fmt, codes_c.data_ptr(), sp(si_c),
-                codes_r.data_ptr(), sp(si_r), ws, pw, st)
-
-    # the GEMMs run one after another on the main stream and share one split scratch
-    gws_len = max(hq.hq_gemm_workspace_bytes(M, N, K), hq.hq_gemm_workspace_bytes(M, K, N),
-                  hq.hq_gemm_workspace_bytes(N, K, M))
-    gws = torch.empty(max(gws_len, 16), dtype=torch.uint8, device=device)
-
-    def gemm(a, ai, b, bi, out):
-        return (a.data_ptr(), sp(ai), b.data_ptr(), sp(bi), a.shape[0], b.shape[0], a.shape[1], fmt,
-                hq.HQ_OUT_BF16, out.data_ptr(), gws.data_ptr(), gws_len, sh)
-
-    pq = hq.hq_quantize_workspace_bytes()
-
-    def single(src, dim, codes, si, ws, st):
-        return (src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt, codes.data_ptr(), sp(si),
-                ws, pq, st)
-
-    q_main = [single(X, 1, qX_K, 0, ws_main, sh), single(W, 1, qW_K, 2, ws_main, sh)]
-    q_side_dual = [dual(dY, qdY_N, 4, qdY_M, 5, ws_side, sh2)]
-    q_side_wn = [single(W, 0, qW_N, 3, ws_side, sh2)]
-    q_side_xm = [single(X, 0, qX_M, 1, ws_side, sh2)]
-    g_fwd, g_dx, g_dw = gemm(qX_K, 0, qW_K, 2, Y), gemm(qdY_N, 4, qW_N, 3, dX), gemm(qdY_M, 5, qX_M, 1, dW)
-
-    def run(calls, fn, what):
-        for c in calls:
-            st = fn(*c)
-            if st:
-                raise hq.HQError(st, what)
-
-    def step(ev_main=None, ev_side=None):
-        rec = (lambda lst, i, s_: lst[i].record(s_)) if ev_main is not None else (lambda *a: None)
-        fork = torch.cuda.Event()
-        fork.record(stream)
-        side.wait_event(fork)
-        rec(ev_side, 0, side)
-        run(q_side_dual, L_.hq_quantize_dual, "hq_quantize_dual")
-        rec(ev_side, 1, side)
-        run(q_side_wn, L_.hq_quantize, "hq_quantize")
-        join_dx = torch.cuda.Event()
-        join_dx.record(side)
-        run(q_side_xm, L_.hq_quantize, "hq_quantize")
-        rec(ev_side, 2, side)
-        join = torch.cuda.Event()
-        join.record(side)
-        rec(ev_main, 0, stream)
-        run(q_main, L_.hq_quantize, "hq_quantize")
-        rec(ev_main, 1, stream)
-        run([g_fwd], L_.hq_gemm_ws, "hq_gemm_ws")
-        rec(ev_main, 2, stream)
-        stream.wait_event(join_dx)
-        rec(ev_main, 3, stream)
-        run([g_dx], L_.hq_gemm_ws, "hq_gemm_ws")
-        stream.wait_event(join)  # X along M, the weight gradient's operand
-        rec(ev_main, 4, stream)
-        run([g_dw], L_.hq_gemm_ws, "hq_gemm_ws")
-        rec(ev_main, 5, stream)
+    # The step: every layer through the public entry point, one after another on one stream.
+    def step(evs=None):
+        for i, l in enumerate(layers):
+            if evs is not None:
+                evs[i].record(stream)
+            hq.hq_linear_fwd_bwd(l["X"], l["W"], l["dY"], k, fmt, Y=l["Y"], dX=l["dX"], dW=l["dW"],
+                                 workspace=l["ws"], stream=stream)
+        if evs is not None:
+            evs[-1].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -353,85 +356,154 @@ def run_gpu(args):
     torch.cuda.synchronize(device)
     if hq.hq_get_error(stream) != 0:
         raise SystemExit("device status error during warm-up")
+    # outputs of an untimed call, compared bit for bit with the timed steps' afterwards
+    ref_out = [tuple(l[n].clone() for n in ("Y", "dX", "dW")) for l in layers]
 
     # ---------------------------------------------------------------- timed region (device)
-    ev_main = [[ev() for _ in range(6)] for _ in range(args.steps)]
-    ev_side = [[ev() for _ in range(3)] for _ in range(args.steps)]
+    evs = [[ev() for _ in range(len(layers) + 1)] for _ in range(args.steps)]
     barrier(world, device)
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.zero_()  # L2 flush (256 MiB > 126 MB L2), outside the step's events
-            step(ev_main[i], ev_side[i])
+            step(evs[i])
         torch.cuda.synchronize(device)
     barrier(world, device)
     torch.cuda.synchronize(device)
     status = hq.hq_get_error(stream)
-    step_ms_local = sum(e[0].elapsed_time(e[5]) for e in ev_main) / args.steps
-    gemm_ms = sum(e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[5]) for e in ev_main)
-    quant_ms = sum(e[0].elapsed_time(e[1]) for e in ev_main) + sum(e[0].elapsed_time(e[2]) for e in ev_side)
-    def mean_ms(pairs):
-        return sum(a.elapsed_time(b) for a, b in pairs) / args.steps
-    phases = {
-        "main_quant_fwd_operands": mean_ms((e[0], e[1]) for e in ev_main),
-        "gemm_fwd": mean_ms((e[1], e[2]) for e in ev_main),
-        "wait_side_dy": mean_ms((e[2], e[3]) for e in ev_main),
-        "gemm_dx": mean_ms((e[3], e[4]) for e in ev_main),
-        "gemm_dw": mean_ms((e[4], e[5]) for e in ev_main),
-        "side_quant_dy_both_rotations": mean_ms((e[0], e[1]) for e in ev_side),
-        "side_quant_w_n_x_m": mean_ms((e[1], e[2]) for e in ev_side),
-    }
+    outputs_match = all(torch.equal(l[n].view(torch.int16), r.view(torch.int16))
+                        for l, rr in zip(layers, ref_out) for n, r in zip(("Y", "dX", "dW"), rr))
+    del ref_out
+    step_ms_local = sum(e[0].elapsed_time(e[-1]) for e in evs) / args.steps
+    layer_ms = {l["L"].name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+                for i, l in enumerate(layers)}
     step_ms = reduce_max(step_ms_local, world, device)
-    gemm_ms_launch = reduce_max(gemm_ms / (3 * args.steps), world, device)
-    quant_ms_step = reduce_max(quant_ms / args.steps, world, device)
-    launches = 13 * args.steps  # per step: 5 quantization calls x 2 kernels + 3 GEMMs
+    # our kernels per layer call: X and W in both rotations and dY in both (2 launches per
+    # rotation pass pair: 5 quantizations x 2) plus the three GEMMs
+    launches = 13 * len(layers) * args.steps
 
-    # ---------------------------------------------------------------- quantizer alone
-    # The three two-rotation quantizations one after another on one stream (nothing
-    # overlapping), L2 flushed before each, to report the quantization kernels' own throughput;
-    # and, for comparison, the six rotations as single-rotation calls (two reads each).
-    def alone(calls, fn, what):
-        tot = 0.0
-        for c in calls:
-            flush.zero_()
-            a, b = ev(), ev()
-            a.record(stream)
-            st = fn(*c)
-            if st:
-                raise hq.HQError(st, what)
-            b.record(stream)
+    # ---------------------------------------------------------------- kernels alone
+    # Every layer's X, W and dY quantized in both rotations by the fused two-rotation kernel
+    # (hq_quantize_dual), each call timed alone with L2 flushed before it; then the three GEMMs
+    # of every layer on those codes (hq_gemm_ws, the same kernels and split rule as the step),
+    # each launch timed alone.
+    reps = max(3, min(args.steps, 5))
+
+    quant = []
+    gemm = []
+    for l in layers:
+        L = l["L"]
+        codes = {}
+        for (nc, nr), src in ((("XK", "XM"), l["X"]), (("WK", "WN"), l["W"]), (("DN", "DM"), l["dY"])):
+            cc = torch.empty(src.shape[0], src.shape[1], dtype=torch.uint8, device=device)
+            cr = torch.empty(src.shape[1], src.shape[0], dtype=torch.uint8, device=device)
+            sc, sr = (torch.empty(1, dtype=torch.float32, device=device) for _ in range(2))
+            qws = torch.empty(hq.hq_quantize_dual_workspace_bytes(), dtype=torch.uint8, device=device)
+            fn = lambda: hq.hq_quantize_dual(src, k, fmt, codes_c=cc, scale_c=sc, codes_r=cr, scale_r=sr,  # noqa: E731
+                                             workspace=qws, stream=stream)
+            fn()
             torch.cuda.synchronize(device)
-            tot += a.elapsed_time(b)
-        return tot
+            ms = []
+            for _ in range(reps):
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                ms.append(a.elapsed_time(b))
+            t = statistics.median(ms)
+            nbytes = 2 * (2 + 1) * src.numel()  # two rotations: bf16 source + 1-byte codes each
+            quant.append({"layer": L.name, "tensor": nc[0] if nc[0] != "D" else "dY",
+                          "shape": list(src.shape), "us": 1e3 * t, "gbs": nbytes / (t * 1e-3) / 1e9})
+            codes[nc], codes[nr] = (cc, sc), (cr, sr)
+        for name, (a_, b_, o) in (("fwd", ("XK", "WK", l["Y"])), ("dX", ("DN", "WN", l["dX"])),
+                                  ("dW", ("DM", "XM", l["dW"]))):
+            (ca, sa), (cb, sb) = codes[a_], codes[b_]
+            Mg, Ng, Kg = ca.shape[0], cb.shape[0], ca.shape[1]
+            gws = torch.empty(max(16, hq.hq_gemm_workspace_bytes(Mg, Ng, Kg)), dtype=torch.uint8, device=device)
+            fn = lambda: hq.hq_gemm(ca, sa, cb, sb, fmt, out=o, workspace=gws, stream=stream)  # noqa: E731
+            fn()
+            ms = []
+            for _ in range(reps):
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                ms.append(a.elapsed_time(b))
+            t = statistics.median(ms)
+            gemm.append({"layer": L.name, "gemm": name, "M": Mg, "N": Ng, "K": Kg, "us": 1e3 * t,
+                         "tops": 2.0 * Mg * Ng * Kg / (t * 1e-3) / 1e12})
+        del codes
+    status |= hq.hq_get_error(stream)
+    gemm_ops = sum(2.0 * g["M"] * g["N"] * g["K"] for g in gemm)
+    gemm_ms = sum(g["us"] for g in gemm) * 1e-3
+    gemm_tops = reduce_max(gemm_ops / (gemm_ms * 1e-3) / 1e12, world, device)
+    quant_bytes = sum(2 * 3 * l[n].numel() for l in layers for n in ("X", "W", "dY"))
+    quant_ms = sum(q["us"] for q in quant) * 1e-3
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    top = max(gemm, key=lambda g: g["us"])
 
-    reps = max(3, min(args.steps, 10))
-    single = [(src.data_ptr(), hq.HQ_BF16, src.shape[0], src.shape[1], dim, k, fmt, codes.data_ptr(), sp(si),
-               ws_main, pq, sh)
-              for src, dim, codes, si in ((X, 1, qX_K, 0), (X, 0, qX_M, 1), (W, 1, qW_K, 2), (W, 0, qW_N, 3),
-                                          (dY, 1, qdY_N, 4), (dY, 0, qdY_M, 5))]
-    dual_calls = [dual(X, qX_K, 0, qX_M, 1, ws_main, sh), dual(W, qW_K, 2, qW_N, 3, ws_main, sh),
-                  dual(dY, qdY_N, 4, qdY_M, 5, ws_main, sh)]
-    alone_ms = sum(alone(dual_calls, L_.hq_quantize_dual, "hq_quantize_dual") for _ in range(reps))
-    alone_ms_step = reduce_max(alone_ms / reps, world, device)
-    single_ms = sum(alone(single, L_.hq_quantize, "hq_quantize") for _ in range(reps))
-    single_ms_step = reduce_max(single_ms / reps, world, device)
+    # pinned host copies of the inputs for the end-to-end leg below
+    hosts = []
+    for l in layers:
+        L = l["L"]
+        hosts.append(dict(X=l["X"].cpu().pin_memory(), W=l["W"].cpu().pin_memory(), dY=l["dY"].cpu().pin_memory(),
+                          Y=torch.empty(L.M, L.N, dtype=torch.bfloat16, pin_memory=True),
+                          dX=torch.empty(L.M, L.K, dtype=torch.bfloat16, pin_memory=True),
+                          dW=torch.empty(L.N, L.K, dtype=torch.bfloat16, pin_memory=True)))
+
+    # ---------------------------------------------------------------- one layer (extra key)
+    wl = synthetic.WORKLOADS[LAYER_WORKLOAD_ID]
+    Ll = wl.layers[0]
+    del layers
+    torch.cuda.empty_cache()
+    dl = synthetic.draw(wl, 0)
+    lX, lW, ldY = dev(dl["X"]), dev(dl["W"]), dev(dl["dY"])
+    lws = torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(Ll.M, Ll.K, Ll.N), dtype=torch.uint8, device=device)
+    lY = torch.empty(Ll.M, Ll.N, dtype=torch.bfloat16, device=device)
+    ldX = torch.empty(Ll.M, Ll.K, dtype=torch.bfloat16, device=device)
+    ldW = torch.empty(Ll.N, Ll.K, dtype=torch.bfloat16, device=device)
+    lfn = lambda: hq.hq_linear_fwd_bwd(lX, lW, ldY, wl.k, fmt, Y=lY, dX=ldX, dW=ldW, workspace=lws,  # noqa: E731
+                                       stream=stream)
+    lfn()
+    lms = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = ev(), ev()
+        a.record(stream)
+        lfn()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        lms.append(a.elapsed_time(b))
+    layer_step_ms = statistics.median(lms)
+    del lX, lW, ldY, lws, lY, ldX, ldW, dl
+    torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- end to end (host buffers)
-    # Every step copies X, W, dY from pinned host memory, runs hq_linear_fwd_bwd and copies Y,
-    # dX, dW back.  Steps are pipelined over two device buffer sets and three streams: the
-    # host->device copy of step i+1 and the device->host copy of step i-1 overlap step i's
-    # kernels (PCIe is full duplex).  Timed from the first copy in to the last copy out.
-    hX = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True).copy_(X)
-    hW = torch.empty(N, K, dtype=torch.bfloat16, pin_memory=True).copy_(W)
-    hdY = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True).copy_(dY)
-    hY = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
-    hdX = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
-    hdW = torch.empty(N, K, dtype=torch.bfloat16, pin_memory=True)
-    e2e_steps = max(2, min(args.steps, 10))
-    bufs = [(X, W, dY, Y, dX, dW)]
-    bufs.append(tuple(torch.empty_like(t) for t in bufs[0]))
+    # Every step copies every layer's X, W, dY from pinned host memory, runs hq_linear_fwd_bwd
+    # for each layer and copies every Y, dX, dW back.  Steps are pipelined over two device
+    # buffer sets and three streams: the host->device copies of step i+1 and the device->host
+    # copies of step i-1 overlap step i's kernels (PCIe is full duplex).  Timed from the first
+    # copy in to the last copy out.
+    e2e_steps = max(2, min(args.steps, 5))
+    bufs = [[], []]
+    for L in w.layers:
+        M, K, N = L.M, L.K, L.N
+        for b in bufs:
+            b.append(dict(X=torch.empty(M, K, dtype=torch.bfloat16, device=device),
+                          W=torch.empty(N, K, dtype=torch.bfloat16, device=device),
+                          dY=torch.empty(M, N, dtype=torch.bfloat16, device=device),
+                          Y=torch.empty(M, N, dtype=torch.bfloat16, device=device),
+                          dX=torch.empty(M, K, dtype=torch.bfloat16, device=device),
+                          dW=torch.empty(N, K, dtype=torch.bfloat16, device=device),
+                          ws=torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(M, K, N), dtype=torch.uint8,
+                                         device=device)))
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     s_cmp = stream
+    h2d = sum(2 * (L.M * L.K + L.N * L.K + L.M * L.N) for L in w.layers)
 
     def e2e_run(nsteps):
         ev_in = [torch.cuda.Event() for _ in range(nsteps)]
@@ -440,24 +512,26 @@ def run_gpu(args):
         t0, t1 = ev(), ev()
         t0.record(s_in)
         for i in range(nsteps):
-            bX, bW, bdY, bY, bdX, bdW = bufs[i % 2]
+            bset = bufs[i % 2]
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(ev_cmp[i - 2])  # step i-2 finished reading these inputs
-                bX.copy_(hX, non_blocking=True)
-                bW.copy_(hW, non_blocking=True)
-                bdY.copy_(hdY, non_blocking=True)
+                for h, b in zip(hosts, bset):
+                    for n in ("X", "W", "dY"):
+                        b[n].copy_(h[n], non_blocking=True)
                 ev_in[i].record(s_in)
             s_cmp.wait_event(ev_in[i])
             if i >= 2:
                 s_cmp.wait_event(ev_out[i - 2])  # step i-2's outputs are on the host
-            hq.hq_linear_fwd_bwd(bX, bW, bdY, k, fmt, Y=bY, dX=bdX, dW=bdW, workspace=lws, stream=s_cmp)
+            for b in bset:
+                hq.hq_linear_fwd_bwd(b["X"], b["W"], b["dY"], k, fmt, Y=b["Y"], dX=b["dX"], dW=b["dW"],
+                                     workspace=b["ws"], stream=s_cmp)
             ev_cmp[i].record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[i])
-                hY.copy_(bY, non_blocking=True)
-                hdX.copy_(bdX, non_blocking=True)
-                hdW.copy_(bdW, non_blocking=True)
+                for h, b in zip(hosts, bset):
+                    for n in ("Y", "dX", "dW"):
+                        h[n].copy_(b[n], non_blocking=True)
                 ev_out[i].record(s_out)
         s_cmp.wait_event(ev_out[nsteps - 1])
         s_cmp.wait_event(ev_in[nsteps - 1])
@@ -471,57 +545,63 @@ def run_gpu(args):
     status |= hq.hq_get_error(stream)
 
     # ---------------------------------------------------------------- report
-    ops = 6.0 * M * N * K
+    ops = block_ops(w)
     value = world * ops / (step_ms * 1e-3) / 1e12
-    peaks = load_peaks()
-    int8_peak = peaks["bf16"] * INT8_OVER_BF16
-    gemm_ops = 2.0 * M * N * K
-    gemm_tops = gemm_ops / (gemm_ms_launch * 1e-3) / 1e12
-    elem = 2  # bf16 source bytes
-    # each rotation: its bf16 source read once + its 1-byte codes written
-    quant_bytes = (elem + 1) * 2 * (M * K + N * K + M * N)
-    quant_gbs = quant_bytes / (quant_ms_step * 1e-3) / 1e9
-    traffic = recorded_traffic("gemm_pair_int8_llama_up_proj")
+    traffic = recorded_traffic(f"gemm_pair_int8_{top['M']}x{top['N']}x{top['K']}")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": f"{w.name}: M={M} K={K} N={N} k={k} {w.fmt} codes, bf16 inputs",
-                   "l2": "flushed between steps (256 MiB write, outside the step timing)",
+        "config": {"workload": f"{w.name}: Llama-2-7B block linears qkv 4096->12288, o 4096->4096, "
+                               f"gate/up 4096->11008, down 11008->4096 at {w.layers[0].M} tokens; "
+                               f"k={k} {w.fmt} codes, bf16 inputs",
+                   "l2": "flushed between steps (256 MiB write, outside the step timing); inputs exceed L2",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<int8,bf16 out> (tcgen05.mma.cta_group::2 kind::i8)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<int8,bf16 out> (tcgen05.mma.cta_group::2 kind::i8), "
+                                                  "the block's 15 GEMM launches each timed alone",
                      "achieved": gemm_tops, "peak": int8_peak, "unit": "TFLOP/s",
                      "frac": gemm_tops / int8_peak, "traffic": traffic,
-                     "peak_note": f"{peaks['src']} burst bf16 {peaks['bf16']} x {INT8_OVER_BF16} (nominal INT8/bf16 ratio; the timed region lasts tens of ms, clocks stay at max); ops = 2*M*N*K per launch"},
-        "fwht_quant": {"achieved_gbs": quant_bytes / (alone_ms_step * 1e-3) / 1e9, "peak_gbs": peaks["hbm"],
-                       "frac": quant_bytes / (alone_ms_step * 1e-3) / 1e9 / peaks["hbm"],
-                       "bytes_per_step": quant_bytes, "ms_per_step": alone_ms_step,
-                       "in_step_gbs": quant_gbs, "in_step_ms": quant_ms_step,
-                       "kernel": "fwhtq_dual_kernel (both rotations of X, W, dY from one read per pass)",
-                       "single_rotation_gbs": quant_bytes / (single_ms_step * 1e-3) / 1e9,
-                       "single_rotation_ms": single_ms_step,
-                       "note": "algorithmic bytes of the six rotations (bf16 source + 1-byte codes each); achieved: the three two-rotation quantizations timed alone with CUDA events, L2 flushed before each; in_step: summed event time of the same launches inside the overlapped step (sharing the GPU with the GEMMs); single_rotation: the six rotations as one-rotation calls"},
-        "phases_ms": phases,
-        "gemm_ms_per_step": gemm_ms_launch * 3,
-        "schedule": "X and W along K + forward GEMM on the main stream; dY in both rotations (one read per pass), W along N and X along M on a side stream overlapping them; the dX GEMM waits for W along N, the dW GEMM for X along M",
+                     "frac_of_nominal": gemm_tops / NOMINAL_INT8_TOPS,
+                     "peak_note": "measured in this run: hq_mma_peak INT8, tcgen05 kind::i8 CTA-pair MMAs with "
+                                  "operands in shared memory, best of ten ~1 ms runs (burst); ops = 2*M*N*K per "
+                                  f"launch; nominal {NOMINAL_INT8_TOPS:.0f} for context",
+                     "largest_launch": top},
+        "mma_peak_tops": {"int8_burst": mma["int8"], "int8_sustained": mma.get("int8_sustained"),
+                          "fp8_burst": mma["fp8"], "bf16_burst_measured_file": peaks_file["bf16"],
+                          "source": "hq_mma_peak in this run"},
+        "fwht_quant": {"achieved_gbs": quant_gbs, "peak_gbs": peaks_file["hbm"], "frac": quant_gbs / peaks_file["hbm"],
+                       "bytes_per_step": quant_bytes, "ms_per_step": quant_ms,
+                       "kernel": "fwhtq_dual_kernel (both rotations of one tensor from one read per pass)",
+                       "per_shape": quant,
+                       "note": "algorithmic bytes of the 30 rotations (bf16 source + 1-byte codes each) over the "
+                               "15 two-rotation calls' CUDA-event times, each call alone with L2 flushed before "
+                               f"it; HBM peak: {peaks_file['src']} copy bandwidth"},
+        "gemms": gemm,
+        "phases_ms": layer_ms,
+        "gemm_ms_per_step": gemm_ms,
         "frac_of_int8_peak_end_to_end": value / world / int8_peak,
+        "frac_of_nominal_end_to_end": value / world / NOMINAL_INT8_TOPS,
+        "outputs_match_untimed_call": bool(outputs_match),
+        "llama_up_proj_layer": {"workload": f"{wl.name}: M={Ll.M} K={Ll.K} N={Ll.N} k={wl.k} {wl.fmt}",
+                                "ms": layer_step_ms,
+                                "tops": 6.0 * Ll.M * Ll.N * Ll.K / (layer_step_ms * 1e-3) / 1e12},
         "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                "h2d_bytes_per_step": elem * (M * K + N * K + M * N),
-                "d2h_bytes_per_step": elem * (M * N + M * K + N * K),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
-                "note": "copies of step i+1 (in) and i-1 (out) overlap step i's kernels"},
+                "note": "hq_linear_fwd_bwd per layer with host buffers; copies of step i+1 (in) and i-1 (out) "
+                        "overlap step i's kernels"},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "device_status": int(status),
     }
     if rank == 0 and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, CPU_SAMPLE_TOKENS)
+        line["cpu_baseline"] = cpu_baseline(w, cpu_sample, CPU_SAMPLE_TOKENS)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-    return 0 if status == 0 else 1
+    return 0 if (status == 0 and outputs_match) else 1
 
 
 def run_sweep(args):
@@ -535,7 +615,7 @@ def run_sweep(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
-    int8_peak = peaks["bf16"] * INT8_OVER_BF16
+    int8_peak = measure_mma_peaks(hq, torch, sustained=False)["int8"]
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     L_ = hq.lib()
     reps = max(3, args.steps)
@@ -624,7 +704,7 @@ def run_reuse(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
-    int8_peak = peaks["bf16"] * INT8_OVER_BF16
+    int8_peak = measure_mma_peaks(hq, torch, sustained=False)["int8"]
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     reps = max(3, args.steps)
 

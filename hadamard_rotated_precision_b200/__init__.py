@@ -39,7 +39,7 @@ EXPORTS = ("hq_quantize_workspace_bytes", "hq_quantize", "hq_quantize_noalloc",
            "hq_linear_bwd_reuse_workspace_bytes", "hq_linear_bwd_reuse",
            "hq_gemm_rotout", "hq_quantize_prerotated_workspace_bytes", "hq_quantize_prerotated",
            "hq_gemm_workspace_bytes", "hq_gemm_ws",
-           "hq_get_error",
+           "hq_workspace_bytes", "hq_mma_peak", "hq_get_error",
            "hq_last_cuda_error", "hq_status_string", "hq_version")
 
 
@@ -127,6 +127,10 @@ def lib() -> ctypes.CDLL:
             f.restype = i32
         L.hq_selftest_gemm_timeout.argtypes = [p, p, p, i64, i64, i64, p]
         L.hq_selftest_gemm_timeout.restype = i32
+        L.hq_workspace_bytes.argtypes = [i64, i64, i64, i32]
+        L.hq_workspace_bytes.restype = sz
+        L.hq_mma_peak.argtypes = [i32, i64, p, p]
+        L.hq_mma_peak.restype = i32
         L.hq_get_error.argtypes = [p]
         L.hq_get_error.restype = i32
         L.hq_last_cuda_error.argtypes = []
@@ -370,6 +374,66 @@ def hq_fsdp_all_gather(w_shard, k: int, fmt, group=None, neg=None):
     full = torch.empty((world * codes.shape[0], codes.shape[1]), dtype=torch.uint8, device=codes.device)
     dist.all_gather_into_tensor(full, codes, group=group)
     return full, scale
+
+
+def fsdp_prefetch_schedule(n_layers: int, start_gather, wait_gather, compute):
+    """Order of a forward pass over a stack of linear layers whose weights are sharded over the
+    ranks and all-gathered as quantized codes (the quantized FSDP communication of HALO): the
+    gather of layer i + 1 is started before layer i computes, so the communication of the next
+    weight overlaps the current layer's GEMMs, and layer i computes only once its own gather
+    has completed.  start_gather(i) issues layer i's gather without waiting for it;
+    wait_gather(i) blocks (or orders the compute stream) until it is done and returns the
+    gathered weight; compute(i, gathered) runs the layer.  Returns the computes' results in
+    layer order.  The callbacks are arguments so the same order runs on CUDA streams with NCCL
+    (hq_fsdp_forward) and, in the CPU tests, with gloo."""
+    out = []
+    if n_layers <= 0:
+        return out
+    start_gather(0)
+    for i in range(n_layers):
+        g = wait_gather(i)
+        if i + 1 < n_layers:
+            start_gather(i + 1)
+        out.append(compute(i, g))
+    return out
+
+
+def hq_fsdp_forward(w_shards, xs, k: int, fmt, group=None, comm_stream=None):
+    """Forward GEMMs Y_i = Q(X_i H) Q(W_i H)^T of a stack of layers with quantized FSDP weights.
+    Rank r holds rows [r n_i, (r + 1) n_i) of every W_i [N_i][K_i] (w_shards[i]); xs[i] is
+    the layer's full input X_i [M][K_i] on this rank.  Each layer's weight is quantized shard by
+    shard with the whole tensor's scale and its 1-byte codes all-gathered (hq_fsdp_all_gather)
+    on `comm_stream` (a new CUDA stream by default), the gather of layer i + 1 overlapping the
+    quantization of X_i and the GEMM of layer i on the current stream (fsdp_prefetch_schedule).
+    Returns the bf16 outputs; each equals hq_linear_fwd(X_i, W_i) bit for bit."""
+    torch = _torch()
+    compute = torch.cuda.current_stream()
+    comm = comm_stream if comm_stream is not None else torch.cuda.Stream()
+    pending = {}
+
+    def start(i):
+        ready = torch.cuda.Event()
+        ready.record(compute)  # the shard as the compute stream left it
+        with torch.cuda.stream(comm):
+            comm.wait_event(ready)
+            codes, scale = hq_fsdp_all_gather(w_shards[i], k, fmt, group=group)
+            done = torch.cuda.Event()
+            done.record(comm)
+        codes.record_stream(compute)
+        scale.record_stream(compute)
+        pending[i] = (codes, scale, done)
+
+    def wait(i):
+        codes, scale, done = pending.pop(i)
+        compute.wait_event(done)
+        return codes, scale
+
+    def run(i, g):
+        wq, sw = g
+        xq, sx = hq_quantize(xs[i], 1, k, fmt)
+        return hq_gemm(xq, sx, wq, sw, fmt)
+
+    return fsdp_prefetch_schedule(len(w_shards), start, wait, run)
 
 
 def hq_quantize_dual_workspace_bytes() -> int:
@@ -714,6 +778,20 @@ def hq_linear_bwd_dw(dY, X, k: int, fmt, out=None, workspace=None, stream=None):
     M, N = dY.shape
     K = X.shape[1]
     return _linear("hq_linear_bwd_dw", dY, X, M, K, N, (N, K), k, fmt, out, workspace, stream)
+
+
+def hq_workspace_bytes(M: int, K: int, N: int, fmt) -> int:
+    """One workspace size for every layer-level call of the shape (any code format)."""
+    return int(lib().hq_workspace_bytes(M, K, N, _fmt(fmt)))
+
+
+def hq_mma_peak(fmt, n_blocks: int, stream=None) -> int:
+    """Launch the dense tensor-core throughput probe (n_blocks x 4 CTA-pair MMAs of 256 x 256 x 32
+    per pair, operands in shared memory) on `stream`; returns the number of CTA pairs.  The
+    caller times it: operations = pairs * n_blocks * 4 * 2 * 256 * 256 * 32."""
+    pairs = ctypes.c_int(0)
+    _check(lib().hq_mma_peak(_fmt(fmt), int(n_blocks), ctypes.byref(pairs), _stream_handle(stream)), "hq_mma_peak")
+    return int(pairs.value)
 
 
 def hq_get_error(stream=None) -> int:

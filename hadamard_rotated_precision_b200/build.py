@@ -11,7 +11,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhq.so")
 SOURCES = ["hq_api.cu"]
-DEPS = ["hq_api.cu", "fwht_quant.cuh", "fwht_dual.cuh", "gemm_tcgen05.cuh", "rotate_out.cuh", "prerot_quant.cuh", "sm100_ptx.cuh"]
+DEPS = ["hq_api.cu", "fwht_quant.cuh", "fwht_dual.cuh", "gemm_tcgen05.cuh", "rotate_out.cuh", "prerot_quant.cuh",
+        "mma_peak.cuh", "sm100_ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -22,6 +22,10 @@
 //   col role  (rotation along the rows): four ldmatrix.trans x4 gathers per 32 rows give a
 //             thread 64 consecutive rows of one column (bits 0..5 in registers, bits 6, 7 in
 //             lane bits 0, 1).
+// The absmax, INT8 and FP8 passes compute in the exchange layout of fwht_quant.cuh (xrotate:
+// packed f32x2 butterflies, the lane bits brought into registers by swapping half of the
+// registers with the partner lane, 32-byte code segments); the FP6 / FP4 code pass keeps
+// butterfly shuffles across lanes (rotate64) and packs its codes per 16-code group.
 // Pass 1 reduces both rotations' absmax into one partial per CTA and role; pass 2 reduces
 // the partials, rotates again and writes both code tensors.  HBM traffic per element and
 // pass is one 2-byte read (plus two 1-byte code writes in pass 2), against two reads when
@@ -74,18 +78,6 @@ __device__ __forceinline__ bool wait_full(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// max(m, fl(|a| + |b|), fl(|c| + |d|)), NaN-propagating.  For a butterfly pair (u, v) the two
-// outputs satisfy max(|fl(u + v)|, |fl(u - v)|) = fl(|u| + |v|) (one of them is the sum of the
-// magnitudes, the other the difference, and rounding is monotone and sign-symmetric), so the
-// absmax pass never forms the last stage's outputs.
-__device__ __forceinline__ float max_abs_sums(float m, float a, float b, float c, float d) {
-  return absmax3(m, __fadd_rn(fabsf(a), fabsf(b)), __fadd_rn(fabsf(c), fabsf(d)));
-}
-
-// Running maxima of the absmax pass: eight independent chains, so consecutive max
-// instructions do not wait on each other.
-constexpr int kAcc = 8;
-
 // Rotation of a thread's 64 values (v[i] = positions 2i, 2i+1 of bits 0..5) for block size K:
 // register stages for bits 0..min(log2 K, 6) - 1, then the lane stages (bit 6: lane xor m6,
 // bit 7: lane xor m7).  ABSMAX: the last stage is folded into the running maxima `am` of the
@@ -121,13 +113,6 @@ __device__ __forceinline__ void rotate64(float2 (&v)[32], int lane, int m6, int 
       stage_lanes<32>(v, ml, lane);
     }
   }
-}
-
-__device__ __forceinline__ void st_global_32B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
-                                              uint32_t f, uint32_t g, uint32_t h) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d),
-               "r"(e), "r"(f), "r"(g), "r"(h)
-               : "memory");
 }
 
 // Codes of a thread's 64 rotated values, 64 contiguous bytes at dst (W32: two 32-byte stores,
@@ -175,6 +160,7 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float2& f) {
   f = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+
 template <int K, int MODE, bool W32, bool SIGNED>
 __global__ void __launch_bounds__(kThreads, 1)
 fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
@@ -183,6 +169,10 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
                   float* __restrict__ scale_c, float* __restrict__ scale_r,
                   unsigned int* __restrict__ status, int reverse,
                   const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r, int lp_fmt) {
+  // programmatic dependent launch: nothing is read or written before the previous grid in the
+  // stream has completed; the next grid may be scheduled from here on
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   // SIGNED: sign flags per column (neg_c) and per row (neg_r); either may be null (all clear)
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
@@ -270,6 +260,21 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
   // i = lane & 7 (same swizzle), matrix mm = lane >> 3
   const int grp = warp >> 3;
   const uint32_t col_lane_off = (8u * (lane >> 3) + swr) * 128u + ((static_cast<uint32_t>(warp & 7) ^ swr) << 4);
+  // exchange layout (absmax, INT8, FP8 passes): chunk / gather swizzles and stage signs
+  constexpr bool XL = MODE != kModeLowp;
+  // row role: position bits 3, 4 of the loaded chunk XOR (A, B) = strip bits (k = 256), bit 4
+  // XOR A (k = 128)
+  const int row_sw = K == 256 ? sr : K == 128 ? 2 * (sr & 1) : 0;
+  // col role: the receiving thread's swizzle (its lane bits 0, 1), and that of the thread
+  // receiving the matrix row this lane addresses (row x of a matrix goes to lane bits x >> 1)
+  const int col_sw = K == 256 ? (lane & 3) : K == 128 ? 2 * (lane & 1) : 0;
+  const int col_sw_addr = K == 256 ? (x >> 1) : K == 128 ? 2 * ((x >> 1) & 1) : 0;
+  const float rgA = (sr & 1) ? -1.0f : 1.0f, rgB = (sr & 2) ? -1.0f : 1.0f;
+  const float cgA = (lane & 1) ? -1.0f : 1.0f, cgB = (lane & 2) ? -1.0f : 1.0f;
+  const float2 rsA = make_float2(rgA, rgA), rnsA = make_float2(-rgA, -rgA);
+  const float2 rsB = make_float2(rgB, rgB), rnsB = make_float2(-rgB, -rgB);
+  const float2 csA = make_float2(cgA, cgA), cnsA = make_float2(-cgA, -cgA);
+  const float2 csB = make_float2(cgB, cgB), cnsB = make_float2(-cgB, -cgB);
 
   for (int64_t i = 0; i < work_tiles; ++i) {
     const int64_t t = tile_of(i);
@@ -285,92 +290,191 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
     }
     if (!ok) break;
 
-    // ---- row role: rotation along the columns, kSteps steps of 8 rows x 256 columns per warp
-    const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+    if constexpr (XL) {
+      // ---- row role (exchange layout): a thread reads one strip row (64 columns) of its strip
+      // sr; position bits 6, 7 of the column are lane bits 3, 4 (A = bit 3, B = bit 4)
+      const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
 #pragma unroll 1
-    for (int st = 0; st < kSteps; ++st) {
-      const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
-      const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
-      // sign flags of the thread's 64 columns (the randomized variant; cols is a multiple of 64,
-      // so they are all inside the tensor or all past its end)
-      uint32_t sm[SIGNED ? 32 : 1];
-      if constexpr (SIGNED) {
-        const int64_t c0 = col0 + kStripCols * sr;
+      for (int st = 0; st < kSteps; ++st) {
+        const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
+        const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+        float2 v[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t m8[8];
-          sign_masks_bf16x16(neg_c != nullptr && c0 < cols ? __ldg(reinterpret_cast<const uint4*>(neg_c + c0 + 16 * c))
-                                                           : make_uint4(0u, 0u, 0u, 0u), m8);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t cq = static_cast<uint32_t>(q ^ row_sw);  // chunk of the x half; the y half's is 4 + cq
+          uint4 rx = ptx::ld_shared_v4(rowaddr + ((cq ^ swr) << 4));
+          uint4 ry = ptx::ld_shared_v4(rowaddr + (((4u + cq) ^ swr) << 4));
+          if constexpr (SIGNED) {
+            const int64_t c0 = col0 + kStripCols * sr + 8 * cq;
+            uint32_t mx[4], my[4];
+            const bool in = neg_c != nullptr && c0 < cols;
+            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0)) : make_uint2(0u, 0u), mx);
+            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0 + 32)) : make_uint2(0u, 0u), my);
+            rx.x ^= mx[0]; rx.y ^= mx[1]; rx.z ^= mx[2]; rx.w ^= mx[3];
+            ry.x ^= my[0]; ry.y ^= my[1]; ry.z ^= my[2]; ry.w ^= my[3];
+          }
+          const uint32_t wxq[4] = {rx.x, rx.y, rx.z, rx.w}, wyq[4] = {ry.x, ry.y, ry.z, ry.w};
+          xunpack(q, wxq, wyq, v);
+        }
+        if (kSteps == 2 && st == 1) {
+          release(q0 + 1 - grp);
+          release(q0 + 3 - grp);
+        }
+        xrotate<K, !QUANT>(v, rsA, rnsA, rsB, rnsB, 8, 16, amc);
+        if constexpr (QUANT) {
+          const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
+          if (!qc.abort) {  // uniform: every lane takes part in the code-word exchange
+            const bool row_in = r < rows;
+            uint32_t wx[8], wy[8];
+            xcodes<MODE>(v, csc, qc.zero, wx, wy);
+            // segment of half h: k <= 64 the thread's strip; k = 128 position bit 6 = A, bit 7 =
+            // the strip's bit 1; k = 256 bits 6, 7 = the strip
+            auto pos_of = [&](int h) -> int64_t {
+              if constexpr (K <= 64) return int64_t(kStripCols) * sr + 32 * h;
+              else if constexpr (K == 128) return 32 * h + 64 * (sr & 1) + 128 * (sr >> 1);
+              else return 32 * h + 64 * sr;
+            };
+            auto ok_pos = [&](int64_t pc) { return row_in && col0 + pc < cols; };
+            xstore<K>(codes_c + r * cols + col0, wx, wy, K == 256 ? sr : (sr & 1), 8, 16, pos_of, ok_pos, W32);
+          }
         }
       }
-      float2 v[32];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
-        if constexpr (SIGNED) {
-          raw.x ^= sm[(4 * j) % (SIGNED ? 32 : 1)];
-          raw.y ^= sm[(4 * j + 1) % (SIGNED ? 32 : 1)];
-          raw.z ^= sm[(4 * j + 2) % (SIGNED ? 32 : 1)];
-          raw.w ^= sm[(4 * j + 3) % (SIGNED ? 32 : 1)];
-        }
-        unpack_bf16x2(raw.x, v[4 * j]);
-        unpack_bf16x2(raw.y, v[4 * j + 1]);
-        unpack_bf16x2(raw.z, v[4 * j + 2]);
-        unpack_bf16x2(raw.w, v[4 * j + 3]);
-      }
-      if (kSteps == 2 && st == 1) {
-        // this warp's last reads of the two strips it has no column step on (with 16 warps a
-        // warp's column steps cover strips grp and grp + 2; with 8 warps all four)
-        release(q0 + 1 - grp);
-        release(q0 + 3 - grp);
-      }
-      if constexpr (!QUANT) {
-        rotate64<K, true>(v, lane, 8, 16, amc);
-      } else {
-        rotate64<K, false>(v, lane, 8, 16, amc);
-        const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
-        const int64_t cc = col0 + kStripCols * sr;
-        if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero, lp_fmt);
-      }
-    }
 
-    // ---- col role: rotation along the rows, 8 columns of one strip per step
+      // ---- col role (exchange layout): ldmatrix.trans gathers; a thread receives rows of one
+      // column whose position bits 6, 7 are its lane bits 0, 1 (A = bit 0, B = bit 1)
 #pragma unroll 1
-    for (int j2 = 0; j2 < kSteps; ++j2) {
-      const int s = grp + (kComputeWarps / 8) * j2;
-      const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
-      // sign flags of the thread's 64 rows (rows is a multiple of 64)
-      uint32_t sm[SIGNED ? 32 : 1];
-      if constexpr (SIGNED) {
-        const int64_t r0t = row0 + 64 * (lane & 3);
+      for (int j2 = 0; j2 < kSteps; ++j2) {
+        const int s = grp + (kComputeWarps / 8) * j2;
+        const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+        float2 v[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t m8[8];
-          sign_masks_bf16x16(neg_r != nullptr && r0t < rows ? __ldg(reinterpret_cast<const uint4*>(neg_r + r0t + 16 * c))
-                                                            : make_uint4(0u, 0u, 0u, 0u), m8);
+        for (int q = 0; q < 4; ++q) {
+          // gather q of the x half reads call (q ^ sw) of 32 rows, the y half call 4 + (q ^ sw);
+          // the swizzle is that of the thread receiving the row this lane addresses
+          uint32_t rx[4], ry[4];
+          ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(q ^ col_sw_addr), rx);
+          ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(4 + (q ^ col_sw_addr)), ry);
+          if constexpr (SIGNED) {
+            const int64_t r0t = row0 + 64 * (lane & 3) + 8 * (q ^ col_sw);
+            uint32_t mx[4], my[4];
+            const bool in = neg_r != nullptr && r0t < rows;
+            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t)) : make_uint2(0u, 0u), mx);
+            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t + 32)) : make_uint2(0u, 0u), my);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+            for (int mm = 0; mm < 4; ++mm) {
+              rx[mm] ^= mx[mm];
+              ry[mm] ^= my[mm];
+            }
+          }
+          xunpack(q, rx, ry, v);
+        }
+        release(q0 + s);
+        xrotate<K, !QUANT>(v, csA, cnsA, csB, cnsB, 1, 2, amr);
+        if constexpr (QUANT) {
+          const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
+          if (!qr.abort) {  // uniform: every lane takes part in the code-word exchange
+            const bool col_in = gc < cols;
+            uint32_t wx[8], wy[8];
+            xcodes<MODE>(v, csr, qr.zero, wx, wy);
+            const int a = lane & 3;
+            auto pos_of = [&](int h) -> int64_t {
+              if constexpr (K <= 64) return 64 * a + 32 * h;
+              else if constexpr (K == 128) return 32 * h + 64 * (a & 1) + 128 * (a >> 1);
+              else return 32 * h + 64 * a;
+            };
+            auto ok_pos = [&](int64_t pr) { return col_in && row0 + pr < rows; };
+            xstore<K>(codes_r + gc * rows + row0, wx, wy, K == 256 ? a : (a & 1), 1, 2, pos_of, ok_pos, W32);
+          }
         }
       }
-      float2 v[32];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        uint32_t r4[4];
-        ldmatrix_x4_trans(lbase + 4096u * n, r4);
-#pragma unroll
-        for (int mm = 0; mm < 4; ++mm)
-          unpack_bf16x2(SIGNED ? r4[mm] ^ sm[(4 * n + mm) % (SIGNED ? 32 : 1)] : r4[mm], v[4 * n + mm]);
+    } else {
+      // ---- row role: rotation along the columns, kSteps steps of 8 rows x 256 columns per warp
+      const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+  #pragma unroll 1
+      for (int st = 0; st < kSteps; ++st) {
+        const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
+        const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+        // sign flags of the thread's 64 columns (the randomized variant; cols is a multiple of 64,
+        // so they are all inside the tensor or all past its end)
+        uint32_t sm[SIGNED ? 32 : 1];
+        if constexpr (SIGNED) {
+          const int64_t c0 = col0 + kStripCols * sr;
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t m8[8];
+            sign_masks_bf16x16(neg_c != nullptr && c0 < cols ? __ldg(reinterpret_cast<const uint4*>(neg_c + c0 + 16 * c))
+                                                             : make_uint4(0u, 0u, 0u, 0u), m8);
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+          }
+        }
+        float2 v[32];
+  #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+          if constexpr (SIGNED) {
+            raw.x ^= sm[(4 * j) % (SIGNED ? 32 : 1)];
+            raw.y ^= sm[(4 * j + 1) % (SIGNED ? 32 : 1)];
+            raw.z ^= sm[(4 * j + 2) % (SIGNED ? 32 : 1)];
+            raw.w ^= sm[(4 * j + 3) % (SIGNED ? 32 : 1)];
+          }
+          unpack_bf16x2(raw.x, v[4 * j]);
+          unpack_bf16x2(raw.y, v[4 * j + 1]);
+          unpack_bf16x2(raw.z, v[4 * j + 2]);
+          unpack_bf16x2(raw.w, v[4 * j + 3]);
+        }
+        if (kSteps == 2 && st == 1) {
+          // this warp's last reads of the two strips it has no column step on (with 16 warps a
+          // warp's column steps cover strips grp and grp + 2; with 8 warps all four)
+          release(q0 + 1 - grp);
+          release(q0 + 3 - grp);
+        }
+        if constexpr (!QUANT) {
+          rotate64<K, true>(v, lane, 8, 16, amc);
+        } else {
+          rotate64<K, false>(v, lane, 8, 16, amc);
+          const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
+          const int64_t cc = col0 + kStripCols * sr;
+          if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero, lp_fmt);
+        }
       }
-      release(q0 + s);
-      if constexpr (!QUANT) {
-        rotate64<K, true>(v, lane, 1, 2, amr);
-      } else {
-        rotate64<K, false>(v, lane, 1, 2, amr);
-        const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
-        const int64_t gr = row0 + 64 * (lane & 3);
-        if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero, lp_fmt);
+
+      // ---- col role: rotation along the rows, 8 columns of one strip per step
+  #pragma unroll 1
+      for (int j2 = 0; j2 < kSteps; ++j2) {
+        const int s = grp + (kComputeWarps / 8) * j2;
+        const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+        // sign flags of the thread's 64 rows (rows is a multiple of 64)
+        uint32_t sm[SIGNED ? 32 : 1];
+        if constexpr (SIGNED) {
+          const int64_t r0t = row0 + 64 * (lane & 3);
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t m8[8];
+            sign_masks_bf16x16(neg_r != nullptr && r0t < rows ? __ldg(reinterpret_cast<const uint4*>(neg_r + r0t + 16 * c))
+                                                              : make_uint4(0u, 0u, 0u, 0u), m8);
+  #pragma unroll
+            for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+          }
+        }
+        float2 v[32];
+  #pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          uint32_t r4[4];
+          ldmatrix_x4_trans(lbase + 4096u * n, r4);
+  #pragma unroll
+          for (int mm = 0; mm < 4; ++mm)
+            unpack_bf16x2(SIGNED ? r4[mm] ^ sm[(4 * n + mm) % (SIGNED ? 32 : 1)] : r4[mm], v[4 * n + mm]);
+        }
+        release(q0 + s);
+        if constexpr (!QUANT) {
+          rotate64<K, true>(v, lane, 1, 2, amr);
+        } else {
+          rotate64<K, false>(v, lane, 1, 2, amr);
+          const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
+          const int64_t gr = row0 + 64 * (lane & 3);
+          if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero, lp_fmt);
+        }
       }
     }
   }

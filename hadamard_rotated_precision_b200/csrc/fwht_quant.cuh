@@ -17,15 +17,18 @@
 //   pass 1 rotates and reduces the absmax into one partial per CTA, pass 2 reduces the
 //   partials, rotates again and writes the 1-byte codes.  Consecutive passes over the same
 //   tensor walk it in opposite directions so each starts on what the previous left in L2.
-//   * along the contiguous dimension (dim = 1): each thread owns 8 consecutive elements
-//     (one 16-byte bf16 load or two fp32 loads), bits 0-2 of the in-block index live in
-//     registers, bits 3.. across lanes (warp shuffles); 8 code bytes per thread, 256
-//     contiguous bytes per warp.
-//   * along the strided dimension (dim = 0): a CTA stages a 256-row x 128-byte tile in
-//     shared memory (16-byte chunks XOR-swizzled by row group so the column gather is
-//     conflict-free), each thread then owns 8 consecutive rows of 8 (bf16) or 4 (fp32)
-//     columns; the codes are written transposed (rotated dimension innermost), 256
-//     contiguous bytes per warp per column.
+//   * along the contiguous dimension (dim = 1, fwhtq_rows_kernel): each thread owns 32
+//     consecutive elements (one warp step = 1024 elements), so in-block index bits 0..4 are
+//     register bits; for k >= 64 the warp swaps its values through a 4 KB shared-memory slice
+//     so that the remaining stages run in registers too (no shuffles); 32 code bytes per
+//     thread.
+//   * along the strided dimension (dim = 0, fwhtq_cols_bf16_kernel for bf16): a CTA stages
+//     256-row x 64-column tiles in shared memory (cp.async, 3-tile ring); ldmatrix.trans gives
+//     each thread 64 rows of one column.  The absmax, INT8 and FP8 passes use the exchange
+//     layout (xrotate): position bits 6, 7 start in lane bits and are brought into registers by
+//     swapping half of the registers with the partner lane; the codes are written transposed
+//     (rotated dimension innermost) in 32-byte segments.
+//     fp32 sources use a simpler shared-memory tile kernel (fwhtq_cols_f32_kernel).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -449,6 +452,10 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
                   float* __restrict__ partials, int n_partials, float* __restrict__ scale_out,
                   unsigned int* __restrict__ status, int reverse, const uint8_t* __restrict__ neg,
                   int64_t cols, int lp_fmt) {
+  // programmatic dependent launch: nothing is read or written before the previous grid in the
+  // stream has completed; the next grid may be scheduled from here on
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   constexpr bool EXCH = K >= 64;
@@ -594,6 +601,307 @@ fwhtq_rows_kernel(const SrcT* __restrict__ src, int64_t n, uint8_t* __restrict__
   if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
 }
 
+// max(m, fl(|a| + |b|), fl(|c| + |d|)), NaN-propagating.  For a butterfly pair (u, v) the two
+// outputs satisfy max(|fl(u + v)|, |fl(u - v)|) = fl(|u| + |v|) (one of them is the sum of the
+// magnitudes, the other the difference, and rounding is monotone and sign-symmetric), so the
+// absmax pass never forms the last stage's outputs.
+__device__ __forceinline__ float max_abs_sums(float m, float a, float b, float c, float d) {
+  return absmax3(m, __fadd_rn(fabsf(a), fabsf(b)), __fadd_rn(fabsf(c), fabsf(d)));
+}
+
+// Running maxima of the absmax pass: eight independent chains, so consecutive max
+// instructions do not wait on each other.
+constexpr int kAcc = 8;
+
+__device__ __forceinline__ void st_global_32B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                              uint32_t f, uint32_t g, uint32_t h) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d),
+               "r"(e), "r"(f), "r"(g), "r"(h)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ exchange layout
+//
+// The absmax, INT8 and FP8 passes hold a thread's 64 values of one k-block slice as v[j].x =
+// in-block position j and v[j].y = position j + 32 (j = position bits 0..4, the float2 half =
+// bit 5), so every butterfly stage except the one on bit 5 pairs two different float2
+// registers and runs as packed f32x2 operations.  For k = 128 / 256 the position bits 6 / 6, 7
+// start in lane bits; they are brought into registers by exchanging half of the registers with
+// the partner lane (one shuffle per two values instead of one per value):
+//   before the exchange, register bit r holds position bit Q and lane bit l holds bit P; lane
+//   l-value b keeps the registers with r-bit 0 and swaps those with r-bit 1 for the partner's.
+//   Afterwards the lane bit holds Q and the register bit holds P.  For this to need no selects,
+//   register bit r is stored "swizzled", holding Q XOR b before and P XOR b after the exchange
+//   (the loads place the data so, from lane-dependent shared-memory addresses).
+// A butterfly stage on a swizzled register bit pairs R0 (r-bit 0) and R1: with b = 0 they hold
+// positions 0 and 1 of the pair, with b = 1 positions 1 and 0, so R0' = fma(s, R0, R1) and
+// R1' = fma(-s, R1, R0) with s = +1 (b = 0) or -1 (b = 1) give u + v and u - v at the right
+// places.  Each is one fp32 rounding of the exact sum or difference: bit-identical to the plain
+// stage.
+// Exchanged bits: k = 256: register bit 3 (position 3) with the lane bit of position 6 ("A"),
+// register bit 4 (position 4) with the lane bit of position 7 ("B"); k = 128: register bit 4
+// with lane bit A.  Afterwards a thread holds 8 (k = 256) or 16 (k = 128) consecutive
+// positions per group of registers, and 4 / 2 lanes together hold 32 consecutive code bytes.
+
+// Plain stage on register bit log2(H): pairs (v[i], v[i + H]).
+template <int H>
+__device__ __forceinline__ void xstage(float2 (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i & H) continue;
+    const float2 a = v[i], b = v[i + H];
+    v[i] = add2(a, b);
+    v[i + H] = sub2(a, b);
+  }
+}
+
+// Stage on a swizzled register bit (s2 = (s, s), ns2 = (-s, -s)).
+template <int H>
+__device__ __forceinline__ void xstage_sw(float2 (&v)[32], float2 s2, float2 ns2) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i & H) continue;
+    const float2 a = v[i], b = v[i + H];
+    v[i] = __ffma2_rn(s2, a, b);
+    v[i + H] = __ffma2_rn(ns2, b, a);
+  }
+}
+
+// Stage on position bit 5 (the two halves of every float2).
+__device__ __forceinline__ void xstage_halves(float2 (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float a = v[i].x, b = v[i].y;
+    v[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+}
+
+// Registers with bit log2(H) set are swapped with lane ^ m's.
+template <int H>
+__device__ __forceinline__ void xexchange(float2 (&v)[32], int m) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (!(i & H)) continue;
+    v[i].x = __shfl_xor_sync(0xFFFFFFFFu, v[i].x, m);
+    v[i].y = __shfl_xor_sync(0xFFFFFFFFu, v[i].y, m);
+  }
+}
+
+// Last stage folded into the running maxima (see max_abs_sums): pairs on register bit log2(H),
+// or the two halves of every float2.
+template <int H>
+__device__ __forceinline__ void xfold(const float2 (&v)[32], float (&am)[kAcc]) {
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i & H) continue;
+    am[n % kAcc] = max_abs_sums(am[n % kAcc], v[i].x, v[i + H].x, v[i].y, v[i + H].y);
+    ++n;
+  }
+}
+__device__ __forceinline__ void xfold_halves(const float2 (&v)[32], float (&am)[kAcc]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2)
+    am[(i / 2) % kAcc] = max_abs_sums(am[(i / 2) % kAcc], v[i].x, v[i].y, v[i + 1].x, v[i + 1].y);
+}
+
+// Whole rotation of a thread's values in the exchange layout (stages in position-bit order
+// 0, 1, ..., log2 K - 1).  ABSMAX: the last stage is folded into `am` instead.
+template <int K, bool ABSMAX>
+__device__ __forceinline__ void xrotate(float2 (&v)[32], float2 sA, float2 nsA, float2 sB, float2 nsB, int mA, int mB,
+                                        float (&am)[kAcc]) {
+  xstage<1>(v);
+  xstage<2>(v);
+  if constexpr (K == 16) {
+    xstage<4>(v);
+    if constexpr (ABSMAX) xfold<8>(v, am); else xstage<8>(v);
+  } else if constexpr (K == 32) {
+    xstage<4>(v);
+    xstage<8>(v);
+    if constexpr (ABSMAX) xfold<16>(v, am); else xstage<16>(v);
+  } else if constexpr (K == 64) {
+    xstage<4>(v);
+    xstage<8>(v);
+    xstage<16>(v);
+    if constexpr (ABSMAX) xfold_halves(v, am); else xstage_halves(v);
+  } else if constexpr (K == 128) {
+    xstage<4>(v);
+    xstage<8>(v);
+    xstage_sw<16>(v, sA, nsA);
+    xstage_halves(v);
+    xexchange<16>(v, mA);
+    if constexpr (ABSMAX) xfold<16>(v, am); else xstage_sw<16>(v, sA, nsA);
+  } else {
+    xstage<4>(v);
+    xstage_sw<8>(v, sA, nsA);
+    xstage_sw<16>(v, sB, nsB);
+    xstage_halves(v);
+    xexchange<8>(v, mA);
+    xstage_sw<8>(v, sA, nsA);
+    xexchange<16>(v, mB);
+    if constexpr (ABSMAX) xfold<16>(v, am); else xstage_sw<16>(v, sB, nsB);
+  }
+}
+
+// Code words of a thread's rotated values: wx[q] = codes of positions 4q .. 4q + 3 (the .x
+// halves of v[4q .. 4q + 3]), wy[q] the same for the .y halves, little-endian.
+template <int MODE>
+__device__ __forceinline__ void xcodes(const float2 (&v)[32], const CodeScale& cs, bool zero, uint32_t (&wx)[8],
+                                       uint32_t (&wy)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float2 z[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      z[i] = cs.one_mul ? mul2(v[4 * q + i], cs.ci2) : mul2(mul2(v[4 * q + i], cs.c2), cs.inv2);
+    if constexpr (MODE == kModeInt8) {
+      // z + 1.5 * 2^23: the low byte is rne(z) in two's complement (see codes4).  The add is
+      // the scalar __fadd_rn: with a packed add the compiler fused it with the packed multiply
+      // into one fused multiply-add, which rounds y * inv only once (a product 74.50000000019
+      // whose fp32 rounding is the tie 74.5 then gave 75 instead of the even 74).
+      constexpr float mg = 12582912.0f;
+      uint32_t bx[4], by[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        bx[i] = __float_as_uint(__fadd_rn(z[i].x, mg));
+        by[i] = __float_as_uint(__fadd_rn(z[i].y, mg));
+      }
+      wx[q] = __byte_perm(__byte_perm(bx[0], bx[1], 0x0040), __byte_perm(bx[2], bx[3], 0x0040), 0x5410);
+      wy[q] = __byte_perm(__byte_perm(by[0], by[1], 0x0040), __byte_perm(by[2], by[3], 0x0040), 0x5410);
+    } else {
+      const uint32_t x01 = __nv_cvt_float2_to_fp8x2(make_float2(z[0].x, z[1].x), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t x23 = __nv_cvt_float2_to_fp8x2(make_float2(z[2].x, z[3].x), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t y01 = __nv_cvt_float2_to_fp8x2(make_float2(z[0].y, z[1].y), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t y23 = __nv_cvt_float2_to_fp8x2(make_float2(z[2].y, z[3].y), __NV_SATFINITE, __NV_E4M3);
+      wx[q] = x01 | (x23 << 16);
+      wy[q] = y01 | (y23 << 16);
+    }
+    if (zero) wx[q] = wy[q] = 0u;
+  }
+}
+
+__device__ __forceinline__ void st_global_8B(void* p, uint32_t a, uint32_t b) {
+  asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void st_global_16B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Stores of a thread's code words.  k <= 64: the thread's 64 codes are consecutive (x half,
+// then y half) at pos0 relative to `base`.  k = 128 / 256: groups of 16 / 8 consecutive codes
+// whose 32-byte segments are shared by the 2 / 4 lanes of the exchanged lane bits (A, B; p =
+// the thread's value of them).  Those lanes first swap code words so that each ends with whole
+// segments: register group g of lane p holds segment pieces of segment pair g ^ p (the swizzle),
+// so in round r every lane sends its group r to lane p ^ r and receives pieces of its own
+// segment pair p; the pieces are then put in address order (piece q comes from lane q, i.e.
+// from round q ^ p) with two layers of selects.  Each lane then writes its segment pair
+// (position bits 6, 7 = p; 5 = the half) as two 32-byte stores.  pos_of(h) gives the in-tile
+// position of the thread's segment for half h; ok(pos) whether it lies inside the tensor.
+__device__ __forceinline__ uint32_t sel(bool c, uint32_t a, uint32_t b) { return c ? a : b; }
+
+// One 32-byte segment: a single 32-byte store when the address is 32-byte aligned (w32), else
+// two 16-byte stores.
+__device__ __forceinline__ void store_seg32(uint8_t* d, const uint32_t (&w)[8], bool w32) {
+  if (w32) {
+    st_global_32B(d, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+  } else {
+    st_global_16B(d, w[0], w[1], w[2], w[3]);
+    st_global_16B(d + 16, w[4], w[5], w[6], w[7]);
+  }
+}
+
+template <int K, class Pos, class Ok>
+__device__ __forceinline__ void xstore(uint8_t* base, const uint32_t (&wx)[8], const uint32_t (&wy)[8], int p, int mA,
+                                       int mB, Pos pos_of, Ok ok, bool w32) {
+  uint32_t o[2][8];
+  if constexpr (K <= 64) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o[0][i] = wx[i];
+      o[1][i] = wy[i];
+    }
+  } else if constexpr (K == 128) {
+    // groups g = 0, 1 (4 words per half); round 1 swaps group 1 with lane ^ mA
+    uint32_t s0[8], s1[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      s0[i] = wx[i];
+      s0[4 + i] = wy[i];
+      s1[i] = __shfl_xor_sync(0xFFFFFFFFu, wx[4 + i], mA);
+      s1[4 + i] = __shfl_xor_sync(0xFFFFFFFFu, wy[4 + i], mA);
+    }
+    const bool sw = p & 1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[0][i] = sel(sw, s1[i], s0[i]);
+      o[0][4 + i] = sel(sw, s0[i], s1[i]);
+      o[1][i] = sel(sw, s1[4 + i], s0[4 + i]);
+      o[1][4 + i] = sel(sw, s0[4 + i], s1[4 + i]);
+    }
+  } else {
+    // groups g = 0..3 (2 words per half); round r swaps group r with lane ^ (A if r & 1, B if r & 2)
+    uint32_t sl[4][4];  // slot: x word 0, x word 1, y word 0, y word 1
+    sl[0][0] = wx[0]; sl[0][1] = wx[1]; sl[0][2] = wy[0]; sl[0][3] = wy[1];
+#pragma unroll
+    for (int r = 1; r < 4; ++r) {
+      const int m = ((r & 1) ? mA : 0) | ((r & 2) ? mB : 0);
+      sl[r][0] = __shfl_xor_sync(0xFFFFFFFFu, wx[2 * r], m);
+      sl[r][1] = __shfl_xor_sync(0xFFFFFFFFu, wx[2 * r + 1], m);
+      sl[r][2] = __shfl_xor_sync(0xFFFFFFFFu, wy[2 * r], m);
+      sl[r][3] = __shfl_xor_sync(0xFFFFFFFFu, wy[2 * r + 1], m);
+    }
+    // piece q of the segment = slot q ^ p: swap by bit 0 of p, then by bit 1
+    const bool b0 = p & 1, b1 = p & 2;
+    uint32_t t[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      t[0][i] = sel(b0, sl[1][i], sl[0][i]);
+      t[1][i] = sel(b0, sl[0][i], sl[1][i]);
+      t[2][i] = sel(b0, sl[3][i], sl[2][i]);
+      t[3][i] = sel(b0, sl[2][i], sl[3][i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sl[0][i] = sel(b1, t[2][i], t[0][i]);
+      sl[1][i] = sel(b1, t[3][i], t[1][i]);
+      sl[2][i] = sel(b1, t[0][i], t[2][i]);
+      sl[3][i] = sel(b1, t[1][i], t[3][i]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      o[0][2 * q] = sl[q][0];
+      o[0][2 * q + 1] = sl[q][1];
+      o[1][2 * q] = sl[q][2];
+      o[1][2 * q + 1] = sl[q][3];
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t ps = pos_of(h);
+    if (ok(ps)) store_seg32(base + ps, o[h], w32);
+  }
+}
+
+// Sign masks of 8 consecutive bf16 positions (4 bf16x2 words) from their 8 flag bytes.
+__device__ __forceinline__ void sign_masks_bf16x8(uint2 f, uint32_t (&m)[4]) {
+  const uint32_t w[2] = {f.x & 0x01010101u, f.y & 0x01010101u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    m[2 * i] = __byte_perm(w[i], 0u, 0x1404) << 7;
+    m[2 * i + 1] = __byte_perm(w[i], 0u, 0x3424) << 7;
+  }
+}
+
+// v[8q + 2i], v[8q + 2i + 1] from words i of chunk q: .x from the chunk's x-half words, .y from
+// its y-half words.
+__device__ __forceinline__ void xunpack(int q, const uint32_t (&wxq)[4], const uint32_t (&wyq)[4], float2 (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[8 * q + 2 * i] = make_float2(__uint_as_float(wxq[i] << 16), __uint_as_float(wyq[i] << 16));
+    v[8 * q + 2 * i + 1] = make_float2(__uint_as_float(wxq[i] & 0xFFFF0000u), __uint_as_float(wyq[i] & 0xFFFF0000u));
+  }
+}
+
 // ------------------------------------------------------------------ dim = 0, bf16 source
 
 // A CTA tile is 256 rows x 64 bf16 columns (32 KB); a 3-tile ring in shared memory is filled
@@ -629,6 +937,10 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
                        uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
                        float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
                        const uint8_t* __restrict__ neg, int lp_fmt) {
+  // programmatic dependent launch: nothing is read or written before the previous grid in the
+  // stream has completed; the next grid may be scheduled from here on
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   constexpr bool QUANT = MODE != kModeAbsmax;
   extern __shared__ __align__(128) uint4 tiles[];  // [3][256 rows][8 chunks]
@@ -647,6 +959,12 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
   const int64_t n_ct = (cols + kColsTileCols2 - 1) / kColsTileCols2;
   const int64_t n_tiles = n_rt * n_ct;
   float amax = 0.0f;
+  float am[kAcc];  // exchange layout: independent running maxima of the unnormalised |t|
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) am[j] = 0.0f;
+  // 32-byte code stores when every segment address is 32-byte aligned (k >= 128: rows is a
+  // multiple of 128)
+  const bool w32 = (reinterpret_cast<uintptr_t>(codes) & 31u) == 0;
 
   // load a tile: thread T copies 16-byte chunk (T & 7) of rows (T >> 3) + 32 j
   auto issue = [&](int buf, int64_t t) {
@@ -684,6 +1002,76 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
         cp_async_wait<0>();
       }
       __syncthreads();
+      if constexpr (MODE != kModeLowp) {
+        // exchange layout (see xrotate): a thread receives rows of column 8 warp + lane / 4
+        // whose position bits 6, 7 are its lane bits 0, 1; gather q of the x half reads 8-row
+        // group (q ^ sw) of each 64-row quarter, the y half group 4 + (q ^ sw), with the swizzle
+        // sw of the thread receiving the row this lane addresses (matrix row lane & 7 goes to
+        // lane bits (lane & 7) >> 1)
+        const int m = lane >> 3, qr = lane & 7;
+        const int sw_addr = K == 256 ? (qr >> 1) : K == 128 ? 2 * ((qr >> 1) & 1) : 0;
+        const int a = lane & 3;
+        const int sw_own = K == 256 ? a : K == 128 ? 2 * (a & 1) : 0;
+        float2 v[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t rx[4], ry[4];
+          const int kx = q ^ sw_addr, ky = 4 + (q ^ sw_addr);
+          const int rhox = (qr & 1) + 2 * m + 8 * kx + 64 * (qr >> 1);
+          const int rhoy = (qr & 1) + 2 * m + 8 * ky + 64 * (qr >> 1);
+          ldmatrix_x4_trans(ptx::smem_u32(&tiles[(buf * kColsTileRows2 + rhox) * 8 + (warp ^ cols_swz(rhox))]), rx);
+          ldmatrix_x4_trans(ptx::smem_u32(&tiles[(buf * kColsTileRows2 + rhoy) * 8 + (warp ^ cols_swz(rhoy))]), ry);
+          if constexpr (SIGNED) {
+            // flags of the thread's own rows: 8-row group (q ^ sw_own) and the one 32 rows on
+            // (16-row chunks are wholly inside or outside: rows is a multiple of 16)
+            const int64_t r0t = (t / n_ct) * kColsTileRows2 + 64 * a + 8 * (q ^ sw_own);
+            uint32_t mx[4], my[4];
+            sign_masks_bf16x8(r0t < rows ? __ldg(reinterpret_cast<const uint2*>(neg + r0t)) : make_uint2(0u, 0u), mx);
+            sign_masks_bf16x8(r0t + 32 < rows ? __ldg(reinterpret_cast<const uint2*>(neg + r0t + 32)) : make_uint2(0u, 0u),
+                              my);
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+              rx[mm] ^= mx[mm];
+              ry[mm] ^= my[mm];
+            }
+          }
+          xunpack(q, rx, ry, v);
+        }
+        __syncthreads();  // buffer free before the copies issued next iteration reuse it
+        const float gA = (lane & 1) ? -1.0f : 1.0f, gB = (lane & 2) ? -1.0f : 1.0f;
+        const float2 sA = make_float2(gA, gA), nsA = make_float2(-gA, -gA);
+        const float2 sB = make_float2(gB, gB), nsB = make_float2(-gB, -gB);
+        xrotate<K, !QUANT>(v, sA, nsA, sB, nsB, 1, 2, am);
+        if constexpr (QUANT) {
+          if (!qp.abort) {  // uniform: every lane takes part in the code-word exchange
+            const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+            const int64_t col = c0 + 8 * warp + (lane >> 2);
+            uint32_t wx[8], wy[8];
+            xcodes<MODE>(v, cs, qp.zero, wx, wy);
+            uint8_t* o = codes + col * rows + r0;
+            if constexpr (K <= 64) {
+              // the thread's 64 consecutive rows, stored per 16 rows (rows is a multiple of 16)
+              const int64_t rb = 64 * a;
+              if (col < cols) {
+                if (r0 + rb < rows) st_global_16B(o + rb, wx[0], wx[1], wx[2], wx[3]);
+                if (r0 + rb + 16 < rows) st_global_16B(o + rb + 16, wx[4], wx[5], wx[6], wx[7]);
+                if (r0 + rb + 32 < rows) st_global_16B(o + rb + 32, wy[0], wy[1], wy[2], wy[3]);
+                if (r0 + rb + 48 < rows) st_global_16B(o + rb + 48, wy[4], wy[5], wy[6], wy[7]);
+              }
+            } else {
+              const bool col_in = col < cols;
+              auto pos_of = [&](int h) -> int64_t {
+                if constexpr (K == 128) return 32 * h + 64 * (a & 1) + 128 * (a >> 1);
+                else return 32 * h + 64 * a;
+              };
+              auto ok_pos = [&](int64_t pr) { return col_in && r0 + pr < rows; };
+              xstore<K>(o, wx, wy, K == 256 ? a : (a & 1), 1, 2, pos_of, ok_pos, w32);
+            }
+          }
+        }
+        buf = buf == 2 ? 0 : buf + 1;
+        continue;
+      }
       // gather: 8 x (ldmatrix.x4.trans) -> 64 consecutive rows of one column per thread
       float2 v[32];
       {
@@ -746,6 +1134,10 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
       buf = buf == 2 ? 0 : buf + 1;
     }
   }
+  if constexpr (!QUANT && MODE != kModeLowp) {
+#pragma unroll
+    for (int j = 0; j < kAcc; ++j) amax = absmax3(amax, am[j], 0.0f);
+  }
   if (!QUANT) write_partial_unnormalised(amax, c, partials, scratch);
 }
 
@@ -760,6 +1152,10 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes, float* __restrict__ partials, int n_partials,
                   float* __restrict__ scale_out, unsigned int* __restrict__ status, int reverse,
                   const uint8_t* __restrict__ neg, int lp_fmt) {
+  // programmatic dependent launch: nothing is read or written before the previous grid in the
+  // stream has completed; the next grid may be scheduled from here on
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
   static_assert(!SIGNED || sizeof(SrcT) == 4, "sign masks of this kernel are for fp32 words");
   constexpr bool QUANT = MODE != kModeAbsmax;

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "hq.h"
 #include "fwht_quant.cuh"
@@ -17,6 +18,7 @@
 #include "gemm_tcgen05.cuh"
 #include "rotate_out.cuh"
 #include "prerot_quant.cuh"
+#include "mma_peak.cuh"
 
 namespace {
 
@@ -164,6 +166,25 @@ cudaError_t cols_bf16_smem_attr(DeviceInfo& d) {
   return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel in the stream is finishing; it waits for that kernel's completion (griddep_wait) before
+// touching memory, so the order of results is that of an ordinary launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Launch one pass; returns its grid through *grid (the absmax pass's grid is the number of
 // partials the code pass reduces).  SIGNED: the randomized variant with sign flags `neg`.
 template <typename SrcT, int K, int MODE, bool SIGNED>
@@ -182,26 +203,30 @@ cudaError_t launch_pass_s(const SrcT* src, int64_t rows, int64_t cols, int dim, 
     if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0) {
       auto fn = fwhtq_rows_kernel<SrcT, K, MODE, true, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
-      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
-                                      reverse, neg, cols, lp_fmt);
+      cudaError_t e = launch_pdl(fn, g, kQuantThreads, 0, st, src, n, codes, partials,
+                                 MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse, neg, cols, lp_fmt);
+      if (e != cudaSuccess) return e;
     } else {
       auto fn = fwhtq_rows_kernel<SrcT, K, MODE, false, SIGNED>;
       g = grid_for(reinterpret_cast<const void*>(fn), 0);
-      fn<<<g, kQuantThreads, 0, st>>>(src, n, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale, d.status,
-                                      reverse, neg, cols, lp_fmt);
+      cudaError_t e = launch_pdl(fn, g, kQuantThreads, 0, st, src, n, codes, partials,
+                                 MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse, neg, cols, lp_fmt);
+      if (e != cudaSuccess) return e;
     }
   } else if constexpr (sizeof(SrcT) == 2) {
     cudaError_t e = cols_bf16_smem_attr<K, MODE, SIGNED>(d);
     if (e != cudaSuccess) return e;
     auto fn = fwhtq_cols_bf16_kernel<K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), kColsSmemBytes2);
-    fn<<<g, kQuantThreads, kColsSmemBytes2, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials,
-                                                  scale, d.status, reverse, neg, lp_fmt);
+    e = launch_pdl(fn, g, kQuantThreads, kColsSmemBytes2, st, src, rows, cols, codes, partials,
+                   MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse, neg, lp_fmt);
+    if (e != cudaSuccess) return e;
   } else {
     auto fn = fwhtq_cols_f32_kernel<SrcT, K, MODE, SIGNED>;
     g = grid_for(reinterpret_cast<const void*>(fn), 0);
-    fn<<<g, kQuantThreads, 0, st>>>(src, rows, cols, codes, partials, MODE == kModeAbsmax ? g : n_partials, scale,
-                                    d.status, reverse, neg, lp_fmt);
+    cudaError_t e = launch_pdl(fn, g, kQuantThreads, 0, st, src, rows, cols, codes, partials,
+                               MODE == kModeAbsmax ? g : n_partials, scale, d.status, reverse, neg, lp_fmt);
+    if (e != cudaSuccess) return e;
   }
   *grid = g;
   return cudaGetLastError();
@@ -316,24 +341,24 @@ hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols
   const int g = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(n_tiles, d.sms)));
   cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32, SIGNED>(d);
   if (e != cudaSuccess) return cuda_fail(e);
-  fwhtq_dual_kernel<K, kModeAbsmax, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-      map, rows, cols, codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r, 0);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  if ((e = launch_pdl(fwhtq_dual_kernel<K, kModeAbsmax, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols,
+                      codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r, 0)) !=
+      cudaSuccess)
+    return cuda_fail(e);
   if (fmt == HQ_INT8) {
     if ((e = dual_smem_attr<K, kModeInt8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
-    fwhtq_dual_kernel<K, kModeInt8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+    e = launch_pdl(fwhtq_dual_kernel<K, kModeInt8, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
   } else if (fmt == HQ_FP8_E4M3) {
     if ((e = dual_smem_attr<K, kModeFp8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
-    fwhtq_dual_kernel<K, kModeFp8, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+    e = launch_pdl(fwhtq_dual_kernel<K, kModeFp8, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
   } else {
     if ((e = dual_smem_attr<K, kModeLowp, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
-    fwhtq_dual_kernel<K, kModeLowp, W32, SIGNED><<<g, kThreads, kSmemBytes, st>>>(
-        map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r,
-        static_cast<int>(fmt));
+    e = launch_pdl(fwhtq_dual_kernel<K, kModeLowp, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, static_cast<int>(fmt));
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  if (e != cudaSuccess) return cuda_fail(e);
   return HQ_OK;
 }
 
@@ -1161,6 +1186,9 @@ hq_status carve_codes_ws(void* ws, size_t ws_bytes, int64_t b0, int64_t b1, int6
 // array every device that loads the library keeps until exit.  Host code never uses the name
 // as an address: the device address comes from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) float g_noalloc_partials[HQ_NOALLOC_MAX_PARTIALS];
+// The quantizer's grids are capped at kMaxPartials CTAs (one partial each); the array must hold
+// that many, whatever the launch-time check below derives.
+static_assert(kMaxPartials <= HQ_NOALLOC_MAX_PARTIALS, "the no-allocation scratch holds every partial maximum");
 
 struct NoAllocSlot {
   bool ready = false;
@@ -1658,6 +1686,46 @@ hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int6
   cudaError_t e = launch_gemm<hq::gemm::kInt8, hq::gemm::kOutAcc>(ta, tb, nullptr, nullptr, out, int(M), int(N),
                                                                   int(K), *d, reinterpret_cast<cudaStream_t>(stream), 0,
                                                                   1);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
+size_t hq_workspace_bytes(int64_t M, int64_t K, int64_t N, hq_fmt fmt) {
+  if (M < 0 || K < 0 || N < 0) return 0;
+  if (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3 && fmt != HQ_FP6_E3M2 && fmt != HQ_FP6_E2M3 && fmt != HQ_FP4_E2M1) return 0;
+  const size_t sizes[] = {hq_linear_workspace_bytes(M, K, N), hq_linear_fwd_bwd_workspace_bytes(M, K, N),
+                          hq_linear_fwd_save_workspace_bytes(M, K, N), hq_linear_bwd_workspace_bytes(M, K, N),
+                          hq_linear_fwd_keep_workspace_bytes(M, K, N), hq_linear_bwd_reuse_workspace_bytes(M, K, N),
+                          hq_linear_bwd_dx_reuse_workspace_bytes(M, K, N)};
+  size_t m = 0;
+  for (size_t v : sizes) m = std::max(m, v);
+  return m;
+}
+
+hq_status hq_mma_peak(hq_fmt fmt, int64_t n_blocks, int* pairs_out, hq_stream_t stream) {
+  if (fmt != HQ_INT8 && fmt != HQ_FP8_E4M3) return HQ_ERR_ARG;
+  if (n_blocks < 1 || n_blocks > (int64_t(1) << 24)) return HQ_ERR_ARG;
+  DeviceInfo* d = nullptr;
+  hq_status s = device_info(&d);
+  if (s != HQ_OK) return s;
+  const int pairs = d->sms / 2;
+  if (pairs_out) *pairs_out = pairs;
+  auto kernel = fmt == HQ_INT8 ? hq::peak::mma_peak_kernel<hq::gemm::kInt8> : hq::peak::mma_peak_kernel<hq::gemm::kFp8>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(hq::peak::kSmemBytes));
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(hq::peak::kThreads);
+  cfg.dynamicSmemBytes = hq::peak::kSmemBytes;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, n_blocks, d->status);
   return e == cudaSuccess ? HQ_OK : cuda_fail(e);
 }
 

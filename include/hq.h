@@ -160,7 +160,17 @@ HQ_API hq_status hq_gemm_ws(const void* A, const float* scale_a, const void* B, 
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
 
-/* Y[M][N] = (X H)(W H)^T: X and W rotated along K. */
+/* One workspace size for every layer-level call of a shape: the largest of
+ * hq_linear_workspace_bytes, hq_linear_fwd_bwd_workspace_bytes, the saved-codes pair
+ * (hq_linear_fwd_save / hq_linear_bwd) and the reuse placement (hq_linear_fwd_keep /
+ * hq_linear_bwd_reuse) for M, K, N.  Every code format stores one byte per element, so `fmt`
+ * only has to be a valid format; 0 for negative sizes or an unknown format. */
+HQ_API size_t hq_workspace_bytes(int64_t M, int64_t K, int64_t N, hq_fmt fmt);
+
+/* Y[M][N] = (X H)(W H)^T: X and W rotated along K.  The forward that also keeps X's codes
+ * rotated along the tokens for the weight gradient (the HALO training flow, where the
+ * activation is stored quantized) is the separate call hq_linear_fwd_save; its backward,
+ * which takes those codes instead of X, is hq_linear_bwd. */
 HQ_API hq_status hq_linear_fwd(const void* X, const void* W, hq_dtype dt, int64_t M, int64_t K,
                         int64_t N, int k, hq_fmt fmt, void* Y, void* workspace, size_t ws_bytes,
                         hq_stream_t stream);
@@ -432,6 +442,20 @@ HQ_API hq_status hq_quantize_noalloc(const void* src, hq_dtype dt, int64_t rows,
  * ---------------------------------------------------------------------------------------- */
 HQ_API hq_status hq_selftest_gemm_timeout(const void* A, const void* B, void* out, int64_t M,
                                           int64_t N, int64_t K, hq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * hq_mma_peak -- dense tensor-core throughput probe (no counterpart on the pages; it measures
+ * the roofline denominator of the GEMMs on the device at hand).
+ *
+ * Runs one CTA pair per TPC (2 * floor(SMs / 2) CTAs), each pair issuing n_blocks x 4
+ * back-to-back tcgen05.mma.cta_group::2 instructions (M = 256, N = 256, K = 32: 4,194,304
+ * operations each) of kind::i8 (fmt HQ_INT8) or kind::f8f6f4 with e4m3 operands
+ * (HQ_FP8_E4M3) on operand tiles resident in shared memory, accumulating in tensor memory:
+ * no global-memory traffic.  The caller times the launch (CUDA events on `stream`); the
+ * operation count is pairs * n_blocks * 4 * 4,194,304, with pairs from *pairs_out (may be
+ * NULL).  1 <= n_blocks <= 2^24 (at most a few seconds); other formats give HQ_ERR_ARG.
+ * ---------------------------------------------------------------------------------------- */
+HQ_API hq_status hq_mma_peak(hq_fmt fmt, int64_t n_blocks, int* pairs_out, hq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Status.

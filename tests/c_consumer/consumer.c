@@ -17,6 +17,14 @@ int main(void) {
   CHECK(hq_quantize_workspace_bytes() > 0);
   CHECK(hq_linear_fwd_bwd_workspace_bytes(4096, 4096, 11008) > (size_t)4096 * 11008);
   CHECK(hq_gemm_workspace_bytes(4096, 11008, 4096) == 0);
+  /* one size covers every layer-level call of a shape, in every code format */
+  CHECK(hq_workspace_bytes(4096, 4096, 11008, HQ_INT8) >= hq_linear_fwd_bwd_workspace_bytes(4096, 4096, 11008));
+  CHECK(hq_workspace_bytes(4096, 4096, 11008, HQ_INT8) >= hq_linear_workspace_bytes(4096, 4096, 11008));
+  CHECK(hq_workspace_bytes(4096, 4096, 11008, HQ_FP4_E2M1) == hq_workspace_bytes(4096, 4096, 11008, HQ_INT8));
+  CHECK(hq_workspace_bytes(4096, 4096, 11008, (hq_fmt)9) == 0);
+  /* the tensor-core probe rejects formats other than INT8 / FP8 before any launch */
+  CHECK(hq_mma_peak(HQ_FP6_E2M3, 16, NULL, NULL) == HQ_ERR_ARG);
+  CHECK(hq_mma_peak(HQ_INT8, 0, NULL, NULL) == HQ_ERR_ARG);
   float scale = 0.0f;
   /* null source: rejected before anything is launched */
   CHECK(hq_quantize(NULL, HQ_BF16, 256, 256, 1, 64, HQ_INT8, (void*)0x10000, &scale, (void*)0x10000,

@@ -50,6 +50,20 @@ def test_workspace_sizes(L):
     need = hq.hq_linear_workspace_bytes(M, K, N)
     assert need >= max(M * K + N * K, M * N + K * N, N * M + K * M) + q
     assert hq.hq_linear_workspace_bytes(-1, 2, 3) == 0
+    # one size for every layer-level call of the shape, whatever the format
+    one = hq.hq_workspace_bytes(M, K, N, "int8")
+    for f in ("hq_linear_workspace_bytes", "hq_linear_fwd_bwd_workspace_bytes", "hq_linear_fwd_save_workspace_bytes",
+              "hq_linear_bwd_workspace_bytes", "hq_linear_fwd_keep_workspace_bytes",
+              "hq_linear_bwd_reuse_workspace_bytes", "hq_linear_bwd_dx_reuse_workspace_bytes"):
+        assert one >= getattr(L, f)(M, K, N), f
+    assert all(hq.hq_workspace_bytes(M, K, N, f) == one for f in ("fp8", "fp6_e3m2", "fp6_e2m3", "fp4_e2m1"))
+    assert L.hq_workspace_bytes(M, K, N, 5) == 0 and L.hq_workspace_bytes(-1, K, N, 0) == 0
+
+
+def test_mma_peak_argument_errors(L):
+    assert L.hq_mma_peak(2, 16, None, None) == 1   # FP6: the probe runs INT8 / FP8 only
+    assert L.hq_mma_peak(0, 0, None, None) == 1
+    assert L.hq_mma_peak(1, (1 << 24) + 1, None, None) == 1
 
 
 def _q(L, src=FAKE, dt=hq.HQ_BF16, rows=64, cols=256, dim=1, k=16, fmt=0, codes=FAKE, scale=FAKE,

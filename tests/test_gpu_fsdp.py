@@ -78,3 +78,26 @@ def test_codes_pass_special_absmax():
     c, s = hq.hq_quantize_codes(W, 1, 64, "int8", torch.full((1,), float("inf"), device="cuda"))
     assert hq.hq_get_error() == 5
     assert not np.isfinite(s.cpu().numpy()[0])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt", ("int8", "fp8"))
+def test_fsdp_forward_flow_one_gpu(fmt):
+    """The quantized-FSDP forward flow (gathers on a communication stream, prefetched one layer
+    ahead) on one GPU, where each rank's shard is the whole weight: every layer's output equals
+    hq_linear_fwd bit for bit."""
+    from hadamard_rotated_precision_b200 import synthetic
+    k = 64
+    xs, ws = [], []
+    for i in range(3):
+        K, N, M = 256 * (i + 1), 128 * (i + 2), 512
+        X = synthetic.tiny_random((M, K), 500 + i)
+        X[:, 3] *= 40.0
+        xs.append(to_device(synthetic.to_bf16_bits(X)))
+        ws.append(to_device(synthetic.to_bf16_bits(synthetic.tiny_random((N, K), 600 + i, scale=0.02))))
+    ys = hq.hq_fsdp_forward(ws, xs, k, fmt)
+    torch.cuda.synchronize()
+    for i, (x, w, y) in enumerate(zip(xs, ws, ys)):
+        want = hq.hq_linear_fwd(x, w, k, fmt)
+        assert torch.equal(y.view(torch.int16), want.view(torch.int16)), f"layer {i}"
+    assert hq.hq_get_error() == 0

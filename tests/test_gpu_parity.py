@@ -307,11 +307,13 @@ def test_gemm_k_zero_writes_zeros():
 
 # ------------------------------------------------------------------------------ the layer
 
-def _layer_check(d, k, fmt, rows_sample=None, tag=""):
+def _layer_check(d, k, fmt, rows_sample=None, tag="", step=False):
     """All three GEMMs of one layer: codes, scales, accumulators (via the split entry points)
-    and the fused linear entry points' bf16 outputs."""
+    and the fused linear entry points' bf16 outputs.  step=True: the whole-layer entry point
+    hq_linear_fwd_bwd's outputs are compared with the oracle on the same rows as well."""
     X, W, dY = d["X"], d["W"], d["dY"]
     Xd, Wd, dYd = to_device(X), to_device(W), to_device(dY)
+    step_out = dict(zip(("fwd", "dx", "dw"), hq.hq_linear_fwd_bwd(Xd, Wd, dYd, k, fmt))) if step else {}
     cases = (
         ("fwd", hq.hq_linear_fwd, (Xd, Wd), oracle.linear_fwd, (X, W), (X, 1), (W, 1)),
         ("dx", hq.hq_linear_bwd_dx, (dYd, Wd), oracle.linear_bwd_dx, (dY, W), (dY, 1), (W, 0)),
@@ -341,6 +343,16 @@ def _layer_check(d, k, fmt, rows_sample=None, tag=""):
         else:
             e = rel_fro(bits_to_f32(got), bits_to_f32(want["ref"]))
             assert e <= FP8_TOL, f"{tag}{name}: fp8 rel fro {e}"
+        if step:
+            gs = bf16_bits(step_out[name])
+            if rows is not None:
+                gs = gs[rows]
+            if fmt == oracle.INT8:
+                np.testing.assert_array_equal(gs, want["fast"], err_msg=f"{tag}{name}: step bf16 formula")
+                assert bf16_ulp_diff(gs, want["ref"]).max() <= 1, f"{tag}{name}: step ulp"
+            else:
+                e = rel_fro(bits_to_f32(gs), bits_to_f32(want["ref"]))
+                assert e <= FP8_TOL, f"{tag}{name}: step fp8 rel fro {e}"
     assert hq.hq_get_error() == 0
 
 
@@ -451,12 +463,13 @@ def test_layer_token_prefix(wid):
 
 @pytest.mark.parametrize("wid", (1, 2, 3, 4))
 def test_layer_full_size(wid):
-    """Each workload at its full size (the bench's launch configuration), outputs compared on
-    sampled rows; codes and scales compared in full."""
+    """Each workload at its full size, outputs of the separate entry points and of the
+    whole-layer step hq_linear_fwd_bwd compared with the oracle on sampled rows; codes and
+    scales compared in full."""
     w = synthetic.WORKLOADS[wid]
     fmt = oracle.INT8 if w.fmt == "int8" else oracle.FP8_E4M3
     for li in range(len(w.layers)):
-        _layer_check(synthetic.draw(w, li), w.k, fmt, rows_sample=True, tag=f"{w.name}/{li}/")
+        _layer_check(synthetic.draw(w, li), w.k, fmt, rows_sample=True, tag=f"{w.name}/{li}/", step=True)
 
 
 @pytest.mark.parametrize("fmt_name,k", synthetic.WORKLOADS[5].sweep)
@@ -467,8 +480,22 @@ def test_llama_block_sweep_o_proj(fmt_name, k):
     _layer_check(synthetic.draw(w, 1), k, fmt, rows_sample=True, tag=f"o/{fmt_name}/{k}/")
 
 
-@pytest.mark.parametrize("li", (0, 2, 4))
-def test_llama_block_other_shapes(li):
-    """qkv (4096 -> 12288), gate (4096 -> 11008) and down (11008 -> 4096) at INT8 k=256."""
+@pytest.mark.parametrize("li", (0, 1, 2, 3, 4))
+def test_llama_block_step_vs_oracle(li):
+    """The bench's headline step: every layer of the Llama-2-7B block (qkv, o, gate, up, down
+    at 8192 tokens) through hq_linear_fwd_bwd at INT8 k = 256, outputs against the oracle on
+    sampled rows, codes and scales in full."""
     w = synthetic.WORKLOADS[5]
-    _layer_check(synthetic.draw(w, li), 256, oracle.INT8, rows_sample=True, tag=f"{li}/")
+    _layer_check(synthetic.draw(w, li), 256, oracle.INT8, rows_sample=True, tag=f"{w.layers[li].name}/", step=True)
+
+
+@pytest.mark.parametrize("li", (0, 2, 3, 4))
+def test_llama_block_sweep_other_layers(li):
+    """The block's sweep over INT8 / FP8 x k = 16 .. 256 on qkv, gate, up and down (8192
+    tokens; the o projection has its own test above): codes and scales in full, the separate
+    entry points' and the whole-layer step's outputs on sampled rows."""
+    w = synthetic.WORKLOADS[5]
+    d = synthetic.draw(w, li)
+    for fmt_name, k in w.sweep:
+        fmt = oracle.INT8 if fmt_name == "int8" else oracle.FP8_E4M3
+        _layer_check(d, k, fmt, rows_sample=True, tag=f"{w.layers[li].name}/{fmt_name}/{k}/", step=(k in (16, 256)))

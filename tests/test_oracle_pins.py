@@ -754,3 +754,45 @@ def test_next_layer_flow_tracks_two_layer_product(oracle_lib):
     qp, sp = oracle.quantize_rotated(y_plain, oracle.INT8)
     bad = oracle.gemm(qp, qw2, oracle.INT8).astype(np.float64) * float(sp) * float(sw2)
     assert _rel_fro(bad, want) > 0.5
+
+
+# ------------------------------------------------------------------ packed minifloat layout
+
+def _lowp_pack_fixture():
+    path = os.path.join(os.path.dirname(__file__), "golden", "lowp_pack16.txt")
+    out = []
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            bits, codes, chunk = (p.strip() for p in line.split("|"))
+            out.append((int(bits), [int(c) for c in codes.split()], bytes(int(b, 16) for b in chunk.split())))
+    return out
+
+
+def test_device_codes_packed_layout_fixture():
+    """oracle.device_codes packs FP6 / FP4 codes as the hand-derived chunks of the fixture
+    (16 codes per 16-byte chunk, LSB first, zero tail), for every minifloat format of the bit
+    width, and leaves INT8 / FP8 codes as they are."""
+    cases = _lowp_pack_fixture()
+    assert len(cases) == 3
+    for bits, codes, chunk in cases:
+        fmts = (oracle.FP6_E3M2, oracle.FP6_E2M3) if bits == 6 else (oracle.FP4_E2M1,)
+        for fmt in fmts:
+            got = oracle.device_codes(np.array([codes], dtype=np.uint8), fmt)
+            assert got.shape == (1, 16) and got.tobytes() == chunk, (fmt, got.tobytes().hex())
+    x = np.arange(64, dtype=np.uint8).reshape(2, 32)
+    for fmt in (oracle.INT8, oracle.FP8_E4M3):
+        assert np.array_equal(oracle.device_codes(x, fmt), x)
+
+
+def test_device_codes_packed_chunk_order():
+    """Chunks follow the code groups in order along the rotated dimension and rows stay rows:
+    a 2 x 32 array of FP4 codes is four fixture-style chunks, group by group."""
+    (_, c6, ch6), _, (_, c4, ch4) = _lowp_pack_fixture()
+    rows = np.array([c4 + [0] * 16, [0] * 16 + c4], dtype=np.uint8)
+    got = oracle.device_codes(rows, oracle.FP4_E2M1)
+    zero = bytes(16)
+    assert got[0].tobytes() == ch4 + zero and got[1].tobytes() == zero + ch4
+    rows6 = np.array([c6 + c6], dtype=np.uint8)
+    assert oracle.device_codes(rows6, oracle.FP6_E2M3)[0].tobytes() == ch6 + ch6
