@@ -816,10 +816,30 @@ def run_kernel_case(args):
     torch.cuda.set_device(0)
     g = torch.Generator(device="cuda").manual_seed(0)
     case = args.kernel_case
+    if case == "block_step":
+        # two steps of the bench's headline workload (every layer of the Llama-2-7B block through
+        # hq_linear_fwd_bwd), for the launch list of the step
+        w = synthetic.WORKLOADS[WORKLOAD_ID]
+        ls = []
+        for li, L in enumerate(w.layers):
+            d = synthetic.draw(w, li)
+            t = {n: torch.from_numpy(d[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("X", "W", "dY")}
+            t["ws"] = torch.empty(hq.hq_linear_fwd_bwd_workspace_bytes(L.M, L.K, L.N), dtype=torch.uint8, device="cuda")
+            ls.append(t)
+        for _ in range(2):
+            for t in ls:
+                hq.hq_linear_fwd_bwd(t["X"], t["W"], t["dY"], w.k, w.fmt, workspace=t["ws"])
+        torch.cuda.synchronize()
+        st = hq.hq_get_error()
+        print(json.dumps({"kernel_case": case, "status": st}))
+        return 0 if st == 0 else 1
     if case.startswith("gemm"):
         fmt = "fp8" if case == "gemm_fp8" else "int8"
-        # the Llama up-projection forward shape, or the ViT-B fc1 forward (contraction 768)
+        # the Llama up-projection forward shape, or the ViT-B fc1 forward (contraction 768), or
+        # --shape M,N,K
         M, N, K = (12608, 3072, 768) if case == "gemm_short_k" else (4096, 11008, 4096)
+        if args.shape:
+            M, N, K = (int(v) for v in args.shape.split(","))
         A = torch.randint(-127, 128, (M, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
         B = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
         if fmt == "fp8":
@@ -860,8 +880,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
     ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual",
-                                              "dx_reuse"),
+                                              "dx_reuse", "block_step"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
+    ap.add_argument("--shape", help="with --kernel-case gemm / gemm_fp8: M,N,K of the GEMM")
     ap.add_argument("--formats", action="store_true",
                     help="with --sweep: the bench workload's layer in every code format (INT8, FP8, FP6, FP4)")
     ap.add_argument("--reuse", action="store_true",

@@ -466,6 +466,25 @@ struct Geo {
       1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
 };
 
+// Tile order of the pair kernel: bands of kRasterBand M-blocks; within a band the M-block
+// varies fastest, then the N-block.  The tiles in flight together (one per CTA pair) then read
+// kRasterBand A panels and about pairs / kRasterBand B panels (256 rows x K each), which stay
+// in L2 while the band sweeps N, so A is read from DRAM about once and B once per band.  With
+// the M-fastest order over the whole of M, the A panels of every M-block were read again for
+// each N-block column once A exceeded what L2 keeps beside the output stream (12288 x 4096 x
+// 8192: 1054 MB of DRAM reads for 134 MB of operands).  A GEMM with at most kRasterBand
+// M-blocks is one band, i.e. the plain M-fastest order.
+constexpr int kRasterBand = 16;
+
+__device__ __forceinline__ void pair_tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
+  const int band = tile / (kRasterBand * num_n);
+  const int m0 = band * kRasterBand;
+  const int gb = min(kRasterBand, num_m - m0);
+  const int idx = tile - band * kRasterBand * num_n;
+  m_blk = m0 + idx % gb;
+  n_blk = idx / gb;
+}
+
 constexpr int kShortKBlocks = 8;  // K <= 1024 bytes: the SHORT_K shape
 
 template <int FMT, int BN_>
@@ -572,6 +591,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   ptx::cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *sh.tmem_holder;
+  // programmatic dependent launch: the set-up above overlaps the previous kernel's end; global
+  // memory (operands, scales, output, split scratch) is touched only once that kernel has
+  // completed.  The next kernel in the stream may be scheduled from here on.
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -582,7 +606,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       bool ok = true;
       for (int item = pair_id; item < num_items && ok; item += num_pairs) {
         const Item it = item_at(item);
-        const int m_blk = it.tile % num_m, n_blk = it.tile / num_m;
+        int m_blk, n_blk;
+        pair_tile_coords(it.tile, num_m, num_n, m_blk, n_blk);
         for (int kb = it.kb_begin; kb < it.kb_end; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, sh.abort_flag, status)) { ok = false; break; }
           const uint32_t fb = ptx::mapa_shared(full_bar(stage), 0);
@@ -660,7 +685,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     uint32_t acc_phase = 0;
     for (int item = pair_id; item < num_items; item += num_pairs) {
       const Item it = item_at(item);
-      const int m_blk = it.tile % num_m, n_blk = it.tile / num_m;
+      int m_blk, n_blk;
+      pair_tile_coords(it.tile, num_m, num_n, m_blk, n_blk);
       int ok = 0;
       if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, sh.abort_flag, status) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);

@@ -212,13 +212,15 @@ HQ_API hq_status hq_quantize_dual(const void* src, hq_dtype dt, int64_t rows, in
  * of hq_linear_fwd, hq_linear_bwd_dx and hq_linear_bwd_dw bit for bit.
  *   X [M][K], W [N][K], dY [M][N] (dtype dt); Y [M][N], dX [M][K], dW [N][K] bf16.
  *   M, K, N: positive multiples of k.  workspace: >= hq_linear_fwd_bwd_workspace_bytes().
- * X and W along K and the forward GEMM run on `stream`; the four rotations the forward GEMM
- * does not use (dY along N and along M together, as in hq_quantize_dual, then W along N and
- * X along M) run on a per-device side stream that the library creates on first use (with
- * three events) and forks from / joins back to `stream` with events, so they overlap the
- * forward quantizations and GEMM.  The dX GEMM waits only for dY along N and W along N; X
- * along M lands while it runs and the dW GEMM waits for it.  Everything is complete when
- * `stream` reaches the end of the call.
+ * dY in both rotations (one two-rotation call, as hq_quantize_dual) runs on a per-device side
+ * stream that the library creates on first use (with three events) and forks from / joins back
+ * to `stream` with events.  When X and W are bf16 with both dimensions >= 2048 (and multiples
+ * of 64) and k <= 128, each is quantized in both rotations by one two-rotation call on `stream`, followed by
+ * the three GEMMs, the backward ones after dY's codes have landed.  Otherwise X and W along K
+ * and the forward GEMM run on `stream` while the side stream also quantizes W along N and X
+ * along M; the dX GEMM waits only for dY along N and W along N, X along M lands while it runs
+ * and the dW GEMM waits for it.  Everything is complete when `stream` reaches the end of the
+ * call.
  * ---------------------------------------------------------------------------------------- */
 HQ_API size_t hq_linear_fwd_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N);
 HQ_API hq_status hq_linear_fwd_bwd(const void* X, const void* W, const void* dY, hq_dtype dt,
