@@ -591,12 +591,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   ptx::cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *sh.tmem_holder;
-  // programmatic dependent launch: the set-up above overlaps the previous kernel's end; global
-  // memory (operands, scales, output, split scratch) is touched only once that kernel has
-  // completed.  The next kernel in the stream may be scheduled from here on.
-  ptx::griddep_wait();
-  ptx::griddep_launch_dependents();
-
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {

@@ -627,15 +627,13 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   cfg.blockDim = dim3(hq::gemm::NUM_THREADS);
   cfg.dynamicSmemBytes = G::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait in the kernel
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   (void)d;
   return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, split_from, part_ws, counters,
                             ab_code, rot_k);
