@@ -623,7 +623,9 @@ def run_sweep(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
-    int8_peak = measure_mma_peaks(hq, torch, sustained=False)["int8"]
+    mma = measure_mma_peaks(hq, torch, sustained=False)
+    # INT8 GEMMs against the measured INT8 peak, the kind::f8f6f4 formats against the FP8 one
+    peak_of = lambda f: mma["int8"] if f == "int8" else mma["fp8"]  # noqa: E731
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     L_ = hq.lib()
     reps = max(3, args.steps)
@@ -687,7 +689,8 @@ def run_sweep(args):
                         "dtype": "bf16" if elem == 2 else "f32",
                         "step_ms": step_ms, "step_tops": ops / (step_ms * 1e-3) / 1e12,
                         "gemm_ms": gemm_ms, "gemm_tops": ops / (gemm_ms * 1e-3) / 1e12,
-                        "gemm_frac_of_peak": ops / (gemm_ms * 1e-3) / 1e12 / int8_peak,
+                        "gemm_frac_of_peak": ops / (gemm_ms * 1e-3) / 1e12 / peak_of(fmt_name),
+                        "peak_tops": peak_of(fmt_name),
                         "quant_ms": quant_ms, "quant_gbs": qbytes / (quant_ms * 1e-3) / 1e9,
                         "quant_frac_of_hbm": qbytes / (quant_ms * 1e-3) / 1e9 / peaks["hbm"],
                         "status": hq.hq_get_error()}
@@ -712,7 +715,7 @@ def run_reuse(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     peaks = load_peaks()
-    int8_peak = measure_mma_peaks(hq, torch, sustained=False)["int8"]
+    mma = measure_mma_peaks(hq, torch, sustained=False)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     reps = max(3, args.steps)
 
@@ -773,7 +776,7 @@ def run_reuse(args):
             line = {"workload": w.name, "layer": Lr.name, "M": M, "K": K, "N": N, "fmt": w.fmt, "k": k,
                     "halo2_step_ms": halo2_ms, "halo2_step_tops": ops / (halo2_ms * 1e-3) / 1e12,
                     "reuse_step_ms": reuse_ms, "reuse_step_tops": ops / (reuse_ms * 1e-3) / 1e12,
-                    "reuse_frac_of_peak": ops / (reuse_ms * 1e-3) / 1e12 / int8_peak,
+                    "reuse_frac_of_peak": ops / (reuse_ms * 1e-3) / 1e12 / (mma["int8"] if fmt == hq.HQ_INT8 else mma["fp8"]),
                     "dx_reuse_ms": dx_reuse_ms, "dx_halo2_gemm_ms": dx_gemm_ms,
                     "derotate_bytes": 14 * M * K,
                     "status": hq.hq_get_error()}
