@@ -591,6 +591,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   ptx::cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *sh.tmem_holder;
+
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {
