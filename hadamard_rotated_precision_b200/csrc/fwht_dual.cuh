@@ -40,6 +40,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 #include "fwht_quant.cuh"
 #include "sm100_ptx.cuh"
 
@@ -161,25 +162,34 @@ __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float2& f) {
 }
 
 
-template <int K, int MODE, bool W32, bool SIGNED>
+// ONCHIP (INT8 / FP8 codes; a cooperative launch of at most one CTA per SM and one tile per
+// CTA): both passes in one launch.  Each CTA keeps its tile in shared memory, runs the absmax
+// pass over it, writes its partial maxima, meets the other CTAs at a grid barrier on
+// *grid_counter (zeroed by the host before the launch; every wait bounded), reduces all the
+// partials and runs the code pass over the same resident tile: the source is read from HBM
+// once, and there is one launch instead of two.
+template <int K, int MODE, bool W32, bool SIGNED, bool ONCHIP = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t cols,
                   uint8_t* __restrict__ codes_c, uint8_t* __restrict__ codes_r,
                   float* __restrict__ part_c, float* __restrict__ part_r, int n_partials,
                   float* __restrict__ scale_c, float* __restrict__ scale_r,
                   unsigned int* __restrict__ status, int reverse,
-                  const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r, int lp_fmt) {
+                  const uint8_t* __restrict__ neg_c, const uint8_t* __restrict__ neg_r, int lp_fmt,
+                  unsigned int* __restrict__ grid_counter) {
   // programmatic dependent launch: nothing is read or written before the previous grid in the
   // stream has completed; the next grid may be scheduled from here on
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
   // SIGNED: sign flags per column (neg_c) and per row (neg_r); either may be null (all clear)
   static_assert(K >= 16 && K <= 256 && (K & (K - 1)) == 0, "k must be a power of two in [16,256]");
+  static_assert(!ONCHIP || MODE == kModeInt8 || MODE == kModeFp8, "single-launch form: INT8 / FP8 codes");
   constexpr bool QUANT = MODE != kModeAbsmax;
   extern __shared__ uint8_t dsmem[];
   __shared__ float scratch[32];
   __shared__ float red[2 * kComputeWarps];
   __shared__ int abort_flag;
+  __shared__ int grid_ok;  // ONCHIP: the grid barrier completed in time
   __shared__ unsigned int released[kSlots];  // warps done with the slot, over all rounds
   __shared__ int issued_round[kSlots];       // round of the slot's latest copy (-1: none)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
@@ -241,13 +251,13 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
 
   const float c = __frsqrt_rn(static_cast<float>(K));
   QuantParams qc{0.0f, false, false}, qr{0.0f, false, false};
-  if constexpr (QUANT) {
+  if constexpr (QUANT && !ONCHIP) {
     qc = finish_absmax<MODE>(part_c, n_partials, scale_c, scratch, status, lp_fmt);
     qr = finish_absmax<MODE>(part_r, n_partials, scale_r, scratch, status, lp_fmt);
   }
-  const int64_t work_tiles = (qc.abort && qr.abort) ? 0 : my_tiles;
+  int64_t work_tiles = (qc.abort && qr.abort) ? 0 : my_tiles;
 
-  const CodeScale csc = code_scale<K>(c, qc.inv), csr = code_scale<K>(c, qr.inv);
+  CodeScale csc = code_scale<K>(c, qc.inv), csr = code_scale<K>(c, qr.inv);
   float amc[kAcc], amr[kAcc];
 #pragma unroll
   for (int j = 0; j < kAcc; ++j) amc[j] = amr[j] = 0.0f;
@@ -276,226 +286,219 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
   const float2 csA = make_float2(cgA, cgA), cnsA = make_float2(-cgA, -cgA);
   const float2 csB = make_float2(cgB, cgB), cnsB = make_float2(-cgB, -cgB);
 
-  for (int64_t i = 0; i < work_tiles; ++i) {
-    const int64_t t = tile_of(i);
-    const int64_t row0 = (t / n_ct) * kTile, col0 = (t % n_ct) * kTile;
-    const int64_t q0 = i * kStripsPerTile;
-    const int slot0 = static_cast<int>(q0 % kSlots);
-    auto slot_of = [&](int s) { return slot0 + s < kSlots ? slot0 + s : slot0 + s - kSlots; };
-    bool ok = true;
-#pragma unroll
-    for (int s = 0; s < kStripsPerTile; ++s) {
-      const int64_t q = q0 + s;
-      ok = ok && wait_full(full_bar(slot_of(s)), static_cast<uint32_t>((q / kSlots) & 1), &abort_flag, status);
-    }
-    if (!ok) break;
-
-    if constexpr (XL) {
-      // ---- row role (exchange layout): a thread reads one strip row (64 columns) of its strip
-      // sr; position bits 6, 7 of the column are lane bits 3, 4 (A = bit 3, B = bit 4)
-      const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
-#pragma unroll 1
-      for (int st = 0; st < kSteps; ++st) {
-        const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
-        const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
-        float2 v[32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t cq = static_cast<uint32_t>(q ^ row_sw);  // chunk of the x half; the y half's is 4 + cq
-          uint4 rx = ptx::ld_shared_v4(rowaddr + ((cq ^ swr) << 4));
-          uint4 ry = ptx::ld_shared_v4(rowaddr + (((4u + cq) ^ swr) << 4));
-          if constexpr (SIGNED) {
-            const int64_t c0 = col0 + kStripCols * sr + 8 * cq;
-            uint32_t mx[4], my[4];
-            const bool in = neg_c != nullptr && c0 < cols;
-            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0)) : make_uint2(0u, 0u), mx);
-            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0 + 32)) : make_uint2(0u, 0u), my);
-            rx.x ^= mx[0]; rx.y ^= mx[1]; rx.z ^= mx[2]; rx.w ^= mx[3];
-            ry.x ^= my[0]; ry.y ^= my[1]; ry.z ^= my[2]; ry.w ^= my[3];
-          }
-          const uint32_t wxq[4] = {rx.x, rx.y, rx.z, rx.w}, wyq[4] = {ry.x, ry.y, ry.z, ry.w};
-          xunpack(q, wxq, wyq, v);
-        }
-        if (kSteps == 2 && st == 1) {
-          release(q0 + 1 - grp);
-          release(q0 + 3 - grp);
-        }
-        xrotate<K, !QUANT>(v, rsA, rnsA, rsB, rnsB, 8, 16, amc);
-        if constexpr (QUANT) {
-          const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
-          if (!qc.abort) {  // uniform: every lane takes part in the code-word exchange
-            const bool row_in = r < rows;
-            uint32_t wx[8], wy[8];
-            xcodes<MODE>(v, csc, qc.zero, wx, wy);
-            // segment of half h: k <= 64 the thread's strip; k = 128 position bit 6 = A, bit 7 =
-            // the strip's bit 1; k = 256 bits 6, 7 = the strip
-            auto pos_of = [&](int h) -> int64_t {
-              if constexpr (K <= 64) return int64_t(kStripCols) * sr + 32 * h;
-              else if constexpr (K == 128) return 32 * h + 64 * (sr & 1) + 128 * (sr >> 1);
-              else return 32 * h + 64 * sr;
-            };
-            auto ok_pos = [&](int64_t pc) { return row_in && col0 + pc < cols; };
-            xstore<K>(codes_c + r * cols + col0, wx, wy, K == 256 ? sr : (sr & 1), 8, 16, pos_of, ok_pos, W32);
-          }
-        }
+  // One sweep over this CTA's tiles: the absmax pass (Q false: both roles' running maxima)
+  // or the code pass (Q true).
+  auto sweep = [&](auto q_tag) {
+    constexpr bool Q = decltype(q_tag)::value;
+    for (int64_t i = 0; i < work_tiles; ++i) {
+      const int64_t t = tile_of(i);
+      const int64_t row0 = (t / n_ct) * kTile, col0 = (t % n_ct) * kTile;
+      const int64_t q0 = i * kStripsPerTile;
+      const int slot0 = static_cast<int>(q0 % kSlots);
+      auto slot_of = [&](int s) { return slot0 + s < kSlots ? slot0 + s : slot0 + s - kSlots; };
+      bool ok = true;
+  #pragma unroll
+      for (int s = 0; s < kStripsPerTile; ++s) {
+        const int64_t q = q0 + s;
+        ok = ok && wait_full(full_bar(slot_of(s)), static_cast<uint32_t>((q / kSlots) & 1), &abort_flag, status);
       }
+      if (!ok) break;
 
-      // ---- col role (exchange layout): ldmatrix.trans gathers; a thread receives rows of one
-      // column whose position bits 6, 7 are its lane bits 0, 1 (A = bit 0, B = bit 1)
-#pragma unroll 1
-      for (int j2 = 0; j2 < kSteps; ++j2) {
-        const int s = grp + (kComputeWarps / 8) * j2;
-        const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
-        float2 v[32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          // gather q of the x half reads call (q ^ sw) of 32 rows, the y half call 4 + (q ^ sw);
-          // the swizzle is that of the thread receiving the row this lane addresses
-          uint32_t rx[4], ry[4];
-          ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(q ^ col_sw_addr), rx);
-          ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(4 + (q ^ col_sw_addr)), ry);
-          if constexpr (SIGNED) {
-            const int64_t r0t = row0 + 64 * (lane & 3) + 8 * (q ^ col_sw);
-            uint32_t mx[4], my[4];
-            const bool in = neg_r != nullptr && r0t < rows;
-            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t)) : make_uint2(0u, 0u), mx);
-            sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t + 32)) : make_uint2(0u, 0u), my);
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm) {
-              rx[mm] ^= mx[mm];
-              ry[mm] ^= my[mm];
+      if constexpr (XL) {
+        // ---- row role (exchange layout): a thread reads one strip row (64 columns) of its strip
+        // sr; position bits 6, 7 of the column are lane bits 3, 4 (A = bit 3, B = bit 4)
+        const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+  #pragma unroll 1
+        for (int st = 0; st < kSteps; ++st) {
+          const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
+          const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+          float2 v[32];
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t cq = static_cast<uint32_t>(q ^ row_sw);  // chunk of the x half; the y half's is 4 + cq
+            uint4 rx = ptx::ld_shared_v4(rowaddr + ((cq ^ swr) << 4));
+            uint4 ry = ptx::ld_shared_v4(rowaddr + (((4u + cq) ^ swr) << 4));
+            if constexpr (SIGNED) {
+              const int64_t c0 = col0 + kStripCols * sr + 8 * cq;
+              uint32_t mx[4], my[4];
+              const bool in = neg_c != nullptr && c0 < cols;
+              sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0)) : make_uint2(0u, 0u), mx);
+              sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_c + c0 + 32)) : make_uint2(0u, 0u), my);
+              rx.x ^= mx[0]; rx.y ^= mx[1]; rx.z ^= mx[2]; rx.w ^= mx[3];
+              ry.x ^= my[0]; ry.y ^= my[1]; ry.z ^= my[2]; ry.w ^= my[3];
+            }
+            const uint32_t wxq[4] = {rx.x, rx.y, rx.z, rx.w}, wyq[4] = {ry.x, ry.y, ry.z, ry.w};
+            xunpack(q, wxq, wyq, v);
+          }
+          if (kSteps == 2 && st == 1) {
+            release(q0 + 1 - grp);
+            release(q0 + 3 - grp);
+          }
+          xrotate<K, !Q>(v, rsA, rnsA, rsB, rnsB, 8, 16, amc);
+          if constexpr (Q) {
+            const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
+            if (!qc.abort) {  // uniform: every lane takes part in the code-word exchange
+              const bool row_in = r < rows;
+              uint32_t wx[8], wy[8];
+              xcodes<MODE>(v, csc, qc.zero, wx, wy);
+              // segment of half h: k <= 64 the thread's strip; k = 128 position bit 6 = A, bit 7 =
+              // the strip's bit 1; k = 256 bits 6, 7 = the strip
+              auto pos_of = [&](int h) -> int64_t {
+                if constexpr (K <= 64) return int64_t(kStripCols) * sr + 32 * h;
+                else if constexpr (K == 128) return 32 * h + 64 * (sr & 1) + 128 * (sr >> 1);
+                else return 32 * h + 64 * sr;
+              };
+              auto ok_pos = [&](int64_t pc) { return row_in && col0 + pc < cols; };
+              xstore<K>(codes_c + r * cols + col0, wx, wy, K == 256 ? sr : (sr & 1), 8, 16, pos_of, ok_pos, W32);
             }
           }
-          xunpack(q, rx, ry, v);
         }
-        release(q0 + s);
-        xrotate<K, !QUANT>(v, csA, cnsA, csB, cnsB, 1, 2, amr);
-        if constexpr (QUANT) {
-          const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
-          if (!qr.abort) {  // uniform: every lane takes part in the code-word exchange
-            const bool col_in = gc < cols;
-            uint32_t wx[8], wy[8];
-            xcodes<MODE>(v, csr, qr.zero, wx, wy);
-            const int a = lane & 3;
-            auto pos_of = [&](int h) -> int64_t {
-              if constexpr (K <= 64) return 64 * a + 32 * h;
-              else if constexpr (K == 128) return 32 * h + 64 * (a & 1) + 128 * (a >> 1);
-              else return 32 * h + 64 * a;
-            };
-            auto ok_pos = [&](int64_t pr) { return col_in && row0 + pr < rows; };
-            xstore<K>(codes_r + gc * rows + row0, wx, wy, K == 256 ? a : (a & 1), 1, 2, pos_of, ok_pos, W32);
-          }
-        }
-      }
-    } else {
-      // ---- row role: rotation along the columns, kSteps steps of 8 rows x 256 columns per warp
-      const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+
+        // ---- col role (exchange layout): ldmatrix.trans gathers; a thread receives rows of one
+        // column whose position bits 6, 7 are its lane bits 0, 1 (A = bit 0, B = bit 1)
   #pragma unroll 1
-      for (int st = 0; st < kSteps; ++st) {
-        const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
-        const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
-        // sign flags of the thread's 64 columns (the randomized variant; cols is a multiple of 64,
-        // so they are all inside the tensor or all past its end)
-        uint32_t sm[SIGNED ? 32 : 1];
-        if constexpr (SIGNED) {
-          const int64_t c0 = col0 + kStripCols * sr;
+        for (int j2 = 0; j2 < kSteps; ++j2) {
+          const int s = grp + (kComputeWarps / 8) * j2;
+          const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+          float2 v[32];
   #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t m8[8];
-            sign_masks_bf16x16(neg_c != nullptr && c0 < cols ? __ldg(reinterpret_cast<const uint4*>(neg_c + c0 + 16 * c))
-                                                             : make_uint4(0u, 0u, 0u, 0u), m8);
+          for (int q = 0; q < 4; ++q) {
+            // gather q of the x half reads call (q ^ sw) of 32 rows, the y half call 4 + (q ^ sw);
+            // the swizzle is that of the thread receiving the row this lane addresses
+            uint32_t rx[4], ry[4];
+            ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(q ^ col_sw_addr), rx);
+            ldmatrix_x4_trans(lbase + 4096u * static_cast<uint32_t>(4 + (q ^ col_sw_addr)), ry);
+            if constexpr (SIGNED) {
+              const int64_t r0t = row0 + 64 * (lane & 3) + 8 * (q ^ col_sw);
+              uint32_t mx[4], my[4];
+              const bool in = neg_r != nullptr && r0t < rows;
+              sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t)) : make_uint2(0u, 0u), mx);
+              sign_masks_bf16x8(in ? __ldg(reinterpret_cast<const uint2*>(neg_r + r0t + 32)) : make_uint2(0u, 0u), my);
   #pragma unroll
-            for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+              for (int mm = 0; mm < 4; ++mm) {
+                rx[mm] ^= mx[mm];
+                ry[mm] ^= my[mm];
+              }
+            }
+            xunpack(q, rx, ry, v);
+          }
+          release(q0 + s);
+          xrotate<K, !Q>(v, csA, cnsA, csB, cnsB, 1, 2, amr);
+          if constexpr (Q) {
+            const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
+            if (!qr.abort) {  // uniform: every lane takes part in the code-word exchange
+              const bool col_in = gc < cols;
+              uint32_t wx[8], wy[8];
+              xcodes<MODE>(v, csr, qr.zero, wx, wy);
+              const int a = lane & 3;
+              auto pos_of = [&](int h) -> int64_t {
+                if constexpr (K <= 64) return 64 * a + 32 * h;
+                else if constexpr (K == 128) return 32 * h + 64 * (a & 1) + 128 * (a >> 1);
+                else return 32 * h + 64 * a;
+              };
+              auto ok_pos = [&](int64_t pr) { return col_in && row0 + pr < rows; };
+              xstore<K>(codes_r + gc * rows + row0, wx, wy, K == 256 ? a : (a & 1), 1, 2, pos_of, ok_pos, W32);
+            }
           }
         }
-        float2 v[32];
-  #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+      } else {
+        // ---- row role: rotation along the columns, kSteps steps of 8 rows x 256 columns per warp
+        const uint32_t my_strip = sbase + static_cast<uint32_t>(slot_of(sr)) * kStripBytes;
+    #pragma unroll 1
+        for (int st = 0; st < kSteps; ++st) {
+          const int g = warp + kComputeWarps * st;  // 0..31: tile rows {2g, 2g+1} + 64 * {0..3}
+          const uint32_t rowaddr = my_strip + (8u * g + swr) * 128u;
+          // sign flags of the thread's 64 columns (the randomized variant; cols is a multiple of 64,
+          // so they are all inside the tensor or all past its end)
+          uint32_t sm[SIGNED ? 32 : 1];
+        (void)sm;
           if constexpr (SIGNED) {
-            raw.x ^= sm[(4 * j) % (SIGNED ? 32 : 1)];
-            raw.y ^= sm[(4 * j + 1) % (SIGNED ? 32 : 1)];
-            raw.z ^= sm[(4 * j + 2) % (SIGNED ? 32 : 1)];
-            raw.w ^= sm[(4 * j + 3) % (SIGNED ? 32 : 1)];
+            const int64_t c0 = col0 + kStripCols * sr;
+    #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t m8[8];
+              sign_masks_bf16x16(neg_c != nullptr && c0 < cols ? __ldg(reinterpret_cast<const uint4*>(neg_c + c0 + 16 * c))
+                                                               : make_uint4(0u, 0u, 0u, 0u), m8);
+    #pragma unroll
+              for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+            }
           }
-          unpack_bf16x2(raw.x, v[4 * j]);
-          unpack_bf16x2(raw.y, v[4 * j + 1]);
-          unpack_bf16x2(raw.z, v[4 * j + 2]);
-          unpack_bf16x2(raw.w, v[4 * j + 3]);
+          float2 v[32];
+    #pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 raw = ptx::ld_shared_v4(rowaddr + ((static_cast<uint32_t>(j) ^ swr) << 4));
+            if constexpr (SIGNED) {
+              raw.x ^= sm[(4 * j) % (SIGNED ? 32 : 1)];
+              raw.y ^= sm[(4 * j + 1) % (SIGNED ? 32 : 1)];
+              raw.z ^= sm[(4 * j + 2) % (SIGNED ? 32 : 1)];
+              raw.w ^= sm[(4 * j + 3) % (SIGNED ? 32 : 1)];
+            }
+            unpack_bf16x2(raw.x, v[4 * j]);
+            unpack_bf16x2(raw.y, v[4 * j + 1]);
+            unpack_bf16x2(raw.z, v[4 * j + 2]);
+            unpack_bf16x2(raw.w, v[4 * j + 3]);
+          }
+          if (kSteps == 2 && st == 1) {
+            // this warp's last reads of the two strips it has no column step on (with 16 warps a
+            // warp's column steps cover strips grp and grp + 2; with 8 warps all four)
+            release(q0 + 1 - grp);
+            release(q0 + 3 - grp);
+          }
+          if constexpr (!Q) {
+            rotate64<K, true>(v, lane, 8, 16, amc);
+          } else {
+            rotate64<K, false>(v, lane, 8, 16, amc);
+            const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
+            const int64_t cc = col0 + kStripCols * sr;
+            if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero, lp_fmt);
+          }
         }
-        if (kSteps == 2 && st == 1) {
-          // this warp's last reads of the two strips it has no column step on (with 16 warps a
-          // warp's column steps cover strips grp and grp + 2; with 8 warps all four)
-          release(q0 + 1 - grp);
-          release(q0 + 3 - grp);
-        }
-        if constexpr (!QUANT) {
-          rotate64<K, true>(v, lane, 8, 16, amc);
-        } else {
-          rotate64<K, false>(v, lane, 8, 16, amc);
-          const int64_t r = row0 + 64 * (x >> 1) + (x & 1) + 2 * g;
-          const int64_t cc = col0 + kStripCols * sr;
-          if (!qc.abort && r < rows && cc < cols) store_codes64<MODE, W32>(codes_c + r * cols + cc, v, csc, qc.zero, lp_fmt);
-        }
-      }
 
-      // ---- col role: rotation along the rows, 8 columns of one strip per step
-  #pragma unroll 1
-      for (int j2 = 0; j2 < kSteps; ++j2) {
-        const int s = grp + (kComputeWarps / 8) * j2;
-        const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
-        // sign flags of the thread's 64 rows (rows is a multiple of 64)
-        uint32_t sm[SIGNED ? 32 : 1];
-        if constexpr (SIGNED) {
-          const int64_t r0t = row0 + 64 * (lane & 3);
-  #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t m8[8];
-            sign_masks_bf16x16(neg_r != nullptr && r0t < rows ? __ldg(reinterpret_cast<const uint4*>(neg_r + r0t + 16 * c))
-                                                              : make_uint4(0u, 0u, 0u, 0u), m8);
-  #pragma unroll
-            for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+        // ---- col role: rotation along the rows, 8 columns of one strip per step
+    #pragma unroll 1
+        for (int j2 = 0; j2 < kSteps; ++j2) {
+          const int s = grp + (kComputeWarps / 8) * j2;
+          const uint32_t lbase = sbase + static_cast<uint32_t>(slot_of(s)) * kStripBytes + col_lane_off;
+          // sign flags of the thread's 64 rows (rows is a multiple of 64)
+          uint32_t sm[SIGNED ? 32 : 1];
+        (void)sm;
+          if constexpr (SIGNED) {
+            const int64_t r0t = row0 + 64 * (lane & 3);
+    #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t m8[8];
+              sign_masks_bf16x16(neg_r != nullptr && r0t < rows ? __ldg(reinterpret_cast<const uint4*>(neg_r + r0t + 16 * c))
+                                                                : make_uint4(0u, 0u, 0u, 0u), m8);
+    #pragma unroll
+              for (int j = 0; j < 8; ++j) sm[8 * c + j] = m8[j];
+            }
           }
-        }
-        float2 v[32];
-  #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          uint32_t r4[4];
-          ldmatrix_x4_trans(lbase + 4096u * n, r4);
-  #pragma unroll
-          for (int mm = 0; mm < 4; ++mm)
-            unpack_bf16x2(SIGNED ? r4[mm] ^ sm[(4 * n + mm) % (SIGNED ? 32 : 1)] : r4[mm], v[4 * n + mm]);
-        }
-        release(q0 + s);
-        if constexpr (!QUANT) {
-          rotate64<K, true>(v, lane, 1, 2, amr);
-        } else {
-          rotate64<K, false>(v, lane, 1, 2, amr);
-          const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
-          const int64_t gr = row0 + 64 * (lane & 3);
-          if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero, lp_fmt);
+          float2 v[32];
+    #pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            uint32_t r4[4];
+            ldmatrix_x4_trans(lbase + 4096u * n, r4);
+    #pragma unroll
+            for (int mm = 0; mm < 4; ++mm)
+              unpack_bf16x2(SIGNED ? r4[mm] ^ sm[(4 * n + mm) % (SIGNED ? 32 : 1)] : r4[mm], v[4 * n + mm]);
+          }
+          release(q0 + s);
+          if constexpr (!Q) {
+            rotate64<K, true>(v, lane, 1, 2, amr);
+          } else {
+            rotate64<K, false>(v, lane, 1, 2, amr);
+            const int64_t gc = col0 + kStripCols * s + 8 * (warp & 7) + (lane >> 2);
+            const int64_t gr = row0 + 64 * (lane & 3);
+            if (!qr.abort && gc < cols && gr < rows) store_codes64<MODE, W32>(codes_r + gc * rows + gr, v, csr, qr.zero, lp_fmt);
+          }
         }
       }
     }
-  }
 
-  // every copy issued has landed before the CTA exits (all are consumed above unless a wait
-  // gave up or both rotations were abandoned)
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      if (issued_round[s] < 0) continue;
-      const uint32_t par = static_cast<uint32_t>(issued_round[s] & 1);
-      const uint64_t t0 = ptx::globaltimer_ns();
-      while (!ptx::mbar_try_wait(full_bar(s), par)) {
-        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-          atomicCAS(status, 0u, 6u);
-          break;
-        }
-      }
-    }
-  }
-  if constexpr (!QUANT) {
+  };
+  // The CTA's partial maxima of both rotations (the unnormalised |t| times fp32(1/sqrt(k)),
+  // +inf when any rotated value was not finite).
+  auto write_partials = [&]() {
     float mc = amc[0], mr = amr[0];
 #pragma unroll
     for (int j = 1; j < kAcc; ++j) {
@@ -521,7 +524,61 @@ fwhtq_dual_kernel(const __grid_constant__ CUtensorMap map, int64_t rows, int64_t
       part_c[b] = __fmul_rn(mc, c);
       part_r[b] = __fmul_rn(mr, c);
     }
+  };
+
+  if constexpr (ONCHIP) {
+    sweep(std::false_type{});
+    write_partials();
+    // grid barrier: every CTA's partials are written before any CTA reduces them (each CTA
+    // fences its write, then counts; all wait, bounded, for the count to reach the grid)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(grid_counter, 1u);
+      const uint64_t t0 = ptx::globaltimer_ns();
+      int ok = 1;
+      while (*reinterpret_cast<volatile unsigned int*>(grid_counter) < gridDim.x) {
+        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicCAS(status, 0u, 6u /* HQ_ERR_TIMEOUT */);
+          ok = 0;
+          break;
+        }
+      }
+      __threadfence();
+      grid_ok = ok;
+    }
+    __syncthreads();
+    if (grid_ok) {
+      qc = finish_absmax<MODE, true>(part_c, static_cast<int>(gridDim.x), scale_c, scratch, status, lp_fmt);
+      qr = finish_absmax<MODE, true>(part_r, static_cast<int>(gridDim.x), scale_r, scratch, status, lp_fmt);
+    } else {
+      qc.abort = qr.abort = true;
+    }
+    csc = code_scale<K>(c, qc.inv);
+    csr = code_scale<K>(c, qr.inv);
+    work_tiles = (qc.abort && qr.abort) ? 0 : my_tiles;
+    sweep(std::true_type{});
+  } else {
+    sweep(std::integral_constant<bool, QUANT>{});
   }
+
+  // every copy issued has landed before the CTA exits (all are consumed above unless a wait
+  // gave up or both rotations were abandoned)
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      if (issued_round[s] < 0) continue;
+      const uint32_t par = static_cast<uint32_t>(issued_round[s] & 1);
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!ptx::mbar_try_wait(full_bar(s), par)) {
+        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicCAS(status, 0u, 6u);
+          break;
+        }
+      }
+    }
+  }
+  if constexpr (!QUANT) write_partials();
 }
 
 }  // namespace dual

@@ -153,12 +153,13 @@ struct QuantParams {
 
 // Pass-2 prologue: reduce the partials to a, publish the scale (CTA 0), set the status
 // word on a non-finite tensor.
-template <int MODE>
+// CG: the partials were written by other CTAs of the same launch (read through L2, past L1).
+template <int MODE, bool CG = false>
 __device__ __forceinline__ QuantParams finish_absmax(const float* partials, int n_partials,
                                                      float* scale_out, float* scratch,
                                                      unsigned int* status, int lp_fmt = 0) {
   float m = 0.0f;
-  for (int i = threadIdx.x; i < n_partials; i += blockDim.x) m = fmaxf(m, partials[i]);
+  for (int i = threadIdx.x; i < n_partials; i += blockDim.x) m = fmaxf(m, CG ? __ldcg(partials + i) : partials[i]);
   const float a = block_max(m, scratch);
   const float QMAX = MODE == kModeInt8 ? 127.0f : MODE == kModeFp8 ? 448.0f : lowp_max(lp_fmt);
   QuantParams p;

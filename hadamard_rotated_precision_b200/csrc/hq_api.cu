@@ -42,6 +42,7 @@ struct DeviceInfo {
   bool cols_attr[5][4][2] = {};  // strided bf16 quantizer instantiations prepared [k][mode][signed]
   unsigned pair_attr_set = 0;  // bit per CTA-pair GEMM instantiation
   bool dual_attr[5][4][2][2] = {};  // fused two-rotation instantiations prepared [k][mode][w32][signed]
+  bool dual_onchip_attr[5][2][2][2] = {};  // its single-launch form [k][int8 / fp8][w32][signed]
   bool mn_attr[2] = {};             // MN-major pair GEMM (fp32 output) prepared [int8 / fp8]
   bool rot_attr[3] = {};            // row de-rotation with its 64 KB tile prepared [k = 64, 128, 256]
   bool rotout_attr[2] = {};         // K-major pair GEMM with fp32 rotated output prepared [int8 / fp8]
@@ -327,6 +328,46 @@ cudaError_t dual_smem_attr(DeviceInfo& d) {
   return e;
 }
 
+// The single-launch form (ONCHIP) for tensors of at most one 256 x 256 tile per SM, INT8 / FP8:
+// a cooperative launch of one CTA per tile (all resident at once, which the grid barrier
+// inside needs); the barrier counter is the last entry of the column rotation's partial array
+// (the grid uses entries 0 .. grid - 1), zeroed here before the launch.
+template <int K, int MODE, bool W32, bool SIGNED>
+hq_status launch_dual_onchip(const CUtensorMap& map, int64_t rows, int64_t cols, uint8_t* codes_c, float* scale_c,
+                             uint8_t* codes_r, float* scale_r, float* part_c, float* part_r, const uint8_t* neg_c,
+                             const uint8_t* neg_r, DeviceInfo& d, cudaStream_t st, int g) {
+  using namespace hq;
+  using namespace hq::dual;
+  auto kernel = fwhtq_dual_kernel<K, MODE, W32, SIGNED, true>;
+  constexpr int kIdx = (K == 16 ? 0 : K == 32 ? 1 : K == 64 ? 2 : K == 128 ? 3 : 4);
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    bool& done = d.dual_onchip_attr[kIdx][MODE == kModeInt8 ? 0 : 1][W32 ? 1 : 0][SIGNED ? 1 : 0];
+    if (!done) {
+      if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(kSmemBytes))) != cudaSuccess)
+        return cuda_fail(e);
+      done = true;
+    }
+  }
+  unsigned int* counter = reinterpret_cast<unsigned int*>(part_c + (kMaxPartials - 1));
+  if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), st)) != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kernel, map, rows, cols, codes_c, codes_r, part_c, part_r, g, scale_c, scale_r, d.status,
+                         0, neg_c, neg_r, 0, counter);
+  return e == cudaSuccess ? HQ_OK : cuda_fail(e);
+}
+
 // Pass 1 (both absmax partials, tiles in order) then pass 2 (both code tensors, tiles in
 // reverse order), one CTA per SM.  W32: both code buffers are 32-byte aligned, so the code
 // stores are whole 32-byte sectors.  SIGNED: the randomized variant (neg_c per column for the
@@ -339,24 +380,31 @@ hq_status launch_dual_fused_w(const CUtensorMap& map, int64_t rows, int64_t cols
   using namespace hq::dual;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
   const int g = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(n_tiles, d.sms)));
+  // at most one tile per SM: both passes in one launch over tiles resident in shared memory
+  if (n_tiles <= d.sms && fmt == HQ_INT8)
+    return launch_dual_onchip<K, kModeInt8, W32, SIGNED>(map, rows, cols, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                         part_r, neg_c, neg_r, d, st, g);
+  if (n_tiles <= d.sms && fmt == HQ_FP8_E4M3)
+    return launch_dual_onchip<K, kModeFp8, W32, SIGNED>(map, rows, cols, codes_c, scale_c, codes_r, scale_r, part_c,
+                                                        part_r, neg_c, neg_r, d, st, g);
   cudaError_t e = dual_smem_attr<K, kModeAbsmax, W32, SIGNED>(d);
   if (e != cudaSuccess) return cuda_fail(e);
   if ((e = launch_pdl(fwhtq_dual_kernel<K, kModeAbsmax, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols,
-                      codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r, 0)) !=
+                      codes_c, codes_r, part_c, part_r, 0, scale_c, scale_r, d.status, 0, neg_c, neg_r, 0, nullptr)) !=
       cudaSuccess)
     return cuda_fail(e);
   if (fmt == HQ_INT8) {
     if ((e = dual_smem_attr<K, kModeInt8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
     e = launch_pdl(fwhtq_dual_kernel<K, kModeInt8, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
-                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0, nullptr);
   } else if (fmt == HQ_FP8_E4M3) {
     if ((e = dual_smem_attr<K, kModeFp8, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
     e = launch_pdl(fwhtq_dual_kernel<K, kModeFp8, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
-                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0);
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, 0, nullptr);
   } else {
     if ((e = dual_smem_attr<K, kModeLowp, W32, SIGNED>(d)) != cudaSuccess) return cuda_fail(e);
     e = launch_pdl(fwhtq_dual_kernel<K, kModeLowp, W32, SIGNED>, g, kThreads, kSmemBytes, st, map, rows, cols, codes_c,
-                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, static_cast<int>(fmt));
+                   codes_r, part_c, part_r, g, scale_c, scale_r, d.status, 1, neg_c, neg_r, static_cast<int>(fmt), nullptr);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   return HQ_OK;

@@ -193,9 +193,14 @@ HQ_API hq_status hq_linear_bwd_dw(const void* dY, const void* X, hq_dtype dt, in
  *   codes_r [cols][rows] + scale_r: rotated along rows  (hq_quantize dim = 0)
  * rows and cols must both be multiples of k.  For a bf16 source with rows and cols multiples
  * of 64 one kernel computes both rotations from a single read of each 256 x 256 tile per pass
- * (2 launches: both absmax partials, then both code tensors); otherwise the four single-
- * rotation passes run back to back in alternating directions so that after the first one most
- * source reads are served by L2.  workspace: >= hq_quantize_dual_workspace_bytes() bytes.
+ * (2 launches: both absmax partials, then both code tensors).  When the tensor has at most one
+ * such tile per SM and the codes are INT8 or FP8, both passes run in one cooperative launch over
+ * tiles kept in shared memory, with a grid barrier between the passes (the source is read from
+ * HBM once; the barrier's counter is the workspace's last 4 bytes of the first partial array,
+ * zeroed by the call, and its wait is bounded: HQ_ERR_TIMEOUT, no codes, if it expires).
+ * Otherwise the four single-rotation passes run back to back in alternating directions so that
+ * after the first one most source reads are served by L2.  workspace: >=
+ * hq_quantize_dual_workspace_bytes() bytes.
  * Device-side errors as for hq_quantize, per rotation (a rotation whose absmax is not finite
  * writes no codes and a NaN scale; the other rotation is still written).
  * ---------------------------------------------------------------------------------------- */
