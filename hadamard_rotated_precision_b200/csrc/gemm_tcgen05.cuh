@@ -440,30 +440,66 @@ namespace pair {
 constexpr int BM = 256;    // rows per pair tile (128 per CTA)
 constexpr int HALF = 128;  // A rows per CTA
 
+// Row `lane` of a 32 x 64 bf16 output box in shared memory (128-byte swizzle: 16-byte chunk q,
+// columns 8q .. 8q+7, at q ^ (lane & 7)) from 64 accumulators (r0: columns 0-31, r1: 32-63):
+// bf16(fp32(acc) * sab).
+template <int FMT>
+__device__ __forceinline__ void write_box_row(uint32_t box, int lane, const uint32_t (&r0)[32],
+                                              const uint32_t (&r1)[32], float sab) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 8 * (q & 3) + 2 * e;
+      const uint32_t u0 = q < 4 ? r0[i] : r1[i], u1 = q < 4 ? r0[i + 1] : r1[i + 1];
+      float x0, x1;
+      if (FMT == kInt8) {
+        x0 = __int2float_rn(static_cast<int>(u0));
+        x1 = __int2float_rn(static_cast<int>(u1));
+      } else {
+        x0 = __uint_as_float(u0);
+        x1 = __uint_as_float(u1);
+      }
+      const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(x0, sab), __fmul_rn(x1, sab));
+      pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    ptx::st_shared_v4(box + uint32_t(lane * 128 + ((q ^ (lane & 7)) << 4)), pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
 // Tile geometry for an N tile of BN_ (256 or 128) columns: each CTA holds BN_/2 rows of B.
 // The bf16 epilogue stages output boxes of 32 rows x 64 columns (4 KB, 128-byte swizzle) in
-// shared memory for TMA stores.  Default shape: a 192 KB operand ring and two boxes per
-// epilogue warp.  SHORT_K (contractions of at most kShortKBlocks k-blocks, where a tile's main
-// loop is shorter than writing its output): a 128 KB ring and room for the warp's whole
-// tile share, so the accumulator is released as soon as it has been read and the stores
-// stream out while the next tiles are computed.
+// shared memory for TMA stores.  Default shape: a 192 KB operand ring, four epilogue warps
+// (one per 32-lane quarter of TMEM) and two boxes per warp.  SHORT_K (contractions of at most
+// kShortKBlocks k-blocks, where a tile's main loop is shorter than writing its output): a
+// 128 KB ring and eight epilogue warps, two per TMEM quarter, each owning half of the tile's
+// columns with room for its whole share, so the accumulator is released as soon as it has
+// been read and the stores stream out while the next tiles are computed.
+constexpr int kShortStages = 5;  // SHORT_K operand ring: stages of 32 KB (BN = 256)
+constexpr int kShortBoxes = 2;   // SHORT_K output boxes per epilogue warp
+
 template <int BN_, bool SHORT_K = false>
 struct Geo {
+  static constexpr int EPI_WARPS = SHORT_K ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;  // producer, MMA issuer, epilogue
   static constexpr int BN = BN_;
   static constexpr int B_ROWS = BN_ / 2;
   static constexpr int A_STAGE_BYTES = HALF * BK;
   static constexpr int B_STAGE_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;  // per CTA
-  static constexpr int STAGES = ((SHORT_K ? 4 : 6) * (16384 + 16384)) / STAGE_BYTES;
+  static constexpr int STAGES = ((SHORT_K ? kShortStages : 6) * (16384 + 16384)) / STAGE_BYTES;
   static constexpr int TMEM_COLS = ACC_BUFS * BN_;                      // 512 or 256
   static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
   static constexpr int BOX_COLS = 64;
   static constexpr int BOX_BYTES = 32 * BOX_COLS * 2;
-  static constexpr int CHUNKS = BN_ / BOX_COLS;         // 64-column chunks per tile and warp
-  static constexpr int NB = SHORT_K ? CHUNKS : 2;       // boxes per epilogue warp
-  static constexpr int EPI_BYTES = 4 * NB * BOX_BYTES;  // four epilogue warps
+  static constexpr int CHUNKS = BN_ / BOX_COLS / (EPI_WARPS / 4);  // 64-column chunks per tile and warp
+  static constexpr int NB = SHORT_K ? (CHUNKS < kShortBoxes ? CHUNKS : kShortBoxes) : 2;  // boxes per epilogue warp
+  static constexpr bool WHOLE = SHORT_K && NB == CHUNKS;  // the boxes hold the warp's whole tile share
+  static constexpr int EPI_BYTES = EPI_WARPS * NB * BOX_BYTES;
   static constexpr size_t SMEM_BYTES =
       1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "more dynamic shared memory than a B200 CTA may have");
 };
 
 // Tile order of the pair kernel: bands of kRasterBand M-blocks; within a band the M-block
@@ -512,7 +548,7 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
 // stride between 8-row groups (now groups along the contraction), and one MMA's 32-deep slice
 // starts 32 rows = 4096 bytes further on.  Needs BN_ = 256 (128 B rows per CTA).
 template <int FMT, int OUT, int BN_, bool SHORT_K, bool MN = false>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Geo<BN_, SHORT_K>::THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const __grid_constant__ CUtensorMap tmap_out, const float* __restrict__ scale_a,
                  const float* __restrict__ scale_b, void* __restrict__ out, int M, int N, int K,
@@ -522,6 +558,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   // before storing (see epi_rot_cols)
   using G = Geo<BN_, SHORT_K>;
   static_assert(!MN || (BN_ == 256 && !SHORT_K && OUT != kOutBf16), "MN-major operands: 256-wide tiles, direct stores");
+  static_assert(!SHORT_K || OUT == kOutBf16, "SHORT_K: bf16 output through TMA stores");
   constexpr int BN = G::BN, STAGES = G::STAGES, A_STAGE_BYTES = G::A_STAGE_BYTES;
   constexpr int B_STAGE_BYTES = G::B_STAGE_BYTES, STAGE_BYTES = G::STAGE_BYTES, TMEM_COLS = G::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -539,7 +576,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   // split; in between: only the last, partial wave's tiles, so that it takes half a tile-time.
   // A half writes its partial accumulator to part_ws; the warp slab that finishes second adds
   // the other half and writes the output (bf16 output only).
-  const int split_f = min(split_from, num_tiles);
+  const int split_f = SHORT_K ? num_tiles : min(split_from, num_tiles);  // SHORT_K never splits
   const int split_t = num_tiles - split_f;
   const int num_items = split_f + 2 * split_t;
   const int kb_half = (num_kb + 1) / 2;
@@ -573,7 +610,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     }
     for (int b = 0; b < ACC_BUFS; ++b) {
       ptx::mbar_init(tfull_bar(b), 1);
-      ptx::mbar_init(tempty_bar(b), 8);  // used in CTA 0: 4 epilogue warps x 2 CTAs
+      ptx::mbar_init(tempty_bar(b), 2 * G::EPI_WARPS);  // used in CTA 0: every epilogue warp of both CTAs
     }
     ptx::mbar_init(drain_bar, 1);
     *sh.abort_flag = 0;
@@ -591,6 +628,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   ptx::cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
   ptx::tc_fence_after_sync();
   const uint32_t tmem_base = *sh.tmem_holder;
+  // programmatic dependent launch: the set-up above overlaps the previous grid's tail; codes,
+  // scales and the output are touched only once that grid has completed
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -666,12 +707,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     }
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;  // the TMEM lanes this warp may read: 32 * quarter ..
+    const int ew = warp - 2;       // epilogue warp 0 .. EPI_WARPS - 1
+    const int chunk0 = (ew >> 2) * G::CHUNKS;  // first 64-column chunk of this warp's columns
     const float sab = (OUT != kOutAcc) ? __fmul_rn(*scale_a, *scale_b) : 0.0f;
     // bf16 output: chunk j (64 columns) of this warp's 32 rows goes TMEM -> registers -> a
     // swizzled 32 x 64 box in shared memory -> TMA store (asynchronous).  Box b of the warp's
-    // NB boxes is rewritten only once the store that last used it has read it.
-    const uint32_t epi_base = ptx::smem_u32(sh.epi) + uint32_t(quarter) * uint32_t(G::NB * G::BOX_BYTES);
+    // NB boxes is rewritten only once the store that last used it has read it.  SHORT_K: the
+    // warp's boxes hold its whole share of the tile; they are all written, made visible to the
+    // TMA engine with one proxy fence and stored as one group.
+    const uint32_t epi_base = ptx::smem_u32(sh.epi) + uint32_t(ew) * uint32_t(G::NB * G::BOX_BYTES);
     int box_group[G::NB];  // commit index of the store that last used each box (-1: none)
 #pragma unroll
     for (int b = 0; b < G::NB; ++b) box_group[b] = -1;
@@ -727,11 +772,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(tempty_bar(acc), 0));
           }
         }
+        if constexpr (G::WHOLE) {  // the previous tile's stores have read every box
+          if (lane == 0 && ncommit > 0) ptx::bulk_wait_read<0>();
+          __syncwarp();
+        }
 #pragma unroll
         for (int j = 0; j < G::CHUNKS && emit; ++j) {
           uint32_t r0[32], r1[32];
-          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64), r0);
-          ptx::tmem_ld_32x32b_x32(t_row + uint32_t(j * 64 + 32), r1);
+          ptx::tmem_ld_32x32b_x32(t_row + uint32_t((chunk0 + j) * 64), r0);
+          ptx::tmem_ld_32x32b_x32(t_row + uint32_t((chunk0 + j) * 64 + 32), r1);
           ptx::tmem_ld_wait(r0);
           ptx::reg_fence(r1);
           if (peer) {  // own + other half: one rounding per element (fp32) or exact (int32)
@@ -753,42 +802,40 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           }
           const int b = j % G::NB;
           const uint32_t box = epi_base + uint32_t(b * G::BOX_BYTES);
-          if (lane == 0 && box_group[b] >= 0) {
-            if (ncommit - 1 - box_group[b] >= G::NB - 1) ptx::bulk_wait_read<G::NB - 1>();
-            else ptx::bulk_wait_read<0>();
+          if constexpr (!G::WHOLE) {
+            if (lane == 0 && box_group[b] >= 0) {
+              if (ncommit - 1 - box_group[b] >= G::NB - 1) ptx::bulk_wait_read<G::NB - 1>();
+              else ptx::bulk_wait_read<0>();
+            }
+            __syncwarp();
           }
-          __syncwarp();
-          // row `lane` of the box: 16-byte chunk q (columns 8q .. 8q+7) at q ^ (lane & 7)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 8 * (q & 3) + 2 * e;
-              const uint32_t u0 = q < 4 ? r0[i] : r1[i], u1 = q < 4 ? r0[i + 1] : r1[i + 1];
-              float x0, x1;
-              if (FMT == kInt8) {
-                x0 = __int2float_rn(static_cast<int>(u0));
-                x1 = __int2float_rn(static_cast<int>(u1));
-              } else {
-                x0 = __uint_as_float(u0);
-                x1 = __uint_as_float(u1);
+          write_box_row<FMT>(box, lane, r0, r1, sab);
+          if constexpr (!G::WHOLE) {
+            ptx::fence_proxy_async_smem();  // the box is visible to the TMA engine
+            __syncwarp();
+            const int col0 = n_blk * BN + (chunk0 + j) * G::BOX_COLS;
+            if (col0 < N && row0 < M) {  // boxes reaching past the edge are clipped by TMA
+              if (lane == 0) {
+                ptx::tma_store_2d(&tmap_out, box, col0, row0);
+                ptx::bulk_commit();
               }
-              const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(x0, sab), __fmul_rn(x1, sab));
-              pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+              box_group[b] = ncommit++;
             }
-            ptx::st_shared_v4(box + uint32_t(lane * 128 + ((q ^ (lane & 7)) << 4)), pk[0], pk[1], pk[2], pk[3]);
           }
-          ptx::fence_proxy_async_smem();  // the box is visible to the TMA engine
+        }
+        if constexpr (G::WHOLE) {
+          ptx::fence_proxy_async_smem();  // the boxes are visible to the TMA engine
           __syncwarp();
-          const int col0 = n_blk * BN + j * G::BOX_COLS;
-          if (col0 < N && row0 < M) {  // boxes reaching past the edge are clipped by TMA
-            if (lane == 0) {
-              ptx::tma_store_2d(&tmap_out, box, col0, row0);
-              ptx::bulk_commit();
+          if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < G::CHUNKS; ++j) {
+              const int col0 = n_blk * BN + (chunk0 + j) * G::BOX_COLS;
+              if (col0 < N && row0 < M)  // boxes reaching past the edge are clipped by TMA
+                ptx::tma_store_2d(&tmap_out, epi_base + uint32_t(j * G::BOX_BYTES), col0, row0);
             }
-            box_group[b] = ncommit++;
+            ptx::bulk_commit();
           }
+          ++ncommit;
         }
         if (peer && lane == 0) *slab_counter = 0;  // both halves counted: ready for the next launch
       } else {

@@ -626,7 +626,7 @@ hq_status check_gemm_args(const void* A, const float* sa, const void* B, const f
 }
 
 // Co-resident 2-CTA clusters of a pair-GEMM instantiation (cached per device).
-int pair_clusters(const void* kernel, size_t smem, int sms) {
+int pair_clusters(const void* kernel, size_t smem, int sms, int threads) {
   static std::mutex mu;
   static const void* keys[64];
   static int devs[64], vals[64];
@@ -638,7 +638,7 @@ int pair_clusters(const void* kernel, size_t smem, int sms) {
     if (keys[i] == kernel && devs[i] == dev) return vals[i];
   cudaLaunchConfig_t q = {};
   q.gridDim = dim3(2 * (sms / 2));
-  q.blockDim = dim3(hq::gemm::NUM_THREADS);
+  q.blockDim = dim3(threads);
   q.dynamicSmemBytes = smem;
   cudaLaunchAttribute qa[1];
   qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -672,16 +672,18 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
   const int pairs = std::max(1, std::min(items, clusters));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(hq::gemm::NUM_THREADS);
+  cfg.blockDim = dim3(G::THREADS);
   cfg.dynamicSmemBytes = G::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait in the kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   (void)d;
   return cudaLaunchKernelEx(&cfg, kernel, ta, tb, to, sa, sb, out, M, N, K, d.status, split_from, part_ws, counters,
                             ab_code, rot_k);
@@ -703,7 +705,7 @@ cudaError_t pair_prepare(DeviceInfo& d, int* clusters) {
       d.pair_attr_set |= bit;
     }
   }
-  *clusters = pair_clusters(reinterpret_cast<const void*>(kernel), G::SMEM_BYTES, d.sms);
+  *clusters = pair_clusters(reinterpret_cast<const void*>(kernel), G::SMEM_BYTES, d.sms, G::THREADS);
   return cudaSuccess;
 }
 
@@ -881,7 +883,7 @@ hq_status gemm_mn_f32_impl(const void* A, const float* sa, const void* B, const 
       d.mn_attr[f] = true;
     }
   }
-  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms);
+  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms, G::THREADS);
   CUtensorMap ta, tb, to;
   std::memset(&to, 0, sizeof(to));
   // boxes of 128 contraction rows x 128 bytes along M (N): the K-major map with the roles of
@@ -975,7 +977,7 @@ hq_status gemm_rotout_impl(const void* A, const float* sa, const void* B, const 
       d.rotout_attr[f] = true;
     }
   }
-  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms);
+  const int clusters = pair_clusters(kernel, G::SMEM_BYTES, d.sms, G::THREADS);
   CUtensorMap ta, tb, to;
   std::memset(&to, 0, sizeof(to));
   hq_status s = encode_codes_map(&ta, A, M, K, gp::HALF);
