@@ -846,9 +846,10 @@ def run_kernel_case(args):
         return 0 if st == 0 else 1
     if case.startswith("gemm"):
         fmt = "fp8" if case == "gemm_fp8" else "int8"
-        # the Llama up-projection forward shape, or the ViT-B fc1 forward (contraction 768), or
-        # --shape M,N,K
-        M, N, K = (12608, 3072, 768) if case == "gemm_short_k" else (4096, 11008, 4096)
+        # the Llama up-projection forward shape, or the ViT-B fc1 forward (contraction 768), or its
+        # dX (contraction 11008: 3.46 waves of tiles, the last wave split along the contraction
+        # through the workspace), or --shape M,N,K
+        M, N, K = {"gemm_short_k": (12608, 3072, 768), "gemm_split": (4096, 4096, 11008)}.get(case, (4096, 11008, 4096))
         if args.shape:
             M, N, K = (int(v) for v in args.shape.split(","))
         A = torch.randint(-127, 128, (M, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
@@ -858,8 +859,25 @@ def run_kernel_case(args):
             B = B & 0x77
         s = torch.full((1,), 0.01, device="cuda")
         out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        ws = None
+        if case == "gemm_split":
+            ws = torch.empty(max(16, hq.hq_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device="cuda")
         for _ in range(2):
-            hq.hq_gemm(A, s, B, s, fmt, out=out)
+            hq.hq_gemm(A, s, B, s, fmt, out=out, workspace=ws)
+    elif case == "rotout":
+        # the next layer's rotation in the epilogue: 4096 x 4096 x 4096 INT8, fp32 output rotated
+        # along its columns in blocks of 256 (64 MB)
+        M = N = K = 4096
+        A = torch.randint(-127, 128, (M, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        B = torch.randint(-127, 128, (N, K), generator=g, device="cuda", dtype=torch.int32).to(torch.int8).view(torch.uint8)
+        s = torch.full((1,), 0.01, device="cuda")
+        for _ in range(2):
+            hq.hq_gemm_rotout(A, s, B, s, 256, "int8")
+    elif case == "prerot":
+        # codes of already-rotated fp32 values, 4096 x 11008 (180 MB)
+        y = torch.randn(4096, 11008, generator=g, device="cuda")
+        for _ in range(2):
+            hq.hq_quantize_prerotated(y, "int8")
     elif case == "dx_reuse":
         # a dX of the reuse placement at 4096 tokens, K = 4096, contraction 8192 (codes 2 x 32 MB,
         # fp32 output 64 MB + bf16 32 MB: more than L2)
@@ -890,7 +908,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("hq", "reference"), default="hq")
-    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "quant_rows", "quant_cols", "quant_dual",
+    ap.add_argument("--kernel-case", choices=("gemm", "gemm_fp8", "gemm_short_k", "gemm_split", "rotout", "prerot",
+                                              "quant_rows", "quant_cols", "quant_dual",
                                               "dx_reuse", "block_step"),
                     help="run one small standalone kernel case (for profiler captures) and exit")
     ap.add_argument("--shape", help="with --kernel-case gemm / gemm_fp8: M,N,K of the GEMM")
