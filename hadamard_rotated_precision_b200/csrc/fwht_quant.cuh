@@ -37,6 +37,7 @@
 #include "sm100_ptx.cuh"
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 
 namespace hq {
 
@@ -282,8 +283,9 @@ __device__ __forceinline__ CodeScale code_scale(float c, float inv) {
   return s;
 }
 
-// Codes of 4 consecutive rotated values (t0.x, t0.y, t1.x, t1.y) at the scale of cs.
-template <int MODE>
+// Codes of 4 consecutive rotated values (t0.x, t0.y, t1.x, t1.y) at the scale of cs, in its
+// one-multiply form (ONE_MUL, valid when cs.one_mul) or its two-multiply form.
+template <int MODE, bool ONE_MUL>
 __device__ __forceinline__ uint32_t scaled_codes4(float2 t0, float2 t1, const CodeScale& cs, int lp_fmt);
 
 // Codes of 4 consecutive elements for any mode (the minifloats' format at run time).
@@ -305,10 +307,10 @@ __device__ __forceinline__ uint32_t codes4x(float2 z0, float2 z1, int lp_fmt) {
   }
 }
 
-template <int MODE>
+template <int MODE, bool ONE_MUL>
 __device__ __forceinline__ uint32_t scaled_codes4(float2 t0, float2 t1, const CodeScale& cs, int lp_fmt) {
-  return cs.one_mul ? codes4x<MODE>(mul2(t0, cs.ci2), mul2(t1, cs.ci2), lp_fmt)
-                    : codes4x<MODE>(mul2(mul2(t0, cs.c2), cs.inv2), mul2(mul2(t1, cs.c2), cs.inv2), lp_fmt);
+  return ONE_MUL ? codes4x<MODE>(mul2(t0, cs.ci2), mul2(t1, cs.ci2), lp_fmt)
+                 : codes4x<MODE>(mul2(mul2(t0, cs.c2), cs.inv2), mul2(mul2(t1, cs.c2), cs.inv2), lp_fmt);
 }
 
 // Tensor-core operand layout of the minifloat codes: each group of 16 consecutive codes along
@@ -746,15 +748,15 @@ __device__ __forceinline__ void xrotate(float2 (&v)[32], float2 sA, float2 nsA, 
 
 // Code words of a thread's rotated values: wx[q] = codes of positions 4q .. 4q + 3 (the .x
 // halves of v[4q .. 4q + 3]), wy[q] the same for the .y halves, little-endian.
-template <int MODE>
-__device__ __forceinline__ void xcodes(const float2 (&v)[32], const CodeScale& cs, bool zero, uint32_t (&wx)[8],
-                                       uint32_t (&wy)[8]) {
+template <int MODE, bool ONE_MUL>
+__device__ __forceinline__ void xcodes_at(const float2 (&v)[32], const CodeScale& cs, bool zero, uint32_t (&wx)[8],
+                                          uint32_t (&wy)[8]) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     float2 z[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      z[i] = cs.one_mul ? mul2(v[4 * q + i], cs.ci2) : mul2(mul2(v[4 * q + i], cs.c2), cs.inv2);
+      z[i] = ONE_MUL ? mul2(v[4 * q + i], cs.ci2) : mul2(mul2(v[4 * q + i], cs.c2), cs.inv2);
     if constexpr (MODE == kModeInt8) {
       // z + 1.5 * 2^23: the low byte is rne(z) in two's complement (see codes4).  The add is
       // the scalar __fadd_rn: with a packed add the compiler fused it with the packed multiply
@@ -779,6 +781,15 @@ __device__ __forceinline__ void xcodes(const float2 (&v)[32], const CodeScale& c
     }
     if (zero) wx[q] = wy[q] = 0u;
   }
+}
+
+// The scale's one-multiply form is chosen once for all of the thread's values (a branch on a
+// warp-uniform flag), so each value takes one multiply by fp32(c * inv) or two.
+template <int MODE>
+__device__ __forceinline__ void xcodes(const float2 (&v)[32], const CodeScale& cs, bool zero, uint32_t (&wx)[8],
+                                       uint32_t (&wy)[8]) {
+  if (cs.one_mul) xcodes_at<MODE, true>(v, cs, zero, wx, wy);
+  else xcodes_at<MODE, false>(v, cs, zero, wx, wy);
 }
 
 __device__ __forceinline__ void st_global_8B(void* p, uint32_t a, uint32_t b) {
@@ -1117,19 +1128,25 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
         const int64_t row = r0 + 64 * (lane & 3);
         if (col < cols) {
           uint8_t* o = codes + col * rows + row;
+          // the scale's form chosen once for the thread's values (a warp-uniform flag)
+          auto emit = [&](auto one_tag) {
+            constexpr bool ONE = decltype(one_tag)::value;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (row + 16 * j < rows) {
-              uint32_t w[4];
+            for (int j = 0; j < 4; ++j) {
+              if (row + 16 * j < rows) {
+                uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int i = 8 * j + 2 * e;
-                w[e] = qp.zero ? 0u : scaled_codes4<MODE>(v[i], v[i + 1], cs, lp_fmt);
+                for (int e = 0; e < 4; ++e) {
+                  const int i = 8 * j + 2 * e;
+                  w[e] = qp.zero ? 0u : scaled_codes4<MODE, ONE>(v[i], v[i + 1], cs, lp_fmt);
+                }
+                *reinterpret_cast<uint4*>(o + 16 * j) = MODE == kModeLowp ? lowp_pack16(w[0], w[1], w[2], w[3], lp_fmt)
+                                                                          : make_uint4(w[0], w[1], w[2], w[3]);
               }
-              *reinterpret_cast<uint4*>(o + 16 * j) =
-                  MODE == kModeLowp ? lowp_pack16(w[0], w[1], w[2], w[3], lp_fmt) : make_uint4(w[0], w[1], w[2], w[3]);
             }
-          }
+          };
+          if (cs.one_mul) emit(std::true_type{});
+          else emit(std::false_type{});
         }
       }
       buf = buf == 2 ? 0 : buf + 1;
