@@ -943,6 +943,27 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
 
+// Row and column block of a tile index t = tr * n_ct + tc that advances by a fixed step (either
+// sign): one 64-bit division at the start, then an add with one carry per step (a 64-bit
+// division per tile cost a few instructions per element in the strided kernel's integer work).
+struct TileWalk {
+  int64_t tr, tc, dr, dc, n_ct;
+  __device__ __forceinline__ void init(int64_t t, int64_t step, int64_t nct) {
+    n_ct = nct;
+    tr = t / nct;
+    tc = t - tr * nct;
+    if (tc < 0) { tc += nct; --tr; }  // floor division for a t before the first tile
+    dr = step / nct;
+    dc = step - dr * nct;
+    if (dc < 0) { dc += nct; --dr; }
+  }
+  __device__ __forceinline__ void advance() {
+    tr += dr;
+    tc += dc;
+    if (tc >= n_ct) { tc -= n_ct; ++tr; }
+  }
+};
+
 template <int K, int MODE, bool SIGNED>
 __global__ void __launch_bounds__(kQuantThreads)
 fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int64_t cols,
@@ -978,9 +999,9 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
   // multiple of 128)
   const bool w32 = (reinterpret_cast<uintptr_t>(codes) & 31u) == 0;
 
-  // load a tile: thread T copies 16-byte chunk (T & 7) of rows (T >> 3) + 32 j
-  auto issue = [&](int buf, int64_t t) {
-    const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+  // load tile (tr, tc): thread T copies 16-byte chunk (T & 7) of rows (T >> 3) + 32 j
+  auto issue = [&](int buf, int64_t tr, int64_t tc) {
+    const int64_t r0 = tr * kColsTileRows2, c0 = tc * kColsTileCols2;
     const int ch = threadIdx.x & 7;
     const int64_t gc = c0 + 8 * ch;
 #pragma unroll
@@ -1001,12 +1022,19 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
     const int64_t step = reverse ? -G : G;
     auto valid = [&](int64_t t) { return reverse ? t >= 0 : t < n_tiles; };
     int buf = 0;
-    issue(0, first);
-    if (valid(first + step)) issue(1, first + step);
-    for (int64_t t = first; valid(t); t += step) {
+    TileWalk cur, ahead;  // tile t and tile t + 2 step
+    cur.init(first, step, n_ct);
+    ahead.init(first + 2 * step, step, n_ct);
+    issue(0, cur.tr, cur.tc);
+    if (valid(first + step)) {
+      TileWalk next;
+      next.init(first + step, step, n_ct);
+      issue(1, next.tr, next.tc);
+    }
+    for (int64_t t = first; valid(t); t += step, cur.advance(), ahead.advance()) {
       // keep two tiles in flight; wait only for this tile's copies
       if (valid(t + 2 * step)) {
-        issue(buf == 0 ? 2 : buf - 1, t + 2 * step);
+        issue(buf == 0 ? 2 : buf - 1, ahead.tr, ahead.tc);
         cp_async_wait<2>();
       } else if (valid(t + step)) {
         cp_async_wait<1>();
@@ -1036,7 +1064,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
           if constexpr (SIGNED) {
             // flags of the thread's own rows: 8-row group (q ^ sw_own) and the one 32 rows on
             // (16-row chunks are wholly inside or outside: rows is a multiple of 16)
-            const int64_t r0t = (t / n_ct) * kColsTileRows2 + 64 * a + 8 * (q ^ sw_own);
+            const int64_t r0t = cur.tr * kColsTileRows2 + 64 * a + 8 * (q ^ sw_own);
             uint32_t mx[4], my[4];
             sign_masks_bf16x8(r0t < rows ? __ldg(reinterpret_cast<const uint2*>(neg + r0t)) : make_uint2(0u, 0u), mx);
             sign_masks_bf16x8(r0t + 32 < rows ? __ldg(reinterpret_cast<const uint2*>(neg + r0t + 32)) : make_uint2(0u, 0u),
@@ -1056,7 +1084,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
         xrotate<K, !QUANT>(v, sA, nsA, sB, nsB, 1, 2, am);
         if constexpr (QUANT) {
           if (!qp.abort) {  // uniform: every lane takes part in the code-word exchange
-            const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+            const int64_t r0 = cur.tr * kColsTileRows2, c0 = cur.tc * kColsTileCols2;
             const int64_t col = c0 + 8 * warp + (lane >> 2);
             uint32_t wx[8], wy[8];
             xcodes<MODE>(v, cs, qp.zero, wx, wy);
@@ -1091,7 +1119,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
         // the tensor: rows is a multiple of 16); rows past the end stay unflipped zeros
         uint32_t sm[SIGNED ? 32 : 1];
         if constexpr (SIGNED) {
-          const int64_t r0t = (t / n_ct) * kColsTileRows2 + 64 * (lane & 3);
+          const int64_t r0t = cur.tr * kColsTileRows2 + 64 * (lane & 3);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t m8[8];
@@ -1123,7 +1151,7 @@ fwhtq_cols_bf16_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, int6
 #pragma unroll
         for (int i = 0; i < 32; ++i) amax = absmax3(amax, v[i].x, v[i].y);
       } else {
-        const int64_t r0 = (t / n_ct) * kColsTileRows2, c0 = (t % n_ct) * kColsTileCols2;
+        const int64_t r0 = cur.tr * kColsTileRows2, c0 = cur.tc * kColsTileCols2;
         const int64_t col = c0 + 8 * warp + (lane >> 2);
         const int64_t row = r0 + 64 * (lane & 3);
         if (col < cols) {
