@@ -1228,9 +1228,12 @@ fwhtq_cols_f32_kernel(const SrcT* __restrict__ src, int64_t rows, int64_t cols,
     const int64_t G = gridDim.x;
     const int64_t b = blockIdx.x;
     const int64_t last = b + G * ((n_tiles - 1 - b) / G);
-    for (int64_t t = reverse ? last : b; reverse ? t >= 0 : t < n_tiles; t += reverse ? -G : G) {
-      const int64_t r0 = (t / n_ct) * kColsTileRows;
-      const int64_t c0 = (t % n_ct) * TCOLS;
+    const int64_t first = reverse ? last : b, step = reverse ? -G : G;
+    TileWalk cur;
+    cur.init(first, step, n_ct);
+    for (int64_t t = first; reverse ? t >= 0 : t < n_tiles; t += step, cur.advance()) {
+      const int64_t r0 = cur.tr * kColsTileRows;
+      const int64_t c0 = cur.tc * TCOLS;
       __syncthreads();  // previous tile's gather is done before the tile is overwritten
       {
         const int ch = threadIdx.x & 7;
