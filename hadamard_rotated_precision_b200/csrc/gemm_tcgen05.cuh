@@ -473,7 +473,7 @@ __device__ __forceinline__ void write_box_row(uint32_t box, int lane, const uint
 // shared memory for TMA stores.  Default shape: a 192 KB operand ring, four epilogue warps
 // (one per 32-lane quarter of TMEM) and two boxes per warp.  SHORT_K (contractions of at most
 // kShortKBlocks k-blocks, where a tile's main loop is shorter than writing its output): a
-// 128 KB ring and eight epilogue warps, two per TMEM quarter, each owning half of the tile's
+// 160 KB ring and eight epilogue warps, two per TMEM quarter, each owning half of the tile's
 // columns with room for its whole share, so the accumulator is released as soon as it has
 // been read and the stores stream out while the next tiles are computed.
 constexpr int kShortStages = 5;  // SHORT_K operand ring: stages of 32 KB (BN = 256)
